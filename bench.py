@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the masked WIDE layer on B200; prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_ffn_3b]
+
+Workload ``decode_ffn_3b`` (default): the Llama-3.2-3B-shaped masked SwiGLU FFN
+in decode -- hidden 3072, intermediate 8192 in 64 channel groups of 128,
+bf16 weights ~ N(0, 0.02), x ~ N(0, 1), per-(token, group) keep mask
+Bernoulli(0.5).  One step runs the three batch sizes of that configuration
+(1, 8 and 32 tokens, each with its own x and mask) through the library's
+C ABI; tokens per step = 41.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
+device synchronise on both sides.  Each call is timed with CUDA events on the
+launch stream after an L2 flush (a 256 MiB write) that sits outside the
+events; ms_per_step is the sum of the call times, maximised over ranks.
+Kernel times for the roofline come from the library's own per-launch events
+(wide_profile_*) recorded during the same timed steps.  SM clocks and
+throttle reasons are sampled through NVML during the timed steps.
+
+Multi-GPU: every rank runs the same workload on its own GPU (replicas, weak
+scaling); value = all ranks' tokens / the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle (oracle/, the per-token loop
+over kept groups) on the host cores, one bounded token sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "masked-layer tok/s @50% sparsity; HBM GB/s (decode), TFLOPS (prefill)"
+BATCHES = (1, 8, 32)
+FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def _workload_desc():
+    return ("decode_ffn_3b: Llama-3.2-3B-shaped masked SwiGLU FFN decode, hidden 3072, "
+            "intermediate 8192 = 64 groups x 128, bf16, Bernoulli(0.5) masks; one step = "
+            "batches 1, 8 and 32 (41 tokens)")
+
+
+def _union_groups(mask_bool):
+    return int(mask_bool.any(axis=0).sum())
+
+
+def algorithmic_bytes(case):
+    """Bytes a call must move at minimum: every weight byte of the batch's
+    union of groups once, plus x, mask, the fp32 h it writes and reads back,
+    and out."""
+    B, H, I, gs = case.T, case.H, case.I, case.gs
+    U = _union_groups(case.mask)
+    pairs = int(case.mask.sum())
+    w_gateup = 2 * U * gs * H * 2
+    w_down = H * U * gs * 2
+    x = B * H * 2
+    m = case.mask_words.nbytes
+    h = pairs * gs * 4
+    out = B * H * 2
+    return {"gateup": w_gateup + x + m + h, "down": w_down + h + m + out,
+            "total": w_gateup + w_down + x + m + 2 * h + out, "union_groups": U}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only)."""
+
+    def __init__(self, index: int, period: float = 0.01):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nv = nv
+            self._h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self.ok = True
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=2)
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "source": "nvml" if self.ok else "unavailable"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def _traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source it was taken on is unchanged."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[workload][kernel]
+        src = os.path.join(ROOT, rec["source"])
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if digest != rec["source_sha256_16"]:
+            return None
+        return rec
+    except Exception:
+        return None
+
+
+def cpu_oracle_baseline(cases, seconds: float = 10.0):
+    """Times the oracle's per-token loop (fp64, OpenMP over tokens) on the
+    host: all tokens of one step, repeated until `seconds` have passed."""
+    import oracle
+    from oracle import _clib
+    tokens, t0, reps = 0, time.perf_counter(), 0
+    while True:
+        for c in cases:
+            oracle.ffn.ffn_token_loop(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs, "bf16")
+            tokens += c.T
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": tokens / el, "unit": "tokens/s", "cores": int(_clib.lib().oracle_num_threads()),
+            "kind": "oracle",
+            "sample": f"{reps} repetitions of one full step ({sum(c.T for c in cases)} tokens: "
+                      f"batches {', '.join(str(c.T) for c in cases)}), fp64 per-token loop over "
+                      f"kept groups, {el:.1f} s"}
+
+
+def _make_cases():
+    import synth
+    base = synth.decode_ffn(BATCHES[0])
+    cases = [base]
+    for b in BATCHES[1:]:
+        c = synth.decode_ffn(b, weights=False)
+        c.w_gate, c.w_up, c.w_down = base.w_gate, base.w_up, base.w_down
+        cases.append(c)
+    return cases
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from oracle import _clib
+    cases = _make_cases()
+    # bounded sample per step: the first token of every batch
+    samples = []
+    for c in cases:
+        s = type(c)(**{**c.__dict__})
+        s.x, s.mask, s.T = c.x[:1], c.mask[:1], 1
+        samples.append(s)
+
+    def step():
+        for s in samples:
+            oracle.ffn.ffn_token_loop(s.x, s.w_gate, s.w_up, s.w_down, s.mask_words, s.gs, "bf16")
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    tok = args.steps * len(samples)
+    v = tok / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": _workload_desc(), "parallelism": "host cores"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": int(_clib.lib().oracle_num_threads()),
+                         "kind": "oracle",
+                         "sample": "per step: token 0 of each of batches 1, 8, 32 (3 tokens), "
+                                   "fp64 per-token loop over kept groups"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(dev)
+
+    import token_level_dynamic_b200 as w
+    from synth.torch_io import to_dev
+
+    cases = _make_cases()
+    base = cases[0]
+    Wg = to_dev(base.w_gate, "bf16", dev)
+    Wu = to_dev(base.w_up, "bf16", dev)
+    Wd = to_dev(base.w_down, "bf16", dev)
+    xs = [to_dev(c.x, "bf16", dev) for c in cases]
+    ms = [to_dev(c.mask_words, "mask", dev) for c in cases]
+    outs = [torch.empty_like(x) for x in xs]
+    ws_bytes = max(w.wide_ffn_workspace_bytes(c.T, c.H, c.I, c.gs) for c in cases)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    gs = base.gs
+    PATH = w.WIDE_PATH_DECODE
+    ab = [algorithmic_bytes(c) for c in cases]
+
+    def call(i, mask=None):
+        w.wide_ffn_masked(xs[i], Wg, Wu, Wd, ms[i] if mask is None else mask, gs, out=outs[i],
+                          workspace=ws, path=PATH, stream=stream)
+
+    def timed_step(fn, nstreams=len(cases)):
+        evs = []
+        for i in range(nstreams):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn(i)
+            e1.record(stream)
+            evs.append((e0, e1))
+        return evs
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # correctness guard: one call each, status word clean
+    w.wide_clear_device_status(stream)
+    for _ in range(args.warmup):
+        timed_step(call)
+    torch.cuda.synchronize(dev)
+    if w.wide_get_device_status(stream) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # ---- timed region
+    w.wide_profile_start(65536)
+    n0 = w.wide_launch_count()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier()
+        all_evs = [timed_step(call) for _ in range(args.steps)]
+        barrier()
+    launches = w.wide_launch_count() - n0
+    w.wide_profile_stop()
+    recs = w.wide_profile_read()
+    per_call = np.array([[e0.elapsed_time(e1) for (e0, e1) in evs] for evs in all_evs])  # [K][3] ms
+    step_ms = float(per_call.sum(axis=1).mean())
+    total_ms = float(per_call.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        step_ms = total_ms / args.steps
+    tokens_per_step = sum(c.T for c in cases)
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # per-kernel durations (the library's own launch events)
+    kern = {}
+    for name, t in recs:
+        kern.setdefault(name, []).append(t)
+    peaks = _peaks()
+    nb = len(cases)
+    kernels = {}
+    for name, key in (("decode_gateup_gemv", "gateup"), ("decode_down_gemv", "down")):
+        ts = kern.get(name, [])
+        if not ts:
+            continue
+        # launches cycle through the batches in step order
+        per_b = [ts[i::nb] for i in range(nb)]
+        bytes_step = sum(a[key] for a in ab)
+        t_step = sum(statistics.mean(p) for p in per_b)
+        gbs = bytes_step / (t_step / 1e3) / 1e9
+        kernels[name] = {
+            "launches": len(ts), "avg_us": 1e3 * statistics.mean(ts),
+            "per_batch_us": {str(c.T): 1e3 * statistics.mean(p) for c, p in zip(cases, per_b)},
+            "algorithmic_bytes_per_step": bytes_step, "achieved_gbs": gbs,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"],
+        }
+    dom = "decode_gateup_gemv"
+    dk = kernels.get(dom)
+    traffic = _traffic_record(dom, "decode_ffn_3b")
+    roofline = None
+    if dk:
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved_gbs"],
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": dk["achieved_gbs"] / peaks["hbm_gbs"],
+                    "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)",
+                    "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                    "note": "achieved = union-of-groups gate/up weight bytes + x + mask + h, "
+                            "summed over the three batch sizes / summed mean launch time"}
+
+    per_batch = {}
+    for i, c in enumerate(cases):
+        t = float(per_call[:, i].mean())
+        per_batch[str(c.T)] = {
+            "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3),
+            "union_groups": ab[i]["union_groups"], "algorithmic_bytes": ab[i]["total"],
+            "achieved_gbs": ab[i]["total"] / (t / 1e3) / 1e9,
+            "frac_of_hbm": ab[i]["total"] / (t / 1e3) / 1e9 / peaks["hbm_gbs"],
+        }
+
+    # ---- dense baselines (same shapes): torch/cuBLAS bf16, and our kernels with all-ones masks
+    ones = [torch.full_like(m, -1) for m in ms]  # 64 groups -> two full words
+    def dense_torch(i):
+        x = xs[i]
+        a = torch.nn.functional.linear(x, Wg)
+        b = torch.nn.functional.linear(x, Wu)
+        outs[i].copy_(torch.nn.functional.linear(torch.nn.functional.silu(a) * b, Wd))
+    def ours_ones(i):
+        call(i, ones[i])
+    dense = {}
+    for name, fn in (("torch_cublas_bf16", dense_torch), ("ours_all_groups_kept", ours_ones)):
+        for _ in range(3):
+            timed_step(fn)
+        evs = [timed_step(fn) for _ in range(max(5, args.steps // 4))]
+        torch.cuda.synchronize(dev)
+        pc = np.array([[a.elapsed_time(b) for a, b in e] for e in evs])
+        dense[name] = {"ms_per_step": float(pc.sum(axis=1).mean()),
+                       "tokens_per_s": tokens_per_step / (float(pc.sum(axis=1).mean()) / 1e3),
+                       "per_batch_us": {str(c.T): 1e3 * float(pc[:, i].mean())
+                                        for i, c in enumerate(cases)}}
+    dense["masked_speedup_vs_torch_dense"] = dense["torch_cublas_bf16"]["ms_per_step"] / step_ms
+
+    # ---- end to end through the public API with host buffers
+    xh = [x.cpu().pin_memory() for x in xs]
+    mh = [m.cpu().pin_memory() for m in ms]
+    oh = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    def e2e_call(i):
+        xs[i].copy_(xh[i], non_blocking=True)
+        ms[i].copy_(mh[i], non_blocking=True)
+        call(i)
+        oh[i].copy_(outs[i], non_blocking=True)
+    for _ in range(3):
+        timed_step(e2e_call)
+    barrier()
+    e_evs = [timed_step(e2e_call) for _ in range(args.steps)]
+    barrier()
+    e_ms = float(np.array([[a.elapsed_time(b) for a, b in e] for e in e_evs]).sum())
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e = {"value": world * tokens_per_step * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(sum(x.numel() * 2 + m.numel() * 4 for x, m in zip(xh, mh))),
+           "d2h_bytes_per_step": int(sum(o.numel() * 2 for o in oh)),
+           "ms_per_step": e_ms / args.steps}
+
+    # ---- parity spot check of this run's outputs (B=8) against the oracle
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_baseline(cases, seconds=args.cpu_seconds)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of the pages' Llama-3.2-3B FFN)",
+        "config": {"workload": _workload_desc(), "global_batch": world * tokens_per_step,
+                   "l2": "flushed (256 MiB write) before every timed call",
+                   "parallelism": f"replicas x{world} (no collective on the data path)"},
+        "roofline": roofline, "kernels": kernels, "per_batch": per_batch,
+        "dense_baseline": dense, "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["decode_ffn_3b"], default="decode_ffn_3b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * wide.h -- C ABI of libwide.so, the B200 (sm_100a) masked-layer library.
+ *
+ * The method: "WIDE: Boosting Adaptive LLM Inference via Token-level Dynamic
+ * Width Pruning".  Every token keeps or skips its own FFN channel groups
+ * (contiguous groups of the intermediate dimension D') and its own attention
+ * head groups (the query heads that share one KV head), technical summary
+ * section 2.A.  Execution follows the pruning-kernel co-design of the
+ * abstract and section 2.C: per-group mask reordering (section 2.B), then
+ * block-level skipping (a tile with no active token does nothing) and
+ * intra-block skipping (inactive rows of a partly active tile are neither
+ * loaded nor multiplied).  Section 1 names the two costs this removes: a
+ * synchronous mask-to-index conversion on the host and explicit
+ * gather-scatter copies of activations; no entry point below synchronises
+ * with the host or copies activations into a compacted buffer.
+ *
+ * Conventions for every entry point
+ *   - Pointers named d_* or documented as "device" are device pointers on the
+ *     current CUDA device; the caller owns every buffer.  The library never
+ *     allocates or frees device memory.
+ *   - stream is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  All work is enqueued asynchronously on it.
+ *   - Return value: WIDE_OK (0) or a negative WIDE_E* code for an error the
+ *     host detects before launching anything (nothing is enqueued then).
+ *     Errors found on the device (a mask bit at or above G, a bounded wait
+ *     that gave up) set bits of a per-device status word, read with
+ *     wide_get_device_status (the only call that synchronises).
+ *   - bf16 tensors are IEEE bfloat16 bit patterns; all accumulation is fp32.
+ *   - Matrices are row-major.  Weights use the nn.Linear layout
+ *     [out_features][in_features].
+ *   - A group mask is bit-packed, token-major: uint32 words[T][W] with
+ *     W = ceil(G / 32); group g of token t is bit (g % 32) of words[t][g/32];
+ *     a set bit means the token executes the group.  Bits at or above G
+ *     must be zero.
+ *   - Outputs must not alias inputs.
+ */
+#ifndef WIDE_H
+#define WIDE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WIDE_ABI_VERSION 1
+
+/* host-side status codes */
+#define WIDE_OK 0
+#define WIDE_EINVAL -1        /* null pointer, negative or inconsistent size */
+#define WIDE_EUNSUPPORTED -2  /* a shape or alignment this build does not run */
+#define WIDE_EWORKSPACE -3    /* workspace smaller than the *_workspace_bytes query */
+#define WIDE_ECUDA -4         /* a CUDA runtime/driver call failed */
+
+/* device status word bits (wide_get_device_status) */
+#define WIDE_DEV_BAD_MASK 0x1 /* a mask word had a bit at or above G set */
+#define WIDE_DEV_TIMEOUT 0x2  /* a bounded wait inside a kernel gave up */
+#define WIDE_DEV_BAD_ITEM 0x4 /* a work-list entry was out of range */
+
+/* element types */
+#define WIDE_BF16 0
+#define WIDE_F32 1
+
+/* FFN execution path */
+#define WIDE_PATH_AUTO 0      /* decode for T <= 32, prefill otherwise */
+#define WIDE_PATH_DECODE 1    /* CUDA-core GEMV over the batch's union of groups */
+#define WIDE_PATH_PREFILL 2   /* reorder + tcgen05 grouped GEMMs (bf16 only) */
+
+/* ------------------------------------------------------------------ status */
+
+/* Human-readable text for a WIDE_* host code or a device status bit set. */
+const char *wide_status_string(int code);
+
+/* ABI version of the loaded library (WIDE_ABI_VERSION). */
+int wide_abi_version(void);
+
+/* Synchronises `stream`, then copies the current device's status word into
+ * *h_status (host pointer).  0 means no device-side error since the last
+ * wide_clear_device_status. */
+int wide_get_device_status(int32_t *h_status, void *stream);
+
+/* Enqueues a reset of the current device's status word on `stream`. */
+int wide_clear_device_status(void *stream);
+
+/* ------------------------------------------------------------ measurement
+ *
+ * Kernel timing for benchmarks.  While profiling is on (host-global switch),
+ * every kernel this library launches is bracketed by a pair of CUDA events
+ * recorded on the launch stream; wide_profile_read synchronises on them and
+ * returns one (kernel id, milliseconds) record per launch.  Off by default;
+ * the events are created once, host side (no device allocation).
+ */
+
+/* Starts recording, keeping at most max_records launches (<= 65536). */
+int wide_profile_start(int32_t max_records);
+
+/* Stops recording new launches (records already taken stay readable). */
+int wide_profile_stop(void);
+
+/* Copies up to `max` records into kernel_ids[] / ms[] (host arrays), sets
+ * *n to the number copied and clears the record list. */
+int wide_profile_read(int32_t *kernel_ids, float *ms, int32_t max, int32_t *n);
+
+/* Name of a kernel id ("?" when unknown). */
+const char *wide_kernel_name(int32_t kernel_id);
+
+/* Number of kernels this library has launched in this process. */
+int64_t wide_launch_count(void);
+
+/* --------------------------------------------------------- mask reordering
+ *
+ * Section 2.B: for each routing group, sort the binary mask along the token
+ * dimension M so that the active tokens form a contiguous prefix; a tile of
+ * that order is then a dense block with a known active prefix.  The sort is
+ * the stable partition (active tokens ascending, then inactive ascending).
+ * Also produced, for the kernels that sum over groups (FFN down projection):
+ * a signature order of the tokens -- stable sort by the mask row read as one
+ * big-endian unsigned key (word W-1 most significant) -- and the OR of the
+ * mask rows of each tile_m-token tile of that order.
+ *
+ * All arrays are device memory inside one caller buffer laid out by
+ * wide_worklist_carve; sizes:
+ *   count[G], perm[G][T], items[G * ceil(T/tile_m)][2] (group, tile index;
+ *   group-major; only tiles that hold an active token), n_items[1],
+ *   sig_perm[T], sig_pos[T] (inverse of sig_perm),
+ *   tile_union[ceil(T/tile_m)][W], plus reorder scratch.
+ */
+typedef struct wide_worklist {
+    int32_t *count;
+    int32_t *perm;
+    int32_t *items;
+    int32_t *n_items;
+    int32_t *sig_perm;
+    int32_t *sig_pos;
+    uint32_t *tile_union;
+    int32_t *scratch;      /* rank partial sums, owned by wide_reorder */
+    int64_t tokens, groups;
+    int32_t tile_m, scratch_splits;
+} wide_worklist;
+
+/* Bytes of device memory a work list for (T, G, tile_m) needs (256-byte
+ * aligned sub-arrays included).  Returns 0 for invalid arguments. */
+size_t wide_worklist_bytes(int64_t T, int64_t G, int32_t tile_m);
+
+/* Lays out the work-list arrays inside the device buffer `d_base` of
+ * `bytes` bytes (>= wide_worklist_bytes; 256-byte aligned) and fills *wl
+ * (host struct).  Enqueues nothing. */
+int wide_worklist_carve(void *d_base, size_t bytes, int64_t T, int64_t G, int32_t tile_m,
+                        wide_worklist *wl);
+
+/* Builds the work list of section 2.B on the device from d_mask[T][W]
+ * (device).  T >= 0, 1 <= G <= 1024, tile_m in {64, 128}.  No host sync;
+ * n_items stays on the device.  A mask bit at or above G sets
+ * WIDE_DEV_BAD_MASK (the outputs are then unspecified). */
+int wide_reorder(const uint32_t *d_mask, int64_t T, int64_t G, int32_t tile_m,
+                 const wide_worklist *wl, void *stream);
+
+/* -------------------------------------------------------------- masked FFN
+ *
+ * Section 2.A, FFN half: for every token t and kept channel group g of
+ * group_size consecutive channels c,
+ *     h[t][c]  = silu(x[t] . W_gate[c]) * (x[t] . W_up[c])
+ *     out[t]   = sum over kept groups g, c in g:  h[t][c] * W_down[:, c]
+ * Skipped groups are never computed (and their W_down columns never read
+ * for that token).
+ *
+ * Shapes: x[T][hidden], W_gate[inter][hidden], W_up[inter][hidden],
+ * W_down[hidden][inter], group_mask[T][W] with G = inter / group_size,
+ * out[T][hidden]; element type `dtype` for x, weights and out.  All device.
+ *
+ * Supported: hidden % 64 == 0; group_size in {32, 64, 128} dividing inter;
+ * G <= 1024; 16-byte aligned pointers.  WIDE_PATH_PREFILL needs bf16,
+ * group_size == 128 and hidden % 256 == 0.  The fp32 type runs the
+ * CUDA-core path at any T.
+ */
+typedef struct wide_ffn_dims {
+    int64_t tokens;        /* T */
+    int64_t hidden;        /* H */
+    int64_t inter;         /* I (D' on the pages) */
+    int64_t group_size;    /* channels per group */
+    int32_t dtype;         /* WIDE_BF16 or WIDE_F32 */
+    int32_t path;          /* WIDE_PATH_* */
+} wide_ffn_dims;
+
+/* Device workspace bytes wide_ffn_masked needs for `d` (0 on bad args). */
+size_t wide_ffn_workspace_bytes(const wide_ffn_dims *d);
+
+/* Masked SwiGLU FFN.  d_workspace: device, >= wide_ffn_workspace_bytes(d)
+ * bytes, 256-byte aligned, contents need not be initialised and are
+ * clobbered.  Calls that share a workspace must be ordered on one stream. */
+int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
+                    const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
+                    const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
+                    void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WIDE_H */

@@ -240,15 +240,16 @@ def ffn_case(T: int, H: int, I: int, gs: int, seed: int = 0, keep: float = 0.5,
     )
 
 
-def decode_ffn(batch: int, seed: int = 0) -> FFNCase:
-    """Llama-3.2-3B-shaped decode FFN; weights independent of the batch size."""
+def decode_ffn(batch: int, seed: int = 0, weights: bool = True) -> FFNCase:
+    """Llama-3.2-3B-shaped decode FFN; weights independent of the batch size
+    (``weights=False`` leaves them as None, for a batch that reuses them)."""
     H, I, gs = 3072, 8192, 128
     return FFNCase(
         f"decode_ffn_3b_b{batch}", batch, H, I, gs, "bf16",
         x=_normal(seed, "x", (batch, H), 1.0, True, batch),
-        w_gate=_normal(seed, "w_gate", (I, H), 0.02),
-        w_up=_normal(seed, "w_up", (I, H), 0.02),
-        w_down=_normal(seed, "w_down", (H, I), 0.02),
+        w_gate=_normal(seed, "w_gate", (I, H), 0.02) if weights else None,
+        w_up=_normal(seed, "w_up", (I, H), 0.02) if weights else None,
+        w_down=_normal(seed, "w_down", (H, I), 0.02) if weights else None,
         mask=bernoulli_mask(_rng(seed, "mask_f", batch), batch, I // gs, 0.5),
     )
 

@@ -19,3 +19,18 @@ def torch_cuda():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch
+
+
+def load_build_module():
+    """token_level_dynamic_b200/build.py, loaded by path (the package's
+    __init__ loads libwide.so, which may not exist yet)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "wide_build", os.path.join(ROOT, "token_level_dynamic_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def pytest_sessionstart(session):
+    load_build_module().build()

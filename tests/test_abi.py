@@ -1,0 +1,109 @@
+"""The C ABI library loads and exports every symbol include/wide.h declares;
+host-side argument checks answer without touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "wide.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(wide_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def native():
+    from token_level_dynamic_b200 import _native
+    return _native
+
+
+def test_library_exports_every_declared_symbol(native):
+    L = native.lib()
+    declared = _header_functions()
+    assert len(declared) >= 9
+    for name in declared:
+        assert hasattr(L, name), name
+        assert name in native.SIGNATURES, f"binding lacks {name}"
+
+
+def test_binding_names_match_c_names(native):
+    import token_level_dynamic_b200 as w
+    for name in _header_functions():
+        if name in ("wide_worklist_carve",):
+            continue
+        assert hasattr(w, name), name
+
+
+def test_constants_match_header(native):
+    src = open(os.path.join(ROOT, "include", "wide.h")).read()
+    for name, val in re.findall(r"#define (WIDE_[A-Z0-9_]+) (-?0x[0-9a-fA-F]+|-?\d+)", src):
+        if hasattr(native, name):
+            assert getattr(native, name) == int(val, 0), name
+
+
+def test_version_and_status_strings(native):
+    L = native.lib()
+    assert L.wide_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, 1, 2, 4):
+        assert L.wide_status_string(code)
+
+
+def test_worklist_bytes_and_carve_validation(native):
+    L = native.lib()
+    assert L.wide_worklist_bytes(4096, 112, 128) > 4 * 112 * 4096
+    assert L.wide_worklist_bytes(4096, 0, 128) == 0
+    assert L.wide_worklist_bytes(4096, 1025, 128) == 0
+    assert L.wide_worklist_bytes(-1, 8, 128) == 0
+    assert L.wide_worklist_bytes(64, 8, 96) == 0
+    wl = native.WideWorklist()
+    # a misaligned base pointer is refused before anything is enqueued
+    assert L.wide_worklist_carve(ctypes.c_void_p(16), 1 << 30, 64, 8, 128, ctypes.byref(wl)) \
+        == native.WIDE_EUNSUPPORTED
+    assert L.wide_worklist_carve(ctypes.c_void_p(256), 16, 64, 8, 128, ctypes.byref(wl)) \
+        == native.WIDE_EWORKSPACE
+    assert L.wide_worklist_carve(ctypes.c_void_p(1 << 20), 1 << 30, 64, 8, 128,
+                                 ctypes.byref(wl)) == 0
+    assert wl.tokens == 64 and wl.groups == 8 and wl.tile_m == 128
+    assert wl.perm - wl.count >= 32 and (wl.perm % 256) == 0
+    assert L.wide_reorder(None, 64, 8, 128, None, None) == native.WIDE_EINVAL
+    assert L.wide_reorder(None, 64, 9, 128, ctypes.byref(wl), None) == native.WIDE_EINVAL
+
+
+def test_ffn_argument_checks(native):
+    L = native.lib()
+    D = native.WideFFNDims
+    ok = D(8, 3072, 8192, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)
+    assert L.wide_ffn_workspace_bytes(ctypes.byref(ok)) >= 8 * 8192 * 4
+    for bad in (D(-1, 3072, 8192, 128, 0, 1), D(8, 3072, 8192, 100, 0, 1),
+                D(8, 3072, 8192, 128, 5, 1), D(8, 3072, 8192, 128, 0, 7),
+                D(8, 3072, 128 * 2000, 128, 0, 1)):
+        assert L.wide_ffn_workspace_bytes(ctypes.byref(bad)) == 0
+        assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(bad),
+                                 None, 0, None) == native.WIDE_EINVAL
+    # null pointers with valid dims
+    assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(ok), None, 0,
+                             None) == native.WIDE_EINVAL
+    # zero tokens is a no-op
+    z = D(0, 3072, 8192, 128, 0, 1)
+    assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(z), None, 0,
+                             None) == native.WIDE_OK
+    # an unsupported shape is refused on the host (hidden not a multiple of 128)
+    p = ctypes.c_void_p(1 << 20)
+    odd = D(8, 3000, 8192, 128, 0, 1)
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(odd), p, 1 << 30, None) \
+        == native.WIDE_EUNSUPPORTED
+    # bf16 group size 32 is not built on the decode path
+    g32 = D(8, 3072, 8192, 32, 0, 1)
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(g32), p, 1 << 30, None) \
+        == native.WIDE_EUNSUPPORTED
+    # misaligned pointer
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    assert L.wide_ffn_masked(mis, p, p, p, p, p, ctypes.byref(ok), p, 1 << 30, None) \
+        == native.WIDE_EUNSUPPORTED
+    # workspace too small
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(ok), p, 16, None) \
+        == native.WIDE_EWORKSPACE

@@ -1,0 +1,81 @@
+"""Decode (CUDA-core GEMV) masked FFN against the fp64 oracle, through the
+C ABI.  WIDE, technical summary section 2.A: a token's skipped FFN channel
+groups contribute nothing; the union of the batch's groups is streamed."""
+import numpy as np
+import pytest
+
+import synth
+from oracle.ffn import ffn_masked
+from tests._util import rel_l2, ffn_to_dev, from_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 5e-3   # relative L2, bf16 storage / fp32 accumulation
+TOL_F32 = 1e-5    # relative L2, fp32 tiny configuration
+
+
+def _run(c, path=None):
+    import torch
+    import token_level_dynamic_b200 as w
+    x, wg, wu, wd, m = ffn_to_dev(c)
+    w.wide_clear_device_status()
+    out = w.wide_ffn_masked(x, wg, wu, wd, m, c.gs,
+                            path=w.WIDE_PATH_DECODE if path is None else path)
+    torch.cuda.synchronize()
+    assert w.wide_get_device_status() == 0
+    return from_dev(out)
+
+
+def _ref(c):
+    return ffn_masked(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs, c.dtype)
+
+
+def test_tiny_fp32_config():
+    c = synth.tiny_ffn()
+    assert rel_l2(_run(c), _ref(c)) <= TOL_F32
+
+
+@pytest.mark.parametrize("batch", [1, 8, 32])
+def test_decode_ffn_3b_config(batch):
+    c = synth.decode_ffn(batch)
+    assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
+
+
+def test_decode_layer_ffn_shape():
+    """The FFN half of the 8B decode layer: B=16, H=4096, I=14336, keep 0.72."""
+    c = synth.ffn_case(16, 4096, 14336, 128, seed=4, keep=0.72)
+    assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("T,H,I,gs,dtype", [
+    (1, 128, 256, 64, "bf16"), (3, 256, 1024, 128, "bf16"), (33, 384, 768, 64, "bf16"),
+    (70, 256, 512, 32, "f32"), (5, 640, 1280, 128, "f32"), (32, 1024, 2048, 64, "bf16"),
+])
+def test_decode_shapes_and_ragged_token_counts(T, H, I, gs, dtype):
+    c = synth.ffn_case(T, H, I, gs, seed=T, dtype=dtype)
+    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    assert rel_l2(_run(c), _ref(c)) <= tol
+
+
+def test_all_zero_mask_gives_exact_zero():
+    c = synth.ffn_case(8, 512, 1024, 128, seed=1, mask_kind="zeros")
+    assert not np.any(_run(c))
+
+
+def test_all_ones_mask_equals_dense():
+    c = synth.ffn_case(8, 512, 1024, 128, seed=2, mask_kind="ones")
+    from oracle.ffn import ffn_dense
+    assert rel_l2(_run(c), ffn_dense(c.x, c.w_gate, c.w_up, c.w_down)) <= TOL_BF16
+
+
+def test_single_token_single_group():
+    c = synth.ffn_case(1, 256, 1024, 128, seed=3)
+    c.mask[:] = False
+    c.mask[0, 5] = True
+    assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
+
+
+def test_repeatable_bitwise():
+    c = synth.decode_ffn(8)
+    a, b = _run(c), _run(c)
+    np.testing.assert_array_equal(a, b)

@@ -1,0 +1,189 @@
+"""token_level_dynamic_b200 -- WIDE's masked transformer layer on B200 (sm_100a).
+
+A thin Python binding over libwide.so (C ABI, include/wide.h).  Each function
+here has the name of the C entry point it calls and only marshals arguments:
+torch tensors supply device memory and the stream; every step of the layer
+runs in the library's CUDA kernels.  Importing the package loads the library
+and fails if it has not been built.
+
+Method: "WIDE: Boosting Adaptive LLM Inference via Token-level Dynamic Width
+Pruning" -- per-token FFN channel groups and GQA head groups (technical
+summary section 2.A), mask reordering (2.B), block-level and intra-block
+skipping (2.C).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _native
+from ._native import (  # noqa: F401
+    WIDE_OK, WIDE_EINVAL, WIDE_EUNSUPPORTED, WIDE_EWORKSPACE, WIDE_ECUDA,
+    WIDE_DEV_BAD_MASK, WIDE_DEV_TIMEOUT, WIDE_DEV_BAD_ITEM,
+    WIDE_BF16, WIDE_F32, WIDE_PATH_AUTO, WIDE_PATH_DECODE, WIDE_PATH_PREFILL,
+    WideWorklist, WideFFNDims,
+)
+
+_L = _native.lib()
+
+
+class WideError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {code} ({wide_status_string(code)})")
+        self.code = code
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != WIDE_OK:
+        raise WideError(fn, rc)
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return WIDE_BF16
+    if t.dtype == torch.float32:
+        return WIDE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _dev_ptr(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+# ------------------------------------------------------------------ status
+
+def wide_status_string(code: int) -> str:
+    return _L.wide_status_string(int(code)).decode()
+
+
+def wide_abi_version() -> int:
+    return _L.wide_abi_version()
+
+
+def wide_get_device_status(stream=None, device=None) -> int:
+    """Synchronises the stream and returns the device status word."""
+    v = ctypes.c_int32(0)
+    _check("wide_get_device_status",
+           _L.wide_get_device_status(ctypes.byref(v), _stream(stream, device)))
+    return v.value
+
+
+def wide_clear_device_status(stream=None, device=None) -> None:
+    _check("wide_clear_device_status", _L.wide_clear_device_status(_stream(stream, device)))
+
+
+# ------------------------------------------------------------ measurement
+
+def wide_profile_start(max_records: int = 4096) -> None:
+    _check("wide_profile_start", _L.wide_profile_start(int(max_records)))
+
+
+def wide_profile_stop() -> None:
+    _check("wide_profile_stop", _L.wide_profile_stop())
+
+
+def wide_profile_read(max_records: int = 65536) -> list:
+    """[(kernel name, milliseconds)] for the launches recorded since start."""
+    import numpy as np
+    ids = np.zeros(max_records, dtype=np.int32)
+    ms = np.zeros(max_records, dtype=np.float32)
+    n = ctypes.c_int32(0)
+    _check("wide_profile_read", _L.wide_profile_read(
+        ids.ctypes.data, ms.ctypes.data, max_records, ctypes.byref(n)))
+    return [(wide_kernel_name(int(ids[i])), float(ms[i])) for i in range(n.value)]
+
+
+def wide_kernel_name(kernel_id: int) -> str:
+    return _L.wide_kernel_name(int(kernel_id)).decode()
+
+
+def wide_launch_count() -> int:
+    return int(_L.wide_launch_count())
+
+
+# --------------------------------------------------------- mask reordering
+
+def wide_worklist_bytes(T: int, G: int, tile_m: int = 128) -> int:
+    return int(_L.wide_worklist_bytes(T, G, tile_m))
+
+
+def wide_reorder(mask_words: torch.Tensor, G: int, tile_m: int = 128, buf: torch.Tensor = None,
+                 stream=None) -> dict:
+    """Device-side mask reordering (section 2.B) of an int32/uint32 [T][W]
+    mask.  Returns tensor views into one device buffer: count, perm,
+    items ([n_cap][2]), n_items ([1]), sig_perm, sig_pos, tile_union."""
+    T, W = mask_words.shape
+    if W != (G + 31) // 32:
+        raise ValueError("mask has the wrong number of words per token")
+    nbytes = wide_worklist_bytes(T, G, tile_m)
+    if nbytes == 0:
+        raise WideError("wide_worklist_bytes", WIDE_EINVAL)
+    dev = mask_words.device
+    if buf is None:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    wl = WideWorklist()
+    _check("wide_worklist_carve", _L.wide_worklist_carve(
+        buf.data_ptr(), buf.numel(), T, G, tile_m, ctypes.byref(wl)))
+    _check("wide_reorder", _L.wide_reorder(
+        _dev_ptr(mask_words, "mask_words"), T, G, tile_m, ctypes.byref(wl), _stream(stream, dev)))
+    base = buf.data_ptr()
+    nt = (T + tile_m - 1) // tile_m
+
+    def view(ptr, n, dt=torch.int32):
+        off = ptr - base
+        return buf[off:off + 4 * n].view(dt)
+
+    return {
+        "count": view(wl.count, G),
+        "perm": view(wl.perm, G * T).view(G, T),
+        "items": view(wl.items, 2 * G * nt).view(G * nt, 2),
+        "n_items": view(wl.n_items, 1),
+        "sig_perm": view(wl.sig_perm, T),
+        "sig_pos": view(wl.sig_pos, T),
+        "tile_union": view(wl.tile_union, nt * W).view(nt, W),
+        "_buf": buf,
+    }
+
+
+# -------------------------------------------------------------- masked FFN
+
+def _ffn_dims(x, w_gate, group_size, path) -> WideFFNDims:
+    T, H = x.shape
+    I = w_gate.shape[0]
+    return WideFFNDims(T, H, I, group_size, _dtype_code(x), path)
+
+
+def wide_ffn_workspace_bytes(T: int, H: int, I: int, group_size: int, dtype=torch.bfloat16,
+                             path: int = WIDE_PATH_AUTO) -> int:
+    d = WideFFNDims(T, H, I, group_size, WIDE_BF16 if dtype == torch.bfloat16 else WIDE_F32, path)
+    return int(_L.wide_ffn_workspace_bytes(ctypes.byref(d)))
+
+
+def wide_ffn_masked(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
+                    w_down: torch.Tensor, mask_words: torch.Tensor, group_size: int,
+                    out: torch.Tensor = None, workspace: torch.Tensor = None,
+                    path: int = WIDE_PATH_AUTO, stream=None) -> torch.Tensor:
+    """Masked SwiGLU FFN (section 2.A).  x[T][H]; W_gate/W_up[I][H];
+    W_down[H][I]; mask_words int32 [T][ceil(G/32)]; returns out[T][H]."""
+    d = _ffn_dims(x, w_gate, group_size, path)
+    if out is None:
+        out = torch.empty_like(x)
+    need = int(_L.wide_ffn_workspace_bytes(ctypes.byref(d)))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    _check("wide_ffn_masked", _L.wide_ffn_masked(
+        _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
+        _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"), _dev_ptr(out, "out"),
+        ctypes.byref(d), workspace.data_ptr(), workspace.numel(), _stream(stream, x.device)))
+    return out

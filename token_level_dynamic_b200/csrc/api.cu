@@ -1,0 +1,295 @@
+// api.cu -- the extern "C" entry points of libwide.so (declared in wide.h):
+// argument validation, work-list layout, tensor-map encoding and the
+// per-device status word.  The kernels live in the other .cu files.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "host.h"
+#include "wide.h"
+
+// Per-device status word: each device that loads this module gets its own
+// copy.  Kernels set WIDE_DEV_* bits in it; wide_get_device_status reads it.
+__device__ int32_t g_wide_status;
+
+namespace wide {
+
+int32_t *status_ptr()
+{
+    static int32_t *ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_wide_status) == cudaSuccess)
+            ptrs[dev] = static_cast<int32_t *>(p);
+    }
+    return ptrs[dev];
+}
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                  uint64_t pitch_elems, uint32_t elem_bytes, uint32_t box_rows, uint32_t box_cols,
+                  bool swizzle128)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows == 0 || cols == 0)
+        return false;
+    const CUtensorMapDataType dt =
+        elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch_elems * elem_bytes};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r =
+        fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE,
+           swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool raise_smem_limit(const void *kernel, size_t bytes)
+{
+    static std::mutex mu;
+    static std::set<std::pair<std::pair<const void *, int>, size_t>> done;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    auto key = std::make_pair(std::make_pair(kernel, dev), bytes);
+    if (done.count(key))
+        return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return false;
+    done.insert(key);
+    return true;
+}
+
+namespace {
+
+struct WorklistLayout {
+    size_t count, perm, items, n_items, sig_perm, sig_pos, tile_union, scratch, total;
+    int splits;
+};
+
+bool worklist_layout(int64_t T, int64_t G, int32_t tile_m, WorklistLayout *L)
+{
+    if (T < 0 || T > (1 << 24) || G < 1 || G > 1024 || (tile_m != 64 && tile_m != 128))
+        return false;
+    const size_t W = (size_t)((G + 31) / 32);
+    const size_t nt = (size_t)((T + tile_m - 1) / tile_m);
+    const size_t t = (size_t)T;
+    L->splits = reorder_splits(T);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += align_up(bytes > 0 ? bytes : 1, 256);
+        return at;
+    };
+    L->count = take(4 * (size_t)G);
+    L->perm = take(4 * (size_t)G * t);
+    L->items = take(8 * (size_t)G * nt);
+    L->n_items = take(4);
+    L->sig_perm = take(4 * t);
+    L->sig_pos = take(4 * t);
+    L->tile_union = take(4 * nt * W);
+    L->scratch = take(4 * (size_t)L->splits * t);
+    L->total = off;
+    return true;
+}
+
+bool ffn_dims_ok(const wide_ffn_dims *d)
+{
+    if (!d || d->tokens < 0 || d->hidden <= 0 || d->inter <= 0 || d->group_size <= 0)
+        return false;
+    if (d->dtype != WIDE_BF16 && d->dtype != WIDE_F32)
+        return false;
+    if (d->path < WIDE_PATH_AUTO || d->path > WIDE_PATH_PREFILL)
+        return false;
+    return d->inter % d->group_size == 0 && d->inter / d->group_size <= 1024;
+}
+
+int ffn_path(const wide_ffn_dims *d)
+{
+    if (d->path != WIDE_PATH_AUTO)
+        return d->path;
+    return (d->dtype == WIDE_F32 || d->tokens <= 32) ? WIDE_PATH_DECODE : WIDE_PATH_PREFILL;
+}
+
+bool ffn_shape_supported(const wide_ffn_dims *d, int path)
+{
+    if (d->hidden % 128 != 0 || d->hidden > (1 << 20) || d->inter > (1 << 22))
+        return false;
+    const int64_t gs = d->group_size;
+    if (path == WIDE_PATH_DECODE)
+        return d->dtype == WIDE_BF16 ? (gs == 64 || gs == 128) : (gs == 32 || gs == 64 || gs == 128);
+    return false;  // the prefill path is built in a later file
+}
+
+}  // namespace
+}  // namespace wide
+
+using namespace wide;
+
+extern "C" {
+
+const char *wide_status_string(int code)
+{
+    switch (code) {
+    case WIDE_OK:
+        return "ok";
+    case WIDE_EINVAL:
+        return "invalid argument (null pointer, negative or inconsistent size)";
+    case WIDE_EUNSUPPORTED:
+        return "unsupported shape, type or alignment";
+    case WIDE_EWORKSPACE:
+        return "workspace too small";
+    case WIDE_ECUDA:
+        return "CUDA runtime or driver call failed";
+    case WIDE_DEV_BAD_MASK:
+        return "device: mask bit at or above G";
+    case WIDE_DEV_TIMEOUT:
+        return "device: bounded wait gave up";
+    case WIDE_DEV_BAD_ITEM:
+        return "device: work item out of range";
+    default:
+        return code > 0 ? "device: several error bits" : "unknown status";
+    }
+}
+
+int wide_abi_version(void) { return WIDE_ABI_VERSION; }
+
+int wide_get_device_status(int32_t *h_status, void *stream)
+{
+    if (!h_status)
+        return WIDE_EINVAL;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return WIDE_ECUDA;
+    if (cudaMemcpyFromSymbol(h_status, g_wide_status, sizeof(int32_t)) != cudaSuccess)
+        return WIDE_ECUDA;
+    return WIDE_OK;
+}
+
+int wide_clear_device_status(void *stream)
+{
+    int32_t *p = status_ptr();
+    if (!p)
+        return WIDE_ECUDA;
+    return cudaMemsetAsync(p, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? WIDE_OK
+               : WIDE_ECUDA;
+}
+
+size_t wide_worklist_bytes(int64_t T, int64_t G, int32_t tile_m)
+{
+    WorklistLayout L;
+    return worklist_layout(T, G, tile_m, &L) ? L.total : 0;
+}
+
+int wide_worklist_carve(void *d_base, size_t bytes, int64_t T, int64_t G, int32_t tile_m,
+                        wide_worklist *wl)
+{
+    WorklistLayout L;
+    if (!wl || !d_base || !worklist_layout(T, G, tile_m, &L))
+        return WIDE_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(d_base) & 255u) != 0)
+        return WIDE_EUNSUPPORTED;
+    if (bytes < L.total)
+        return WIDE_EWORKSPACE;
+    char *b = static_cast<char *>(d_base);
+    wl->count = reinterpret_cast<int32_t *>(b + L.count);
+    wl->perm = reinterpret_cast<int32_t *>(b + L.perm);
+    wl->items = reinterpret_cast<int32_t *>(b + L.items);
+    wl->n_items = reinterpret_cast<int32_t *>(b + L.n_items);
+    wl->sig_perm = reinterpret_cast<int32_t *>(b + L.sig_perm);
+    wl->sig_pos = reinterpret_cast<int32_t *>(b + L.sig_pos);
+    wl->tile_union = reinterpret_cast<uint32_t *>(b + L.tile_union);
+    wl->scratch = reinterpret_cast<int32_t *>(b + L.scratch);
+    wl->tokens = T;
+    wl->groups = G;
+    wl->tile_m = tile_m;
+    wl->scratch_splits = L.splits;
+    return WIDE_OK;
+}
+
+int wide_reorder(const uint32_t *d_mask, int64_t T, int64_t G, int32_t tile_m,
+                 const wide_worklist *wl, void *stream)
+{
+    WorklistLayout L;
+    if (!wl || !worklist_layout(T, G, tile_m, &L))
+        return WIDE_EINVAL;
+    if (wl->tokens != T || wl->groups != G || wl->tile_m != tile_m ||
+        wl->scratch_splits != L.splits)
+        return WIDE_EINVAL;
+    if ((T > 0 && !d_mask) || !wl->count || !wl->perm || !wl->items || !wl->n_items ||
+        !wl->sig_perm || !wl->sig_pos || !wl->tile_union || !wl->scratch)
+        return WIDE_EINVAL;
+    return reorder_launch(d_mask, T, G, tile_m, wl, static_cast<cudaStream_t>(stream));
+}
+
+size_t wide_ffn_workspace_bytes(const wide_ffn_dims *d)
+{
+    if (!ffn_dims_ok(d))
+        return 0;
+    const int path = ffn_path(d);
+    if (path == WIDE_PATH_DECODE)
+        return ffn_decode_workspace(d);
+    return 0;
+}
+
+int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
+                    const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
+                    const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
+                    void *stream)
+{
+    if (!ffn_dims_ok(d))
+        return WIDE_EINVAL;
+    if (d->tokens == 0)
+        return WIDE_OK;
+    if (!d_x || !d_w_gate || !d_w_up || !d_w_down || !d_group_mask || !d_out || !d_workspace)
+        return WIDE_EINVAL;
+    const int path = ffn_path(d);
+    if (!ffn_shape_supported(d, path))
+        return WIDE_EUNSUPPORTED;
+    if (!aligned16(d_x) || !aligned16(d_w_gate) || !aligned16(d_w_up) || !aligned16(d_w_down) ||
+        !aligned16(d_out) || (reinterpret_cast<uintptr_t>(d_workspace) & 255u) != 0)
+        return WIDE_EUNSUPPORTED;
+    if (workspace_bytes < wide_ffn_workspace_bytes(d))
+        return WIDE_EWORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (path == WIDE_PATH_DECODE)
+        return ffn_decode_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d,
+                                 d_workspace, s);
+    return WIDE_EUNSUPPORTED;
+}
+
+}  // extern "C"

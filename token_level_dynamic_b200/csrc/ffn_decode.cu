@@ -1,0 +1,476 @@
+// ffn_decode.cu -- masked SwiGLU FFN for small token counts (decode).
+//
+// WIDE, technical summary section 2.A (contiguous FFN channel groups chosen
+// per token) and section 2.C (block-level early exit, intra-block skipping)
+// applied to the bandwidth-bound decode case: the weights of a channel group
+// are streamed from HBM once per call, and only when at least one token of
+// the batch executes the group (the batch's union); inside a streamed tile,
+// only the tokens that execute the group do arithmetic.
+//
+// gate/up kernel: grid (KS, G), cluster (KS, 1, 1), GS threads.
+//   The cluster owns channel group g; CTA s owns the K-slice
+//   [s*H/KS, (s+1)*H/KS).  If no token executes g the cluster exits at once
+//   (block-level skip).  Gate and up tiles (GS rows x 128 bytes, 128-byte
+//   swizzle) arrive by TMA through a 3-stage mbarrier ring; thread c owns
+//   channel c of the group and accumulates, in fp32, the gate and up dot
+//   products of every executing token against x held in shared memory as
+//   fp32.  The KS partial sums are added through distributed shared memory,
+//   and h = silu(gate) * up is written (fp32) for executing tokens only.
+// down kernel: grid (KS, H/128), cluster (KS, 1, 1), 128 threads.
+//   CTA (s, nb) owns output rows [nb*128, nb*128+128) and the groups of
+//   slice s.  It streams W_down tiles (128 rows x 128 bytes) only for groups
+//   some token executes, with the matching h tile, and thread n adds
+//   h[t][c] * W_down[n][c] only for tokens t that execute the group.  The KS
+//   partial outputs are added through distributed shared memory.
+//
+// Tokens are processed 32 at a time (one mask bit per lane).
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "host.h"
+
+namespace cg = cooperative_groups;
+
+namespace wide {
+namespace {
+
+constexpr int kNTok = 32;
+constexpr int kStages = 3;
+constexpr int kDownRows = 128;
+
+template <typename TIn> struct ElemTraits;
+template <> struct ElemTraits<__nv_bfloat16> {
+    static constexpr int EPC = 8;  // elements per 16-byte chunk
+};
+template <> struct ElemTraits<float> {
+    static constexpr int EPC = 4;
+};
+
+template <typename TIn>
+__device__ __forceinline__ void chunk_to_f32(const uint4 v, float (&f)[ElemTraits<TIn>::EPC]);
+template <>
+__device__ __forceinline__ void chunk_to_f32<__nv_bfloat16>(const uint4 v, float (&f)[8])
+{
+    bf16x8_to_f32(v, f);
+}
+template <> __device__ __forceinline__ void chunk_to_f32<float>(const uint4 v, float (&f)[4])
+{
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// Token mask of group g over tokens [0, T), T <= 32 (one lane per token).
+__device__ __forceinline__ uint32_t group_token_mask(const uint32_t *mask, int T, int W, int g)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t a = lane < T ? (mask[(size_t)lane * W + (g >> 5)] >> (g & 31)) & 1u : 0u;
+    return __ballot_sync(0xffffffffu, a);
+}
+
+template <typename TIn, int GS>
+__global__ void __launch_bounds__(GS)
+    ffn_decode_gateup(const __grid_constant__ CUtensorMap tm_gate,
+                      const __grid_constant__ CUtensorMap tm_up, const TIn *__restrict__ x,
+                      const uint32_t *__restrict__ mask, float *__restrict__ h, int T, int H,
+                      int I, int W, int kslice, int32_t *status)
+{
+    constexpr int EPC = ElemTraits<TIn>::EPC;
+    constexpr int KT = 8 * EPC;                 // elements in one 128-byte tile row
+    constexpr uint32_t kTileBytes = GS * 128u;  // one operand tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *stages = smem;                                          // [kStages][2][GS][128]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * 2 * kTileBytes);
+    int *act = reinterpret_cast<int *>(full + kStages);              // [32]
+    float *xs = reinterpret_cast<float *>(smem + kStages * 2 * kTileBytes + 256);  // [nact][kslice]
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int KS = (int)gridDim.x;
+    const int s = (int)blockIdx.x;
+    const int g = (int)blockIdx.y;
+    const int c = (int)threadIdx.x;
+
+    const uint32_t tmask = group_token_mask(mask, T, W, g);
+    if (tmask == 0u)
+        return;  // block-level skip: the whole cluster leaves together
+    const int nact = __popc(tmask);
+    const int k0 = s * kslice;
+    const int ntile = kslice / KT;
+
+    if (c < 32 && ((tmask >> c) & 1u))
+        act[__popc(tmask & ((1u << c) - 1u))] = c;
+    if (c == 0) {
+        for (int st = 0; st < kStages; ++st)
+            mbar_init(&full[st], 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_gate);
+        tma_prefetch_desc(&tm_up);
+    }
+    __syncthreads();
+
+    auto issue = [&](int kt) {
+        const int st = kt % kStages;
+        uint8_t *dst = stages + st * 2 * kTileBytes;
+        mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
+        tma_load_2d(dst, &tm_gate, k0 + kt * KT, g * GS, &full[st]);
+        tma_load_2d(dst + kTileBytes, &tm_up, k0 + kt * KT, g * GS, &full[st]);
+    };
+    int issued = 0;
+    if (c == 0) {
+        for (; issued < kStages && issued < ntile; ++issued)
+            issue(issued);
+    }
+
+    // x of the executing tokens over this K-slice, widened to fp32
+    const int chunks_per_row = kslice / EPC;
+    for (int idx = c; idx < nact * chunks_per_row; idx += GS) {
+        const int i = idx / chunks_per_row, q = idx % chunks_per_row;
+        const uint4 v = *reinterpret_cast<const uint4 *>(x + (size_t)act[i] * H + k0 + q * EPC);
+        float f[EPC];
+        chunk_to_f32<TIn>(v, f);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e)
+            xs[i * kslice + q * EPC + e] = f[e];
+    }
+    __syncthreads();
+
+    float accg[kNTok], accu[kNTok];
+#pragma unroll
+    for (int i = 0; i < kNTok; ++i) {
+        accg[i] = 0.f;
+        accu[i] = 0.f;
+    }
+    bool timeout = false;
+    int consumed = 0;
+    for (int kt = 0; kt < ntile; ++kt) {
+        const int st = kt % kStages;
+        const uint32_t par = (uint32_t)(kt / kStages) & 1u;
+        if (!mbar_wait(&full[st], par))
+            timeout = true;
+        if (!timeout) {
+            const uint8_t *tg = stages + st * 2 * kTileBytes;
+            const uint8_t *tu = tg + kTileBytes;
+#pragma unroll 2
+            for (int j = 0; j < 8; ++j) {
+                float wg[EPC], wu[EPC];
+                chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tg + swz128(c, j)), wg);
+                chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tu + swz128(c, j)), wu);
+                const float *xk = xs + kt * KT + j * EPC;
+#pragma unroll
+                for (int i = 0; i < kNTok; ++i) {
+                    if (i >= nact)
+                        break;
+                    const float *xp = xk + i * kslice;
+                    float xv[EPC];
+#pragma unroll
+                    for (int e = 0; e < EPC; e += 4) {
+                        const float4 t4 = *reinterpret_cast<const float4 *>(xp + e);
+                        xv[e] = t4.x;
+                        xv[e + 1] = t4.y;
+                        xv[e + 2] = t4.z;
+                        xv[e + 3] = t4.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e) {
+                        accg[i] = fmaf(wg[e], xv[e], accg[i]);
+                        accu[i] = fmaf(wu[e], xv[e], accu[i]);
+                    }
+                }
+            }
+        }
+        consumed = kt + 1;
+        if (__syncthreads_or(timeout)) {
+            timeout = true;
+            break;
+        }
+        if (c == 0 && issued < ntile)
+            issue(issued++);
+    }
+    if (timeout) {
+        // let copies already in flight land before this CTA's smem is reused
+        if (c == 0) {
+            set_status(status, WIDE_DEV_TIMEOUT);
+            for (int kt = consumed; kt < issued; ++kt)
+                mbar_wait(&full[kt % kStages], (uint32_t)(kt / kStages) & 1u);
+        }
+        __syncthreads();
+    }
+
+    // partial sums -> this CTA's shared memory, then a cluster-wide add
+    float *pg = reinterpret_cast<float *>(stages);  // [kNTok][GS]
+    float *pu = pg + kNTok * GS;
+#pragma unroll
+    for (int i = 0; i < kNTok; ++i) {
+        if (i >= nact)
+            break;
+        pg[i * GS + c] = timeout ? 0.f : accg[i];
+        pu[i * GS + c] = timeout ? 0.f : accu[i];
+    }
+    cluster.sync();
+    for (int i = s; i < nact; i += KS) {
+        float gs = 0.f, us = 0.f;
+        for (int q = 0; q < KS; ++q) {
+            const float *rg = cluster.map_shared_rank(pg, q);
+            const float *ru = cluster.map_shared_rank(pu, q);
+            gs += rg[i * GS + c];
+            us += ru[i * GS + c];
+        }
+        h[(size_t)act[i] * I + (size_t)g * GS + c] = silu_f32(gs) * us;
+    }
+    cluster.sync();
+}
+
+template <typename TIn, int GS>
+__global__ void __launch_bounds__(kDownRows)
+    ffn_decode_down(const __grid_constant__ CUtensorMap tm_down,
+                    const __grid_constant__ CUtensorMap tm_h, const uint32_t *__restrict__ mask,
+                    TIn *__restrict__ out, int T, int H, int I, int W, int G, int32_t *status)
+{
+    constexpr int EPC = ElemTraits<TIn>::EPC;
+    constexpr int KT = 8 * EPC;
+    constexpr int TPG = GS / KT;                          // tiles per group
+    constexpr uint32_t kWBytes = kDownRows * 128u;        // W_down tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    const uint32_t hbytes = (uint32_t)T * KT * 4u;        // h tile (fp32, unswizzled)
+    const uint32_t stage_bytes = kWBytes + ((hbytes + 1023u) & ~1023u);
+    uint8_t *stages = smem;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * stage_bytes);
+    uint32_t *gmask = reinterpret_cast<uint32_t *>(full + kStages);  // [gq]
+    int *live = reinterpret_cast<int *>(gmask + 1024);              // [gq]
+    __shared__ int n_live;
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int KS = (int)gridDim.x;
+    const int s = (int)blockIdx.x;
+    const int nb = (int)blockIdx.y;
+    const int n = (int)threadIdx.x;
+    const int warp = n >> 5, lane = n & 31;
+    const int gq = (G + KS - 1) / KS;
+    const int gbeg = s * gq, gend = min(G, gbeg + gq);
+
+    for (int gi = warp; gi < gend - gbeg; gi += kDownRows / 32) {
+        const uint32_t m = group_token_mask(mask, T, W, gbeg + gi);
+        if (lane == 0)
+            gmask[gi] = m;
+    }
+    if (n == 0) {
+        for (int st = 0; st < kStages; ++st)
+            mbar_init(&full[st], 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_down);
+        tma_prefetch_desc(&tm_h);
+    }
+    __syncthreads();
+    if (n == 0) {
+        int k = 0;
+        for (int gi = 0; gi < gend - gbeg; ++gi)
+            if (gmask[gi])
+                live[k++] = gi;
+        n_live = k;
+    }
+    __syncthreads();
+    const int ntile = n_live * TPG;
+
+    auto issue = [&](int kt) {
+        const int st = kt % kStages;
+        const int gg = gbeg + live[kt / TPG];
+        const int col = gg * GS + (kt % TPG) * KT;
+        uint8_t *dst = stages + st * stage_bytes;
+        mbar_arrive_expect_tx(&full[st], kWBytes + hbytes);
+        tma_load_2d(dst, &tm_down, col, nb * kDownRows, &full[st]);
+        tma_load_2d(dst + kWBytes, &tm_h, col, 0, &full[st]);
+    };
+    int issued = 0;
+    if (n == 0) {
+        for (; issued < kStages && issued < ntile; ++issued)
+            issue(issued);
+    }
+
+    float acc[kNTok];
+#pragma unroll
+    for (int t = 0; t < kNTok; ++t)
+        acc[t] = 0.f;
+    bool timeout = false;
+    int consumed = 0;
+    for (int kt = 0; kt < ntile; ++kt) {
+        const int st = kt % kStages;
+        const uint32_t par = (uint32_t)(kt / kStages) & 1u;
+        if (!mbar_wait(&full[st], par))
+            timeout = true;
+        if (!timeout) {
+            const uint32_t tm = gmask[live[kt / TPG]];
+            const uint8_t *tw = stages + st * stage_bytes;
+            const float *hs = reinterpret_cast<const float *>(tw + kWBytes);
+#pragma unroll 2
+            for (int j = 0; j < 8; ++j) {
+                float w[EPC];
+                chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tw + swz128(n, j)), w);
+#pragma unroll
+                for (int t = 0; t < kNTok; ++t) {
+                    if (t >= T)
+                        break;
+                    if ((tm >> t) & 1u) {
+                        const float *hp = hs + t * KT + j * EPC;
+#pragma unroll
+                        for (int e = 0; e < EPC; e += 4) {
+                            const float4 v = *reinterpret_cast<const float4 *>(hp + e);
+                            acc[t] = fmaf(w[e], v.x, acc[t]);
+                            acc[t] = fmaf(w[e + 1], v.y, acc[t]);
+                            acc[t] = fmaf(w[e + 2], v.z, acc[t]);
+                            acc[t] = fmaf(w[e + 3], v.w, acc[t]);
+                        }
+                    }
+                }
+            }
+        }
+        consumed = kt + 1;
+        if (__syncthreads_or(timeout)) {
+            timeout = true;
+            break;
+        }
+        if (n == 0 && issued < ntile)
+            issue(issued++);
+    }
+    if (timeout) {
+        if (n == 0) {
+            set_status(status, WIDE_DEV_TIMEOUT);
+            for (int kt = consumed; kt < issued; ++kt)
+                mbar_wait(&full[kt % kStages], (uint32_t)(kt / kStages) & 1u);
+        }
+        __syncthreads();
+    }
+
+    float *part = reinterpret_cast<float *>(stages);  // [kNTok][128]
+#pragma unroll
+    for (int t = 0; t < kNTok; ++t) {
+        if (t >= T)
+            break;
+        part[t * kDownRows + n] = timeout ? 0.f : acc[t];
+    }
+    cluster.sync();
+    for (int t = s; t < T; t += KS) {
+        float sum = 0.f;
+        for (int q = 0; q < KS; ++q)
+            sum += cluster.map_shared_rank(part, q)[t * kDownRows + n];
+        out[(size_t)t * H + (size_t)nb * kDownRows + n] = from_f32<TIn>(sum);
+    }
+    cluster.sync();
+}
+
+template <typename... KArgs, typename... Args>
+int launch_cluster(int32_t kid, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                   int cluster_x, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!raise_smem_limit(reinterpret_cast<const void *>(kernel), smem))
+        return WIDE_ECUDA;
+    LaunchScope scope(kid, s);
+    if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess)
+        return WIDE_ECUDA;
+    return WIDE_OK;
+}
+
+template <typename TIn, int GS>
+int decode_chunk(const TIn *x, const TIn *wg, const TIn *wu, const TIn *wd, const uint32_t *mask,
+                 TIn *out, int T, int H, int I, float *h, cudaStream_t s)
+{
+    constexpr int EPC = ElemTraits<TIn>::EPC;
+    constexpr int KT = 8 * EPC;
+    const int G = I / GS, W = (G + 31) / 32;
+    int KS = 8;
+    while (KS > 1 && (H % (KS * KT)) != 0)
+        KS >>= 1;
+    const int kslice = H / KS;
+
+    CUtensorMap tg, tu, td, th;
+    if (!make_tmap_2d(&tg, wg, I, H, H, sizeof(TIn), GS, KT, true) ||
+        !make_tmap_2d(&tu, wu, I, H, H, sizeof(TIn), GS, KT, true) ||
+        !make_tmap_2d(&td, wd, H, I, I, sizeof(TIn), kDownRows, KT, true) ||
+        !make_tmap_2d(&th, h, T, I, I, 4, T, KT, false))
+        return WIDE_ECUDA;
+
+    const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 256 + (size_t)T * kslice * 4;
+    int rc = launch_cluster(KID_DECODE_GATEUP, ffn_decode_gateup<TIn, GS>, dim3(KS, G), dim3(GS), smem1, KS, s, tg,
+                            tu, x, mask, h, T, H, I, W, kslice, status_ptr());
+    if (rc)
+        return rc;
+
+    const int KSd = G < 8 ? G : 8;
+    const size_t hb = (size_t)T * KT * 4;
+    const size_t stage = (size_t)kDownRows * 128 + ((hb + 1023) & ~(size_t)1023);
+    const size_t smem2 = 1024 + kStages * stage + 64 + 1024 * 4 + 1024 * 4;
+    return launch_cluster(KID_DECODE_DOWN, ffn_decode_down<TIn, GS>, dim3(KSd, H / kDownRows), dim3(kDownRows),
+                          smem2, KSd, s, td, th, mask, out, T, H, I, W, G, status_ptr());
+}
+
+template <typename TIn, int GS>
+int decode_all(const void *x, const void *wg, const void *wu, const void *wd,
+               const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
+               cudaStream_t s)
+{
+    const int64_t T = d->tokens, H = d->hidden, I = d->inter;
+    const int W = (int)((I / GS + 31) / 32);
+    for (int64_t t0 = 0; t0 < T; t0 += kNTok) {
+        const int Tc = (int)(T - t0 < kNTok ? T - t0 : kNTok);
+        int rc = decode_chunk<TIn, GS>(
+            static_cast<const TIn *>(x) + t0 * H, static_cast<const TIn *>(wg),
+            static_cast<const TIn *>(wu), static_cast<const TIn *>(wd), mask + t0 * W,
+            static_cast<TIn *>(out) + t0 * H, Tc, (int)H, (int)I, static_cast<float *>(ws), s);
+        if (rc)
+            return rc;
+    }
+    return WIDE_OK;
+}
+
+}  // namespace
+
+size_t ffn_decode_workspace(const wide_ffn_dims *d)
+{
+    const int64_t T = d->tokens < kNTok ? d->tokens : kNTok;
+    return align_up((size_t)(T > 0 ? T : 1) * (size_t)d->inter * sizeof(float), 256);
+}
+
+int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
+                      const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
+                      cudaStream_t s)
+{
+    if (d->tokens == 0)
+        return WIDE_OK;
+    const int64_t gs = d->group_size;
+    if (d->dtype == WIDE_BF16) {
+        if (gs == 128)
+            return decode_all<__nv_bfloat16, 128>(x, wg, wu, wd, mask, out, d, ws, s);
+        if (gs == 64)
+            return decode_all<__nv_bfloat16, 64>(x, wg, wu, wd, mask, out, d, ws, s);
+    } else {
+        if (gs == 128)
+            return decode_all<float, 128>(x, wg, wu, wd, mask, out, d, ws, s);
+        if (gs == 64)
+            return decode_all<float, 64>(x, wg, wu, wd, mask, out, d, ws, s);
+        if (gs == 32)
+            return decode_all<float, 32>(x, wg, wu, wd, mask, out, d, ws, s);
+    }
+    return WIDE_EUNSUPPORTED;
+}
+
+}  // namespace wide
