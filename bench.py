@@ -13,8 +13,8 @@ C ABI; tokens per step = 41.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronise on both sides.  Each call is timed with CUDA events on the
-launch stream after an L2 flush (a 256 MiB write) that sits outside the
-events; ms_per_step is the sum of the call times, maximised over ranks.
+launch stream after an L2 flush (a 256 MiB write, then a read of it so that L2
+holds clean lines) that sits outside the events; ms_per_step is the sum of the call times, maximised over ranks.
 Kernel times for the roofline come from the library's own per-launch events
 (wide_profile_*) recorded during the same timed steps.  SM clocks and
 throttle reasons are sampled through NVML during the timed steps.
@@ -83,6 +83,17 @@ def algorithmic_bytes(case):
             "total": w_gateup + w_down + x + m + 2 * h + out, "union_groups": U}
 
 
+def _nvml_handle(nv, cuda_index: int):
+    """NVML handle of CUDA device `cuda_index`, honouring CUDA_VISIBLE_DEVICES."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ent = vis.split(",")[cuda_index].strip()
+        if ent.startswith("GPU-") or ent.startswith("MIG-"):
+            return nv.nvmlDeviceGetHandleByUUID(ent)
+        return nv.nvmlDeviceGetHandleByIndex(int(ent))
+    return nv.nvmlDeviceGetHandleByIndex(cuda_index)
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML (read-only)."""
 
@@ -99,7 +110,7 @@ class ClockSampler:
             import pynvml as nv
             nv.nvmlInit()
             self._nv = nv
-            self._h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self._h = _nvml_handle(nv, self.index)
             self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
             self.ok = True
             self._t = threading.Thread(target=self._run, daemon=True)
@@ -261,6 +272,7 @@ def run_ours(args):
     ws_bytes = max(w.wide_ffn_workspace_bytes(c.T, c.H, c.I, c.gs) for c in cases)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream(dev)
     gs = base.gs
     PATH = w.WIDE_PATH_DECODE
@@ -273,7 +285,11 @@ def run_ours(args):
     def timed_step(fn, nstreams=len(cases)):
         evs = []
         for i in range(nstreams):
+            # flush L2: write a buffer larger than L2, then read it back so
+            # the lines left behind are clean (a timed kernel should not pay
+            # for writing back the flush's own dirty lines)
             flush.zero_()
+            flush_sink.copy_(flush.view(torch.int64).sum())
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn(i)
@@ -346,7 +362,8 @@ def run_ours(args):
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": dk["achieved_gbs"] / peaks["hbm_gbs"],
                     "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)",
-                    "traffic": traffic["dram_bytes_per_launch"] if traffic else None,
+                    "traffic": traffic["dram_bytes_per_step"] if traffic else None,
+                    "traffic_unit": "DRAM bytes per step (one launch per batch size), ncu",
                     "note": "achieved = union-of-groups gate/up weight bytes + x + mask + h, "
                             "summed over the three batch sizes / summed mean launch time"}
 
@@ -423,7 +440,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; shapes of the pages' Llama-3.2-3B FFN)",
         "config": {"workload": _workload_desc(), "global_batch": world * tokens_per_step,
-                   "l2": "flushed (256 MiB write) before every timed call",
+                   "l2": "flushed before every timed call (256 MiB write, then read back)",
                    "parallelism": f"replicas x{world} (no collective on the data path)"},
         "roofline": roofline, "kernels": kernels, "per_batch": per_batch,
         "dense_baseline": dense, "e2e": e2e, "cpu_baseline": cpu,

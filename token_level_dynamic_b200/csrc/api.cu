@@ -77,16 +77,29 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
 
 bool raise_smem_limit(const void *kernel, size_t bytes)
 {
+    // The attribute is an upper bound, so it is raised once per (kernel,
+    // device) to the device's opt-in maximum; lowering it for a smaller
+    // launch would break a later, larger one.
     static std::mutex mu;
-    static std::set<std::pair<std::pair<const void *, int>, size_t>> done;
+    static std::set<std::pair<const void *, int>> done;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return false;
     std::lock_guard<std::mutex> lock(mu);
-    auto key = std::make_pair(std::make_pair(kernel, dev), bytes);
+    const auto key = std::make_pair(kernel, dev);
+    int optin = 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+        return false;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+        return false;
+    const int limit = optin - (int)fa.sharedSizeBytes;  // static + dynamic <= opt-in
+    if (bytes > (size_t)limit)
+        return false;
     if (done.count(key))
         return true;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit) !=
         cudaSuccess)
         return false;
     done.insert(key);

@@ -19,7 +19,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxWords = 32;  // G <= 1024
 
 __device__ __forceinline__ uint32_t lanemask_lt()
 {
@@ -205,15 +204,8 @@ int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
     const int S = wl->scratch_splits;
     const int tiles = (int)((T + kThreads - 1) / kThreads);
     const size_t smem = (size_t)2 * W * kThreads * sizeof(uint32_t);
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(reorder_k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(2 * kMaxWords * kThreads * sizeof(uint32_t))) != cudaSuccess)
-            return WIDE_ECUDA;
-        attr_set[dev] = true;
-    }
+    if (!raise_smem_limit(reinterpret_cast<const void *>(reorder_k1), smem))
+        return WIDE_ECUDA;
     {
         LaunchScope scope(KID_REORDER_PARTITION_RANK, s);
         reorder_k1<<<(unsigned)(G + (int64_t)tiles * S), kThreads, smem, s>>>(
