@@ -52,6 +52,7 @@ extern "C" {
 #define WIDE_EUNSUPPORTED -2  /* a shape or alignment this build does not run */
 #define WIDE_EWORKSPACE -3    /* workspace smaller than the *_workspace_bytes query */
 #define WIDE_ECUDA -4         /* a CUDA runtime/driver call failed */
+#define WIDE_ETOOLARGE -5     /* exceeds the fixed scratch of wide_ffn_masked_noalloc */
 
 /* device status word bits (wide_get_device_status) */
 #define WIDE_DEV_BAD_MASK 0x1 /* a mask word had a bit at or above G set */
@@ -193,6 +194,33 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                     const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
                     const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
                     void *stream);
+
+/* ------------------------------------------- FFN without device allocation
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory or hand the library a workspace (for
+ * example code inside a host framework that owns the whole device memory
+ * pool, or a latency-critical loop where cudaMalloc/cudaFree would
+ * synchronise the device).
+ *
+ * Same operation, arguments and layouts as wide_ffn_masked on its decode
+ * path (CUDA-core GEMV over the batch's union of groups), minus the
+ * workspace: the kernels' scratch (fp32 h for up to 32 tokens x inter
+ * channels) lives in a fixed device array inside the library of
+ * WIDE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * holds until the process exits.  Limit: min(tokens, 32) * inter * 4 bytes
+ * must not exceed it (inter <= 16384); larger problems return
+ * WIDE_ETOOLARGE before anything is enqueued.  The call allocates nothing.
+ * Its first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls on a device share the array, which keeps the last
+ * call's contents (nothing in it needs to start at zero); calls that overlap
+ * on the GPU -- on streams not ordered with each other -- race on it.
+ * d->path must be WIDE_PATH_AUTO or WIDE_PATH_DECODE. */
+#define WIDE_NOALLOC_SCRATCH_BYTES 2097152
+int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, const void *d_w_up,
+                            const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
+                            const wide_ffn_dims *d, void *stream);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,8 @@ import torch
 
 from . import _native
 from ._native import (  # noqa: F401
-    WIDE_OK, WIDE_EINVAL, WIDE_EUNSUPPORTED, WIDE_EWORKSPACE, WIDE_ECUDA,
+    WIDE_OK, WIDE_EINVAL, WIDE_EUNSUPPORTED, WIDE_EWORKSPACE, WIDE_ECUDA, WIDE_ETOOLARGE,
+    WIDE_NOALLOC_SCRATCH_BYTES,
     WIDE_DEV_BAD_MASK, WIDE_DEV_TIMEOUT, WIDE_DEV_BAD_ITEM,
     WIDE_BF16, WIDE_F32, WIDE_PATH_AUTO, WIDE_PATH_DECODE, WIDE_PATH_PREFILL,
     WideWorklist, WideFFNDims,
@@ -186,4 +187,21 @@ def wide_ffn_masked(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
         _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
         _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"), _dev_ptr(out, "out"),
         ctypes.byref(d), workspace.data_ptr(), workspace.numel(), _stream(stream, x.device)))
+    return out
+
+
+def wide_ffn_masked_noalloc(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
+                            w_down: torch.Tensor, mask_words: torch.Tensor, group_size: int,
+                            out: torch.Tensor, stream=None) -> torch.Tensor:
+    """The decode-path masked FFN for callers that cannot allocate device
+    memory: no workspace argument, and `out` must be given (this wrapper
+    allocates nothing either).  The library keeps the kernels' scratch in a
+    fixed device array of WIDE_NOALLOC_SCRATCH_BYTES bytes shared by all
+    calls on a device; calls that overlap on the GPU race on it.  Raises
+    WideError (WIDE_ETOOLARGE) when min(T, 32) * I * 4 exceeds that size."""
+    d = _ffn_dims(x, w_gate, group_size, WIDE_PATH_DECODE)
+    _check("wide_ffn_masked_noalloc", _L.wide_ffn_masked_noalloc(
+        _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
+        _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"), _dev_ptr(out, "out"),
+        ctypes.byref(d), _stream(stream, x.device)))
     return out

@@ -19,6 +19,8 @@ WIDE_EINVAL = -1
 WIDE_EUNSUPPORTED = -2
 WIDE_EWORKSPACE = -3
 WIDE_ECUDA = -4
+WIDE_ETOOLARGE = -5
+WIDE_NOALLOC_SCRATCH_BYTES = 2097152
 WIDE_DEV_BAD_MASK = 0x1
 WIDE_DEV_TIMEOUT = 0x2
 WIDE_DEV_BAD_ITEM = 0x4
@@ -61,6 +63,8 @@ SIGNATURES = {
     "wide_ffn_workspace_bytes": (c_size_t, [ctypes.POINTER(WideFFNDims)]),
     "wide_ffn_masked": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 ctypes.POINTER(WideFFNDims), c_void_p, c_size_t, c_void_p]),
+    "wide_ffn_masked_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                        c_void_p, ctypes.POINTER(WideFFNDims), c_void_p]),
 }
 
 _lib = None

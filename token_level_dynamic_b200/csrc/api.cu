@@ -139,6 +139,8 @@ bool worklist_layout(int64_t T, int64_t G, int32_t tile_m, WorklistLayout *L)
     return true;
 }
 
+}  // namespace
+
 bool ffn_dims_ok(const wide_ffn_dims *d)
 {
     if (!d || d->tokens < 0 || d->hidden <= 0 || d->inter <= 0 || d->group_size <= 0)
@@ -167,7 +169,6 @@ bool ffn_shape_supported(const wide_ffn_dims *d, int path)
     return false;  // the prefill path is built in a later file
 }
 
-}  // namespace
 }  // namespace wide
 
 using namespace wide;
@@ -187,6 +188,8 @@ const char *wide_status_string(int code)
         return "workspace too small";
     case WIDE_ECUDA:
         return "CUDA runtime or driver call failed";
+    case WIDE_ETOOLARGE:
+        return "problem larger than the fixed scratch of wide_ffn_masked_noalloc";
     case WIDE_DEV_BAD_MASK:
         return "device: mask bit at or above G";
     case WIDE_DEV_TIMEOUT:

@@ -59,6 +59,11 @@ class LaunchScope {
     cudaStream_t s_;
 };
 
+// FFN argument checks shared by the FFN entry points (api.cu).
+bool ffn_dims_ok(const wide_ffn_dims *d);
+int ffn_path(const wide_ffn_dims *d);
+bool ffn_shape_supported(const wide_ffn_dims *d, int path);
+
 // Internal entry points of the kernel files.
 int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
                    const wide_worklist *wl, cudaStream_t s);
