@@ -1,0 +1,97 @@
+"""Prefill (tcgen05) masked FFN against the fp64 oracle, through the C ABI.
+
+WIDE, technical summary sections 2.B/2.C: groups run as dense tensor-core
+tiles over their reordered active-token prefixes; tiles with no active token
+are never issued; the down projection visits only the groups some token of a
+signature tile keeps."""
+import numpy as np
+import pytest
+
+import synth
+from oracle.ffn import ffn_masked, ffn_dense
+from tests._util import rel_l2, ffn_to_dev, from_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+
+
+def _run(c, x=None):
+    import torch
+    import token_level_dynamic_b200 as w
+    x_, wg, wu, wd, m = ffn_to_dev(c)
+    w.wide_clear_device_status()
+    out = w.wide_ffn_masked(x_ if x is None else x, wg, wu, wd, m, c.gs,
+                            path=w.WIDE_PATH_PREFILL)
+    torch.cuda.synchronize()
+    assert w.wide_get_device_status() == 0
+    return from_dev(out)
+
+
+def _ref(c):
+    return ffn_masked(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs)
+
+
+@pytest.mark.parametrize("T,H,I,kind,keep", [
+    (128, 256, 256, "bernoulli", 0.5),        # one full tile per group
+    (300, 256, 512, "bernoulli", 0.5),        # ragged tails, 4 groups
+    (1000, 512, 1024, "prototype", 0.5),      # prototype masks, several tiles
+    (777, 768, 1408, "bernoulli", 0.3),       # 11 groups (one partial word)
+    (513, 1024, 4352, "prototype", 0.25),     # 34 groups over two mask words
+])
+def test_prefill_parity_small(T, H, I, kind, keep):
+    c = synth.ffn_case(T, H, I, 128, seed=T, keep=keep, mask_kind=kind)
+    assert rel_l2(_run(c), _ref(c)) <= TOL
+
+
+def test_prefill_single_token_and_tiny():
+    for T in (1, 3, 5):
+        c = synth.ffn_case(T, 256, 512, 128, seed=10 + T)
+        assert rel_l2(_run(c), _ref(c)) <= TOL
+
+
+def test_prefill_all_zero_mask_is_exact_zero():
+    c = synth.ffn_case(200, 256, 512, 128, seed=3, mask_kind="zeros")
+    assert not np.any(_run(c))
+
+
+def test_prefill_all_ones_equals_dense():
+    c = synth.ffn_case(260, 512, 1024, 128, seed=4, mask_kind="ones")
+    assert rel_l2(_run(c), ffn_dense(c.x, c.w_gate, c.w_up, c.w_down)) <= TOL
+
+
+def test_prefill_one_group_per_token():
+    c = synth.ffn_case(333, 256, 1024, 128, seed=5)
+    c.mask[:] = False
+    c.mask[np.arange(c.T), np.arange(c.T) % c.G] = True
+    assert rel_l2(_run(c), _ref(c)) <= TOL
+
+
+def test_prefill_matches_decode_path():
+    """Both paths compute the same masked FFN (different kernels)."""
+    import torch
+    import token_level_dynamic_b200 as w
+    c = synth.ffn_case(32, 512, 1024, 128, seed=6)
+    x, wg, wu, wd, m = ffn_to_dev(c)
+    a = from_dev(w.wide_ffn_masked(x, wg, wu, wd, m, 128, path=w.WIDE_PATH_PREFILL))
+    b = from_dev(w.wide_ffn_masked(x, wg, wu, wd, m, 128, path=w.WIDE_PATH_DECODE))
+    torch.cuda.synchronize()
+    assert rel_l2(a, b) <= TOL
+
+
+def test_prefill_repeatable_bitwise():
+    c = synth.ffn_case(400, 512, 1024, 128, seed=7, mask_kind="prototype")
+    np.testing.assert_array_equal(_run(c), _run(c))
+
+
+def test_prefill_ffn_8b_full_size_sampled():
+    """The full Llama-3.1-8B-shaped prefill FFN (T=4096, H=4096, I=14336,
+    8 prototypes + 0.1 flips), checked on 48 sampled tokens whose outputs
+    the oracle computes one by one (tokens are independent)."""
+    c = synth.prefill_ffn()
+    out = _run(c)
+    rows = np.random.default_rng(0).choice(c.T, 48, replace=False)
+    sub = synth.FFNCase("s", len(rows), c.H, c.I, c.gs, "bf16", c.x[rows], c.w_gate, c.w_up,
+                        c.w_down, c.mask[rows])
+    assert rel_l2(out[rows], _ref(sub)) <= TOL
+    assert np.isfinite(out).all()

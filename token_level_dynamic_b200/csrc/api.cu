@@ -166,7 +166,8 @@ bool ffn_shape_supported(const wide_ffn_dims *d, int path)
     const int64_t gs = d->group_size;
     if (path == WIDE_PATH_DECODE)
         return d->dtype == WIDE_BF16 ? (gs == 64 || gs == 128) : (gs == 32 || gs == 64 || gs == 128);
-    return false;  // the prefill path is built in a later file
+    // prefill: tcgen05 kernels with 128-channel groups and 256-column output blocks
+    return d->dtype == WIDE_BF16 && gs == 128 && d->hidden % 256 == 0 && d->tokens <= (1 << 24);
 }
 
 }  // namespace wide
@@ -279,7 +280,7 @@ size_t wide_ffn_workspace_bytes(const wide_ffn_dims *d)
     const int path = ffn_path(d);
     if (path == WIDE_PATH_DECODE)
         return ffn_decode_workspace(d);
-    return 0;
+    return ffn_prefill_workspace(d);
 }
 
 int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
@@ -305,7 +306,8 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
     if (path == WIDE_PATH_DECODE)
         return ffn_decode_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d,
                                  d_workspace, s);
-    return WIDE_EUNSUPPORTED;
+    return ffn_prefill_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d,
+                              d_workspace, s);
 }
 
 }  // extern "C"

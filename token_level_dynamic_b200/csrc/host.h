@@ -69,6 +69,11 @@ int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
                    const wide_worklist *wl, cudaStream_t s);
 int reorder_splits(int64_t T);
 
+size_t ffn_prefill_workspace(const wide_ffn_dims *d);
+int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void *wd,
+                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
+                       cudaStream_t s);
+
 size_t ffn_decode_workspace(const wide_ffn_dims *d);
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
