@@ -2,22 +2,28 @@
 """Benchmark of the masked WIDE layer on B200; prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_ffn_3b]
+                    [--workload decode_ffn_3b|prefill_ffn_8b]
 
-Workload ``decode_ffn_3b`` (default): the Llama-3.2-3B-shaped masked SwiGLU FFN
-in decode -- hidden 3072, intermediate 8192 in 64 channel groups of 128,
-bf16 weights ~ N(0, 0.02), x ~ N(0, 1), per-(token, group) keep mask
-Bernoulli(0.5).  One step runs the three batch sizes of that configuration
-(1, 8 and 32 tokens, each with its own x and mask) through the library's
-C ABI; tokens per step = 41.
+Workloads (seeded synthetic inputs with the shapes the pages name):
+  decode_ffn_3b (default)  Llama-3.2-3B-shaped masked SwiGLU FFN in decode:
+      hidden 3072, intermediate 8192 in 64 groups of 128, bf16, Bernoulli(0.5)
+      masks.  One step = the three batch sizes of the configuration (1, 8
+      and 32 tokens, each with its own x and mask): 41 tokens.  HBM-bound;
+      the roofline is union-of-groups weight bytes over measured HBM GB/s.
+  prefill_ffn_8b  Llama-3.1-8B-shaped masked SwiGLU FFN in prefill: 4096
+      tokens, hidden 4096, intermediate 14336 in 112 groups of 128, 8
+      prototype masks (56 groups each) with 0.1 bit flips.  One step = one
+      call (mask reordering, zero fill, tcgen05 gate/up and down).  Tensor
+      bound; the roofline is kept FLOPs over the measured bf16 tensor peak.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronise on both sides.  Each call is timed with CUDA events on the
-launch stream after an L2 flush (a 256 MiB write, then a read of it so that L2
-holds clean lines) that sits outside the events; ms_per_step is the sum of the call times, maximised over ranks.
-Kernel times for the roofline come from the library's own per-launch events
-(wide_profile_*) recorded during the same timed steps.  SM clocks and
-throttle reasons are sampled through NVML during the timed steps.
+launch stream after an L2 flush (a 256 MiB write, then a read of it so that
+L2 holds clean lines) that sits outside the events; ms_per_step is the sum
+of the call times, maximised over ranks.  Kernel times for the roofline come
+from the library's own per-launch events (wide_profile_*) recorded during the
+same timed steps.  SM clocks and throttle reasons are sampled through NVML
+during the timed steps.
 
 Multi-GPU: every rank runs the same workload on its own GPU (replicas, weak
 scaling); value = all ranks' tokens / the slowest rank's time.
@@ -40,7 +46,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "masked-layer tok/s @50% sparsity; HBM GB/s (decode), TFLOPS (prefill)"
-BATCHES = (1, 8, 32)
 FLUSH_BYTES = 256 << 20
 
 
@@ -54,33 +59,6 @@ def _peaks():
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
-
-
-def _workload_desc():
-    return ("decode_ffn_3b: Llama-3.2-3B-shaped masked SwiGLU FFN decode, hidden 3072, "
-            "intermediate 8192 = 64 groups x 128, bf16, Bernoulli(0.5) masks; one step = "
-            "batches 1, 8 and 32 (41 tokens)")
-
-
-def _union_groups(mask_bool):
-    return int(mask_bool.any(axis=0).sum())
-
-
-def algorithmic_bytes(case):
-    """Bytes a call must move at minimum: every weight byte of the batch's
-    union of groups once, plus x, mask, the fp32 h it writes and reads back,
-    and out."""
-    B, H, I, gs = case.T, case.H, case.I, case.gs
-    U = _union_groups(case.mask)
-    pairs = int(case.mask.sum())
-    w_gateup = 2 * U * gs * H * 2
-    w_down = H * U * gs * 2
-    x = B * H * 2
-    m = case.mask_words.nbytes
-    h = pairs * gs * 4
-    out = B * H * 2
-    return {"gateup": w_gateup + x + m + h, "down": w_down + h + m + out,
-            "total": w_gateup + w_down + x + m + 2 * h + out, "union_groups": U}
 
 
 def _nvml_handle(nv, cuda_index: int):
@@ -153,7 +131,7 @@ class ClockSampler:
 
 
 def _traffic_record(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    """DRAM bytes per step from the committed ncu summary, if the kernel
     source it was taken on is unchanged."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
@@ -168,51 +146,111 @@ def _traffic_record(kernel: str, workload: str):
         return None
 
 
-def cpu_oracle_baseline(cases, seconds: float = 10.0):
+# --------------------------------------------------------------- workloads
+
+class DecodeFFN3B:
+    name = "decode_ffn_3b"
+    desc = ("decode_ffn_3b: Llama-3.2-3B-shaped masked SwiGLU FFN decode, hidden 3072, "
+            "intermediate 8192 = 64 groups x 128, bf16, Bernoulli(0.5) masks; one step = "
+            "batches 1, 8 and 32 (41 tokens)")
+    bound = "hbm"
+    dominant = "decode_gateup_gemv"
+    path_name = "WIDE_PATH_DECODE"
+
+    def make_cases(self):
+        import synth
+        base = synth.decode_ffn(1)
+        cases = [base]
+        for b in (8, 32):
+            c = synth.decode_ffn(b, weights=False)
+            c.w_gate, c.w_up, c.w_down = base.w_gate, base.w_up, base.w_down
+            cases.append(c)
+        return cases
+
+    @staticmethod
+    def units(case):
+        """Algorithmic bytes per call, per kernel: every weight byte of the
+        batch's union of groups once, plus x, mask, fp32 h and out."""
+        B, H, I, gs = case.T, case.H, case.I, case.gs
+        U = int(case.mask.any(axis=0).sum())
+        pairs = int(case.mask.sum())
+        m = case.mask_words.nbytes
+        h = pairs * gs * 4
+        gateup = 2 * U * gs * H * 2 + B * H * 2 + m + h
+        down = H * U * gs * 2 + h + m + B * H * 2
+        return {"decode_gateup_gemv": gateup, "decode_down_gemv": down,
+                "total": gateup + down, "union_groups": U}
+
+    def reference_sample(self, cases):
+        out = []
+        for c in cases:
+            s = type(c)(**{**c.__dict__})
+            s.x, s.mask, s.T = c.x[:1], c.mask[:1], 1
+            out.append(s)
+        return out, "per step: token 0 of each of batches 1, 8, 32 (3 tokens)"
+
+
+class PrefillFFN8B:
+    name = "prefill_ffn_8b"
+    desc = ("prefill_ffn_8b: Llama-3.1-8B-shaped masked SwiGLU FFN prefill, 4096 tokens, hidden "
+            "4096, intermediate 14336 = 112 groups x 128, bf16, 8 prototype masks (56 groups) + "
+            "0.1 flips; one step = one call")
+    bound = "tensor"
+    dominant = "prefill_gateup_tcgen05"
+    path_name = "WIDE_PATH_PREFILL"
+
+    def make_cases(self):
+        import synth
+        return [synth.prefill_ffn()]
+
+    @staticmethod
+    def units(case):
+        """Kept FLOPs per call: 2 flops per multiply-add, only (token, kept
+        group) work; gate and up in the first kernel, down in the second."""
+        H, gs = case.H, case.gs
+        pairs = int(case.mask.sum())
+        gateup = 2 * 2 * H * gs * pairs
+        down = 2 * H * gs * pairs
+        return {"prefill_gateup_tcgen05": gateup, "prefill_down_tcgen05": down,
+                "total": gateup + down, "pairs": pairs,
+                "dense_flops": 6 * case.T * H * case.I}
+
+    def reference_sample(self, cases):
+        c = cases[0]
+        s = type(c)(**{**c.__dict__})
+        s.x, s.mask, s.T = c.x[:8], c.mask[:8], 8
+        return [s], "per step: the first 8 tokens of the 4096-token batch"
+
+
+WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B())}
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_baseline(samples, seconds: float):
     """Times the oracle's per-token loop (fp64, OpenMP over tokens) on the
-    host: all tokens of one step, repeated until `seconds` have passed."""
+    host cores, repeating the sample until `seconds` have passed."""
     import oracle
     from oracle import _clib
     tokens, t0, reps = 0, time.perf_counter(), 0
     while True:
-        for c in cases:
+        for c in samples:
             oracle.ffn.ffn_token_loop(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs, "bf16")
             tokens += c.T
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": tokens / el, "unit": "tokens/s", "cores": int(_clib.lib().oracle_num_threads()),
-            "kind": "oracle",
-            "sample": f"{reps} repetitions of one full step ({sum(c.T for c in cases)} tokens: "
-                      f"batches {', '.join(str(c.T) for c in cases)}), fp64 per-token loop over "
-                      f"kept groups, {el:.1f} s"}
+    return tokens / el, int(_clib.lib().oracle_num_threads()), reps, el
 
 
-def _make_cases():
-    import synth
-    base = synth.decode_ffn(BATCHES[0])
-    cases = [base]
-    for b in BATCHES[1:]:
-        c = synth.decode_ffn(b, weights=False)
-        c.w_gate, c.w_up, c.w_down = base.w_gate, base.w_up, base.w_down
-        cases.append(c)
-    return cases
-
-
-def run_reference(args):
+def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import oracle
     from oracle import _clib
-    cases = _make_cases()
-    # bounded sample per step: the first token of every batch
-    samples = []
-    for c in cases:
-        s = type(c)(**{**c.__dict__})
-        s.x, s.mask, s.T = c.x[:1], c.mask[:1], 1
-        samples.append(s)
+    samples, what = wl.reference_sample(wl.make_cases())
 
     def step():
         for s in samples:
@@ -224,25 +262,26 @@ def run_reference(args):
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
-    tok = args.steps * len(samples)
+    tok = args.steps * sum(s.T for s in samples)
     v = tok / el
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": _workload_desc(), "parallelism": "host cores"},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": int(_clib.lib().oracle_num_threads()),
-                         "kind": "oracle",
-                         "sample": "per step: token 0 of each of batches 1, 8, 32 (3 tokens), "
-                                   "fp64 per-token loop over kept groups"},
+        "config": {"workload": wl.desc, "parallelism": "host cores"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s",
+                         "cores": int(_clib.lib().oracle_num_threads()), "kind": "oracle",
+                         "sample": what + ", fp64 per-token loop over kept groups"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def run_ours(args):
+# ------------------------------------------------------------------- ours
+
+def run_ours(args, wl):
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -261,7 +300,7 @@ def run_ours(args):
     import token_level_dynamic_b200 as w
     from synth.torch_io import to_dev
 
-    cases = _make_cases()
+    cases = wl.make_cases()
     base = cases[0]
     Wg = to_dev(base.w_gate, "bf16", dev)
     Wu = to_dev(base.w_up, "bf16", dev)
@@ -269,22 +308,24 @@ def run_ours(args):
     xs = [to_dev(c.x, "bf16", dev) for c in cases]
     ms = [to_dev(c.mask_words, "mask", dev) for c in cases]
     outs = [torch.empty_like(x) for x in xs]
-    ws_bytes = max(w.wide_ffn_workspace_bytes(c.T, c.H, c.I, c.gs) for c in cases)
+    PATH = getattr(w, wl.path_name)
+    ws_bytes = max(w.wide_ffn_workspace_bytes(c.T, c.H, c.I, c.gs, path=PATH) for c in cases)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream(dev)
     gs = base.gs
-    PATH = w.WIDE_PATH_DECODE
-    ab = [algorithmic_bytes(c) for c in cases]
+    units = [wl.units(c) for c in cases]
+    ncalls = len(cases)
+    tokens_per_step = sum(c.T for c in cases)
 
     def call(i, mask=None):
         w.wide_ffn_masked(xs[i], Wg, Wu, Wd, ms[i] if mask is None else mask, gs, out=outs[i],
                           workspace=ws, path=PATH, stream=stream)
 
-    def timed_step(fn, nstreams=len(cases)):
+    def timed_step(fn):
         evs = []
-        for i in range(nstreams):
+        for i in range(ncalls):
             # flush L2: write a buffer larger than L2, then read it back so
             # the lines left behind are clean (a timed kernel should not pay
             # for writing back the flush's own dirty lines)
@@ -302,7 +343,9 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # correctness guard: one call each, status word clean
+    def ms_of(evs_list):
+        return np.array([[a.elapsed_time(b) for a, b in evs] for evs in evs_list])
+
     w.wide_clear_device_status(stream)
     for _ in range(args.warmup):
         timed_step(call)
@@ -320,100 +363,121 @@ def run_ours(args):
     launches = w.wide_launch_count() - n0
     w.wide_profile_stop()
     recs = w.wide_profile_read()
-    per_call = np.array([[e0.elapsed_time(e1) for (e0, e1) in evs] for evs in all_evs])  # [K][3] ms
-    step_ms = float(per_call.sum(axis=1).mean())
+    if w.wide_get_device_status(stream) != 0:
+        raise RuntimeError("device status set during the timed steps")
+    per_call = ms_of(all_evs)                       # [K][ncalls] ms
     total_ms = float(per_call.sum())
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-        step_ms = total_ms / args.steps
-    tokens_per_step = sum(c.T for c in cases)
+    step_ms = total_ms / args.steps
     value = world * tokens_per_step * args.steps / (total_ms / 1e3)
 
-    # per-kernel durations (the library's own launch events)
+    # ---- per-kernel figures from the library's launch events
+    peaks = _peaks()
     kern = {}
     for name, t in recs:
         kern.setdefault(name, []).append(t)
-    peaks = _peaks()
-    nb = len(cases)
     kernels = {}
-    for name, key in (("decode_gateup_gemv", "gateup"), ("decode_down_gemv", "down")):
-        ts = kern.get(name, [])
-        if not ts:
-            continue
-        # launches cycle through the batches in step order
-        per_b = [ts[i::nb] for i in range(nb)]
-        bytes_step = sum(a[key] for a in ab)
-        t_step = sum(statistics.mean(p) for p in per_b)
-        gbs = bytes_step / (t_step / 1e3) / 1e9
-        kernels[name] = {
-            "launches": len(ts), "avg_us": 1e3 * statistics.mean(ts),
-            "per_batch_us": {str(c.T): 1e3 * statistics.mean(p) for c, p in zip(cases, per_b)},
-            "algorithmic_bytes_per_step": bytes_step, "achieved_gbs": gbs,
-            "frac_of_hbm": gbs / peaks["hbm_gbs"],
-        }
-    dom = "decode_gateup_gemv"
-    dk = kernels.get(dom)
-    traffic = _traffic_record(dom, "decode_ffn_3b")
-    roofline = None
-    if dk:
-        roofline = {"kernel": dom, "bound": "hbm", "achieved": dk["achieved_gbs"],
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": dk["achieved_gbs"] / peaks["hbm_gbs"],
-                    "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)",
-                    "traffic": traffic["dram_bytes_per_step"] if traffic else None,
-                    "traffic_unit": "DRAM bytes per step (one launch per batch size), ncu",
-                    "note": "achieved = union-of-groups gate/up weight bytes + x + mask + h, "
-                            "summed over the three batch sizes / summed mean launch time"}
+    for name, ts in kern.items():
+        per_call_ts = [ts[i::ncalls] for i in range(ncalls)] if len(ts) % ncalls == 0 else [ts]
+        t_step = sum(statistics.mean(p) for p in per_call_ts)
+        entry = {"launches": len(ts), "avg_us": 1e3 * statistics.mean(ts),
+                 "us_per_step": 1e3 * t_step}
+        if name in units[0]:
+            u_step = sum(u[name] for u in units)
+            if wl.bound == "hbm":
+                a = u_step / (t_step / 1e3) / 1e9
+                entry.update({"algorithmic_bytes_per_step": u_step, "achieved_gbs": a,
+                              "frac_of_hbm": a / peaks["hbm_gbs"]})
+            else:
+                a = u_step / (t_step / 1e3) / 1e12
+                entry.update({"kept_flops_per_step": u_step, "achieved_tflops": a,
+                              "frac_of_bf16_peak": a / peaks["bf16_tflops"],
+                              "frac_of_bf16_sustained": a / peaks["bf16_tflops_sustained"]})
+        kernels[name] = entry
+    tot_k = sum(k["us_per_step"] for k in kernels.values())
+    for k in kernels.values():
+        k["share_of_library_time"] = k["us_per_step"] / tot_k if tot_k else None
 
-    per_batch = {}
+    dk = kernels.get(wl.dominant, {})
+    traffic = _traffic_record(wl.dominant, wl.name)
+    if wl.bound == "hbm":
+        roofline = {"kernel": wl.dominant, "bound": "hbm", "achieved": dk.get("achieved_gbs"),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": dk.get("frac_of_hbm"),
+                    "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"}
+    else:
+        roofline = {"kernel": wl.dominant, "bound": "tensor", "achieved": dk.get("achieved_tflops"),
+                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": dk.get("frac_of_bf16_peak"),
+                    "frac_of_sustained": dk.get("frac_of_bf16_sustained"),
+                    "peak_source": f"{peaks['source']} bf16_tflops burst (MEASURED_PEAKS.json)"}
+    roofline["traffic"] = traffic["dram_bytes_per_step"] if traffic else None
+    roofline["traffic_unit"] = "DRAM bytes per step of the dominant kernel (ncu)"
+
+    per_call_out = {}
     for i, c in enumerate(cases):
         t = float(per_call[:, i].mean())
-        per_batch[str(c.T)] = {
-            "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3),
-            "union_groups": ab[i]["union_groups"], "algorithmic_bytes": ab[i]["total"],
-            "achieved_gbs": ab[i]["total"] / (t / 1e3) / 1e9,
-            "frac_of_hbm": ab[i]["total"] / (t / 1e3) / 1e9 / peaks["hbm_gbs"],
-        }
+        d = {"tokens": c.T, "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3)}
+        if wl.bound == "hbm":
+            d.update({"union_groups": units[i]["union_groups"],
+                      "algorithmic_bytes": units[i]["total"],
+                      "achieved_gbs": units[i]["total"] / (t / 1e3) / 1e9})
+            d["frac_of_hbm"] = d["achieved_gbs"] / peaks["hbm_gbs"]
+        else:
+            d.update({"kept_flops": units[i]["total"],
+                      "achieved_tflops_whole_call": units[i]["total"] / (t / 1e3) / 1e12,
+                      "kept_fraction_of_dense": units[i]["total"] / units[i]["dense_flops"]})
+        per_call_out[c.name] = d
 
-    # ---- dense baselines (same shapes): torch/cuBLAS bf16, and our kernels with all-ones masks
-    ones = [torch.full_like(m, -1) for m in ms]  # 64 groups -> two full words
+    # ---- dense baselines: torch/cuBLAS bf16 and our kernels with every group kept
+    ones = [torch.full_like(m, -1) for m in ms]
+    G = base.I // gs
+    if G % 32:
+        for o in ones:
+            o[:, -1] = (1 << (G % 32)) - 1
+
     def dense_torch(i):
         x = xs[i]
         a = torch.nn.functional.linear(x, Wg)
         b = torch.nn.functional.linear(x, Wu)
         outs[i].copy_(torch.nn.functional.linear(torch.nn.functional.silu(a) * b, Wd))
+
     def ours_ones(i):
         call(i, ones[i])
+
     dense = {}
+    nd = max(3, min(args.steps, 20))
     for name, fn in (("torch_cublas_bf16", dense_torch), ("ours_all_groups_kept", ours_ones)):
         for _ in range(3):
             timed_step(fn)
-        evs = [timed_step(fn) for _ in range(max(5, args.steps // 4))]
+        evs = [timed_step(fn) for _ in range(nd)]
         torch.cuda.synchronize(dev)
-        pc = np.array([[a.elapsed_time(b) for a, b in e] for e in evs])
+        pc = ms_of(evs)
         dense[name] = {"ms_per_step": float(pc.sum(axis=1).mean()),
-                       "tokens_per_s": tokens_per_step / (float(pc.sum(axis=1).mean()) / 1e3),
-                       "per_batch_us": {str(c.T): 1e3 * float(pc[:, i].mean())
-                                        for i, c in enumerate(cases)}}
+                       "tokens_per_s": tokens_per_step / (float(pc.sum(axis=1).mean()) / 1e3)}
     dense["masked_speedup_vs_torch_dense"] = dense["torch_cublas_bf16"]["ms_per_step"] / step_ms
+    dense["masked_speedup_vs_ours_all_kept"] = dense["ours_all_groups_kept"]["ms_per_step"] / step_ms
 
     # ---- end to end through the public API with host buffers
     xh = [x.cpu().pin_memory() for x in xs]
     mh = [m.cpu().pin_memory() for m in ms]
     oh = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
     def e2e_call(i):
         xs[i].copy_(xh[i], non_blocking=True)
         ms[i].copy_(mh[i], non_blocking=True)
         call(i)
         oh[i].copy_(outs[i], non_blocking=True)
+
     for _ in range(3):
         timed_step(e2e_call)
     barrier()
     e_evs = [timed_step(e2e_call) for _ in range(args.steps)]
     barrier()
-    e_ms = float(np.array([[a.elapsed_time(b) for a, b in e] for e in e_evs]).sum())
+    e_ms = float(ms_of(e_evs).sum())
     if world > 1:
         t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -423,28 +487,30 @@ def run_ours(args):
            "d2h_bytes_per_step": int(sum(o.numel() * 2 for o in oh)),
            "ms_per_step": e_ms / args.steps}
 
-    # ---- parity spot check of this run's outputs (B=8) against the oracle
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_baseline(cases, seconds=args.cpu_seconds)
+        samples, what = wl.reference_sample(cases)
+        v, cores, reps, el = cpu_oracle_baseline(samples, args.cpu_seconds)
+        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{what}; repeated {reps}x over {el:.1f} s; fp64 per-token loop over "
+                         f"kept groups"}
 
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    clocks = clk.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; shapes of the pages' Llama-3.2-3B FFN)",
-        "config": {"workload": _workload_desc(), "global_batch": world * tokens_per_step,
+        "data": "synthetic (seeded; shapes of the pages' Llama workloads)",
+        "config": {"workload": wl.desc, "global_batch": world * tokens_per_step,
                    "l2": "flushed before every timed call (256 MiB write, then read back)",
                    "parallelism": f"replicas x{world} (no collective on the data path)"},
-        "roofline": roofline, "kernels": kernels, "per_batch": per_batch,
+        "roofline": roofline, "kernels": kernels, "per_call": per_call_out,
         "dense_baseline": dense, "e2e": e2e, "cpu_baseline": cpu,
-        "gpu_launches": int(launches), "clocks": clocks,
+        "gpu_launches": int(launches), "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -453,18 +519,19 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode_ffn_3b"], default="decode_ffn_3b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_ffn_3b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
     if args.impl == "reference":
-        return run_reference(args)
-    return run_ours(args)
+        return run_reference(args, wl)
+    return run_ours(args, wl)
 
 
 if __name__ == "__main__":

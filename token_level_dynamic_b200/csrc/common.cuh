@@ -114,6 +114,25 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ------------------------------------------------------------- cp.async
+// 16-byte global -> shared copy that bypasses L1.
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gsrc)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc)
+                 : "memory");
+}
+// Arrive on the mbarrier once every cp.async this thread issued so far has
+// completed; the barrier's expected count already includes this arrive.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Byte offset of 16-byte chunk j of row r in a tile of 128-byte rows written
 // by TMA with CU_TENSOR_MAP_SWIZZLE_128B (tile base 1024-byte aligned).
 __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t j)

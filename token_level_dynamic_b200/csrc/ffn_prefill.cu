@@ -12,8 +12,10 @@
 //               token skips, so that the down projection can treat every
 //               tile of H as dense.
 //   gateup      persistent, warp-specialised.  Work item (g, i) = rows
-//               perm[g][128 i : 128 i + 128) of x (gathered four rows per TMA
-//               gather4) times the 256-row slab [W_gate[g]; W_up[g]]; one
+//               perm[g][128 i : 128 i + 128) of x (gathered 16 bytes at a time
+//               with cp.async by two warps, straight into the swizzled
+//               operand layout) times the 256-row slab [W_gate[g]; W_up[g]]
+//               (TMA); one
 //               M=128, N=256, K=16 tcgen05 MMA per 16 columns of K into an
 //               fp32 TMEM accumulator (two accumulators, 512 columns, so the
 //               epilogue of one item overlaps the MMAs of the next).  The
@@ -25,9 +27,9 @@
 //               visited group are the zeros written by zero_dead.  The
 //               epilogue writes bf16 rows of out at the tokens' own rows.
 //
-// Warp roles in both tcgen05 kernels (192 threads): warp 0 = TMA producer,
-// warp 1 = TMEM owner and single-thread MMA issuer, warps 2..5 = epilogue
-// (warp w reads TMEM lanes 32 * (w % 4) .. +31).  Every mbarrier wait is
+// Warp roles in both tcgen05 kernels: warp 0 = TMA producer, warp 1 = TMEM
+// owner and single-thread MMA issuer, warps 2..5 = epilogue (warp w reads
+// TMEM lanes 32 * (w % 4) .. +31); gate/up adds warps 6..7 for the row gather.  Every mbarrier wait is
 // bounded; on expiry the kernel records WIDE_DEV_TIMEOUT, drains what it
 // issued (bounded), frees its TMEM and returns.
 #include "common.cuh"
@@ -45,7 +47,9 @@ constexpr int kStages = 4;
 constexpr uint32_t kATile = kBM * 128;   // 16 KB
 constexpr uint32_t kBTile = kBN * 128;   // 32 KB
 constexpr uint32_t kStageBytes = kATile + kBTile;
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;      // down kernel: producer, MMA, 4 epilogue warps
+constexpr int kThreadsGU = 256;    // gate/up: + 2 warps that gather x rows with cp.async
+constexpr int kGatherThreads = 64;
 constexpr uint32_t kTmemCols = 512;
 
 struct __align__(8) Ctl {
@@ -56,7 +60,6 @@ struct __align__(8) Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    int idx[kBM];                   // producer's gathered row indices
 };
 
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + sizeof(Ctl);
@@ -123,8 +126,8 @@ __global__ void __launch_bounds__(128)
 }
 
 // --------------------------------------------------------------- gate/up
-__global__ void __launch_bounds__(kThreads, 1)
-    prefill_gateup(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_g,
+__global__ void __launch_bounds__(kThreadsGU, 1)
+    prefill_gateup(const __nv_bfloat16 *__restrict__ x, const __grid_constant__ CUtensorMap tm_g,
                    const __grid_constant__ CUtensorMap tm_u, const int32_t *__restrict__ count,
                    const int32_t *__restrict__ perm, const int32_t *__restrict__ items,
                    const int32_t *__restrict__ n_items_p, const int32_t *__restrict__ sig_pos,
@@ -139,7 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&ctl->full[s], 1);
+            // one arrive (with the weight-tile bytes) from the TMA producer
+            // plus one cp.async-completion arrive from each gather thread
+            mbar_init(&ctl->full[s], 1 + kGatherThreads);
             mbar_init(&ctl->empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -149,7 +154,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_g);
         tma_prefetch_desc(&tm_u);
     }
@@ -163,36 +167,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        uint32_t stage = 0, phase = 0;
-        uint32_t armed[kStages] = {0, 0, 0, 0};
+        // ------------------------------------------------ weight producer
+        // The 256-row slab [W_gate[g]; W_up[g]] of each K stage by TMA.
+        uint32_t stage = 0, phase = 0, issued = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const int g = items[2 * it], ti = items[2 * it + 1];
-            const int base = ti * kBM;
-            const int nrows = min(kBM, count[g] - base);
-            const int32_t *prow = perm + (size_t)g * T + base;
-            const int pad = prow[0];
-            for (int j = lane; j < kBM; j += 32)
-                ctl->idx[j] = j < nrows ? prow[j] : pad;
-            __syncwarp();
-            const int nq = (nrows + 3) >> 2;
+            const int g = items[2 * it];
             for (int kt = 0; kt < KT && ok; ++kt) {
                 if (lane == 0) {
                     if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, status)) {
                         ok = false;
                     } else {
-                        uint8_t *a = smem + stage * kStageBytes;
-                        uint8_t *b = a + kATile;
-                        mbar_arrive_expect_tx(&ctl->full[stage], (uint32_t)nq * 512u + kBTile);
-                        armed[stage]++;
-                        const int x0 = kt * kBK;
-                        for (int q = 0; q < nq; ++q)
-                            umma::tma_gather4(a + q * 512, &tm_x, x0, ctl->idx[4 * q],
-                                              ctl->idx[4 * q + 1], ctl->idx[4 * q + 2],
-                                              ctl->idx[4 * q + 3], &ctl->full[stage]);
-                        tma_load_2d(b, &tm_g, x0, g * kGS, &ctl->full[stage]);
-                        tma_load_2d(b + kBTile / 2, &tm_u, x0, g * kGS, &ctl->full[stage]);
+                        uint8_t *b = smem + stage * kStageBytes + kATile;
+                        mbar_arrive_expect_tx(&ctl->full[stage], kBTile);
+                        tma_load_2d(b, &tm_g, kt * kBK, g * kGS, &ctl->full[stage]);
+                        tma_load_2d(b + kBTile / 2, &tm_u, kt * kBK, g * kGS, &ctl->full[stage]);
+                        ++issued;
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -201,14 +191,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                     phase ^= 1u;
                 }
             }
-            __syncwarp();
         }
         if (!ok && lane == 0) {
-            // let copies still in flight land before the CTA's smem goes away
-            for (int s = 0; s < kStages; ++s)
-                if (armed[s])
-                    mbar_wait(&ctl->full[s], (armed[s] - 1u) & 1u);
+            // let copies still in flight land before the CTA's smem goes away:
+            // stage s was armed for the issued uses s, s + kStages, ...
+            for (uint32_t s = 0; s < kStages && s < issued; ++s) {
+                const uint32_t uses = (issued - s + kStages - 1) / kStages;
+                mbar_wait(&ctl->full[s], (uses - 1u) & 1u);
+            }
         }
+    } else if (warp >= 6) {
+        // ------------------------------------------------ x-row gather
+        // Load-stage skipping: thread p copies tile rows p and p + 64 of
+        // the item -- the tokens perm[g][128 i + row] -- 16 bytes at a time
+        // into the 128-byte-swizzled A tile; rows past the active prefix
+        // are not loaded (their accumulator rows are never stored).  Each
+        // thread's cp.async completions arrive on the stage's barrier.
+        const int p = threadIdx.x - 6 * 32;
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const int g = items[2 * it], ti = items[2 * it + 1];
+            const int base = ti * kBM;
+            const int nrows = min(kBM, count[g] - base);
+            const int32_t *prow = perm + (size_t)g * T + base;
+            const __nv_bfloat16 *src0 = p < nrows ? x + (size_t)prow[p] * H : nullptr;
+            const __nv_bfloat16 *src1 = p + 64 < nrows ? x + (size_t)prow[p + 64] * H : nullptr;
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t a = smem_u32(smem + stage * kStageBytes);
+                const int k0 = kt * kBK;
+                if (src0) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        cp_async16(a + swz128(p, c), src0 + k0 + 8 * c);
+                }
+                if (src1) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        cp_async16(a + swz128(p + 64, c), src1 + k0 + 8 * c);
+                }
+                cp_async_arrive_noinc(&ctl->full[stage]);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        cp_async_wait_all();
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = umma::idesc_bf16_f32(kBM, kBN);
@@ -225,6 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    // the A tile was written by cp.async (generic proxy) and is
+                    // read by the tensor core (async proxy)
+                    fence_proxy_async_smem();
                     umma::fence_after_sync();
                     const uint32_t a = smem_u32(smem + stage * kStageBytes);
                     const uint32_t b = a + kATile;
@@ -254,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(&ctl->drain, 0);
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ------------------------------------------------ epilogue
         const int q = warp & 3;             // TMEM lane quadrant of this warp
         const int j = q * 32 + lane;        // tile row = TMEM lane
@@ -346,8 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto union_word = [&](int s, int w) { return tile_union[(size_t)s * W + w]; };
 
     if (warp == 0) {
-        uint32_t stage = 0, phase = 0;
-        uint32_t armed[kStages] = {0, 0, 0, 0};
+        uint32_t stage = 0, phase = 0, issued = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
             int s, nb;
@@ -364,13 +399,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             } else {
                                 uint8_t *a = smem + stage * kStageBytes;
                                 mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
-                                armed[stage]++;
                                 const int col = g * kGS + half * kBK;
                                 tma_load_2d(a, &tm_h, col, s * kBM, &ctl->full[stage]);
                                 tma_load_2d(a + kATile, &tm_d, col, nb * kBN, &ctl->full[stage]);
                             }
                         }
                         ok = __shfl_sync(0xffffffffu, ok, 0);
+                        issued += ok ? 1u : 0u;
                         if (++stage == kStages) {
                             stage = 0;
                             phase ^= 1u;
@@ -380,9 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (!ok && lane == 0) {
-            for (int s = 0; s < kStages; ++s)
-                if (armed[s])
-                    mbar_wait(&ctl->full[s], (armed[s] - 1u) & 1u);
+            for (uint32_t s = 0; s < kStages && s < issued; ++s) {
+                const uint32_t uses = (issued - s + kStages - 1) / kStages;
+                mbar_wait(&ctl->full[s], (uses - 1u) & 1u);
+            }
         }
     } else if (warp == 1) {
         constexpr uint32_t idesc = umma::idesc_bf16_f32(kBM, kBN);
@@ -517,9 +553,8 @@ int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void
     __nv_bfloat16 *hbuf =
         reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + align_up(wl_bytes, 1024));
 
-    CUtensorMap tx, tg, tu, th, td;
-    if (!make_tmap_2d(&tx, x, T, H, H, 2, 1, kBK, true) ||
-        !make_tmap_2d(&tg, wg, I, H, H, 2, kGS, kBK, true) ||
+    CUtensorMap tg, tu, th, td;
+    if (!make_tmap_2d(&tg, wg, I, H, H, 2, kGS, kBK, true) ||
         !make_tmap_2d(&tu, wu, I, H, H, 2, kGS, kBK, true) ||
         !make_tmap_2d(&th, hbuf, T, I, I, 2, kBM, kBK, true) ||
         !make_tmap_2d(&td, wd, H, I, I, 2, kBN, kBK, true))
@@ -545,8 +580,8 @@ int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void
         const int64_t max_items = G * ((T + kBM - 1) / kBM);
         const int grid = (int)(max_items < sms ? max_items : sms);
         LaunchScope scope(KID_PREFILL_GATEUP, s);
-        prefill_gateup<<<grid, kThreads, kSmemBytes, s>>>(
-            tx, tg, tu, wl.count, wl.perm, wl.items, wl.n_items, wl.sig_pos, hbuf, (int)T, (int)H,
+        prefill_gateup<<<grid, kThreadsGU, kSmemBytes, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), tg, tu, wl.count, wl.perm, wl.items, wl.n_items, wl.sig_pos, hbuf, (int)T, (int)H,
             (int)I, status_ptr());
     }
     if ((rc = launch_status()))
