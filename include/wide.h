@@ -195,6 +195,67 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                     const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
                     void *stream);
 
+/* --------------------------------------------------- masked attention / layer
+ *
+ * Section 2.A, attention half: a token that skips head group j (the
+ * n_q_heads / n_kv_heads query heads sharing KV head j) computes neither
+ * those query heads nor their attention, and their o_proj columns are not
+ * read for it.  K and V are computed for every token and group and written
+ * to the cache.  The pages fix nothing else about the layer; it is the
+ * Llama pre-norm block (RMSNorm, rotate-half RoPE with base rope_theta,
+ * softmax scale 1/sqrt(head_dim), SwiGLU FFN):
+ *     h1  = x + o_proj(attn(RMSNorm(x) * gamma1))        (attn_out = o_proj(...))
+ *     out = h1 + FFN(RMSNorm(h1) * gamma2)               (ffn_out = FFN(...))
+ * with the FFN masked per token as in wide_ffn_masked.
+ *
+ * Token t = s * seq_len + i is token i of sequence s, at position
+ * cache_len + i; its K/V go to the caches at that position.  Caches are
+ * bf16 [n_seq][n_kv_heads][cache_cap][head_dim]; positions < cache_len must
+ * already hold (post-RoPE) keys and values.  Masks: head_mask [T][W] over
+ * n_kv_heads groups; ffn_mask [T][W] over inter / ffn_group_size groups.
+ *
+ * Supported: bf16; head_dim == 128; decode (seq_len == 1, n_seq <= 32,
+ * n_q_heads / n_kv_heads in {1, 2, 4}, hidden % 512 == 0, ffn_group_size in
+ * {64, 128}).
+ */
+typedef struct wide_layer_dims {
+    int64_t n_seq;           /* sequences */
+    int64_t seq_len;         /* new tokens per sequence (1 = decode) */
+    int64_t cache_len;       /* positions already in the cache */
+    int64_t cache_cap;       /* cache capacity per (sequence, KV head) */
+    int64_t hidden;
+    int64_t inter;           /* FFN intermediate size (ignored by wide_attn_masked) */
+    int64_t ffn_group_size;
+    int32_t n_q_heads, n_kv_heads, head_dim;
+    float rope_theta;
+    float eps;               /* RMSNorm epsilon */
+} wide_layer_dims;
+
+typedef struct wide_layer_weights {
+    const void *gamma1, *wq, *wk, *wv, *wo;       /* attention half (device) */
+    const void *gamma2, *w_gate, *w_up, *w_down;  /* FFN half (device) */
+} wide_layer_weights;
+
+/* Device workspace bytes for wide_layer_masked / wide_attn_masked (0 on
+ * invalid or unsupported dims). */
+size_t wide_layer_workspace_bytes(const wide_layer_dims *d);
+
+/* The masked layer.  out [T][hidden] (required); attn_out and ffn_out
+ * [T][hidden] are optional (NULL = not written).  Appends K/V to the caches.
+ * Workspace: >= wide_layer_workspace_bytes(d), 256-byte aligned. */
+int wide_layer_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cache,
+                      void *d_v_cache, const uint32_t *d_head_mask, const uint32_t *d_ffn_mask,
+                      void *d_out, void *d_attn_out, void *d_ffn_out, const wide_layer_dims *d,
+                      void *d_workspace, size_t workspace_bytes, void *stream);
+
+/* The attention half only: attn_out = o_proj(attn(RMSNorm(x) * gamma1)) with
+ * the head-group mask; appends K/V to the caches.  w->gamma2 and the FFN
+ * weights are ignored. */
+int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cache,
+                     void *d_v_cache, const uint32_t *d_head_mask, void *d_attn_out,
+                     const wide_layer_dims *d, void *d_workspace, size_t workspace_bytes,
+                     void *stream);
+
 /* ------------------------------------------- FFN without device allocation
  *
  * The paper has no counterpart to this entry point; it exists for callers

@@ -23,7 +23,7 @@ from ._native import (  # noqa: F401
     WIDE_NOALLOC_SCRATCH_BYTES,
     WIDE_DEV_BAD_MASK, WIDE_DEV_TIMEOUT, WIDE_DEV_BAD_ITEM,
     WIDE_BF16, WIDE_F32, WIDE_PATH_AUTO, WIDE_PATH_DECODE, WIDE_PATH_PREFILL,
-    WideWorklist, WideFFNDims,
+    WideWorklist, WideFFNDims, WideLayerDims, WideLayerWeights,
 )
 
 _L = _native.lib()
@@ -205,3 +205,70 @@ def wide_ffn_masked_noalloc(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.T
         _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"), _dev_ptr(out, "out"),
         ctypes.byref(d), _stream(stream, x.device)))
     return out
+
+
+# ----------------------------------------------------------- masked layer
+
+LAYER_WEIGHT_NAMES = ("gamma1", "wq", "wk", "wv", "wo", "gamma2", "w_gate", "w_up", "w_down")
+
+
+def wide_layer_dims(n_seq: int, seq_len: int, cache_len: int, cache_cap: int, hidden: int,
+                    inter: int, ffn_group_size: int, n_q_heads: int, n_kv_heads: int,
+                    head_dim: int = 128, rope_theta: float = 5e5,
+                    eps: float = 1e-5) -> WideLayerDims:
+    return WideLayerDims(n_seq, seq_len, cache_len, cache_cap, hidden, inter, ffn_group_size,
+                         n_q_heads, n_kv_heads, head_dim, rope_theta, eps)
+
+
+def _weights(w: dict, names=LAYER_WEIGHT_NAMES) -> WideLayerWeights:
+    vals = {}
+    for n in LAYER_WEIGHT_NAMES:
+        t = w.get(n)
+        vals[n] = _dev_ptr(t, n) if (t is not None and n in names) else None
+    return WideLayerWeights(**vals)
+
+
+def wide_layer_workspace_bytes(d: WideLayerDims) -> int:
+    return int(_L.wide_layer_workspace_bytes(ctypes.byref(d)))
+
+
+def wide_layer_masked(x: torch.Tensor, weights: dict, k_cache: torch.Tensor,
+                      v_cache: torch.Tensor, head_mask: torch.Tensor, ffn_mask: torch.Tensor,
+                      d: WideLayerDims, out: torch.Tensor = None, attn_out: torch.Tensor = None,
+                      ffn_out: torch.Tensor = None, workspace: torch.Tensor = None,
+                      stream=None) -> torch.Tensor:
+    """The masked layer (pre-norm block); appends K/V to the caches.
+    weights: dict with gamma1, wq, wk, wv, wo, gamma2, w_gate, w_up, w_down."""
+    if out is None:
+        out = torch.empty_like(x)
+    need = wide_layer_workspace_bytes(d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    w = _weights(weights)
+    _check("wide_layer_masked", _L.wide_layer_masked(
+        _dev_ptr(x, "x"), ctypes.byref(w), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(head_mask, "head_mask"),
+        _dev_ptr(ffn_mask, "ffn_mask"), _dev_ptr(out, "out"),
+        None if attn_out is None else _dev_ptr(attn_out, "attn_out"),
+        None if ffn_out is None else _dev_ptr(ffn_out, "ffn_out"),
+        ctypes.byref(d), workspace.data_ptr(), workspace.numel(), _stream(stream, x.device)))
+    return out
+
+
+def wide_attn_masked(x: torch.Tensor, weights: dict, k_cache: torch.Tensor,
+                     v_cache: torch.Tensor, head_mask: torch.Tensor, d: WideLayerDims,
+                     attn_out: torch.Tensor = None, workspace: torch.Tensor = None,
+                     stream=None) -> torch.Tensor:
+    """The masked attention half: attn_out = o_proj(attn(RMSNorm(x) * gamma1))."""
+    if attn_out is None:
+        attn_out = torch.empty_like(x)
+    need = wide_layer_workspace_bytes(d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    w = _weights(weights, names=("gamma1", "wq", "wk", "wv", "wo"))
+    _check("wide_attn_masked", _L.wide_attn_masked(
+        _dev_ptr(x, "x"), ctypes.byref(w), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(head_mask, "head_mask"),
+        _dev_ptr(attn_out, "attn_out"), ctypes.byref(d), workspace.data_ptr(), workspace.numel(),
+        _stream(stream, x.device)))
+    return attn_out

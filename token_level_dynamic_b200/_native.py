@@ -44,6 +44,18 @@ class WideFFNDims(ctypes.Structure):
                 ("group_size", c_int64), ("dtype", c_int32), ("path", c_int32)]
 
 
+class WideLayerDims(ctypes.Structure):
+    _fields_ = [("n_seq", c_int64), ("seq_len", c_int64), ("cache_len", c_int64),
+                ("cache_cap", c_int64), ("hidden", c_int64), ("inter", c_int64),
+                ("ffn_group_size", c_int64), ("n_q_heads", c_int32), ("n_kv_heads", c_int32),
+                ("head_dim", c_int32), ("rope_theta", ctypes.c_float), ("eps", ctypes.c_float)]
+
+
+class WideLayerWeights(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("gamma1", "wq", "wk", "wv", "wo",
+                                        "gamma2", "w_gate", "w_up", "w_down")]
+
+
 # name -> (restype, argtypes); every symbol include/wide.h declares
 SIGNATURES = {
     "wide_status_string": (ctypes.c_char_p, [c_int]),
@@ -65,6 +77,13 @@ SIGNATURES = {
                                 ctypes.POINTER(WideFFNDims), c_void_p, c_size_t, c_void_p]),
     "wide_ffn_masked_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, ctypes.POINTER(WideFFNDims), c_void_p]),
+    "wide_layer_workspace_bytes": (c_size_t, [ctypes.POINTER(WideLayerDims)]),
+    "wide_layer_masked": (c_int, [c_void_p, ctypes.POINTER(WideLayerWeights), c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  ctypes.POINTER(WideLayerDims), c_void_p, c_size_t, c_void_p]),
+    "wide_attn_masked": (c_int, [c_void_p, ctypes.POINTER(WideLayerWeights), c_void_p, c_void_p,
+                                 c_void_p, c_void_p, ctypes.POINTER(WideLayerDims), c_void_p,
+                                 c_size_t, c_void_p]),
 }
 
 _lib = None

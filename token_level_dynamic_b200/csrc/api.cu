@@ -310,4 +310,91 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                               d_workspace, s);
 }
 
+static bool layer_dims_ok(const wide_layer_dims *d, bool ffn)
+{
+    if (!d || d->n_seq < 1 || d->seq_len < 1 || d->cache_len < 0 || d->hidden <= 0 ||
+        d->n_q_heads <= 0 || d->n_kv_heads <= 0 || d->head_dim <= 0 ||
+        d->n_q_heads % d->n_kv_heads != 0 || d->cache_cap < d->cache_len + d->seq_len ||
+        !(d->eps >= 0.f) || !(d->rope_theta > 0.f))
+        return false;
+    if (ffn && (d->inter <= 0 || d->ffn_group_size <= 0 || d->inter % d->ffn_group_size != 0 ||
+                d->inter / d->ffn_group_size > 1024))
+        return false;
+    return true;
+}
+
+static wide_layer_dims attn_only_dims(const wide_layer_dims *d)
+{
+    wide_layer_dims a = *d;
+    a.inter = 128;
+    a.ffn_group_size = 128;
+    return a;
+}
+
+size_t wide_layer_workspace_bytes(const wide_layer_dims *d)
+{
+    if (!layer_dims_ok(d, true))
+        return 0;
+    if (layer_decode_supported(d))
+        return layer_decode_workspace(d);
+    return 0;
+}
+
+static int layer_call(const LayerPtrs &p, const wide_layer_dims *d, void *ws, size_t ws_bytes,
+                      void *stream)
+{
+    if (!layer_decode_supported(d))
+        return WIDE_EUNSUPPORTED;
+    const void *ptrs[] = {p.x, p.gamma1, p.wq, p.wk, p.wv, p.wo, p.k_cache, p.v_cache};
+    for (const void *q : ptrs)
+        if (!q)
+            return WIDE_EINVAL;
+    if (!p.head_mask || !ws)
+        return WIDE_EINVAL;
+    if (p.ffn && (!p.gamma2 || !p.w_gate || !p.w_up || !p.w_down || !p.ffn_mask || !p.out))
+        return WIDE_EINVAL;
+    if (!p.ffn && !p.attn_out)
+        return WIDE_EINVAL;
+    const void *al[] = {p.x, p.gamma1, p.wq, p.wk, p.wv, p.wo, p.k_cache, p.v_cache};
+    for (const void *q : al)
+        if (!aligned16(q))
+            return WIDE_EUNSUPPORTED;
+    if ((p.out && !aligned16(p.out)) || (p.attn_out && !aligned16(p.attn_out)) ||
+        (p.ffn_out && !aligned16(p.ffn_out)) ||
+        (p.ffn && (!aligned16(p.gamma2) || !aligned16(p.w_gate) || !aligned16(p.w_up) ||
+                   !aligned16(p.w_down))) ||
+        (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return WIDE_EUNSUPPORTED;
+    if (ws_bytes < layer_decode_workspace(d))
+        return WIDE_EWORKSPACE;
+    return layer_decode_launch(p, d, ws, static_cast<cudaStream_t>(stream));
+}
+
+int wide_layer_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cache,
+                      void *d_v_cache, const uint32_t *d_head_mask, const uint32_t *d_ffn_mask,
+                      void *d_out, void *d_attn_out, void *d_ffn_out, const wide_layer_dims *d,
+                      void *d_workspace, size_t workspace_bytes, void *stream)
+{
+    if (!w || !layer_dims_ok(d, true))
+        return WIDE_EINVAL;
+    LayerPtrs p = {d_x, w->gamma1, w->wq, w->wk, w->wv, w->wo, w->gamma2, w->w_gate, w->w_up,
+                   w->w_down, d_k_cache, d_v_cache, d_head_mask, d_ffn_mask, d_out, d_attn_out,
+                   d_ffn_out, true};
+    return layer_call(p, d, d_workspace, workspace_bytes, stream);
+}
+
+int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cache,
+                     void *d_v_cache, const uint32_t *d_head_mask, void *d_attn_out,
+                     const wide_layer_dims *d, void *d_workspace, size_t workspace_bytes,
+                     void *stream)
+{
+    if (!w || !layer_dims_ok(d, false))
+        return WIDE_EINVAL;
+    const wide_layer_dims a = attn_only_dims(d);
+    LayerPtrs p = {d_x, w->gamma1, w->wq, w->wk, w->wv, w->wo, nullptr, nullptr, nullptr,
+                   nullptr, d_k_cache, d_v_cache, d_head_mask, nullptr, nullptr, d_attn_out,
+                   nullptr, false};
+    return layer_call(p, &a, d_workspace, workspace_bytes, stream);
+}
+
 }  // extern "C"

@@ -232,7 +232,7 @@ template <typename TIn, int GS>
 __global__ void __launch_bounds__(kDownRows)
     ffn_decode_down(const __grid_constant__ CUtensorMap tm_down,
                     const __grid_constant__ CUtensorMap tm_h, const uint32_t *__restrict__ mask,
-                    TIn *__restrict__ out, int T, int H, int I, int W, int G, int32_t *status)
+                    const DownOutputs o, int T, int H, int I, int W, int G, int32_t *status)
 {
     constexpr int EPC = ElemTraits<TIn>::EPC;
     constexpr int KT = 8 * EPC;
@@ -361,7 +361,20 @@ __global__ void __launch_bounds__(kDownRows)
         float sum = 0.f;
         for (int q = 0; q < KS; ++q)
             sum += cluster.map_shared_rank(part, q)[t * kDownRows + n];
-        out[(size_t)t * H + (size_t)nb * kDownRows + n] = from_f32<TIn>(sum);
+        const size_t at = (size_t)t * H + (size_t)nb * kDownRows + n;
+        if (o.out_sum)
+            static_cast<TIn *>(o.out_sum)[at] = from_f32<TIn>(sum);
+        if (o.out_total || o.out_total_f32) {
+            float tot = sum;
+            if (o.res_in)
+                tot += to_f32(static_cast<const TIn *>(o.res_in)[at]);
+            if (o.res_f32)
+                tot += o.res_f32[at];
+            if (o.out_total)
+                static_cast<TIn *>(o.out_total)[at] = from_f32<TIn>(tot);
+            if (o.out_total_f32)
+                o.out_total_f32[at] = tot;
+        }
     }
     cluster.sync();
 }
@@ -391,8 +404,8 @@ int launch_cluster(int32_t kid, void (*kernel)(KArgs...), dim3 grid, dim3 block,
 }
 
 template <typename TIn, int GS>
-int decode_chunk(const TIn *x, const TIn *wg, const TIn *wu, const TIn *wd, const uint32_t *mask,
-                 TIn *out, int T, int H, int I, float *h, cudaStream_t s)
+int gateup_chunk(const TIn *x, const TIn *wg, const TIn *wu, const uint32_t *mask, float *h, int T,
+                 int H, int I, cudaStream_t s)
 {
     constexpr int EPC = ElemTraits<TIn>::EPC;
     constexpr int KT = 8 * EPC;
@@ -401,26 +414,45 @@ int decode_chunk(const TIn *x, const TIn *wg, const TIn *wu, const TIn *wd, cons
     while (KS > 1 && (H % (KS * KT)) != 0)
         KS >>= 1;
     const int kslice = H / KS;
-
-    CUtensorMap tg, tu, td, th;
+    CUtensorMap tg, tu;
     if (!make_tmap_2d(&tg, wg, I, H, H, sizeof(TIn), GS, KT, true) ||
-        !make_tmap_2d(&tu, wu, I, H, H, sizeof(TIn), GS, KT, true) ||
-        !make_tmap_2d(&td, wd, H, I, I, sizeof(TIn), kDownRows, KT, true) ||
+        !make_tmap_2d(&tu, wu, I, H, H, sizeof(TIn), GS, KT, true))
+        return WIDE_ECUDA;
+    const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 256 + (size_t)T * kslice * 4;
+    return launch_cluster(KID_DECODE_GATEUP, ffn_decode_gateup<TIn, GS>, dim3(KS, G), dim3(GS),
+                          smem1, KS, s, tg, tu, x, mask, h, T, H, I, W, kslice, status_ptr());
+}
+
+template <typename TIn, int GS>
+int down_chunk(const TIn *wd, const float *h, const uint32_t *mask, const DownOutputs &o, int T,
+               int H, int I, cudaStream_t s)
+{
+    constexpr int EPC = ElemTraits<TIn>::EPC;
+    constexpr int KT = 8 * EPC;
+    const int G = I / GS, W = (G + 31) / 32;
+    CUtensorMap td, th;
+    if (!make_tmap_2d(&td, wd, H, I, I, sizeof(TIn), kDownRows, KT, true) ||
         !make_tmap_2d(&th, h, T, I, I, 4, T, KT, false))
         return WIDE_ECUDA;
-
-    const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 256 + (size_t)T * kslice * 4;
-    int rc = launch_cluster(KID_DECODE_GATEUP, ffn_decode_gateup<TIn, GS>, dim3(KS, G), dim3(GS), smem1, KS, s, tg,
-                            tu, x, mask, h, T, H, I, W, kslice, status_ptr());
-    if (rc)
-        return rc;
-
     const int KSd = G < 8 ? G : 8;
     const size_t hb = (size_t)T * KT * 4;
     const size_t stage = (size_t)kDownRows * 128 + ((hb + 1023) & ~(size_t)1023);
     const size_t smem2 = 1024 + kStages * stage + 64 + 1024 * 4 + 1024 * 4;
-    return launch_cluster(KID_DECODE_DOWN, ffn_decode_down<TIn, GS>, dim3(KSd, H / kDownRows), dim3(kDownRows),
-                          smem2, KSd, s, td, th, mask, out, T, H, I, W, G, status_ptr());
+    return launch_cluster(KID_DECODE_DOWN, ffn_decode_down<TIn, GS>, dim3(KSd, H / kDownRows),
+                          dim3(kDownRows), smem2, KSd, s, td, th, mask, o, T, H, I, W, G,
+                          status_ptr());
+}
+
+template <typename TIn, int GS>
+int decode_chunk(const TIn *x, const TIn *wg, const TIn *wu, const TIn *wd, const uint32_t *mask,
+                 TIn *out, int T, int H, int I, float *h, cudaStream_t s)
+{
+    int rc = gateup_chunk<TIn, GS>(x, wg, wu, mask, h, T, H, I, s);
+    if (rc)
+        return rc;
+    DownOutputs o = {};
+    o.out_sum = out;
+    return down_chunk<TIn, GS>(wd, h, mask, o, T, H, I, s);
 }
 
 template <typename TIn, int GS>
@@ -443,6 +475,38 @@ int decode_all(const void *x, const void *wg, const void *wu, const void *wd,
 }
 
 }  // namespace
+
+int decode_gateup_bf16(const void *x, const void *wg, const void *wu, const uint32_t *mask,
+                       float *h, int T, int H, int I, int gs, cudaStream_t s)
+{
+    if (T <= 0 || T > kNTok)
+        return WIDE_EINVAL;
+    const auto *xb = static_cast<const __nv_bfloat16 *>(x);
+    const auto *gb = static_cast<const __nv_bfloat16 *>(wg);
+    const auto *ub = static_cast<const __nv_bfloat16 *>(wu);
+    if (gs == 128)
+        return gateup_chunk<__nv_bfloat16, 128>(xb, gb, ub, mask, h, T, H, I, s);
+    if (gs == 64)
+        return gateup_chunk<__nv_bfloat16, 64>(xb, gb, ub, mask, h, T, H, I, s);
+    return WIDE_EUNSUPPORTED;
+}
+
+int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const DownOutputs &o,
+                     int T, int H, int I, int gs, cudaStream_t s)
+{
+    if (T <= 0 || T > kNTok)
+        return WIDE_EINVAL;
+    const auto *db = static_cast<const __nv_bfloat16 *>(wd);
+    if (gs == 128)
+        return down_chunk<__nv_bfloat16, 128>(db, h, mask, o, T, H, I, s);
+    if (gs == 64)
+        return down_chunk<__nv_bfloat16, 64>(db, h, mask, o, T, H, I, s);
+    if (gs == 256)
+        return down_chunk<__nv_bfloat16, 256>(db, h, mask, o, T, H, I, s);
+    if (gs == 512)
+        return down_chunk<__nv_bfloat16, 512>(db, h, mask, o, T, H, I, s);
+    return WIDE_EUNSUPPORTED;
+}
 
 size_t ffn_decode_workspace(const wide_ffn_dims *d)
 {

@@ -45,6 +45,18 @@ enum KernelId : int32_t {
     KID_PREFILL_ZERO = 5,
     KID_PREFILL_GATEUP = 6,
     KID_PREFILL_DOWN = 7,
+    KID_DECODE_QKV = 8,
+    KID_DECODE_ATTN = 9,
+    KID_RMSNORM = 10,
+};
+
+// Pointers of one masked-layer call (FFN pointers unused when !ffn).
+struct LayerPtrs {
+    const void *x, *gamma1, *wq, *wk, *wv, *wo, *gamma2, *w_gate, *w_up, *w_down;
+    void *k_cache, *v_cache;
+    const uint32_t *head_mask, *ffn_mask;
+    void *out, *attn_out, *ffn_out;
+    bool ffn;
 };
 
 // Brackets one kernel launch: counts it and, while profiling is on, records
@@ -64,6 +76,18 @@ bool ffn_dims_ok(const wide_ffn_dims *d);
 int ffn_path(const wide_ffn_dims *d);
 bool ffn_shape_supported(const wide_ffn_dims *d, int path);
 
+// Outputs of the decode down-projection GEMV (each pointer may be null):
+// out_sum = the projection; out_total (element type of the weights) and
+// out_total_f32 = the projection plus the residuals res_in (element type of
+// the weights) and res_f32.  All [T][H] row-major.
+struct DownOutputs {
+    void *out_sum;
+    const void *res_in;
+    const float *res_f32;
+    void *out_total;
+    float *out_total_f32;
+};
+
 // Internal entry points of the kernel files.
 int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
                    const wide_worklist *wl, cudaStream_t s);
@@ -74,7 +98,17 @@ int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void
                        const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                        cudaStream_t s);
 
+bool layer_decode_supported(const wide_layer_dims *d);
+size_t layer_decode_workspace(const wide_layer_dims *d);
+int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, cudaStream_t s);
+
 size_t ffn_decode_workspace(const wide_ffn_dims *d);
+// bf16 decode GEMVs for T <= 32 tokens (one chunk): gate/up writes fp32 h for
+// kept (token, group) pairs; down reads h of kept pairs (group size gs).
+int decode_gateup_bf16(const void *x, const void *wg, const void *wu, const uint32_t *mask,
+                       float *h, int T, int H, int I, int gs, cudaStream_t s);
+int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const DownOutputs &o,
+                     int T, int H, int I, int gs, cudaStream_t s);
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s);

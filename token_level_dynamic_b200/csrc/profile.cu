@@ -109,6 +109,12 @@ const char *wide_kernel_name(int32_t id)
         return "prefill_gateup_tcgen05";
     case KID_PREFILL_DOWN:
         return "prefill_down_tcgen05";
+    case KID_DECODE_QKV:
+        return "decode_qkv_rope_gemv";
+    case KID_DECODE_ATTN:
+        return "decode_attention";
+    case KID_RMSNORM:
+        return "rmsnorm";
     default:
         return "?";
     }
