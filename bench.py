@@ -2,7 +2,7 @@
 """Benchmark of the masked WIDE layer on B200; prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_ffn_3b|prefill_ffn_8b]
+                    [--workload decode_ffn_3b|prefill_ffn_8b|decode_layer_8b]
 
 Workloads (seeded synthetic inputs with the shapes the pages name):
   decode_ffn_3b (default)  Llama-3.2-3B-shaped masked SwiGLU FFN in decode:
@@ -10,6 +10,10 @@ Workloads (seeded synthetic inputs with the shapes the pages name):
       masks.  One step = the three batch sizes of the configuration (1, 8
       and 32 tokens, each with its own x and mask): 41 tokens.  HBM-bound;
       the roofline is union-of-groups weight bytes over measured HBM GB/s.
+  decode_layer_8b  Llama-3.1-8B-shaped masked decode layer, batch 16 with a
+      2048-entry KV cache: attention (QKV+RoPE, GQA over the cache, o_proj)
+      with head groups kept at 0.34 and the FFN with groups kept at 0.72.
+      HBM-bound; the roofline is union weight bytes + kept KV bytes.
   prefill_ffn_8b  Llama-3.1-8B-shaped masked SwiGLU FFN in prefill: 4096
       tokens, hidden 4096, intermediate 14336 in 112 groups of 128, 8
       prototype masks (56 groups each) with 0.1 bit flips.  One step = one
@@ -147,6 +151,63 @@ def _traffic_record(kernel: str, workload: str):
 
 
 # --------------------------------------------------------------- workloads
+# A workload builds its seeded cases, states the algorithmic units of every
+# library kernel it launches, runs the oracle on a bounded sample, and sets
+# up device buffers with the calls that the timing loop makes.
+
+class FFNDevice:
+    """Device buffers and calls of a masked-FFN workload (one call per case)."""
+
+    def __init__(self, wl, cases, dev, stream):
+        import torch
+        import token_level_dynamic_b200 as w
+        from synth.torch_io import to_dev
+        self.w, self.stream, self.cases = w, stream, cases
+        base = cases[0]
+        self.Wg = to_dev(base.w_gate, "bf16", dev)
+        self.Wu = to_dev(base.w_up, "bf16", dev)
+        self.Wd = to_dev(base.w_down, "bf16", dev)
+        self.xs = [to_dev(c.x, "bf16", dev) for c in cases]
+        self.ms = [to_dev(c.mask_words, "mask", dev) for c in cases]
+        self.outs = [torch.empty_like(x) for x in self.xs]
+        self.path = getattr(w, wl.path_name)
+        ws_bytes = max(w.wide_ffn_workspace_bytes(c.T, c.H, c.I, c.gs, path=self.path)
+                       for c in cases)
+        self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        self.ones = [_all_ones(m, base.I // base.gs) for m in self.ms]
+        self.ncalls = len(cases)
+        # e2e: pinned host copies of each call's inputs and output
+        self.xh = [x.cpu().pin_memory() for x in self.xs]
+        self.mh = [m.cpu().pin_memory() for m in self.ms]
+        self.oh = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
+        self.h2d_bytes = int(sum(x.numel() * 2 + m.numel() * 4 for x, m in zip(self.xh, self.mh)))
+        self.d2h_bytes = int(sum(o.numel() * 2 for o in self.oh))
+
+    def call(self, i, all_kept=False):
+        self.w.wide_ffn_masked(self.xs[i], self.Wg, self.Wu, self.Wd,
+                               self.ones[i] if all_kept else self.ms[i], self.cases[i].gs,
+                               out=self.outs[i], workspace=self.ws, path=self.path,
+                               stream=self.stream)
+
+    def e2e_call(self, i):
+        self.xs[i].copy_(self.xh[i], non_blocking=True)
+        self.ms[i].copy_(self.mh[i], non_blocking=True)
+        self.call(i)
+        self.oh[i].copy_(self.outs[i], non_blocking=True)
+
+    def dense_torch(self, i):
+        import torch.nn.functional as F
+        x = self.xs[i]
+        self.outs[i].copy_(F.linear(F.silu(F.linear(x, self.Wg)) * F.linear(x, self.Wu), self.Wd))
+
+
+def _all_ones(m, G):
+    import torch
+    o = torch.full_like(m, -1)
+    if G % 32:
+        o[:, -1] = (1 << (G % 32)) - 1
+    return o
+
 
 class DecodeFFN3B:
     name = "decode_ffn_3b"
@@ -156,6 +217,7 @@ class DecodeFFN3B:
     bound = "hbm"
     dominant = "decode_gateup_gemv"
     path_name = "WIDE_PATH_DECODE"
+    device = FFNDevice
 
     def make_cases(self):
         import synth
@@ -171,15 +233,7 @@ class DecodeFFN3B:
     def units(case):
         """Algorithmic bytes per call, per kernel: every weight byte of the
         batch's union of groups once, plus x, mask, fp32 h and out."""
-        B, H, I, gs = case.T, case.H, case.I, case.gs
-        U = int(case.mask.any(axis=0).sum())
-        pairs = int(case.mask.sum())
-        m = case.mask_words.nbytes
-        h = pairs * gs * 4
-        gateup = 2 * U * gs * H * 2 + B * H * 2 + m + h
-        down = H * U * gs * 2 + h + m + B * H * 2
-        return {"decode_gateup_gemv": gateup, "decode_down_gemv": down,
-                "total": gateup + down, "union_groups": U}
+        return _ffn_decode_bytes(case)
 
     def reference_sample(self, cases):
         out = []
@@ -188,6 +242,27 @@ class DecodeFFN3B:
             s.x, s.mask, s.T = c.x[:1], c.mask[:1], 1
             out.append(s)
         return out, "per step: token 0 of each of batches 1, 8, 32 (3 tokens)"
+
+    reference_step = staticmethod(lambda samples: _ffn_oracle_step(samples))
+
+
+def _ffn_decode_bytes(case, prefix=""):
+    B, H, I, gs = case.T, case.H, case.I, case.gs
+    U = int(case.mask.any(axis=0).sum())
+    pairs = int(case.mask.sum())
+    m = case.mask_words.nbytes
+    h = pairs * gs * 4
+    gateup = 2 * U * gs * H * 2 + B * H * 2 + m + h
+    down = H * U * gs * 2 + h + m + B * H * 2
+    return {"decode_gateup_gemv": gateup, "decode_down_gemv": down,
+            "total": gateup + down, "union_groups": U}
+
+
+def _ffn_oracle_step(samples):
+    import oracle
+    for c in samples:
+        oracle.ffn.ffn_token_loop(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs, "bf16")
+    return sum(c.T for c in samples)
 
 
 class PrefillFFN8B:
@@ -198,6 +273,7 @@ class PrefillFFN8B:
     bound = "tensor"
     dominant = "prefill_gateup_tcgen05"
     path_name = "WIDE_PATH_PREFILL"
+    device = FFNDevice
 
     def make_cases(self):
         import synth
@@ -221,48 +297,173 @@ class PrefillFFN8B:
         s.x, s.mask, s.T = c.x[:8], c.mask[:8], 8
         return [s], "per step: the first 8 tokens of the 4096-token batch"
 
+    reference_step = staticmethod(lambda samples: _ffn_oracle_step(samples))
 
-WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B())}
+
+class LayerDevice:
+    """Device buffers and calls of a masked-layer workload (one call)."""
+
+    def __init__(self, wl, cases, dev, stream):
+        import torch
+        import token_level_dynamic_b200 as w
+        from synth.torch_io import layer_to_dev
+        self.w, self.stream = w, stream
+        lc = cases[0]
+        self.lc = lc
+        self.x, self.wts, self.kc, self.vc, self.hm, self.fm, cap = layer_to_dev(lc, device=dev)
+        a, f = lc.attn, lc.ffn
+        self.d = w.wide_layer_dims(a.n_seq, a.seq_len, a.cache_len, cap, a.H, f.I, f.gs, a.n_q,
+                                   a.n_kv, a.hd, a.theta, a.eps)
+        self.out = torch.empty_like(self.x)
+        self.ws = torch.empty(max(256, w.wide_layer_workspace_bytes(self.d)), dtype=torch.uint8,
+                              device=dev)
+        self.hm1 = _all_ones(self.hm, lc.attn.n_kv)
+        self.fm1 = _all_ones(self.fm, lc.ffn.I // lc.ffn.gs)
+        self.ncalls = 1
+        self.xh = self.x.cpu().pin_memory()
+        self.hmh = self.hm.cpu().pin_memory()
+        self.fmh = self.fm.cpu().pin_memory()
+        self.oh = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.h2d_bytes = int(self.x.numel() * 2 + self.hm.numel() * 4 + self.fm.numel() * 4)
+        self.d2h_bytes = int(self.out.numel() * 2)
+
+    def call(self, i, all_kept=False):
+        self.w.wide_layer_masked(self.x, self.wts, self.kc, self.vc,
+                                 self.hm1 if all_kept else self.hm,
+                                 self.fm1 if all_kept else self.fm, self.d, out=self.out,
+                                 workspace=self.ws, stream=self.stream)
+
+    def e2e_call(self, i):
+        self.x.copy_(self.xh, non_blocking=True)
+        self.hm.copy_(self.hmh, non_blocking=True)
+        self.fm.copy_(self.fmh, non_blocking=True)
+        self.call(i)
+        self.oh.copy_(self.out, non_blocking=True)
+
+    def dense_torch(self, i):
+        """The same layer unmasked with torch/cuBLAS ops (bf16)."""
+        import torch
+        import torch.nn.functional as F
+        a = self.lc.attn
+        W = self.wts
+        x = self.x
+        B, H, nq, nkv, hd = a.n_seq, a.H, a.n_q, a.n_kv, a.hd
+        L = a.cache_len
+        xf = x.float()
+        xn = (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + a.eps)).to(x.dtype) * W["gamma1"]
+        q = F.linear(xn, W["wq"]).view(B, nq, 1, hd)
+        k = F.linear(xn, W["wk"]).view(B, nkv, 1, hd)
+        v = F.linear(xn, W["wv"]).view(B, nkv, 1, hd)
+        pos = torch.full((1,), float(L), device=x.device)
+        inv = a.theta ** (-torch.arange(0, hd, 2, device=x.device, dtype=torch.float32) / hd)
+        ang = pos[:, None] * inv[None, :]
+        cos, sin = torch.cos(ang).to(x.dtype), torch.sin(ang).to(x.dtype)
+        def rope(t):
+            t1, t2 = t[..., :hd // 2], t[..., hd // 2:]
+            return torch.cat([t1 * cos - t2 * sin, t2 * cos + t1 * sin], -1)
+        q, k = rope(q), rope(k)
+        self.kc[:, :, L:L + 1] = k
+        self.vc[:, :, L:L + 1] = v
+        o = F.scaled_dot_product_attention(q, self.kc[:, :, :L + 1], self.vc[:, :, :L + 1],
+                                           enable_gqa=True)
+        h1 = x + F.linear(o.reshape(B, nq * hd), W["wo"])
+        hf = h1.float()
+        xn2 = (hf * torch.rsqrt(hf.pow(2).mean(-1, keepdim=True) + a.eps)).to(x.dtype) * W["gamma2"]
+        f = F.linear(F.silu(F.linear(xn2, W["w_gate"])) * F.linear(xn2, W["w_up"]), W["w_down"])
+        self.out.copy_(h1 + f)
+
+
+class DecodeLayer8B:
+    name = "decode_layer_8b"
+    desc = ("decode_layer_8b: Llama-3.1-8B-shaped masked decode layer (RMSNorm, QKV with 32 "
+            "query / 8 KV heads of 128, RoPE theta 5e5, GQA attention over a 2048-entry KV "
+            "cache, o_proj, RMSNorm, SwiGLU FFN 14336 = 112 groups x 128), batch 16, head "
+            "groups Bernoulli(0.34), FFN groups Bernoulli(0.72); one step = one call")
+    bound = "hbm"
+    dominant = "decode_gateup_gemv"
+    device = LayerDevice
+
+    def make_cases(self):
+        import synth
+        return [synth.decode_layer()]
+
+    @staticmethod
+    def units(lc):
+        """Algorithmic bytes per call, per kernel: union-of-groups weight
+        bytes (each byte once per call), dense Wk/Wv, the kept K/V cache
+        bytes, and the activations each kernel must read or write."""
+        a, f = lc.attn, lc.ffn
+        T, H, hd, nq, nkv = a.T, a.H, a.hd, a.n_q, a.n_kv
+        rep = nq // nkv
+        Ua = int(a.mask.any(axis=0).sum())
+        kept_pairs = int(a.mask.sum())
+        keys = a.cache_len + 1
+        qkv = (Ua * rep * hd * H * 2 + 2 * nkv * hd * H * 2 + T * H * 2 + H * 2
+               + kept_pairs * rep * hd * 4 + 2 * T * nkv * hd * 2)
+        attn = kept_pairs * 2 * keys * hd * 2 + kept_pairs * rep * hd * 4 * 2
+        oproj = H * Ua * rep * hd * 2 + kept_pairs * rep * hd * 4 + T * H * 2 * 2 + T * H * 4
+        ffn = _ffn_decode_bytes(f)
+        down = oproj + ffn["decode_down_gemv"]
+        norm = T * H * 4 + T * H * 2
+        total = qkv + attn + down + ffn["decode_gateup_gemv"] + norm
+        return {"decode_qkv_rope_gemv": qkv, "decode_attention": attn, "decode_down_gemv": down,
+                "decode_gateup_gemv": ffn["decode_gateup_gemv"], "rmsnorm": norm,
+                "total": total, "union_groups": ffn["union_groups"]}
+
+    def reference_sample(self, cases):
+        import copy
+        lc = copy.deepcopy(cases[0])
+        a = lc.attn
+        keep = 2
+        a.n_seq, a.x, a.mask = keep, a.x[:keep], a.mask[:keep]
+        a.k_cache, a.v_cache = a.k_cache[:keep], a.v_cache[:keep]
+        lc.ffn.mask, lc.ffn.T, lc.ffn.x = lc.ffn.mask[:keep], keep, lc.ffn.x[:keep]
+        return [lc], "per step: sequences 0 and 1 of the 16 (2 tokens), fp64 definition form"
+
+    @staticmethod
+    def reference_step(samples):
+        import oracle
+        for lc in samples:
+            oracle.attention.layer_masked(lc)
+        return sum(lc.attn.T for lc in samples)
+
+
+WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B(), DecodeLayer8B())}
 
 
 # ------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_baseline(samples, seconds: float):
-    """Times the oracle's per-token loop (fp64, OpenMP over tokens) on the
-    host cores, repeating the sample until `seconds` have passed."""
-    import oracle
+def cpu_oracle_baseline(wl, samples, seconds: float):
+    """Times the oracle on the host cores, repeating the sample until
+    `seconds` have passed."""
     from oracle import _clib
     tokens, t0, reps = 0, time.perf_counter(), 0
     while True:
-        for c in samples:
-            oracle.ffn.ffn_token_loop(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs, "bf16")
-            tokens += c.T
+        tokens += wl.reference_step(samples)
         reps += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return tokens / el, int(_clib.lib().oracle_num_threads()), reps, el
+    return tokens / el, _host_cores(), reps, el
+
+
+def _host_cores():
+    from oracle import _clib
+    return int(_clib.lib().oracle_num_threads())
 
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import oracle
-    from oracle import _clib
     samples, what = wl.reference_sample(wl.make_cases())
-
-    def step():
-        for s in samples:
-            oracle.ffn.ffn_token_loop(s.x, s.w_gate, s.w_up, s.w_down, s.mask_words, s.gs, "bf16")
-
     for _ in range(args.warmup):
-        step()
+        wl.reference_step(samples)
     t0 = time.perf_counter()
+    tok = 0
     for _ in range(args.steps):
-        step()
+        tok += wl.reference_step(samples)
     el = time.perf_counter() - t0
-    tok = args.steps * sum(s.T for s in samples)
     v = tok / el
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
@@ -270,9 +471,8 @@ def run_reference(args, wl):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": wl.desc, "parallelism": "host cores"},
-        "cpu_baseline": {"value": v, "unit": "tokens/s",
-                         "cores": int(_clib.lib().oracle_num_threads()), "kind": "oracle",
-                         "sample": what + ", fp64 per-token loop over kept groups"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _host_cores(), "kind": "oracle",
+                         "sample": what},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -298,30 +498,16 @@ def run_ours(args, wl):
     torch.cuda.set_device(dev)
 
     import token_level_dynamic_b200 as w
-    from synth.torch_io import to_dev
 
     cases = wl.make_cases()
-    base = cases[0]
-    Wg = to_dev(base.w_gate, "bf16", dev)
-    Wu = to_dev(base.w_up, "bf16", dev)
-    Wd = to_dev(base.w_down, "bf16", dev)
-    xs = [to_dev(c.x, "bf16", dev) for c in cases]
-    ms = [to_dev(c.mask_words, "mask", dev) for c in cases]
-    outs = [torch.empty_like(x) for x in xs]
-    PATH = getattr(w, wl.path_name)
-    ws_bytes = max(w.wide_ffn_workspace_bytes(c.T, c.H, c.I, c.gs, path=PATH) for c in cases)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_sink = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream(dev)
-    gs = base.gs
+    D = wl.device(wl, cases, dev, stream)
     units = [wl.units(c) for c in cases]
-    ncalls = len(cases)
+    ncalls = D.ncalls
     tokens_per_step = sum(c.T for c in cases)
-
-    def call(i, mask=None):
-        w.wide_ffn_masked(xs[i], Wg, Wu, Wd, ms[i] if mask is None else mask, gs, out=outs[i],
-                          workspace=ws, path=PATH, stream=stream)
+    call = D.call
 
     def timed_step(fn):
         evs = []
@@ -419,6 +605,15 @@ def run_ours(args, wl):
 
     per_call_out = {}
     for i, c in enumerate(cases):
+        if not hasattr(c, "mask"):
+            t = float(per_call[:, i].mean())
+            per_call_out[wl.name] = {"tokens": c.T, "us_per_call": 1e3 * t,
+                                     "tokens_per_s": c.T / (t / 1e3),
+                                     "algorithmic_bytes": units[i]["total"],
+                                     "achieved_gbs": units[i]["total"] / (t / 1e3) / 1e9,
+                                     "frac_of_hbm": units[i]["total"] / (t / 1e3) / 1e9
+                                     / peaks["hbm_gbs"]}
+            continue
         t = float(per_call[:, i].mean())
         d = {"tokens": c.T, "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3)}
         if wl.bound == "hbm":
@@ -433,24 +628,10 @@ def run_ours(args, wl):
         per_call_out[c.name] = d
 
     # ---- dense baselines: torch/cuBLAS bf16 and our kernels with every group kept
-    ones = [torch.full_like(m, -1) for m in ms]
-    G = base.I // gs
-    if G % 32:
-        for o in ones:
-            o[:, -1] = (1 << (G % 32)) - 1
-
-    def dense_torch(i):
-        x = xs[i]
-        a = torch.nn.functional.linear(x, Wg)
-        b = torch.nn.functional.linear(x, Wu)
-        outs[i].copy_(torch.nn.functional.linear(torch.nn.functional.silu(a) * b, Wd))
-
-    def ours_ones(i):
-        call(i, ones[i])
-
     dense = {}
     nd = max(3, min(args.steps, 20))
-    for name, fn in (("torch_cublas_bf16", dense_torch), ("ours_all_groups_kept", ours_ones)):
+    for name, fn in (("torch_cublas_bf16", D.dense_torch),
+                     ("ours_all_groups_kept", lambda i: D.call(i, all_kept=True))):
         for _ in range(3):
             timed_step(fn)
         evs = [timed_step(fn) for _ in range(nd)]
@@ -462,20 +643,10 @@ def run_ours(args, wl):
     dense["masked_speedup_vs_ours_all_kept"] = dense["ours_all_groups_kept"]["ms_per_step"] / step_ms
 
     # ---- end to end through the public API with host buffers
-    xh = [x.cpu().pin_memory() for x in xs]
-    mh = [m.cpu().pin_memory() for m in ms]
-    oh = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-
-    def e2e_call(i):
-        xs[i].copy_(xh[i], non_blocking=True)
-        ms[i].copy_(mh[i], non_blocking=True)
-        call(i)
-        oh[i].copy_(outs[i], non_blocking=True)
-
     for _ in range(3):
-        timed_step(e2e_call)
+        timed_step(D.e2e_call)
     barrier()
-    e_evs = [timed_step(e2e_call) for _ in range(args.steps)]
+    e_evs = [timed_step(D.e2e_call) for _ in range(args.steps)]
     barrier()
     e_ms = float(ms_of(e_evs).sum())
     if world > 1:
@@ -483,17 +654,15 @@ def run_ours(args, wl):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e_ms = float(t.item())
     e2e = {"value": world * tokens_per_step * args.steps / (e_ms / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(sum(x.numel() * 2 + m.numel() * 4 for x, m in zip(xh, mh))),
-           "d2h_bytes_per_step": int(sum(o.numel() * 2 for o in oh)),
+           "h2d_bytes_per_step": D.h2d_bytes, "d2h_bytes_per_step": D.d2h_bytes,
            "ms_per_step": e_ms / args.steps}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         samples, what = wl.reference_sample(cases)
-        v, cores, reps, el = cpu_oracle_baseline(samples, args.cpu_seconds)
+        v, cores, reps, el = cpu_oracle_baseline(wl, samples, args.cpu_seconds)
         cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{what}; repeated {reps}x over {el:.1f} s; fp64 per-token loop over "
-                         f"kept groups"}
+               "sample": f"{what}; repeated {reps}x over {el:.1f} s (fp64 oracle)"}
 
     if world > 1:
         dist.barrier()

@@ -114,4 +114,51 @@ def layer_masked(lc, ret_parts: bool = False):
     return out
 
 
-__all__ = ["rmsnorm", "rope", "softmax_rows", "attention_masked", "layer_masked"]
+def layer_masked_rows(lc, rows):
+    """The layer's outputs for the token rows ``rows`` only: the same
+    definition as ``layer_masked``, evaluated row by row (K and V are still
+    computed for every token a selected query can see).  Returns (out[rows],
+    parts) with attn_out, ffn_out, h1 for those rows and k, v (after RoPE)
+    for all tokens."""
+    a = lc.attn
+    T, nq, nkv, hd = a.T, a.n_q, a.n_kv, a.hd
+    rep = nq // nkv
+    rows = np.asarray(rows)
+    x = widen(a.x, "bf16")
+    xn = rmsnorm(x, widen(a.gamma1, "bf16"), a.eps)
+    pos = a.positions
+    k = rope((xn @ widen(a.wk, "bf16").T).reshape(T, nkv, hd).transpose(1, 0, 2), pos,
+             a.theta).transpose(1, 0, 2)
+    v = (xn @ widen(a.wv, "bf16").T).reshape(T, nkv, hd)
+    q = (xn[rows] @ widen(a.wq, "bf16").T).reshape(len(rows), nq, hd)
+    q = rope(q.transpose(1, 0, 2), pos[rows], a.theta).transpose(1, 0, 2)
+    m = mask_bool(a.mask_words, nkv)
+    S = a.seq_len
+    o = np.zeros((len(rows), nq, hd))
+    for n, t in enumerate(rows):
+        b, i = divmod(int(t), S)
+        for j in range(nkv):
+            if not m[t, j]:
+                continue
+            Kn, Vn = k[b * S:b * S + i + 1, j], v[b * S:b * S + i + 1, j]
+            if a.mode == "decode" and a.cache_len > 0:
+                Kn = np.concatenate([widen(a.k_cache[b, j], "bf16"), Kn], axis=0)
+                Vn = np.concatenate([widen(a.v_cache[b, j], "bf16"), Vn], axis=0)
+            for hh in range(rep):
+                h = j * rep + hh
+                s = (Kn @ q[n, h]) / np.sqrt(hd)
+                p = np.exp(s - s.max())
+                o[n, h] = (p / p.sum()) @ Vn
+    attn_out = o.reshape(len(rows), nq * hd) @ widen(a.wo, "bf16").T
+    h1 = x[rows] + attn_out
+    xn2 = rmsnorm(h1, widen(lc.gamma2, "bf16"), a.eps)
+    f = lc.ffn
+    ffn_out = ffn_masked_f64(xn2, widen(f.w_gate, "bf16"), widen(f.w_up, "bf16"),
+                             widen(f.w_down, "bf16"), mask_bool(f.mask_words, f.I // f.gs)[rows],
+                             f.gs)
+    out = h1 + ffn_out
+    return out, {"attn_out": attn_out, "ffn_out": ffn_out, "h1": h1, "k": k, "v": v}
+
+
+__all__ = ["rmsnorm", "rope", "softmax_rows", "attention_masked", "layer_masked",
+           "layer_masked_rows"]

@@ -201,6 +201,10 @@ class LayerCase:
     ffn: FFNCase               # ffn.x is unused (the FFN input is computed)
     gamma2: np.ndarray         # [H] bf16 bits
 
+    @property
+    def T(self) -> int:
+        return self.attn.T
+
 
 def tiny_ffn(seed: int = 0) -> FFNCase:
     T, H, I, gs = 64, 256, 1024, 64

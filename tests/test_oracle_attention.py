@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 
 import synth
-from oracle.attention import rmsnorm, rope, attention_masked, layer_masked
+from oracle.attention import rmsnorm, rope, attention_masked, layer_masked, layer_masked_rows
 from oracle.ffn import widen
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -157,3 +157,17 @@ def test_sequence_permutation_in_decode():
     q.attn.k_cache, q.attn.v_cache = lc.attn.k_cache[p], lc.attn.v_cache[p]
     q.ffn.mask = lc.ffn.mask[p]
     np.testing.assert_array_equal(layer_masked(q), out[p])
+
+
+@pytest.mark.parametrize("mode,kw", [("prefill", dict(n_seq=3, seq_len=20)),
+                                     ("decode", dict(n_seq=5, cache_len=30))])
+def test_row_form_equals_full_layer(mode, kw):
+    """The per-row form (used for full-size sampled checks) is the same
+    definition: it matches the full layer on every row."""
+    lc = synth.small_layer(mode, seed=21, **kw)
+    full, parts = layer_masked(lc, ret_parts=True)
+    rows = np.arange(lc.attn.T)[::2]
+    out, rp = layer_masked_rows(lc, rows)
+    np.testing.assert_allclose(out, full[rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(rp["attn_out"], parts["attn_out"][rows], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(rp["k"], parts["k"], rtol=1e-12, atol=1e-13)

@@ -337,13 +337,16 @@ size_t wide_layer_workspace_bytes(const wide_layer_dims *d)
         return 0;
     if (layer_decode_supported(d))
         return layer_decode_workspace(d);
+    if (layer_prefill_supported(d))
+        return layer_prefill_workspace(d);
     return 0;
 }
 
 static int layer_call(const LayerPtrs &p, const wide_layer_dims *d, void *ws, size_t ws_bytes,
                       void *stream)
 {
-    if (!layer_decode_supported(d))
+    const bool decode = layer_decode_supported(d);
+    if (!decode && !layer_prefill_supported(d))
         return WIDE_EUNSUPPORTED;
     const void *ptrs[] = {p.x, p.gamma1, p.wq, p.wk, p.wv, p.wo, p.k_cache, p.v_cache};
     for (const void *q : ptrs)
@@ -365,9 +368,11 @@ static int layer_call(const LayerPtrs &p, const wide_layer_dims *d, void *ws, si
                    !aligned16(p.w_down))) ||
         (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
         return WIDE_EUNSUPPORTED;
-    if (ws_bytes < layer_decode_workspace(d))
+    if (ws_bytes < (decode ? layer_decode_workspace(d) : layer_prefill_workspace(d)))
         return WIDE_EWORKSPACE;
-    return layer_decode_launch(p, d, ws, static_cast<cudaStream_t>(stream));
+    if (decode)
+        return layer_decode_launch(p, d, ws, static_cast<cudaStream_t>(stream));
+    return layer_prefill_launch(p, d, ws, static_cast<cudaStream_t>(stream));
 }
 
 int wide_layer_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cache,

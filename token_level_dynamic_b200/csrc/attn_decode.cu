@@ -22,7 +22,6 @@
 //                 scores, a partial softmax and P.V for the group's query
 //                 heads; the slices are merged with log-sum-exp weights
 //                 through distributed shared memory.
-//   rmsnorm_rows  the FFN's input norm on the residual stream.
 // o_proj and the FFN run through the decode down/gate-up GEMVs (groups of
 // rep*head_dim o_proj columns), with the residual adds in their epilogues.
 #include <cooperative_groups.h>
@@ -350,31 +349,6 @@ __global__ void __launch_bounds__(kHD)
     cluster.sync();
 }
 
-// ------------------------------------------------------------ rmsnorm_rows
-// y[t] = x[t] / sqrt(mean(x[t]^2) + eps) * gamma, fp32 in, bf16 out.
-__global__ void __launch_bounds__(256)
-    rmsnorm_rows(const float *__restrict__ x, const __nv_bfloat16 *__restrict__ gamma,
-                 __nv_bfloat16 *__restrict__ y, int H, float eps)
-{
-    __shared__ float red[8];
-    const int t = blockIdx.x;
-    const float *xr = x + (size_t)t * H;
-    float ss = 0.f;
-    for (int k = threadIdx.x; k < H; k += 256)
-        ss = fmaf(xr[k], xr[k], ss);
-    for (int off = 16; off; off >>= 1)
-        ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if ((threadIdx.x & 31) == 0)
-        red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    float tot = 0.f;
-    for (int w = 0; w < 8; ++w)
-        tot += red[w];
-    const float r = 1.0f / sqrtf(tot / (float)H + eps);
-    for (int k = threadIdx.x; k < H; k += 256)
-        y[(size_t)t * H + k] = __float2bfloat16_rn(xr[k] * r * __bfloat162float(gamma[k]));
-}
-
 template <typename... KArgs, typename... Args>
 int launch_cluster(int32_t kid, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                    int cluster_x, cudaStream_t s, Args... args)
@@ -516,12 +490,7 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
         return rc;
 
     // 4. FFN input norm
-    {
-        LaunchScope scope(KID_RMSNORM, s);
-        rmsnorm_rows<<<T, 256, 0, s>>>(w.h1, static_cast<const __nv_bfloat16 *>(p.gamma2), w.xn2,
-                                       H, d->eps);
-    }
-    if ((rc = launch_status()))
+    if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
         return rc;
 
     // 5-6. masked FFN; out = h1 + ffn_out

@@ -1,0 +1,477 @@
+// attn_prefill.cu -- causal attention over compacted queries on tcgen05, and
+// the whole masked prefill layer.
+//
+// WIDE, technical summary section 2.A (per-token GQA head groups) with the
+// reordering of section 2.B: the tokens that keep head group j form the
+// prefix perm_a[j][0 : count_a[j]) in ascending token order, so the queries
+// of group j in sequence s are one contiguous range of that prefix.  Their
+// RoPE'd query rows were written contiguously (compacted, group-major) by
+// the Q projection, and attention works on dense 128-query tiles of that
+// range; skipped (token, group) pairs are never computed.
+//
+// prefill_attn: one CTA per (query tile, query head of the group, sequence x
+// KV head); 128 threads, thread r = query row r = TMEM lane r.  Per 128-key
+// tile up to the tile's last query position:
+//   S  = Q K^T           tcgen05, M=128 N=128 K=128, fp32 in TMEM columns 0..127
+//   P  = online softmax of S with the causal mask (key position <= query
+//        position), exp2 domain, row max/sum and the O rescale in registers;
+//        P is written as bf16 to a 128B-swizzled K-major tile
+//   PV = P V             tcgen05, B = V read MN-major from the cache tile,
+//                        fp32 in TMEM columns 128..255, added to O (registers)
+// then O / l is written (bf16) at the token's signature-order row of the
+// o_proj input.  Tiles with no query (ragged counts) exit at once.
+#include "common.cuh"
+#include "host.h"
+#include "umma.cuh"
+
+namespace wide {
+namespace {
+
+constexpr int kHD = 128;
+constexpr int kBQ = 128;       // queries per tile
+constexpr int kBKV = 128;      // keys per tile
+constexpr uint32_t kHalf = 128 * 128;   // one 64-column, 128-row swizzled sub-tile (16 KB)
+constexpr uint32_t kTile = 2 * kHalf;   // 128 x 128 bf16
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct AttnPArgs {
+    const int32_t *count, *perm, *sig_pos;   // head-group work list
+    int T, seq_len, n_kv, rep, qcols, ocols;
+    int64_t cache_cap;
+    float scale_log2;                        // log2(e) / sqrt(hd)
+    __nv_bfloat16 *o_sig;                    // [T][n_q * hd]
+    int32_t *status;
+};
+
+struct __align__(8) ACtl {
+    uint64_t bar_q, bar_kv, bar_mma;
+    uint32_t tmem_base;
+    int lo, nq, pmax;
+};
+
+constexpr size_t kAttnSmem = 1024 + 4 * kTile + sizeof(ACtl);
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// first index i in [0, n) with v[i] >= key (v ascending)
+__device__ __forceinline__ int lower_bound(const int32_t *v, int n, int key)
+{
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (v[mid] < key)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(128, 1)
+    prefill_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const AttnPArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    uint8_t *sq = smem, *sk = smem + kTile, *sv = smem + 2 * kTile, *sp = smem + 3 * kTile;
+    ACtl *ctl = reinterpret_cast<ACtl *>(smem + 4 * kTile);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int qt = blockIdx.x, hh = blockIdx.y;
+    const int s = blockIdx.z / a.n_kv, j = blockIdx.z % a.n_kv;
+    const int32_t *pj = a.perm + (size_t)j * a.T;
+
+    if (tid == 0) {
+        const int cnt = a.count[j];
+        const int lo = lower_bound(pj, cnt, s * a.seq_len);
+        const int hi = lower_bound(pj, cnt, (s + 1) * a.seq_len);
+        ctl->lo = lo;
+        ctl->nq = hi - lo;
+        const int last = min(hi - 1, lo + (qt + 1) * kBQ - 1);
+        ctl->pmax = last >= lo ? pj[last] - s * a.seq_len : -1;
+        mbar_init(&ctl->bar_q, 1);
+        mbar_init(&ctl->bar_kv, 1);
+        mbar_init(&ctl->bar_mma, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int lo = ctl->lo, nq = ctl->nq, pmax = ctl->pmax;
+    if (qt * kBQ >= nq)
+        return;  // no query of this group in this tile: nothing to compute
+    if (warp == 0) {
+        umma::tmem_alloc(&ctl->tmem_base, 256);
+        umma::tmem_relinquish();
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t t_s = tmem, t_pv = tmem + 128;
+
+    const int nvalid = min(kBQ, nq - qt * kBQ);
+    const int idx = lo + qt * kBQ + tid;                       // row of this thread
+    const bool live = tid < nvalid;
+    const int tok = live ? pj[idx] : 0;
+    const int pos = live ? tok - s * a.seq_len : -1;
+    const int64_t kvrow0 = ((int64_t)s * a.n_kv + j) * a.cache_cap;
+    const int nkt = pmax / kBKV + 1;
+
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&ctl->bar_q, kTile);
+        const int qrow = j * a.T + lo + qt * kBQ;
+        tma_load_2d(sq, &tm_q, hh * kHD, qrow, &ctl->bar_q);
+        tma_load_2d(sq + kHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
+    }
+
+    float o[kHD];
+#pragma unroll
+    for (int d = 0; d < kHD; ++d)
+        o[d] = 0.f;
+    float m = -INFINITY, l = 0.f;
+    uint32_t mma_phase = 0, kv_phase = 0;
+    bool ok = true;
+    constexpr uint32_t idesc_s = umma::idesc_bf16_f32(kBQ, kBKV);
+    constexpr uint32_t idesc_pv = umma::idesc_bf16_f32_bmn(kBQ, kHD);
+
+    for (int kt = 0; kt < nkt && ok; ++kt) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&ctl->bar_kv, 2 * kTile);
+            const int krow = (int)(kvrow0 + (int64_t)kt * kBKV);
+            tma_load_2d(sk, &tm_k, 0, krow, &ctl->bar_kv);
+            tma_load_2d(sk + kHalf, &tm_k, 64, krow, &ctl->bar_kv);
+            tma_load_2d(sv, &tm_v, 0, krow, &ctl->bar_kv);
+            tma_load_2d(sv + kHalf, &tm_v, 64, krow, &ctl->bar_kv);
+        }
+        if (!mbar_wait(&ctl->bar_kv, kv_phase)) {
+            set_status(a.status, WIDE_DEV_TIMEOUT);
+            ok = false;
+        }
+        kv_phase ^= 1u;
+        if (__syncthreads_or(!ok)) {
+            ok = false;
+            break;
+        }
+        // keys past the sequence's last position may be uninitialised cache
+        // memory: clear those V rows so that 0 * garbage cannot reach P V
+        {
+            const int kmax = a.seq_len - 1 - kt * kBKV;      // last valid key row in tile
+            if (kmax < kBKV - 1) {
+                for (int rr = max(kmax + 1, 0) + warp; rr < kBKV; rr += 4)
+                    for (int c = (tid & 31); c < 16; c += 32) {
+                        const int sub = c >> 3, ch = c & 7;
+                        *reinterpret_cast<uint4 *>(sv + sub * kHalf + rr * 128 + ch * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
+                fence_proxy_async_smem();
+                __syncthreads();
+            }
+        }
+        // S = Q K^T
+        if (tid == 0) {
+            if (kt == 0 && !mbar_wait(&ctl->bar_q, 0)) {
+                set_status(a.status, WIDE_DEV_TIMEOUT);
+                ok = false;
+            }
+            umma::fence_after_sync();
+            const uint32_t q0 = smem_u32(sq), k0 = smem_u32(sk);
+#pragma unroll
+            for (int k = 0; k < kHD / 16; ++k) {
+                const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
+                umma::mma_bf16(t_s, umma::desc_kmajor_sw128(q0 + off),
+                               umma::desc_kmajor_sw128(k0 + off), idesc_s, k != 0);
+            }
+            umma::commit(&ctl->bar_mma);
+        }
+        if (!mbar_wait(&ctl->bar_mma, mma_phase)) {
+            set_status(a.status, WIDE_DEV_TIMEOUT);
+            ok = false;
+        }
+        mma_phase ^= 1u;
+        umma::fence_after_sync();
+        // online softmax of this thread's row (two passes over TMEM: the
+        // row max, then the probabilities); P row -> swizzled smem
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        float mt = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < kBKV / 32; ++c) {
+            float v[32];
+            umma::tmem_ld32(t_s + lane_off + c * 32, v);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int kp = kt * kBKV + c * 32 + e;
+                if (live && kp <= pos)
+                    mt = fmaxf(mt, v[e] * a.scale_log2);
+            }
+        }
+        const float mn = fmaxf(m, mt);
+        const float alpha = (live && m > -INFINITY) ? exp2f(m - mn) : (live ? 0.f : 1.f);
+        float lsum = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kBKV / 32; ++c) {
+            float v[32];
+            umma::tmem_ld32(t_s + lane_off + c * 32, v);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+                float p[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int kp = kt * kBKV + c * 32 + g8 * 8 + e;
+                    p[e] = (live && kp <= pos) ? exp2f(v[g8 * 8 + e] * a.scale_log2 - mn) : 0.f;
+                    lsum += p[e];
+                }
+                __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]);
+                __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
+                __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
+                const int chunk = c * 4 + g8;            // 16-byte chunk of the 256-byte row
+                const int sub = chunk >> 3, ch = chunk & 7;
+                *reinterpret_cast<uint4 *>(sp + sub * kHalf + swz128(tid, ch)) = make_uint4(
+                    *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                    *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
+            }
+        }
+        if (live) {
+            l = l * alpha + lsum;
+            m = mn;
+#pragma unroll
+            for (int d = 0; d < kHD; ++d)
+                o[d] *= alpha;
+        }
+        fence_proxy_async_smem();       // P written by threads, read by the tensor core
+        umma::fence_before_sync();
+        __syncthreads();
+        // PV = P V
+        if (tid == 0 && ok) {
+            umma::fence_after_sync();
+            const uint32_t p0 = smem_u32(sp), v0 = smem_u32(sv);
+#pragma unroll
+            for (int k = 0; k < kBKV / 16; ++k) {
+                const uint32_t aoff = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
+                const uint32_t boff = (uint32_t)k * 16u * 128u;   // 16 key rows
+                umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
+                               umma::desc_mnmajor_sw128(v0 + boff, kHalf), idesc_pv, k != 0);
+            }
+            umma::commit(&ctl->bar_mma);
+        }
+        if (!mbar_wait(&ctl->bar_mma, mma_phase)) {
+            set_status(a.status, WIDE_DEV_TIMEOUT);
+            ok = false;
+        }
+        mma_phase ^= 1u;
+        umma::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < kHD / 32; ++c) {
+            float v[32];
+            umma::tmem_ld32(t_pv + lane_off + c * 32, v);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                o[c * 32 + e] += v[e];
+        }
+        umma::fence_before_sync();
+        // all TMEM reads are done before the next tile's MMAs; a failed wait
+        // anywhere ends the loop for every thread together
+        if (__syncthreads_or(!ok)) {
+            ok = false;
+            break;
+        }
+    }
+
+    if (live && ok) {
+        const float inv = 1.f / l;
+        __nv_bfloat16 *dst = a.o_sig + (size_t)a.sig_pos[tok] * a.ocols +
+                             (size_t)(j * a.rep + hh) * kHD;
+#pragma unroll
+        for (int c = 0; c < kHD / 8; ++c) {
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(o[c * 8] * inv, o[c * 8 + 1] * inv);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
+            __nv_bfloat162 b3 = __floats2bfloat162_rn(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
+            reinterpret_cast<uint4 *>(dst)[c] =
+                make_uint4(*reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                           *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
+        }
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, 256);
+    }
+}
+
+struct PrefillWs {
+    char *wl_a;
+    __nv_bfloat16 *xn, *qc, *o_sig;
+    float *h1;
+    char *ffn;
+    size_t wl_bytes, total;
+};
+
+PrefillWs prefill_ws(const wide_layer_dims *d, void *base)
+{
+    const size_t T = (size_t)(d->n_seq * d->seq_len);
+    const size_t H = (size_t)d->hidden;
+    const size_t qd = (size_t)d->n_q_heads * d->head_dim;
+    const size_t qcols = qd / d->n_kv_heads;
+    PrefillWs w = {};
+    char *p = static_cast<char *>(base);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *at = p ? p + off : nullptr;
+        off += align_up(bytes > 0 ? bytes : 1, 1024);
+        return at;
+    };
+    w.wl_bytes = wide_worklist_bytes((int64_t)T, d->n_kv_heads, kBQ);
+    w.wl_a = take(w.wl_bytes);
+    w.xn = reinterpret_cast<__nv_bfloat16 *>(take(T * H * 2));
+    w.qc = reinterpret_cast<__nv_bfloat16 *>(take((size_t)d->n_kv_heads * T * qcols * 2));
+    w.o_sig = reinterpret_cast<__nv_bfloat16 *>(take(T * qd * 2));
+    w.h1 = reinterpret_cast<float *>(take(T * H * 4));
+    wide_ffn_dims fd = {(int64_t)T, (int64_t)H, d->inter, d->ffn_group_size, WIDE_BF16,
+                        WIDE_PATH_PREFILL};
+    w.ffn = take(ffn_prefill_workspace(&fd));
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+bool layer_prefill_supported(const wide_layer_dims *d)
+{
+    const int64_t T = d->n_seq * d->seq_len;
+    const int rep = d->n_kv_heads > 0 ? d->n_q_heads / d->n_kv_heads : 0;
+    return d->cache_len == 0 && d->seq_len >= 1 && T >= 1 && T <= (1 << 24) &&
+           d->head_dim == kHD && d->n_kv_heads >= 2 && d->n_kv_heads % 2 == 0 &&
+           d->n_kv_heads <= 1024 && (rep == 2 || rep == 4) && d->hidden % 256 == 0 &&
+           d->ffn_group_size == 128 && d->inter % 128 == 0 && d->inter / 128 <= 1024 &&
+           d->cache_cap >= d->seq_len && (int64_t)d->n_kv_heads * T <= (1ll << 31) / 512;
+}
+
+size_t layer_prefill_workspace(const wide_layer_dims *d) { return prefill_ws(d, nullptr).total; }
+
+int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, cudaStream_t s)
+{
+    const int64_t T = d->n_seq * d->seq_len, H = d->hidden;
+    const int n_q = d->n_q_heads, n_kv = d->n_kv_heads, rep = n_q / n_kv;
+    const int qd = n_q * kHD, qcols = rep * kHD;
+    PrefillWs w = prefill_ws(d, ws);
+    int rc;
+
+    // 1. head-group mask reordering (no host sync)
+    wide_worklist wl;
+    if ((rc = wide_worklist_carve(w.wl_a, w.wl_bytes, T, n_kv, kBQ, &wl)))
+        return rc;
+    if ((rc = reorder_launch(p.head_mask, T, n_kv, kBQ, &wl, s)))
+        return rc;
+
+    // 2. attention input norm
+    if ((rc = rmsnorm_bf16_launch(p.x, p.gamma1, w.xn, (int)T, (int)H, d->eps, s)))
+        return rc;
+
+    // 3. Q for kept (token, group) pairs, compacted per group, RoPE applied
+    CUtensorMap tq, tk, tv, tqc, tkc, tvc, to_a, to_b;
+    const uint64_t kv_rows = (uint64_t)d->n_seq * n_kv * d->cache_cap;
+    if (!make_tmap_2d(&tq, p.wq, qd, H, H, 2, 128, 64, true) ||
+        !make_tmap_2d(&tk, p.wk, (uint64_t)n_kv * kHD, H, H, 2, 128, 64, true) ||
+        !make_tmap_2d(&tv, p.wv, (uint64_t)n_kv * kHD, H, H, 2, 128, 64, true) ||
+        !make_tmap_2d(&tqc, w.qc, (uint64_t)n_kv * T, qcols, qcols, 2, kBQ, 64, true) ||
+        !make_tmap_2d(&tkc, p.k_cache, kv_rows, kHD, kHD, 2, kBKV, 64, true) ||
+        !make_tmap_2d(&tvc, p.v_cache, kv_rows, kHD, kHD, 2, kBKV, 64, true) ||
+        !make_tmap_2d(&to_a, w.o_sig, T, qd, qd, 2, 128, 64, true) ||
+        !make_tmap_2d(&to_b, p.wo, H, qd, qd, 2, 256, 64, true))
+        return WIDE_ECUDA;
+    const float log2_theta = log2f(d->rope_theta);
+    GemmArgs ga = {};
+    ga.a = w.xn;
+    ga.count = wl.count;
+    ga.perm = wl.perm;
+    ga.items = wl.items;
+    ga.n_items_p = wl.n_items;
+    ga.sig_pos = wl.sig_pos;
+    ga.out0 = w.qc;
+    ga.T = (int)T;
+    ga.K = (int)H;
+    ga.group_cols = qcols;
+    ga.seq_len = (int)d->seq_len;
+    ga.n_kv = n_kv;
+    ga.cache_len = 0;
+    ga.cache_cap = d->cache_cap;
+    ga.log2_theta = log2_theta;
+    ga.status = status_ptr();
+    const int m_tiles = (int)((T + 127) / 128);
+    if ((rc = gather_gemm_launch(GEMM_ROPE_Q, tq, tq, ga, (qcols / 256) * n_kv * m_tiles,
+                                 KID_PREFILL_Q, s)))
+        return rc;
+
+    // 4. K and V for every token, RoPE on K, into the caches
+    GemmArgs gk = ga;
+    gk.out0 = static_cast<__nv_bfloat16 *>(p.k_cache);
+    gk.out1 = static_cast<__nv_bfloat16 *>(p.v_cache);
+    gk.kv_blocks = n_kv;          // n_kv/2 blocks of two K heads, then of two V heads
+    gk.m_tiles = m_tiles;
+    if ((rc = gather_gemm_launch(GEMM_KV, tk, tv, gk, n_kv * m_tiles, KID_PREFILL_KV, s)))
+        return rc;
+
+    // 5. attention on compacted queries -> o_sig (zeros at skipped pairs)
+    if ((rc = zero_dead_launch(p.head_mask, wl.sig_pos, w.o_sig, (int)T, qd, n_kv, qcols, s)))
+        return rc;
+    AttnPArgs aa;
+    aa.count = wl.count;
+    aa.perm = wl.perm;
+    aa.sig_pos = wl.sig_pos;
+    aa.T = (int)T;
+    aa.seq_len = (int)d->seq_len;
+    aa.n_kv = n_kv;
+    aa.rep = rep;
+    aa.qcols = qcols;
+    aa.ocols = qd;
+    aa.cache_cap = d->cache_cap;
+    aa.scale_log2 = kLog2e / sqrtf((float)kHD);
+    aa.o_sig = w.o_sig;
+    aa.status = status_ptr();
+    if (!raise_smem_limit(reinterpret_cast<const void *>(prefill_attn), kAttnSmem))
+        return WIDE_ECUDA;
+    {
+        LaunchScope scope(KID_PREFILL_ATTN, s);
+        const dim3 grid((unsigned)((d->seq_len + kBQ - 1) / kBQ), (unsigned)rep,
+                        (unsigned)(d->n_seq * n_kv));
+        prefill_attn<<<grid, 128, kAttnSmem, s>>>(tqc, tkc, tvc, aa);
+    }
+    if ((rc = launch_status()))
+        return rc;
+
+    // 6. o_proj over each signature tile's kept groups; h1 = x + attn (fp32)
+    UnionArgs ua = {};
+    ua.tile_union = wl.tile_union;
+    ua.sig_perm = wl.sig_perm;
+    ua.T = (int)T;
+    ua.N = (int)H;
+    ua.W = (n_kv + 31) / 32;
+    ua.gs = qcols;
+    ua.out_sum = static_cast<__nv_bfloat16 *>(p.attn_out);
+    if (p.ffn) {
+        ua.res_in = static_cast<const __nv_bfloat16 *>(p.x);
+        ua.out_total_f32 = w.h1;
+    }
+    ua.status = status_ptr();
+    if ((rc = tile_union_gemm_launch(to_a, to_b, ua, KID_PREFILL_OPROJ, s)) || !p.ffn)
+        return rc;
+
+    // 7. FFN input norm, masked FFN, out = h1 + ffn_out
+    if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn, (int)T, (int)H, d->eps, s)))
+        return rc;
+    FfnPrefillOut fo = {};
+    fo.out_sum = static_cast<__nv_bfloat16 *>(p.ffn_out);
+    fo.res_f32 = w.h1;
+    fo.out_total = static_cast<__nv_bfloat16 *>(p.out);
+    return ffn_prefill_core(w.xn, p.w_gate, p.w_up, p.w_down, p.ffn_mask, fo, T, H, d->inter,
+                            w.ffn, s);
+}
+
+}  // namespace wide

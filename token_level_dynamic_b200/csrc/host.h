@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -48,6 +49,10 @@ enum KernelId : int32_t {
     KID_DECODE_QKV = 8,
     KID_DECODE_ATTN = 9,
     KID_RMSNORM = 10,
+    KID_PREFILL_Q = 11,
+    KID_PREFILL_KV = 12,
+    KID_PREFILL_ATTN = 13,
+    KID_PREFILL_OPROJ = 14,
 };
 
 // Pointers of one masked-layer call (FFN pointers unused when !ffn).
@@ -88,14 +93,69 @@ struct DownOutputs {
     float *out_total_f32;
 };
 
+// ---- tcgen05 grouped GEMMs of the prefill path (prefill_gemm.cu)
+enum GemmMode : int { GEMM_SWIGLU = 0, GEMM_ROPE_Q = 1, GEMM_KV = 2 };
+
+struct GemmArgs {
+    const __nv_bfloat16 *a;                   // [T][K] activation rows
+    const int32_t *count, *perm, *items, *n_items_p, *sig_pos;  // work list (gathered modes)
+    __nv_bfloat16 *out0, *out1;
+    int T, K;
+    int out_ld;          // SwiGLU: row stride of H (= inter)
+    int group_cols;      // RoPE-Q: columns of one head group (rep * head_dim)
+    int seq_len, n_kv, kv_blocks, m_tiles;
+    int64_t cache_len, cache_cap;
+    float log2_theta;
+    int32_t *status;
+};
+
+struct UnionArgs {
+    const uint32_t *tile_union;
+    const int32_t *sig_perm;
+    int T, N, W, gs;
+    __nv_bfloat16 *out_sum;          // projection (optional)
+    const __nv_bfloat16 *res_in;     // residual, bf16 (optional)
+    const float *res_f32;            // residual, fp32 (optional)
+    __nv_bfloat16 *out_total;        // projection + residuals, bf16 (optional)
+    float *out_total_f32;            // projection + residuals, fp32 (optional)
+    int32_t *status;
+};
+
+int zero_dead_launch(const uint32_t *mask, const int32_t *sig_pos, void *buf, int T, int ld,
+                     int G, int gs, cudaStream_t s);
+int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
+                       const GemmArgs &a, int max_work, int32_t kid, cudaStream_t s);
+int tile_union_gemm_launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const UnionArgs &a,
+                           int32_t kid, cudaStream_t s);
+
 // Internal entry points of the kernel files.
 int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
                    const wide_worklist *wl, cudaStream_t s);
 int reorder_splits(int64_t T);
 
 size_t ffn_prefill_workspace(const wide_ffn_dims *d);
+// Outputs of the prefill FFN (each optional): out_sum = FFN(x); out_total =
+// FFN(x) + res_f32.
+struct FfnPrefillOut {
+    __nv_bfloat16 *out_sum;
+    const float *res_f32;
+    __nv_bfloat16 *out_total;
+};
+int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *wd,
+                     const uint32_t *mask, const FfnPrefillOut &o, int64_t T, int64_t H,
+                     int64_t I, void *ws, cudaStream_t s);
 int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void *wd,
                        const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
+                       cudaStream_t s);
+
+bool layer_prefill_supported(const wide_layer_dims *d);
+size_t layer_prefill_workspace(const wide_layer_dims *d);
+int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, cudaStream_t s);
+
+// RMSNorm of rows: y = x / sqrt(mean(x^2) + eps) * gamma, bf16 out.
+int rmsnorm_bf16_launch(const void *x, const void *gamma, void *y, int T, int H, float eps,
+                        cudaStream_t s);
+int rmsnorm_f32_launch(const float *x, const void *gamma, void *y, int T, int H, float eps,
                        cudaStream_t s);
 
 bool layer_decode_supported(const wide_layer_dims *d);

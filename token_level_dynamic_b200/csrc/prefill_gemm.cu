@@ -1,0 +1,731 @@
+// prefill_gemm.cu -- the tcgen05 grouped GEMMs of the prefill path.
+//
+// WIDE, technical summary section 2.B: after mask reordering, the active
+// tokens of group g are the prefix perm[g][0 : count[g]), so each group is a
+// dense GEMM over ceil(count[g] / 128) row tiles with a known active prefix;
+// section 2.C: tiles with no active token are never issued (block-level
+// skip) and rows past the active prefix are not loaded (load-stage skip).
+//
+// gather_gemm<mode>: persistent, warp-specialised, M=128 x N=256 tiles.
+//   warp 0     weight producer: two 128-row TMA tiles (128-byte swizzle) per
+//              64-column K stage
+//   warp 1     TMEM owner (512 columns: two 256-column fp32 accumulators, so
+//              the epilogue of one tile overlaps the MMAs of the next) and
+//              single-thread tcgen05.mma issuer
+//   warps 2-5  epilogue (warp w reads TMEM lanes 32 * (w % 4) .. +31)
+//   warps 6-7  row gather: 16-byte cp.async copies of the tile's token rows
+//              straight into the swizzled operand layout; each thread's copy
+//              completions arrive on the stage barrier
+//   modes
+//     SwiGLU  work item (g, i) of the FFN work list; B = [W_gate[g]; W_up[g]];
+//             epilogue h = silu(gate) * up, stored bf16 at the token's
+//             signature-order row of H.
+//     RopeQ   work item (j, i) of the head-group work list, 256-column part
+//             hf of the group (group_cols / 256 parts); B = 256 rows of Wq
+//             for two query heads of group j; epilogue RoPE,
+//             stored bf16 at row i*128 + r of group j's compacted q buffer.
+//     KV      dense: every token tile times 256 rows of Wk (two KV heads,
+//             RoPE in the epilogue) or Wv; stored into the caches.
+// tile_union_gemm: persistent, M=128 tokens of one signature tile x N=256
+//   outputs; the K loop visits only the groups (gs columns each) in the
+//   tile's union of kept groups; inactive rows inside a visited group read
+//   the zeros written by zero_dead.  Epilogue: projection and/or projection
+//   plus residuals (bf16 and fp32), written at the tokens' own rows.
+//
+// Every mbarrier wait is bounded; on expiry the kernel records
+// WIDE_DEV_TIMEOUT, drains what it issued (bounded), frees TMEM and returns.
+#include "common.cuh"
+#include "host.h"
+#include "umma.cuh"
+
+namespace wide {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+constexpr uint32_t kATile = kBM * 128;
+constexpr uint32_t kBTile = kBN * 128;
+constexpr uint32_t kStageBytes = kATile + kBTile;
+constexpr int kThreadsDown = 192;
+constexpr int kThreadsGather = 256;
+constexpr int kGatherThreads = 64;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kHD = 128;
+
+struct __align__(8) Ctl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + sizeof(Ctl);
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
+{
+    const uint32_t a = smem_u32(p);
+    return p + (((a + 1023u) & ~1023u) - a);
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Ctl *ctl,
+                                              int32_t *status)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 255u) == 0) {
+            if (*(volatile int *)&ctl->abort)
+                return false;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                set_status(status, WIDE_DEV_TIMEOUT);
+                *(volatile int *)&ctl->abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&v)[32])
+{
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t *>(&p);
+    }
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
+__device__ __forceinline__ void init_ctl(Ctl *ctl, uint32_t full_count)
+{
+    for (int s = 0; s < kStages; ++s) {
+        mbar_init(&ctl->full[s], full_count);
+        mbar_init(&ctl->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+        mbar_init(&ctl->tfull[a], 1);
+        mbar_init(&ctl->tempty[a], 128);
+    }
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_mbar_init();
+}
+
+// Rotate-half RoPE of a head held as 128 fp32 TMEM columns starting at
+// taddr; writes the rotated head as bf16 to dst[0..127].  Angles are
+// pos * theta^(-2p/128) in fp32, p the pair index.
+__device__ __forceinline__ void rope_head_store(uint32_t taddr, int pos, float log2_theta,
+                                                __nv_bfloat16 *dst, bool store)
+{
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
+        float x1[32], x2[32];
+        umma::tmem_ld32(taddr + cc * 32, x1);
+        umma::tmem_ld32(taddr + 64 + cc * 32, x2);
+        umma::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int p = cc * 32 + e;
+            const float inv = exp2f(-(float)(2 * p) / (float)kHD * log2_theta);
+            float sn, cs;
+            sincosf((float)pos * inv, &sn, &cs);
+            const float a = x1[e], b = x2[e];
+            x1[e] = a * cs - b * sn;
+            x2[e] = b * cs + a * sn;
+        }
+        if (store) {
+            store_bf16x32(dst + cc * 32, x1);
+            store_bf16x32(dst + 64 + cc * 32, x2);
+        }
+    }
+}
+
+__device__ __forceinline__ void copy_head_store(uint32_t taddr, __nv_bfloat16 *dst, bool store)
+{
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        umma::tmem_ld32(taddr + cc * 32, v);
+        umma::tmem_ld_wait();
+        if (store)
+            store_bf16x32(dst + cc * 32, v);
+    }
+}
+
+// ------------------------------------------------------------- zero_dead
+// One block per token: clears the gs-column slice of every group the token
+// skips, in row sig_pos[t] of a [T][ld] bf16 buffer.
+__global__ void __launch_bounds__(128)
+    zero_dead(const uint32_t *__restrict__ mask, const int32_t *__restrict__ sig_pos,
+              __nv_bfloat16 *__restrict__ buf, int T, int ld, int G, int W, int gs)
+{
+    const int t = blockIdx.x;
+    if (t >= T)
+        return;
+    const size_t row = (size_t)sig_pos[t] * ld;
+    const int per = gs / 8;                      // 16-byte chunks per group slice
+    for (int idx = threadIdx.x; idx < G * per; idx += 128) {
+        const int g = idx / per, q = idx % per;
+        if ((mask[(size_t)t * W + (g >> 5)] >> (g & 31)) & 1u)
+            continue;
+        reinterpret_cast<uint4 *>(buf + row + (size_t)g * gs)[q] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// --------------------------------------------------------- gather_gemm
+struct Work {
+    int g, base, nrows, hf, nb;
+};
+
+template <int MODE>
+__device__ __forceinline__ int n_work(const GemmArgs &a, int n_items)
+{
+    if (MODE == GEMM_SWIGLU)
+        return n_items;
+    if (MODE == GEMM_ROPE_Q)
+        return (a.group_cols / kBN) * n_items;    // 256-column parts per group
+    return a.kv_blocks * a.m_tiles;
+}
+
+template <int MODE>
+__device__ __forceinline__ Work decode_work(const GemmArgs &a, int it)
+{
+    Work w;
+    w.hf = 0;
+    w.nb = 0;
+    if (MODE == GEMM_KV) {
+        w.nb = it / a.m_tiles;
+        const int ti = it % a.m_tiles;
+        w.g = 0;
+        w.base = ti * kBM;
+        w.nrows = min(kBM, a.T - w.base);
+        return w;
+    }
+    int item = it;
+    if (MODE == GEMM_ROPE_Q) {
+        const int parts = a.group_cols / kBN;
+        item = it / parts;
+        w.hf = it % parts;
+    }
+    w.g = a.items[2 * item];
+    w.base = a.items[2 * item + 1] * kBM;
+    w.nrows = min(kBM, a.count[w.g] - w.base);
+    return w;
+}
+
+// token of tile row r (r < nrows)
+template <int MODE>
+__device__ __forceinline__ int row_token(const GemmArgs &a, const Work &w, int r)
+{
+    if (MODE == GEMM_KV)
+        return w.base + r;
+    return a.perm[(size_t)w.g * a.T + w.base + r];
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsGather, 1)
+    gather_gemm(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+                const GemmArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + kStages * kStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = (MODE == GEMM_KV) ? 0 : *a.n_items_p;
+    const int nw = n_work<MODE>(a, n_items);
+    const int KT = a.K / kBK;
+
+    if (threadIdx.x == 0) {
+        // one arrive (with the weight bytes) from the producer plus one
+        // cp.async-completion arrive from each gather thread
+        init_ctl(ctl, 1 + kGatherThreads);
+        tma_prefetch_desc(&tm0);
+        tma_prefetch_desc(&tm1);
+    }
+    if (warp == 1) {
+        umma::tmem_alloc(&ctl->tmem_base, kTmemCols);
+        umma::tmem_relinquish();
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        // -------------------------------------------- weight producer
+        uint32_t stage = 0, phase = 0, issued = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
+            const Work w = decode_work<MODE>(a, it);
+            const CUtensorMap *m0 = &tm0, *m1 = &tm1;
+            int r0, r1;
+            if (MODE == GEMM_SWIGLU) {
+                r0 = r1 = w.g * 128;                         // [W_gate[g]; W_up[g]]
+            } else if (MODE == GEMM_ROPE_Q) {
+                r0 = w.g * a.group_cols + w.hf * kBN;        // two query heads of group g
+                r1 = r0 + 128;
+                m1 = &tm0;
+            } else {
+                const int half = a.kv_blocks / 2;            // first half: Wk, then Wv
+                const bool is_k = w.nb < half;
+                m0 = m1 = is_k ? &tm0 : &tm1;
+                r0 = (is_k ? w.nb : w.nb - half) * kBN;
+                r1 = r0 + 128;
+            }
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                if (lane == 0) {
+                    if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, a.status)) {
+                        ok = false;
+                    } else {
+                        uint8_t *b = smem + stage * kStageBytes + kATile;
+                        mbar_arrive_expect_tx(&ctl->full[stage], kBTile);
+                        tma_load_2d(b, m0, kt * kBK, r0, &ctl->full[stage]);
+                        tma_load_2d(b + kBTile / 2, m1, kt * kBK, r1, &ctl->full[stage]);
+                        ++issued;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            for (uint32_t s = 0; s < kStages && s < issued; ++s) {
+                const uint32_t uses = (issued - s + kStages - 1) / kStages;
+                mbar_wait(&ctl->full[s], (uses - 1u) & 1u);
+            }
+        }
+    } else if (warp >= 6) {
+        // -------------------------------------------- token-row gather
+        const int p = threadIdx.x - 6 * 32;
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
+            const Work w = decode_work<MODE>(a, it);
+            const __nv_bfloat16 *src0 =
+                p < w.nrows ? a.a + (size_t)row_token<MODE>(a, w, p) * a.K : nullptr;
+            const __nv_bfloat16 *src1 =
+                p + 64 < w.nrows ? a.a + (size_t)row_token<MODE>(a, w, p + 64) * a.K : nullptr;
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, a.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                const int k0 = kt * kBK;
+                if (src0) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        cp_async16(sa + swz128(p, c), src0 + k0 + 8 * c);
+                }
+                if (src1) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        cp_async16(sa + swz128(p + 64, c), src1 + k0 + 8 * c);
+                }
+                cp_async_arrive_noinc(&ctl->full[stage]);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        cp_async_wait_all();
+    } else if (warp == 1) {
+        // -------------------------------------------- MMA issuer
+        constexpr uint32_t idesc = umma::idesc_bf16_f32(kBM, kBN);
+        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
+            if (lane == 0) {
+                if (!wait_or_abort(&ctl->tempty[acc], acc_phase ^ 1u, ctl, a.status))
+                    ok = false;
+                umma::fence_after_sync();
+                const uint32_t d = tmem + acc * (uint32_t)kBN;
+                for (int kt = 0; kt < KT && ok; ++kt) {
+                    if (!wait_or_abort(&ctl->full[stage], phase, ctl, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    // the A tile was written by cp.async (generic proxy) and
+                    // is read by the tensor core (async proxy)
+                    fence_proxy_async_smem();
+                    umma::fence_after_sync();
+                    const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t sb = sa + kATile;
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma::mma_bf16(d, umma::desc_kmajor_sw128(sa + 32u * k),
+                                       umma::desc_kmajor_sw128(sb + 32u * k), idesc,
+                                       (kt | k) != 0);
+                    umma::commit(&ctl->empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok)
+                    umma::commit(&ctl->tfull[acc]);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) {
+            umma::commit(&ctl->drain);
+            mbar_wait(&ctl->drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // -------------------------------------------- epilogue (warps 2-5)
+        const int q = warp & 3;
+        const int r = q * 32 + lane;          // tile row = TMEM lane
+        uint32_t acc = 0, acc_phase = 0;
+        for (int it = blockIdx.x; it < nw; it += gridDim.x) {
+            const Work w = decode_work<MODE>(a, it);
+            const bool live = r < w.nrows;
+            const int t = live ? row_token<MODE>(a, w, r) : 0;
+            if (!wait_or_abort(&ctl->tfull[acc], acc_phase, ctl, a.status))
+                break;
+            umma::fence_after_sync();
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * (uint32_t)kBN;
+            if (MODE == GEMM_SWIGLU) {
+                __nv_bfloat16 *dst = a.out0 + (size_t)(live ? a.sig_pos[t] : 0) * a.out_ld +
+                                     (size_t)w.g * 128;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float gv[32], uv[32];
+                    umma::tmem_ld32(taddr + c * 32, gv);
+                    umma::tmem_ld32(taddr + 128 + c * 32, uv);
+                    umma::tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        gv[e] = silu_f32(gv[e]) * uv[e];
+                    if (live)
+                        store_bf16x32(dst + c * 32, gv);
+                }
+            } else if (MODE == GEMM_ROPE_Q) {
+                const int pos = (int)(t % a.seq_len + a.cache_len);
+                __nv_bfloat16 *dst = a.out0 + ((size_t)w.g * a.T + w.base + r) * a.group_cols +
+                                     (size_t)w.hf * kBN;
+                rope_head_store(taddr, pos, a.log2_theta, dst, live);
+                rope_head_store(taddr + kHD, pos, a.log2_theta, dst + kHD, live);
+            } else {
+                const int half = a.kv_blocks / 2;
+                const bool is_k = w.nb < half;
+                const int seq = t / a.seq_len;
+                const int pos = (int)(t % a.seq_len + a.cache_len);
+                __nv_bfloat16 *cache = is_k ? a.out0 : a.out1;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    const int kvh = (is_k ? w.nb : w.nb - half) * 2 + h;
+                    __nv_bfloat16 *dst =
+                        cache + (((size_t)seq * a.n_kv + kvh) * (size_t)a.cache_cap + pos) * kHD;
+                    if (is_k)
+                        rope_head_store(taddr + h * kHD, pos, a.log2_theta, dst, live);
+                    else
+                        copy_head_store(taddr + h * kHD, dst, live);
+                }
+            }
+            umma::fence_before_sync();
+            mbar_arrive(&ctl->tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ----------------------------------------------------- tile_union_gemm
+__global__ void __launch_bounds__(kThreadsDown, 1)
+    tile_union_gemm(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b, const UnionArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align1024(smem_raw);
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + kStages * kStageBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_sig = (a.T + kBM - 1) / kBM;
+    const int n_tiles = n_sig * (a.N / kBN);
+    const int spg = a.gs / kBK;            // K stages per group
+
+    if (threadIdx.x == 0) {
+        init_ctl(ctl, 1);
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_b);
+    }
+    if (warp == 1) {
+        umma::tmem_alloc(&ctl->tmem_base, kTmemCols);
+        umma::tmem_relinquish();
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    // all signature tiles of one output block, then the next block, so that
+    // concurrently running CTAs share the weight slab
+    auto coords = [&](int tile, int &s, int &nb) {
+        nb = tile / n_sig;
+        s = tile % n_sig;
+    };
+    auto uword = [&](int s, int w) { return a.tile_union[(size_t)s * a.W + w]; };
+
+    if (warp == 0) {
+        uint32_t stage = 0, phase = 0, issued = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            int s, nb;
+            coords(tile, s, nb);
+            for (int w = 0; w < a.W && ok; ++w) {
+                uint32_t bits = uword(s, w);
+                while (bits && ok) {
+                    const int g = w * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    for (int sub = 0; sub < spg && ok; ++sub) {
+                        if (lane == 0) {
+                            if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, a.status)) {
+                                ok = false;
+                            } else {
+                                uint8_t *sa = smem + stage * kStageBytes;
+                                mbar_arrive_expect_tx(&ctl->full[stage], kStageBytes);
+                                const int col = g * a.gs + sub * kBK;
+                                tma_load_2d(sa, &tm_a, col, s * kBM, &ctl->full[stage]);
+                                tma_load_2d(sa + kATile, &tm_b, col, nb * kBN, &ctl->full[stage]);
+                            }
+                        }
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        issued += ok ? 1u : 0u;
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            for (uint32_t s = 0; s < kStages && s < issued; ++s) {
+                const uint32_t uses = (issued - s + kStages - 1) / kStages;
+                mbar_wait(&ctl->full[s], (uses - 1u) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        constexpr uint32_t idesc = umma::idesc_bf16_f32(kBM, kBN);
+        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            int s, nb;
+            coords(tile, s, nb);
+            if (lane == 0) {
+                if (!wait_or_abort(&ctl->tempty[acc], acc_phase ^ 1u, ctl, a.status))
+                    ok = false;
+                umma::fence_after_sync();
+                const uint32_t d = tmem + acc * (uint32_t)kBN;
+                int kstep = 0;
+                for (int w = 0; w < a.W && ok; ++w) {
+                    const int nsteps = __popc(uword(s, w)) * spg;
+                    for (int n = 0; n < nsteps && ok; ++n) {
+                        if (!wait_or_abort(&ctl->full[stage], phase, ctl, a.status)) {
+                            ok = false;
+                            break;
+                        }
+                        umma::fence_after_sync();
+                        const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                        const uint32_t sb = sa + kATile;
+#pragma unroll
+                        for (int k = 0; k < kBK / 16; ++k)
+                            umma::mma_bf16(d, umma::desc_kmajor_sw128(sa + 32u * k),
+                                           umma::desc_kmajor_sw128(sb + 32u * k), idesc,
+                                           (kstep | k) != 0);
+                        umma::commit(&ctl->empty[stage]);
+                        ++kstep;
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+                if (ok)
+                    umma::commit(&ctl->tfull[acc]);
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+        if (lane == 0) {
+            umma::commit(&ctl->drain);
+            mbar_wait(&ctl->drain, 0);
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        uint32_t acc = 0, acc_phase = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            int s, nb;
+            coords(tile, s, nb);
+            int nk = 0;
+            for (int w = 0; w < a.W; ++w)
+                nk += __popc(uword(s, w));
+            const int sr = s * kBM + r;
+            const long long orow = sr < a.T ? (long long)a.sig_perm[sr] : -1;
+            if (!wait_or_abort(&ctl->tfull[acc], acc_phase, ctl, a.status))
+                break;
+            umma::fence_after_sync();
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * (uint32_t)kBN;
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                float v[32];
+                if (nk > 0) {
+                    umma::tmem_ld32(taddr + c * 32, v);
+                    umma::tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        v[e] = 0.f;
+                }
+                if (orow < 0)
+                    continue;
+                const size_t at = (size_t)orow * a.N + (size_t)nb * kBN + c * 32;
+                if (a.out_sum)
+                    store_bf16x32(a.out_sum + at, v);
+                if (a.out_total || a.out_total_f32) {
+                    if (a.res_in) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 8) {
+                            float rv[8];
+                            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(a.res_in + at + e), rv);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                v[e + k] += rv[k];
+                        }
+                    }
+                    if (a.res_f32) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 rv = *reinterpret_cast<const float4 *>(a.res_f32 + at + e);
+                            v[e] += rv.x;
+                            v[e + 1] += rv.y;
+                            v[e + 2] += rv.z;
+                            v[e + 3] += rv.w;
+                        }
+                    }
+                    if (a.out_total)
+                        store_bf16x32(a.out_total + at, v);
+                    if (a.out_total_f32) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4 *>(a.out_total_f32 + at + e) =
+                                make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    }
+                }
+            }
+            umma::fence_before_sync();
+            mbar_arrive(&ctl->tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        umma::fence_after_sync();
+        umma::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+int num_sms()
+{
+    static int n[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 0;
+    if (!n[dev])
+        cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
+    return n[dev];
+}
+
+}  // namespace
+
+int zero_dead_launch(const uint32_t *mask, const int32_t *sig_pos, void *buf, int T, int ld,
+                     int G, int gs, cudaStream_t s)
+{
+    if (T <= 0)
+        return WIDE_OK;
+    LaunchScope scope(KID_PREFILL_ZERO, s);
+    zero_dead<<<(unsigned)T, 128, 0, s>>>(mask, sig_pos, static_cast<__nv_bfloat16 *>(buf), T, ld,
+                                          G, (G + 31) / 32, gs);
+    return launch_status();
+}
+
+int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
+                       const GemmArgs &a, int max_work, int32_t kid, cudaStream_t s)
+{
+    const int sms = num_sms();
+    if (sms <= 0 || max_work < 0)
+        return WIDE_ECUDA;
+    if (max_work == 0)
+        return WIDE_OK;
+    const int grid = max_work < sms ? max_work : sms;
+    const void *k = mode == GEMM_SWIGLU ? reinterpret_cast<const void *>(gather_gemm<GEMM_SWIGLU>)
+                    : mode == GEMM_ROPE_Q ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROPE_Q>)
+                                          : reinterpret_cast<const void *>(gather_gemm<GEMM_KV>);
+    if (!raise_smem_limit(k, kSmemBytes))
+        return WIDE_ECUDA;
+    LaunchScope scope(kid, s);
+    if (mode == GEMM_SWIGLU)
+        gather_gemm<GEMM_SWIGLU><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
+    else if (mode == GEMM_ROPE_Q)
+        gather_gemm<GEMM_ROPE_Q><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
+    else
+        gather_gemm<GEMM_KV><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
+    return launch_status();
+}
+
+int tile_union_gemm_launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const UnionArgs &a,
+                           int32_t kid, cudaStream_t s)
+{
+    const int sms = num_sms();
+    if (sms <= 0)
+        return WIDE_ECUDA;
+    const int64_t tiles = (int64_t)((a.T + kBM - 1) / kBM) * (a.N / kBN);
+    if (tiles == 0)
+        return WIDE_OK;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    if (!raise_smem_limit(reinterpret_cast<const void *>(tile_union_gemm), kSmemBytes))
+        return WIDE_ECUDA;
+    LaunchScope scope(kid, s);
+    tile_union_gemm<<<grid, kThreadsDown, kSmemBytes, s>>>(tm_a, tm_b, a);
+    return launch_status();
+}
+
+}  // namespace wide

@@ -115,6 +115,14 @@ const char *wide_kernel_name(int32_t id)
         return "decode_attention";
     case KID_RMSNORM:
         return "rmsnorm";
+    case KID_PREFILL_Q:
+        return "prefill_q_rope_tcgen05";
+    case KID_PREFILL_KV:
+        return "prefill_kv_rope_tcgen05";
+    case KID_PREFILL_ATTN:
+        return "prefill_attention_tcgen05";
+    case KID_PREFILL_OPROJ:
+        return "prefill_oproj_tcgen05";
     default:
         return "?";
     }

@@ -52,6 +52,20 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr)
            | ((uint64_t)2 << 61);                // 128-byte swizzle, bits [61,64)
 }
 
+// Shared-memory matrix descriptor for an MN-major operand tile written by
+// TMA with 128-byte swizzle: 128-byte rows hold 64 consecutive M/N elements
+// for one K index, 8-row atoms of 1024 bytes step along K (stride byte
+// offset 1024), and successive 64-element M/N atoms are lbo bytes apart
+// (leading byte offset).  A K step of 16 moves the start by 16 rows.
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t lbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu)
+           | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16)
+           | ((uint64_t)(1024u >> 4) << 32)
+           | ((uint64_t)1 << 46)
+           | ((uint64_t)2 << 61);
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, both
 // K-major, shape M x N (M in {64, 128}, N a multiple of 16 up to 256).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N)
@@ -61,6 +75,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N)
            | (1u << 10)            // B format: bf16
            | ((N >> 3) << 17)      // N / 8
            | ((M >> 4) << 24);     // M / 16
+}
+
+// The same with B read MN-major (B[n][k] stored with n contiguous).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(uint32_t M, uint32_t N)
+{
+    return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
