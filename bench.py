@@ -2,7 +2,8 @@
 """Benchmark of the masked WIDE layer on B200; prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_ffn_3b|prefill_ffn_8b|decode_layer_8b]
+                    [--workload decode_ffn_3b|prefill_ffn_8b|decode_layer_8b|
+                                prefill_layer_8b [--keep K]]
 
 Workloads (seeded synthetic inputs with the shapes the pages name):
   decode_ffn_3b (default)  Llama-3.2-3B-shaped masked SwiGLU FFN in decode:
@@ -14,6 +15,9 @@ Workloads (seeded synthetic inputs with the shapes the pages name):
       2048-entry KV cache: attention (QKV+RoPE, GQA over the cache, o_proj)
       with head groups kept at 0.34 and the FFN with groups kept at 0.72.
       HBM-bound; the roofline is union weight bytes + kept KV bytes.
+  prefill_layer_8b  Llama-3.1-8B-shaped masked prefill layer, 4 sequences
+      x 2048 tokens, head and FFN groups from 16 prototypes at keep 0.5 (0.25,
+      0.75, 1.0 with --keep) + 0.1 flips.  Tensor bound on kept FLOPs.
   prefill_ffn_8b  Llama-3.1-8B-shaped masked SwiGLU FFN in prefill: 4096
       tokens, hidden 4096, intermediate 14336 in 112 groups of 128, 8
       prototype masks (56 groups each) with 0.1 bit flips.  One step = one
@@ -347,26 +351,31 @@ class LayerDevice:
         a = self.lc.attn
         W = self.wts
         x = self.x
-        B, H, nq, nkv, hd = a.n_seq, a.H, a.n_q, a.n_kv, a.hd
+        B, S, nq, nkv, hd = a.n_seq, a.seq_len, a.n_q, a.n_kv, a.hd
         L = a.cache_len
         xf = x.float()
         xn = (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + a.eps)).to(x.dtype) * W["gamma1"]
-        q = F.linear(xn, W["wq"]).view(B, nq, 1, hd)
-        k = F.linear(xn, W["wk"]).view(B, nkv, 1, hd)
-        v = F.linear(xn, W["wv"]).view(B, nkv, 1, hd)
-        pos = torch.full((1,), float(L), device=x.device)
+        q = F.linear(xn, W["wq"]).view(B, S, nq, hd).transpose(1, 2)
+        k = F.linear(xn, W["wk"]).view(B, S, nkv, hd).transpose(1, 2)
+        v = F.linear(xn, W["wv"]).view(B, S, nkv, hd).transpose(1, 2)
+        pos = torch.arange(L, L + S, device=x.device, dtype=torch.float32)
         inv = a.theta ** (-torch.arange(0, hd, 2, device=x.device, dtype=torch.float32) / hd)
         ang = pos[:, None] * inv[None, :]
         cos, sin = torch.cos(ang).to(x.dtype), torch.sin(ang).to(x.dtype)
+
         def rope(t):
             t1, t2 = t[..., :hd // 2], t[..., hd // 2:]
             return torch.cat([t1 * cos - t2 * sin, t2 * cos + t1 * sin], -1)
+
         q, k = rope(q), rope(k)
-        self.kc[:, :, L:L + 1] = k
-        self.vc[:, :, L:L + 1] = v
-        o = F.scaled_dot_product_attention(q, self.kc[:, :, :L + 1], self.vc[:, :, :L + 1],
-                                           enable_gqa=True)
-        h1 = x + F.linear(o.reshape(B, nq * hd), W["wo"])
+        self.kc[:, :, L:L + S] = k
+        self.vc[:, :, L:L + S] = v
+        if S == 1:
+            o = F.scaled_dot_product_attention(q, self.kc[:, :, :L + 1], self.vc[:, :, :L + 1],
+                                               enable_gqa=True)
+        else:
+            o = F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)
+        h1 = x + F.linear(o.transpose(1, 2).reshape(B * S, nq * hd), W["wo"])
         hf = h1.float()
         xn2 = (hf * torch.rsqrt(hf.pow(2).mean(-1, keepdim=True) + a.eps)).to(x.dtype) * W["gamma2"]
         f = F.linear(F.silu(F.linear(xn2, W["w_gate"])) * F.linear(xn2, W["w_up"]), W["w_down"])
@@ -428,7 +437,72 @@ class DecodeLayer8B:
         return sum(lc.attn.T for lc in samples)
 
 
-WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B(), DecodeLayer8B())}
+class PrefillLayer8B:
+    name = "prefill_layer_8b"
+    bound = "tensor"
+    dominant = "prefill_gateup_tcgen05"
+    device = LayerDevice
+
+    def __init__(self, keep: float = 0.5):
+        self.keep = keep
+        self.desc = ("prefill_layer_8b: Llama-3.1-8B-shaped masked prefill layer, 4 sequences x "
+                     "2048 tokens (RMSNorm, QKV with 32 query / 8 KV heads of 128, RoPE theta "
+                     "5e5, causal GQA attention, o_proj, RMSNorm, SwiGLU FFN 14336 = 112 groups "
+                     f"x 128), 16 prototype masks at keep {keep} + 0.1 flips; one step = one call")
+
+    def make_cases(self):
+        import synth
+        return [synth.prefill_layer(keep=self.keep)]
+
+    @staticmethod
+    def units(lc):
+        """Kept FLOPs per call, per kernel (2 per multiply-add): Q only for
+        kept (token, head group) pairs; K/V for every token; attention for
+        kept pairs over their causal keys; o_proj for kept pairs; the FFN
+        for kept (token, channel group) pairs."""
+        import numpy as np
+        a, f = lc.attn, lc.ffn
+        T, H, hd, nq, nkv = a.T, a.H, a.hd, a.n_q, a.n_kv
+        rep = nq // nkv
+        pairs_a = int(a.mask.sum())
+        pos = np.tile(np.arange(a.seq_len), a.n_seq) + a.cache_len
+        keys = int((a.mask * (pos[:, None] + 1)).sum())
+        q = 2 * H * rep * hd * pairs_a
+        kv = 2 * H * 2 * nkv * hd * T
+        att = 4 * rep * hd * keys
+        oproj = 2 * H * rep * hd * pairs_a
+        pairs_f = int(f.mask.sum())
+        gateup = 4 * H * f.gs * pairs_f
+        down = 2 * H * f.gs * pairs_f
+        dense = (2 * H * (nq + 2 * nkv) * hd * T + 4 * nq * hd * int((pos + 1).sum())
+                 + 2 * H * nq * hd * T + 6 * H * f.I * T)
+        total = q + kv + att + oproj + gateup + down
+        return {"prefill_q_rope_tcgen05": q, "prefill_kv_rope_tcgen05": kv,
+                "prefill_attention_tcgen05": att, "prefill_oproj_tcgen05": oproj,
+                "prefill_gateup_tcgen05": gateup, "prefill_down_tcgen05": down,
+                "total": total, "dense_flops": dense}
+
+    def reference_sample(self, cases):
+        import copy
+        lc = copy.deepcopy(cases[0])
+        a, f = lc.attn, lc.ffn
+        n = 32
+        a.n_seq, a.seq_len = 1, n
+        a.x, a.mask = a.x[:n], a.mask[:n]
+        f.x, f.mask, f.T = f.x[:n], f.mask[:n], n
+        return [lc], ("per step: the first 32 tokens of sequence 0 (causal, so their outputs "
+                      "equal the full problem's), fp64 definition form")
+
+    @staticmethod
+    def reference_step(samples):
+        import oracle
+        for lc in samples:
+            oracle.attention.layer_masked(lc)
+        return sum(lc.attn.T for lc in samples)
+
+
+WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B(), DecodeLayer8B(),
+                                 PrefillLayer8B())}
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -607,12 +681,18 @@ def run_ours(args, wl):
     for i, c in enumerate(cases):
         if not hasattr(c, "mask"):
             t = float(per_call[:, i].mean())
-            per_call_out[wl.name] = {"tokens": c.T, "us_per_call": 1e3 * t,
-                                     "tokens_per_s": c.T / (t / 1e3),
-                                     "algorithmic_bytes": units[i]["total"],
-                                     "achieved_gbs": units[i]["total"] / (t / 1e3) / 1e9,
-                                     "frac_of_hbm": units[i]["total"] / (t / 1e3) / 1e9
-                                     / peaks["hbm_gbs"]}
+            d = {"tokens": c.T, "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3)}
+            if wl.bound == "hbm":
+                d.update({"algorithmic_bytes": units[i]["total"],
+                          "achieved_gbs": units[i]["total"] / (t / 1e3) / 1e9,
+                          "frac_of_hbm": units[i]["total"] / (t / 1e3) / 1e9 / peaks["hbm_gbs"]})
+            else:
+                d.update({"kept_flops": units[i]["total"],
+                          "achieved_tflops_whole_call": units[i]["total"] / (t / 1e3) / 1e12,
+                          "frac_of_bf16_peak_whole_call":
+                              units[i]["total"] / (t / 1e3) / 1e12 / peaks["bf16_tflops"],
+                          "kept_fraction_of_dense": units[i]["total"] / units[i]["dense_flops"]})
+            per_call_out[wl.name] = d
             continue
         t = float(per_call[:, i].mean())
         d = {"tokens": c.T, "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3)}
@@ -694,10 +774,14 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_ffn_3b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--keep", type=float, default=0.5,
+                    help="keep rate of the prefill_layer_8b masks (0.25, 0.5, 0.75, 1.0)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]
+    if args.workload == "prefill_layer_8b":
+        wl = PrefillLayer8B(args.keep)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

@@ -261,8 +261,13 @@ __global__ void __launch_bounds__(kHD)
     const int b = (int)blockIdx.z;          // sequence (= token)
     const int tid = (int)threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rep = a.n_q / a.n_kv;         // query heads per group (<= 4 here)
-    if (((a.head_mask[(size_t)b * a.Wh + (j >> 5)] >> (j & 31)) & 1u) == 0u)
-        return;  // the token skips this head group: no K/V bytes are read
+    if (((a.head_mask[(size_t)b * a.Wh + (j >> 5)] >> (j & 31)) & 1u) == 0u) {
+        // the token skips this head group: no K/V bytes are read; its output
+        // is 0 (o_proj reads 4-token blocks without per-token predication)
+        if (s < rep)
+            a.o[(size_t)b * a.n_q * kHD + (size_t)(j * rep + s) * kHD + tid] = 0.f;
+        return;
+    }
 
     const int64_t C = (a.nkeys + kSplits - 1) / kSplits;
     const int64_t kb = s * C, ke = min(a.nkeys, kb + C);

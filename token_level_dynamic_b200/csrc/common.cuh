@@ -96,8 +96,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 }
 
 // ------------------------------------------------------------ TMA copies
-// Tile-mode tensor copies global -> shared completing on an mbarrier.  No
-// multicast form is used anywhere in this library.
+// Tile-mode tensor copies global -> shared completing on an mbarrier; each
+// CTA loads its own tiles from this GPU's memory.
 
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int32_t x,
                                             int32_t y, uint64_t *bar)

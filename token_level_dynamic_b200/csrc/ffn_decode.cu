@@ -75,8 +75,72 @@ __device__ __forceinline__ uint32_t group_token_mask(const uint32_t *mask, int T
     return __ballot_sync(0xffffffffu, a);
 }
 
-template <typename TIn, int GS>
-__global__ void __launch_bounds__(GS)
+// Dot products of one weight chunk (EPC elements of two rows wa, wb) with
+// the x chunks of TB tokens (rows 0..TB-1 of xk, row stride ld): 2*TB
+// independent fp32 accumulation chains.
+template <int EPC, int TB>
+__device__ __forceinline__ void fma2_tb(const float (&wa)[EPC], const float (&wb)[EPC],
+                                        const float *xk, int ld, float *a, float *b)
+{
+#pragma unroll
+    for (int e = 0; e < EPC; e += 4) {
+        float xv[TB][4];
+#pragma unroll
+        for (int r = 0; r < TB; ++r) {
+            const float4 v = *reinterpret_cast<const float4 *>(xk + r * ld + e);
+            xv[r][0] = v.x;
+            xv[r][1] = v.y;
+            xv[r][2] = v.z;
+            xv[r][3] = v.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int r = 0; r < TB; ++r) {
+                a[r] = fmaf(wa[e + q], xv[r][q], a[r]);
+                b[r] = fmaf(wb[e + q], xv[r][q], b[r]);
+            }
+    }
+}
+
+// One weight row chunk with TB token chunks: TB independent chains.
+template <int EPC, int TB>
+__device__ __forceinline__ void fma1_tb(const float (&w)[EPC], const float *xk, int ld,
+                                        float *acc)
+{
+#pragma unroll
+    for (int e = 0; e < EPC; e += 4) {
+        float xv[TB][4];
+#pragma unroll
+        for (int r = 0; r < TB; ++r) {
+            const float4 v = *reinterpret_cast<const float4 *>(xk + r * ld + e);
+            xv[r][0] = v.x;
+            xv[r][1] = v.y;
+            xv[r][2] = v.z;
+            xv[r][3] = v.w;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int r = 0; r < TB; ++r)
+                acc[r] = fmaf(w[e + q], xv[r][q], acc[r]);
+    }
+}
+
+// Warp 0 of a decode CTA streams weight (and h) tiles through the stage
+// ring; the consumer warps release a stage by one arrive per warp on its
+// empty barrier, so the producer runs ahead without a block-wide barrier.
+struct Ring {
+    uint64_t *full, *empty;
+};
+
+// gate/up: block = 32 + 2*GS threads.  Warp 0 = TMA producer.  Consumer
+// thread (half, c) owns channel c of group g (its gate and up rows) and the
+// 16-byte chunks half*4 .. half*4+3 of every 128-byte K tile row.  Tokens
+// are taken TB at a time from the group's executing tokens (x rows past
+// them are zero), so consecutive FMAs are independent.
+template <typename TIn, int GS, int TB>
+__global__ void __launch_bounds__(32 + 2 * GS)
     ffn_decode_gateup(const __grid_constant__ CUtensorMap tm_gate,
                       const __grid_constant__ CUtensorMap tm_up, const TIn *__restrict__ x,
                       const uint32_t *__restrict__ mask, float *__restrict__ h, int T, int H,
@@ -85,31 +149,39 @@ __global__ void __launch_bounds__(GS)
     constexpr int EPC = ElemTraits<TIn>::EPC;
     constexpr int KT = 8 * EPC;                 // elements in one 128-byte tile row
     constexpr uint32_t kTileBytes = GS * 128u;  // one operand tile
+    constexpr int kConsumerWarps = 2 * GS / 32;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     uint8_t *stages = smem;                                          // [kStages][2][GS][128]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * 2 * kTileBytes);
-    int *act = reinterpret_cast<int *>(full + kStages);              // [32]
-    float *xs = reinterpret_cast<float *>(smem + kStages * 2 * kTileBytes + 256);  // [nact][kslice]
+    uint64_t *empty = full + kStages;
+    int *act = reinterpret_cast<int *>(empty + kStages);             // [32]
+    float *xs = reinterpret_cast<float *>(smem + kStages * 2 * kTileBytes + 512);  // [nactTB][kslice]
 
     cg::cluster_group cluster = cg::this_cluster();
     const int KS = (int)gridDim.x;
     const int s = (int)blockIdx.x;
     const int g = (int)blockIdx.y;
-    const int c = (int)threadIdx.x;
+    const int tid = (int)threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ct = tid - 32;                    // consumer index (valid when warp > 0)
+    const int c = ct % GS, half = ct / GS;
 
     const uint32_t tmask = group_token_mask(mask, T, W, g);
     if (tmask == 0u)
         return;  // block-level skip: the whole cluster leaves together
     const int nact = __popc(tmask);
+    const int nactb = (nact + TB - 1) / TB * TB;
     const int k0 = s * kslice;
     const int ntile = kslice / KT;
 
-    if (c < 32 && ((tmask >> c) & 1u))
-        act[__popc(tmask & ((1u << c) - 1u))] = c;
-    if (c == 0) {
-        for (int st = 0; st < kStages; ++st)
+    if (tid < 32 && ((tmask >> tid) & 1u))
+        act[__popc(tmask & ((1u << tid) - 1u))] = tid;
+    if (tid == 0) {
+        for (int st = 0; st < kStages; ++st) {
             mbar_init(&full[st], 1);
+            mbar_init(&empty[st], kConsumerWarps);
+        }
         fence_mbar_init();
         tma_prefetch_desc(&tm_gate);
         tma_prefetch_desc(&tm_up);
@@ -123,24 +195,46 @@ __global__ void __launch_bounds__(GS)
         tma_load_2d(dst, &tm_gate, k0 + kt * KT, g * GS, &full[st]);
         tma_load_2d(dst + kTileBytes, &tm_up, k0 + kt * KT, g * GS, &full[st]);
     };
-    int issued = 0;
-    if (c == 0) {
-        for (; issued < kStages && issued < ntile; ++issued)
-            issue(issued);
-    }
+    // the first ring's worth of tiles goes out before x is staged (no slot
+    // is in use yet, so nothing to wait for)
+    if (tid == 0)
+        for (int kt = 0; kt < kStages && kt < ntile; ++kt)
+            issue(kt);
 
     // x of the executing tokens over this K-slice, widened to fp32
     const int chunks_per_row = kslice / EPC;
-    for (int idx = c; idx < nact * chunks_per_row; idx += GS) {
+    for (int idx = tid; idx < nactb * chunks_per_row; idx += 32 + 2 * GS) {
         const int i = idx / chunks_per_row, q = idx % chunks_per_row;
-        const uint4 v = *reinterpret_cast<const uint4 *>(x + (size_t)act[i] * H + k0 + q * EPC);
         float f[EPC];
-        chunk_to_f32<TIn>(v, f);
+        if (i < nact) {
+            const uint4 v =
+                *reinterpret_cast<const uint4 *>(x + (size_t)act[i] * H + k0 + q * EPC);
+            chunk_to_f32<TIn>(v, f);
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPC; ++e)
+                f[e] = 0.f;
+        }
 #pragma unroll
         for (int e = 0; e < EPC; ++e)
             xs[i * kslice + q * EPC + e] = f[e];
     }
     __syncthreads();
+
+    bool timeout = false;
+    if (warp == 0) {
+        // ---------------------------------------------- TMA producer
+        if (lane == 0) {
+            for (int kt = kStages; kt < ntile; ++kt) {
+                const int st = kt % kStages;
+                if (!mbar_wait(&empty[st], (uint32_t)(kt / kStages - 1) & 1u)) {
+                    timeout = true;
+                    break;
+                }
+                issue(kt);
+            }
+        }
+    }
 
     float accg[kNTok], accu[kNTok];
 #pragma unroll
@@ -148,88 +242,90 @@ __global__ void __launch_bounds__(GS)
         accg[i] = 0.f;
         accu[i] = 0.f;
     }
-    bool timeout = false;
-    int consumed = 0;
-    for (int kt = 0; kt < ntile; ++kt) {
-        const int st = kt % kStages;
-        const uint32_t par = (uint32_t)(kt / kStages) & 1u;
-        if (!mbar_wait(&full[st], par))
-            timeout = true;
-        if (!timeout) {
+    if (warp > 0) {
+        // ---------------------------------------------- consumers
+        for (int kt = 0; kt < ntile; ++kt) {
+            const int st = kt % kStages;
+            if (!mbar_wait(&full[st], (uint32_t)(kt / kStages) & 1u)) {
+                timeout = true;
+                break;
+            }
             const uint8_t *tg = stages + st * 2 * kTileBytes;
             const uint8_t *tu = tg + kTileBytes;
-#pragma unroll 2
-            for (int j = 0; j < 8; ++j) {
+#pragma unroll 1
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = half * 4 + jj;
                 float wg[EPC], wu[EPC];
                 chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tg + swz128(c, j)), wg);
                 chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tu + swz128(c, j)), wu);
                 const float *xk = xs + kt * KT + j * EPC;
 #pragma unroll
-                for (int i = 0; i < kNTok; ++i) {
-                    if (i >= nact)
+                for (int i0 = 0; i0 < kNTok; i0 += TB) {
+                    if (i0 >= nactb)
                         break;
-                    const float *xp = xk + i * kslice;
-                    float xv[EPC];
-#pragma unroll
-                    for (int e = 0; e < EPC; e += 4) {
-                        const float4 t4 = *reinterpret_cast<const float4 *>(xp + e);
-                        xv[e] = t4.x;
-                        xv[e + 1] = t4.y;
-                        xv[e + 2] = t4.z;
-                        xv[e + 3] = t4.w;
-                    }
-#pragma unroll
-                    for (int e = 0; e < EPC; ++e) {
-                        accg[i] = fmaf(wg[e], xv[e], accg[i]);
-                        accu[i] = fmaf(wu[e], xv[e], accu[i]);
-                    }
+                    fma2_tb<EPC, TB>(wg, wu, xk + i0 * kslice, kslice, &accg[i0], &accu[i0]);
                 }
             }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[st]);
         }
-        consumed = kt + 1;
-        if (__syncthreads_or(timeout)) {
-            timeout = true;
-            break;
-        }
-        if (c == 0 && issued < ntile)
-            issue(issued++);
     }
-    if (timeout) {
-        // let copies already in flight land before this CTA's smem is reused
-        if (c == 0) {
+    if (__syncthreads_or(timeout)) {
+        timeout = true;
+        if (tid == 0) {
             set_status(status, WIDE_DEV_TIMEOUT);
-            for (int kt = consumed; kt < issued; ++kt)
-                mbar_wait(&full[kt % kStages], (uint32_t)(kt / kStages) & 1u);
+            // let copies in flight land before the stage memory is reused
+            for (int st = 0; st < kStages && st < ntile; ++st) {
+                const int last = st + (ntile - 1 - st) / kStages * kStages;
+                mbar_wait(&full[st], (uint32_t)(last / kStages) & 1u);
+            }
         }
         __syncthreads();
     }
 
     // partial sums -> this CTA's shared memory, then a cluster-wide add
-    float *pg = reinterpret_cast<float *>(stages);  // [kNTok][GS]
-    float *pu = pg + kNTok * GS;
+    float *pg = reinterpret_cast<float *>(stages);  // [2][kNTok][GS]
+    float *pu = pg + 2 * kNTok * GS;
+    if (warp > 0) {
 #pragma unroll
-    for (int i = 0; i < kNTok; ++i) {
-        if (i >= nact)
-            break;
-        pg[i * GS + c] = timeout ? 0.f : accg[i];
-        pu[i * GS + c] = timeout ? 0.f : accu[i];
+        for (int i = 0; i < kNTok; ++i) {
+            if (i >= nact)
+                break;
+            pg[(half * kNTok + i) * GS + c] = timeout ? 0.f : accg[i];
+            pu[(half * kNTok + i) * GS + c] = timeout ? 0.f : accu[i];
+        }
     }
     cluster.sync();
-    for (int i = s; i < nact; i += KS) {
-        float gs = 0.f, us = 0.f;
-        for (int q = 0; q < KS; ++q) {
-            const float *rg = cluster.map_shared_rank(pg, q);
-            const float *ru = cluster.map_shared_rank(pu, q);
-            gs += rg[i * GS + c];
-            us += ru[i * GS + c];
+    if (warp > 0 && half == 0) {
+        for (int i = s; i < nact; i += KS) {
+            float gs = 0.f, us = 0.f;
+            for (int q = 0; q < KS; ++q) {
+                const float *rg = cluster.map_shared_rank(pg, q);
+                const float *ru = cluster.map_shared_rank(pu, q);
+                gs += rg[i * GS + c] + rg[(kNTok + i) * GS + c];
+                us += ru[i * GS + c] + ru[(kNTok + i) * GS + c];
+            }
+            h[(size_t)act[i] * I + (size_t)g * GS + c] = silu_f32(gs) * us;
         }
-        h[(size_t)act[i] * I + (size_t)g * GS + c] = silu_f32(gs) * us;
+    } else if (warp > 0) {
+        // tokens that skip this group get h = 0, so that the down projection
+        // can run token blocks without per-token predication
+        for (int t = s; t < T; t += KS)
+            if (((tmask >> t) & 1u) == 0u)
+                h[(size_t)t * I + (size_t)g * GS + c] = 0.f;
     }
     cluster.sync();
 }
 
-template <typename TIn, int GS>
-__global__ void __launch_bounds__(kDownRows)
+// down: block = 32 + 256 threads.  Warp 0 = TMA producer (W_down tile and
+// the matching h tile per stage).  Consumer thread (half, n) owns output row
+// nb*128 + n and the chunks half*4 .. half*4+3 of every streamed row.  The K
+// loop visits only groups some token keeps; inside a group, blocks of TB
+// tokens none of which keeps the group are skipped (h is 0 for skipped
+// pairs, written by the gate/up kernel or the attention kernel).
+template <typename TIn, int GS, int TB>
+__global__ void __launch_bounds__(32 + 2 * kDownRows)
     ffn_decode_down(const __grid_constant__ CUtensorMap tm_down,
                     const __grid_constant__ CUtensorMap tm_h, const uint32_t *__restrict__ mask,
                     const DownOutputs o, int T, int H, int I, int W, int G, int32_t *status)
@@ -238,39 +334,54 @@ __global__ void __launch_bounds__(kDownRows)
     constexpr int KT = 8 * EPC;
     constexpr int TPG = GS / KT;                          // tiles per group
     constexpr uint32_t kWBytes = kDownRows * 128u;        // W_down tile
+    constexpr int kConsumerWarps = 2 * kDownRows / 32;
+    constexpr uint32_t kBlockMask = TB >= 32 ? 0xffffffffu : ((1u << TB) - 1u);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
+    const int TT = (T + TB - 1) / TB * TB;
     const uint32_t hbytes = (uint32_t)T * KT * 4u;        // h tile (fp32, unswizzled)
-    const uint32_t stage_bytes = kWBytes + ((hbytes + 1023u) & ~1023u);
+    const uint32_t hstride = (uint32_t)TT * KT * 4u;
+    const uint32_t stage_bytes = kWBytes + ((hstride + 1023u) & ~1023u);
     uint8_t *stages = smem;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kStages * stage_bytes);
-    uint32_t *gmask = reinterpret_cast<uint32_t *>(full + kStages);  // [gq]
-    int *live = reinterpret_cast<int *>(gmask + 1024);              // [gq]
+    uint64_t *empty = full + kStages;
+    uint32_t *gmask = reinterpret_cast<uint32_t *>(empty + kStages);  // [gq]
+    int *live = reinterpret_cast<int *>(gmask + 1024);               // [gq]
     __shared__ int n_live;
 
     cg::cluster_group cluster = cg::this_cluster();
     const int KS = (int)gridDim.x;
     const int s = (int)blockIdx.x;
     const int nb = (int)blockIdx.y;
-    const int n = (int)threadIdx.x;
-    const int warp = n >> 5, lane = n & 31;
+    const int tid = (int)threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int ct = tid - 32;
+    const int n = ct % kDownRows, half = ct / kDownRows;
     const int gq = (G + KS - 1) / KS;
     const int gbeg = s * gq, gend = min(G, gbeg + gq);
 
-    for (int gi = warp; gi < gend - gbeg; gi += kDownRows / 32) {
+    for (int gi = warp; gi < gend - gbeg; gi += (32 + 2 * kDownRows) / 32) {
         const uint32_t m = group_token_mask(mask, T, W, gbeg + gi);
         if (lane == 0)
             gmask[gi] = m;
     }
-    if (n == 0) {
-        for (int st = 0; st < kStages; ++st)
+    if (tid == 0) {
+        for (int st = 0; st < kStages; ++st) {
             mbar_init(&full[st], 1);
+            mbar_init(&empty[st], kConsumerWarps);
+        }
         fence_mbar_init();
         tma_prefetch_desc(&tm_down);
         tma_prefetch_desc(&tm_h);
     }
+    // token rows T..TT-1 of every h stage stay zero (TMA writes rows < T)
+    if (TT > T) {
+        for (int st = 0; st < kStages; ++st)
+            for (int i = tid; i < (TT - T) * KT; i += 32 + 2 * kDownRows)
+                reinterpret_cast<float *>(stages + st * stage_bytes + kWBytes)[T * KT + i] = 0.f;
+    }
     __syncthreads();
-    if (n == 0) {
+    if (tid == 0) {
         int k = 0;
         for (int gi = 0; gi < gend - gbeg; ++gi)
             if (gmask[gi])
@@ -280,100 +391,99 @@ __global__ void __launch_bounds__(kDownRows)
     __syncthreads();
     const int ntile = n_live * TPG;
 
-    auto issue = [&](int kt) {
-        const int st = kt % kStages;
-        const int gg = gbeg + live[kt / TPG];
-        const int col = gg * GS + (kt % TPG) * KT;
-        uint8_t *dst = stages + st * stage_bytes;
-        mbar_arrive_expect_tx(&full[st], kWBytes + hbytes);
-        tma_load_2d(dst, &tm_down, col, nb * kDownRows, &full[st]);
-        tma_load_2d(dst + kWBytes, &tm_h, col, 0, &full[st]);
-    };
-    int issued = 0;
-    if (n == 0) {
-        for (; issued < kStages && issued < ntile; ++issued)
-            issue(issued);
-    }
-
+    bool timeout = false;
     float acc[kNTok];
 #pragma unroll
     for (int t = 0; t < kNTok; ++t)
         acc[t] = 0.f;
-    bool timeout = false;
-    int consumed = 0;
-    for (int kt = 0; kt < ntile; ++kt) {
-        const int st = kt % kStages;
-        const uint32_t par = (uint32_t)(kt / kStages) & 1u;
-        if (!mbar_wait(&full[st], par))
-            timeout = true;
-        if (!timeout) {
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kt = 0; kt < ntile; ++kt) {
+                const int st = kt % kStages;
+                if (kt >= kStages && !mbar_wait(&empty[st], (uint32_t)(kt / kStages - 1) & 1u)) {
+                    timeout = true;
+                    break;
+                }
+                const int gg = gbeg + live[kt / TPG];
+                const int col = gg * GS + (kt % TPG) * KT;
+                uint8_t *dst = stages + st * stage_bytes;
+                mbar_arrive_expect_tx(&full[st], kWBytes + hbytes);
+                tma_load_2d(dst, &tm_down, col, nb * kDownRows, &full[st]);
+                tma_load_2d(dst + kWBytes, &tm_h, col, 0, &full[st]);
+            }
+        }
+    } else {
+        for (int kt = 0; kt < ntile; ++kt) {
+            const int st = kt % kStages;
+            if (!mbar_wait(&full[st], (uint32_t)(kt / kStages) & 1u)) {
+                timeout = true;
+                break;
+            }
             const uint32_t tm = gmask[live[kt / TPG]];
             const uint8_t *tw = stages + st * stage_bytes;
             const float *hs = reinterpret_cast<const float *>(tw + kWBytes);
-#pragma unroll 2
-            for (int j = 0; j < 8; ++j) {
+#pragma unroll 1
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = half * 4 + jj;
                 float w[EPC];
                 chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tw + swz128(n, j)), w);
 #pragma unroll
-                for (int t = 0; t < kNTok; ++t) {
-                    if (t >= T)
+                for (int t0 = 0; t0 < kNTok; t0 += TB) {
+                    if (t0 >= TT)
                         break;
-                    if ((tm >> t) & 1u) {
-                        const float *hp = hs + t * KT + j * EPC;
-#pragma unroll
-                        for (int e = 0; e < EPC; e += 4) {
-                            const float4 v = *reinterpret_cast<const float4 *>(hp + e);
-                            acc[t] = fmaf(w[e], v.x, acc[t]);
-                            acc[t] = fmaf(w[e + 1], v.y, acc[t]);
-                            acc[t] = fmaf(w[e + 2], v.z, acc[t]);
-                            acc[t] = fmaf(w[e + 3], v.w, acc[t]);
-                        }
-                    }
+                    if (((tm >> t0) & kBlockMask) == 0u)
+                        continue;
+                    fma1_tb<EPC, TB>(w, hs + t0 * KT + j * EPC, KT, &acc[t0]);
                 }
             }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[st]);
         }
-        consumed = kt + 1;
-        if (__syncthreads_or(timeout)) {
-            timeout = true;
-            break;
-        }
-        if (n == 0 && issued < ntile)
-            issue(issued++);
     }
-    if (timeout) {
-        if (n == 0) {
+    if (__syncthreads_or(timeout)) {
+        timeout = true;
+        if (tid == 0) {
             set_status(status, WIDE_DEV_TIMEOUT);
-            for (int kt = consumed; kt < issued; ++kt)
-                mbar_wait(&full[kt % kStages], (uint32_t)(kt / kStages) & 1u);
+            for (int st = 0; st < kStages && st < ntile; ++st) {
+                const int last = st + (ntile - 1 - st) / kStages * kStages;
+                mbar_wait(&full[st], (uint32_t)(last / kStages) & 1u);
+            }
         }
         __syncthreads();
     }
 
-    float *part = reinterpret_cast<float *>(stages);  // [kNTok][128]
+    float *part = reinterpret_cast<float *>(stages);  // [2][kNTok][128]
+    if (warp > 0) {
 #pragma unroll
-    for (int t = 0; t < kNTok; ++t) {
-        if (t >= T)
-            break;
-        part[t * kDownRows + n] = timeout ? 0.f : acc[t];
+        for (int t = 0; t < kNTok; ++t) {
+            if (t >= T)
+                break;
+            part[(half * kNTok + t) * kDownRows + n] = timeout ? 0.f : acc[t];
+        }
     }
     cluster.sync();
-    for (int t = s; t < T; t += KS) {
-        float sum = 0.f;
-        for (int q = 0; q < KS; ++q)
-            sum += cluster.map_shared_rank(part, q)[t * kDownRows + n];
-        const size_t at = (size_t)t * H + (size_t)nb * kDownRows + n;
-        if (o.out_sum)
-            static_cast<TIn *>(o.out_sum)[at] = from_f32<TIn>(sum);
-        if (o.out_total || o.out_total_f32) {
-            float tot = sum;
-            if (o.res_in)
-                tot += to_f32(static_cast<const TIn *>(o.res_in)[at]);
-            if (o.res_f32)
-                tot += o.res_f32[at];
-            if (o.out_total)
-                static_cast<TIn *>(o.out_total)[at] = from_f32<TIn>(tot);
-            if (o.out_total_f32)
-                o.out_total_f32[at] = tot;
+    if (warp > 0 && half == 0) {
+        for (int t = s; t < T; t += KS) {
+            float sum = 0.f;
+            for (int q = 0; q < KS; ++q) {
+                const float *rp = cluster.map_shared_rank(part, q);
+                sum += rp[t * kDownRows + n] + rp[(kNTok + t) * kDownRows + n];
+            }
+            const size_t at = (size_t)t * H + (size_t)nb * kDownRows + n;
+            if (o.out_sum)
+                static_cast<TIn *>(o.out_sum)[at] = from_f32<TIn>(sum);
+            if (o.out_total || o.out_total_f32) {
+                float tot = sum;
+                if (o.res_in)
+                    tot += to_f32(static_cast<const TIn *>(o.res_in)[at]);
+                if (o.res_f32)
+                    tot += o.res_f32[at];
+                if (o.out_total)
+                    static_cast<TIn *>(o.out_total)[at] = from_f32<TIn>(tot);
+                if (o.out_total_f32)
+                    o.out_total_f32[at] = tot;
+            }
         }
     }
     cluster.sync();
@@ -418,9 +528,19 @@ int gateup_chunk(const TIn *x, const TIn *wg, const TIn *wu, const uint32_t *mas
     if (!make_tmap_2d(&tg, wg, I, H, H, sizeof(TIn), GS, KT, true) ||
         !make_tmap_2d(&tu, wu, I, H, H, sizeof(TIn), GS, KT, true))
         return WIDE_ECUDA;
-    const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 256 + (size_t)T * kslice * 4;
-    return launch_cluster(KID_DECODE_GATEUP, ffn_decode_gateup<TIn, GS>, dim3(KS, G), dim3(GS),
-                          smem1, KS, s, tg, tu, x, mask, h, T, H, I, W, kslice, status_ptr());
+    const int TB = T >= 4 ? 4 : (T >= 2 ? 2 : 1);
+    const size_t TT = (size_t)((T + TB - 1) / TB * TB);
+    const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 512 + TT * kslice * 4;
+    const dim3 grid(KS, G), block(32 + 2 * GS);
+#define WIDE_GU(TBV)                                                                               \
+    launch_cluster(KID_DECODE_GATEUP, ffn_decode_gateup<TIn, GS, TBV>, grid, block, smem1, KS, s, \
+                   tg, tu, x, mask, h, T, H, I, W, kslice, status_ptr())
+    if (TB == 4)
+        return WIDE_GU(4);
+    if (TB == 2)
+        return WIDE_GU(2);
+    return WIDE_GU(1);
+#undef WIDE_GU
 }
 
 template <typename TIn, int GS>
@@ -435,12 +555,22 @@ int down_chunk(const TIn *wd, const float *h, const uint32_t *mask, const DownOu
         !make_tmap_2d(&th, h, T, I, I, 4, T, KT, false))
         return WIDE_ECUDA;
     const int KSd = G < 8 ? G : 8;
-    const size_t hb = (size_t)T * KT * 4;
+    const int TB = T >= 8 ? 8 : (T >= 4 ? 4 : (T >= 2 ? 2 : 1));
+    const size_t hb = (size_t)((T + TB - 1) / TB * TB) * KT * 4;
     const size_t stage = (size_t)kDownRows * 128 + ((hb + 1023) & ~(size_t)1023);
     const size_t smem2 = 1024 + kStages * stage + 64 + 1024 * 4 + 1024 * 4;
-    return launch_cluster(KID_DECODE_DOWN, ffn_decode_down<TIn, GS>, dim3(KSd, H / kDownRows),
-                          dim3(kDownRows), smem2, KSd, s, td, th, mask, o, T, H, I, W, G,
-                          status_ptr());
+    const dim3 grid(KSd, H / kDownRows), block(32 + 2 * kDownRows);
+#define WIDE_DN(TBV)                                                                               \
+    launch_cluster(KID_DECODE_DOWN, ffn_decode_down<TIn, GS, TBV>, grid, block, smem2, KSd, s, td, \
+                   th, mask, o, T, H, I, W, G, status_ptr())
+    if (TB == 8)
+        return WIDE_DN(8);
+    if (TB == 4)
+        return WIDE_DN(4);
+    if (TB == 2)
+        return WIDE_DN(2);
+    return WIDE_DN(1);
+#undef WIDE_DN
 }
 
 template <typename TIn, int GS>

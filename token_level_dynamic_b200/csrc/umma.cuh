@@ -1,7 +1,7 @@
 // umma.cuh -- 5th-generation tensor core (tcgen05) helpers for sm_100a:
 // TMEM allocation, shared-memory matrix descriptors, the instruction
-// descriptor of the bf16 x bf16 -> fp32 MMA, MMA issue/commit, TMEM loads
-// and the TMA gather of four rows.  Inline PTX only.
+// descriptor of the bf16 x bf16 -> fp32 MMA, MMA issue/commit and TMEM
+// loads.  Inline PTX only.
 #pragma once
 
 #include "common.cuh"
@@ -128,22 +128,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
 __device__ __forceinline__ void tmem_ld_wait()
 {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// -------------------------------------------------------------- TMA gather
-// Four rows (row0..row3) of a 2-D tensor map whose box is one row high and
-// 64 bf16 wide, starting at column x, into 4 consecutive 128-byte rows of a
-// 128-byte-swizzled shared tile.  No multicast.
-__device__ __forceinline__ void tma_gather4(void *smem_dst, const CUtensorMap *map, int32_t x,
-                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3,
-                                            uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(smem_dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(smem_u32(bar))
-        : "memory");
 }
 
 }  // namespace umma
