@@ -219,7 +219,7 @@ class DecodeFFN3B:
             "intermediate 8192 = 64 groups x 128, bf16, Bernoulli(0.5) masks; one step = "
             "batches 1, 8 and 32 (41 tokens)")
     bound = "hbm"
-    dominant = "decode_gateup_gemv"
+    dominant = None          # the kernel with the largest share of the step
     path_name = "WIDE_PATH_DECODE"
     device = FFNDevice
 
@@ -235,8 +235,8 @@ class DecodeFFN3B:
 
     @staticmethod
     def units(case):
-        """Algorithmic bytes per call, per kernel: every weight byte of the
-        batch's union of groups once, plus x, mask, fp32 h and out."""
+        """Algorithmic bytes per call and kernel: every weight byte (gate, up,
+        down) of the batch's union of groups once, plus activations."""
         return _ffn_decode_bytes(case)
 
     def reference_sample(self, cases):
@@ -250,14 +250,30 @@ class DecodeFFN3B:
     reference_step = staticmethod(lambda samples: _ffn_oracle_step(samples))
 
 
-def _ffn_decode_bytes(case, prefix=""):
+def _fused_decode_used(T, H, I, gs, sms=148):
+    """Mirror of the library's dispatch: the fused decode kernel runs for up
+    to 8 tokens when H % 256 == 0, gs in 64..256 and the W_down rows of one
+    CTA fit its box (ceil(H / SMs) <= 96)."""
+    return (1 <= T <= 8 and H % 256 == 0 and gs % 64 == 0 and gs <= 256 and I % gs == 0
+            and I // gs <= 1024 and -(-H // sms) <= 96)
+
+
+def _ffn_decode_bytes(case, res_bytes=0, x_bytes=None):
+    """Algorithmic bytes per kernel of one decode FFN call: every weight byte
+    of the batch's union of groups once, plus activations in and out (h of
+    the two-kernel path goes through memory; the fused kernel keeps it in
+    L2)."""
     B, H, I, gs = case.T, case.H, case.I, case.gs
     U = int(case.mask.any(axis=0).sum())
-    pairs = int(case.mask.sum())
     m = case.mask_words.nbytes
+    xb = B * H * 2 if x_bytes is None else x_bytes
+    if _fused_decode_used(B, H, I, gs):
+        fused = 3 * U * gs * H * 2 + xb + m + B * H * 2 + res_bytes
+        return {"decode_ffn_fused_gemv": fused, "total": fused, "union_groups": U}
+    pairs = int(case.mask.sum())
     h = pairs * gs * 4
-    gateup = 2 * U * gs * H * 2 + B * H * 2 + m + h
-    down = H * U * gs * 2 + h + m + B * H * 2
+    gateup = 2 * U * gs * H * 2 + xb + m + h
+    down = H * U * gs * 2 + h + m + B * H * 2 + res_bytes
     return {"decode_gateup_gemv": gateup, "decode_down_gemv": down,
             "total": gateup + down, "union_groups": U}
 
@@ -389,7 +405,7 @@ class DecodeLayer8B:
             "cache, o_proj, RMSNorm, SwiGLU FFN 14336 = 112 groups x 128), batch 16, head "
             "groups Bernoulli(0.34), FFN groups Bernoulli(0.72); one step = one call")
     bound = "hbm"
-    dominant = "decode_gateup_gemv"
+    dominant = None          # the kernel with the largest share of the step
     device = LayerDevice
 
     def make_cases(self):
@@ -411,13 +427,22 @@ class DecodeLayer8B:
                + kept_pairs * rep * hd * 4 + 2 * T * nkv * hd * 2)
         attn = kept_pairs * 2 * keys * hd * 2 + kept_pairs * rep * hd * 4 * 2
         oproj = H * Ua * rep * hd * 2 + kept_pairs * rep * hd * 4 + T * H * 2 * 2 + T * H * 4
-        ffn = _ffn_decode_bytes(f)
-        down = oproj + ffn["decode_down_gemv"]
-        norm = T * H * 4 + T * H * 2
-        total = qkv + attn + down + ffn["decode_gateup_gemv"] + norm
-        return {"decode_qkv_rope_gemv": qkv, "decode_attention": attn, "decode_down_gemv": down,
-                "decode_gateup_gemv": ffn["decode_gateup_gemv"], "rmsnorm": norm,
-                "total": total, "union_groups": ffn["union_groups"]}
+        out = {"decode_qkv_rope_gemv": qkv, "decode_attention": attn}
+        if _fused_decode_used(T, H, f.I, f.gs):
+            # FFN with its input norm: h1 (fp32) and gamma2 in, ffn_out and out back
+            ffn = _ffn_decode_bytes(f, res_bytes=T * H * 2, x_bytes=T * H * 4 + H * 2)
+            out["decode_down_gemv"] = oproj
+        else:
+            norm = T * H * 4 + T * H * 2 + H * 2
+            ffn = _ffn_decode_bytes(f, res_bytes=T * H * 4 + T * H * 2)
+            out["rmsnorm"] = norm
+            out["decode_down_gemv"] = oproj + ffn.pop("decode_down_gemv")
+        for k, v in ffn.items():
+            if k not in ("total", "union_groups"):
+                out[k] = v
+        out["total"] = sum(v for k, v in out.items())
+        out["union_groups"] = ffn["union_groups"]
+        return out
 
     def reference_sample(self, cases):
         import copy
@@ -641,12 +666,11 @@ def run_ours(args, wl):
         kern.setdefault(name, []).append(t)
     kernels = {}
     for name, ts in kern.items():
-        per_call_ts = [ts[i::ncalls] for i in range(ncalls)] if len(ts) % ncalls == 0 else [ts]
-        t_step = sum(statistics.mean(p) for p in per_call_ts)
+        t_step = sum(ts) / args.steps
         entry = {"launches": len(ts), "avg_us": 1e3 * statistics.mean(ts),
                  "us_per_step": 1e3 * t_step}
-        if name in units[0]:
-            u_step = sum(u[name] for u in units)
+        if any(name in u for u in units):
+            u_step = sum(u.get(name, 0) for u in units)
             if wl.bound == "hbm":
                 a = u_step / (t_step / 1e3) / 1e9
                 entry.update({"algorithmic_bytes_per_step": u_step, "achieved_gbs": a,
@@ -661,15 +685,18 @@ def run_ours(args, wl):
     for k in kernels.values():
         k["share_of_library_time"] = k["us_per_step"] / tot_k if tot_k else None
 
-    dk = kernels.get(wl.dominant, {})
-    traffic = _traffic_record(wl.dominant, wl.name)
+    dominant = wl.dominant or max(
+        (k for k in kernels if any(k in u for u in units)),
+        key=lambda k: kernels[k]["us_per_step"], default=None)
+    dk = kernels.get(dominant, {})
+    traffic = _traffic_record(dominant, wl.name)
     if wl.bound == "hbm":
-        roofline = {"kernel": wl.dominant, "bound": "hbm", "achieved": dk.get("achieved_gbs"),
+        roofline = {"kernel": dominant, "bound": "hbm", "achieved": dk.get("achieved_gbs"),
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": dk.get("frac_of_hbm"),
                     "peak_source": f"{peaks['source']} hbm_gbs (MEASURED_PEAKS.json)"}
     else:
-        roofline = {"kernel": wl.dominant, "bound": "tensor", "achieved": dk.get("achieved_tflops"),
+        roofline = {"kernel": dominant, "bound": "tensor", "achieved": dk.get("achieved_tflops"),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": dk.get("frac_of_bf16_peak"),
                     "frac_of_sustained": dk.get("frac_of_bf16_sustained"),

@@ -76,6 +76,12 @@ const char *wide_status_string(int code);
 /* ABI version of the loaded library (WIDE_ABI_VERSION). */
 int wide_abi_version(void);
 
+/* After a call returned WIDE_ECUDA: "file:line: <CUDA error text>" of the
+ * failing runtime or driver call, for the calling host thread ("" if none
+ * yet).  The string is owned by the library and valid until the thread's
+ * next failing call. */
+const char *wide_last_error(void);
+
 /* Synchronises `stream`, then copies the current device's status word into
  * *h_status (host pointer).  0 means no device-side error since the last
  * wide_clear_device_status. */
@@ -268,7 +274,8 @@ int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cac
  * path (CUDA-core GEMV over the batch's union of groups), minus the
  * workspace: the kernels' scratch (fp32 h for up to 32 tokens x inter
  * channels) lives in a fixed device array inside the library of
- * WIDE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * WIDE_NOALLOC_SCRATCH_BYTES bytes, and the decode kernel's grid-barrier
+ * words in a second one of 256 bytes, which every GPU that loads the library
  * holds until the process exits.  Limit: min(tokens, 32) * inter * 4 bytes
  * must not exceed it (inter <= 16384); larger problems return
  * WIDE_ETOOLARGE before anything is enqueued.  The call allocates nothing.

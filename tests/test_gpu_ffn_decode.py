@@ -79,3 +79,42 @@ def test_repeatable_bitwise():
     c = synth.decode_ffn(8)
     a, b = _run(c), _run(c)
     np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("T", [9, 17, 24, 31])
+def test_token_blocks_share_weight_tiles(T):
+    """Batches of more than 8 tokens run as blocks of 8 tokens whose CTAs
+    read the same weight rows; a ragged last block included."""
+    c = synth.ffn_case(T, 1024, 4096, 128, seed=40 + T)
+    assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
+
+
+def test_union_of_one_group_with_a_full_batch():
+    """Only token 19 keeps anything (group 3): every other token's output is
+    exactly zero and the one kept group is right."""
+    c = synth.ffn_case(20, 512, 2048, 128, seed=9)
+    c.mask[:] = False
+    c.mask[19, 3] = True
+    out = _run(c)
+    assert not np.any(out[:19])
+    assert rel_l2(out, _ref(c)) <= TOL_BF16
+
+
+def test_output_rows_split_unevenly_over_the_grid():
+    """A hidden size whose output rows do not split evenly over the grid."""
+    c = synth.ffn_case(5, 2816, 3072, 64, seed=11)
+    assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
+
+
+def test_bad_mask_bit_sets_device_status():
+    """A bit at or above G in the decode mask sets WIDE_DEV_BAD_MASK."""
+    import torch
+    import token_level_dynamic_b200 as w
+    c = synth.ffn_case(2, 256, 1024, 128, seed=5)          # G = 8
+    x, wg, wu, wd, m = ffn_to_dev(c)
+    m[1, 0] |= 1 << 9
+    w.wide_clear_device_status()
+    w.wide_ffn_masked(x, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_DECODE)
+    torch.cuda.synchronize()
+    assert w.wide_get_device_status() & w.WIDE_DEV_BAD_MASK
+    w.wide_clear_device_status()

@@ -31,7 +31,10 @@ _L = _native.lib()
 
 class WideError(RuntimeError):
     def __init__(self, fn: str, code: int):
-        super().__init__(f"{fn}: {code} ({wide_status_string(code)})")
+        msg = f"{fn}: {code} ({wide_status_string(code)})"
+        if code == WIDE_ECUDA:
+            msg += f" at {wide_last_error()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -70,6 +73,10 @@ def wide_status_string(code: int) -> str:
 
 def wide_abi_version() -> int:
     return _L.wide_abi_version()
+
+
+def wide_last_error() -> str:
+    return _L.wide_last_error().decode()
 
 
 def wide_get_device_status(stream=None, device=None) -> int:

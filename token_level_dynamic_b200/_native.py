@@ -60,6 +60,7 @@ class WideLayerWeights(ctypes.Structure):
 SIGNATURES = {
     "wide_status_string": (ctypes.c_char_p, [c_int]),
     "wide_abi_version": (c_int, []),
+    "wide_last_error": (ctypes.c_char_p, []),
     "wide_get_device_status": (c_int, [c_void_p, c_void_p]),
     "wide_clear_device_status": (c_int, [c_void_p]),
     "wide_profile_start": (c_int, [c_int32]),

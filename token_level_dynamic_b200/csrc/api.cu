@@ -3,6 +3,8 @@
 // per-device status word.  The kernels live in the other .cu files.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdio.h>
+#include <string.h>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -15,6 +17,19 @@
 __device__ int32_t g_wide_status;
 
 namespace wide {
+
+// Text of the calling thread's last CUDA failure (wide_last_error).
+thread_local char g_last_error[256] = "";
+
+int cuda_fail(const char *file, int line)
+{
+    const cudaError_t e = cudaGetLastError();
+    const char *base = strrchr(file, '/');
+    snprintf(g_last_error, sizeof g_last_error, "%s:%d: %s", base ? base + 1 : file, line,
+             e == cudaSuccess ? "a CUDA driver call failed (no runtime error recorded)"
+                              : cudaGetErrorString(e));
+    return WIDE_ECUDA;
+}
 
 int32_t *status_ptr()
 {
@@ -71,6 +86,23 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
         fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE,
            swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                      uint64_t pitch_elems, uint32_t box_chunks, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows == 0 || cols == 0 || cols % 64 != 0)
+        return false;
+    const cuuint64_t dims[3] = {64, cols / 64, rows};
+    const cuuint64_t strides[2] = {128, pitch_elems * 2};
+    const cuuint32_t box[3] = {64, box_chunks, box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r =
+        fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -204,14 +236,16 @@ const char *wide_status_string(int code)
 
 int wide_abi_version(void) { return WIDE_ABI_VERSION; }
 
+const char *wide_last_error(void) { return wide::g_last_error; }
+
 int wide_get_device_status(int32_t *h_status, void *stream)
 {
     if (!h_status)
         return WIDE_EINVAL;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     if (cudaMemcpyFromSymbol(h_status, g_wide_status, sizeof(int32_t)) != cudaSuccess)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     return WIDE_OK;
 }
 
@@ -219,11 +253,11 @@ int wide_clear_device_status(void *stream)
 {
     int32_t *p = status_ptr();
     if (!p)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     return cudaMemsetAsync(p, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)) ==
                    cudaSuccess
                ? WIDE_OK
-               : WIDE_ECUDA;
+               : WIDE_CUDA_FAIL();
 }
 
 size_t wide_worklist_bytes(int64_t T, int64_t G, int32_t tile_m)

@@ -371,16 +371,17 @@ int launch_cluster(int32_t kid, void (*kernel)(KArgs...), dim3 grid, dim3 block,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (!raise_smem_limit(reinterpret_cast<const void *>(kernel), smem))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     LaunchScope scope(kid, s);
     if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     return WIDE_OK;
 }
 
 struct DecodeWs {
     float *q, *o, *h1, *hffn;
     __nv_bfloat16 *xn2;
+    uint32_t *bar;
     size_t total;
 };
 
@@ -401,6 +402,7 @@ DecodeWs decode_ws(const wide_layer_dims *d, void *base)
     w.h1 = reinterpret_cast<float *>(take(T * (size_t)d->hidden * 4));
     w.hffn = reinterpret_cast<float *>(take(T * (size_t)d->inter * 4));
     w.xn2 = reinterpret_cast<__nv_bfloat16 *>(take(T * (size_t)d->hidden * 2));
+    w.bar = reinterpret_cast<uint32_t *>(take(256));
     w.total = off;
     return w;
 }
@@ -435,7 +437,7 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
     if (!make_tmap_2d(&tq, p.wq, qd, H, H, 2, kHD, 64, true) ||
         !make_tmap_2d(&tk, p.wk, (uint64_t)n_kv * kHD, H, H, 2, kHD, 64, true) ||
         !make_tmap_2d(&tv, p.wv, (uint64_t)n_kv * kHD, H, H, 2, kHD, 64, true))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     int KS = 8;
     while (KS > 1 && H % (KS * 64) != 0)
         KS >>= 1;
@@ -494,20 +496,30 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
     if (rc || !p.ffn)
         return rc;
 
-    // 4. FFN input norm
-    if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
-        return rc;
-
-    // 5-6. masked FFN; out = h1 + ffn_out
-    rc = decode_gateup_bf16(w.xn2, p.w_gate, p.w_up, p.ffn_mask, w.hffn, T, H, I,
-                            (int)d->ffn_group_size, s);
-    if (rc)
-        return rc;
+    // 4-6. FFN input norm and masked FFN; out = h1 + ffn_out
+    const int gsf = (int)d->ffn_group_size;
     DownOutputs fo = {};
     fo.out_sum = p.ffn_out;
     fo.res_f32 = w.h1;
     fo.out_total = p.out;
-    return decode_down_bf16(p.w_down, w.hffn, p.ffn_mask, fo, T, H, I, (int)d->ffn_group_size, s);
+    if (decode_ffn_fused_preferred(T, H, I, gsf)) {
+        // one persistent kernel: the norm is applied while x is staged
+        FusedInput in = {};
+        in.x_f32 = w.h1;
+        in.gamma = p.gamma2;
+        in.eps = d->eps;
+        in.w_gate = p.w_gate;
+        in.w_up = p.w_up;
+        in.w_down = p.w_down;
+        in.mask = p.ffn_mask;
+        return decode_ffn_fused(in, fo, T, H, I, gsf, w.hffn, w.bar, s);
+    }
+    if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
+        return rc;
+    rc = decode_gateup_bf16(w.xn2, p.w_gate, p.w_up, p.ffn_mask, w.hffn, T, H, I, gsf, s);
+    if (rc)
+        return rc;
+    return decode_down_bf16(p.w_down, w.hffn, p.ffn_mask, fo, T, H, I, gsf, s);
 }
 
 }  // namespace wide

@@ -385,7 +385,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
         !make_tmap_2d(&tvc, p.v_cache, kv_rows, kHD, kHD, 2, kBKV, 64, true) ||
         !make_tmap_2d(&to_a, w.o_sig, T, qd, qd, 2, 128, 64, true) ||
         !make_tmap_2d(&to_b, p.wo, H, qd, qd, 2, 256, 64, true))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     const float log2_theta = log2f(d->rope_theta);
     GemmArgs ga = {};
     ga.a = w.xn;
@@ -436,7 +436,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
     aa.o_sig = w.o_sig;
     aa.status = status_ptr();
     if (!raise_smem_limit(reinterpret_cast<const void *>(prefill_attn), kAttnSmem))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     {
         LaunchScope scope(KID_PREFILL_ATTN, s);
         const dim3 grid((unsigned)((d->seq_len + kBQ - 1) / kBQ), (unsigned)rep,

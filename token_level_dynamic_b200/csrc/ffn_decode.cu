@@ -506,10 +506,10 @@ int launch_cluster(int32_t kid, void (*kernel)(KArgs...), dim3 grid, dim3 block,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (!raise_smem_limit(reinterpret_cast<const void *>(kernel), smem))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     LaunchScope scope(kid, s);
     if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     return WIDE_OK;
 }
 
@@ -527,7 +527,7 @@ int gateup_chunk(const TIn *x, const TIn *wg, const TIn *wu, const uint32_t *mas
     CUtensorMap tg, tu;
     if (!make_tmap_2d(&tg, wg, I, H, H, sizeof(TIn), GS, KT, true) ||
         !make_tmap_2d(&tu, wu, I, H, H, sizeof(TIn), GS, KT, true))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     const int TB = T >= 4 ? 4 : (T >= 2 ? 2 : 1);
     const size_t TT = (size_t)((T + TB - 1) / TB * TB);
     const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 512 + TT * kslice * 4;
@@ -553,7 +553,7 @@ int down_chunk(const TIn *wd, const float *h, const uint32_t *mask, const DownOu
     CUtensorMap td, th;
     if (!make_tmap_2d(&td, wd, H, I, I, sizeof(TIn), kDownRows, KT, true) ||
         !make_tmap_2d(&th, h, T, I, I, 4, T, KT, false))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     const int KSd = G < 8 ? G : 8;
     const int TB = T >= 8 ? 8 : (T >= 4 ? 4 : (T >= 2 ? 2 : 1));
     const size_t hb = (size_t)((T + TB - 1) / TB * TB) * KT * 4;
@@ -638,33 +638,65 @@ int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const
     return WIDE_EUNSUPPORTED;
 }
 
-size_t ffn_decode_workspace(const wide_ffn_dims *d)
+size_t ffn_decode_h_bytes(const wide_ffn_dims *d)
 {
     const int64_t T = d->tokens < kNTok ? d->tokens : kNTok;
     return align_up((size_t)(T > 0 ? T : 1) * (size_t)d->inter * sizeof(float), 256);
+}
+
+// h scratch, then 256 bytes holding the fused kernel's grid-barrier words.
+size_t ffn_decode_workspace(const wide_ffn_dims *d) { return ffn_decode_h_bytes(d) + 256; }
+
+int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
+                   const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
+                   uint32_t *bar, cudaStream_t s)
+{
+    if (d->tokens == 0)
+        return WIDE_OK;
+    const int64_t gs = d->group_size;
+    if (d->dtype == WIDE_BF16) {
+        const int H = (int)d->hidden, I = (int)d->inter;
+        const int64_t T = d->tokens;
+        const int W = (int)((I / gs + 31) / 32);
+        if (decode_ffn_fused_preferred((int)(T < kNTok ? T : kNTok), H, I, (int)gs)) {
+            for (int64_t t0 = 0; t0 < T; t0 += kNTok) {
+                const int Tc = (int)(T - t0 < kNTok ? T - t0 : kNTok);
+                FusedInput in = {};
+                in.x = static_cast<const __nv_bfloat16 *>(x) + t0 * H;
+                in.w_gate = wg;
+                in.w_up = wu;
+                in.w_down = wd;
+                in.mask = mask + t0 * W;
+                DownOutputs o = {};
+                o.out_sum = static_cast<__nv_bfloat16 *>(out) + t0 * H;
+                const int rc = decode_ffn_fused(in, o, Tc, H, I, (int)gs, h, bar, s);
+                if (rc)
+                    return rc;
+            }
+            return WIDE_OK;
+        }
+        if (gs == 128)
+            return decode_all<__nv_bfloat16, 128>(x, wg, wu, wd, mask, out, d, h, s);
+        if (gs == 64)
+            return decode_all<__nv_bfloat16, 64>(x, wg, wu, wd, mask, out, d, h, s);
+    } else {
+        if (gs == 128)
+            return decode_all<float, 128>(x, wg, wu, wd, mask, out, d, h, s);
+        if (gs == 64)
+            return decode_all<float, 64>(x, wg, wu, wd, mask, out, d, h, s);
+        if (gs == 32)
+            return decode_all<float, 32>(x, wg, wu, wd, mask, out, d, h, s);
+    }
+    return WIDE_EUNSUPPORTED;
 }
 
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s)
 {
-    if (d->tokens == 0)
-        return WIDE_OK;
-    const int64_t gs = d->group_size;
-    if (d->dtype == WIDE_BF16) {
-        if (gs == 128)
-            return decode_all<__nv_bfloat16, 128>(x, wg, wu, wd, mask, out, d, ws, s);
-        if (gs == 64)
-            return decode_all<__nv_bfloat16, 64>(x, wg, wu, wd, mask, out, d, ws, s);
-    } else {
-        if (gs == 128)
-            return decode_all<float, 128>(x, wg, wu, wd, mask, out, d, ws, s);
-        if (gs == 64)
-            return decode_all<float, 64>(x, wg, wu, wd, mask, out, d, ws, s);
-        if (gs == 32)
-            return decode_all<float, 32>(x, wg, wu, wd, mask, out, d, ws, s);
-    }
-    return WIDE_EUNSUPPORTED;
+    char *base = static_cast<char *>(ws);
+    return ffn_decode_run(x, wg, wu, wd, mask, out, d, reinterpret_cast<float *>(base),
+                          reinterpret_cast<uint32_t *>(base + ffn_decode_h_bytes(d)), s);
 }
 
 }  // namespace wide

@@ -6,8 +6,9 @@
 // latency-critical loop where cudaMalloc/cudaFree would synchronise the
 // device.  This entry point runs the same decode kernels as
 // wide_ffn_masked's decode path, but keeps their scratch -- the fp32
-// intermediate h = silu(gate) * up of up to 32 tokens -- in the file-scope
-// device array below instead of a caller workspace.
+// intermediate h = silu(gate) * up of up to 32 tokens, and the two words of
+// the fused kernel's grid barrier -- in the file-scope device arrays below
+// instead of a caller workspace.
 //
 // The array is a module global: every GPU that loads the library holds
 // WIDE_NOALLOC_SCRATCH_BYTES of device memory for it until the process exits.
@@ -22,28 +23,34 @@
 #include "wide.h"
 
 static __device__ __align__(256) float g_noalloc_scratch[WIDE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+static __device__ __align__(256) uint32_t g_noalloc_bar[64];
 
 namespace wide {
 namespace {
 
-// Device address of this device's copy of g_noalloc_scratch.  In host code
-// the array's name is only a host-side stand-in, so the address is looked up
-// with cudaGetSymbolAddress once per device, with that device current.
-float *noalloc_scratch()
+// Device addresses of this device's copies of g_noalloc_scratch and
+// g_noalloc_bar.  In host code the arrays' names are only host-side
+// stand-ins, so the addresses are looked up with cudaGetSymbolAddress once
+// per device, with that device current.
+bool noalloc_arrays(float **scratch, uint32_t **bar)
 {
     static std::mutex mu;
-    static float *ptrs[64] = {};
+    static void *ptrs[64][2] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return nullptr;
+        return false;
     std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess)
-            return nullptr;
-        ptrs[dev] = static_cast<float *>(p);
+    if (!ptrs[dev][0]) {
+        void *p = nullptr, *q = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess ||
+            cudaGetSymbolAddress(&q, g_noalloc_bar) != cudaSuccess)
+            return false;
+        ptrs[dev][0] = p;
+        ptrs[dev][1] = q;
     }
-    return ptrs[dev];
+    *scratch = static_cast<float *>(ptrs[dev][0]);
+    *bar = static_cast<uint32_t *>(ptrs[dev][1]);
+    return true;
 }
 
 }  // namespace
@@ -68,11 +75,12 @@ extern "C" int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, co
     if (!aligned16(d_x) || !aligned16(d_w_gate) || !aligned16(d_w_up) || !aligned16(d_w_down) ||
         !aligned16(d_out))
         return WIDE_EUNSUPPORTED;
-    if (ffn_decode_workspace(d) > (size_t)WIDE_NOALLOC_SCRATCH_BYTES)
+    if (ffn_decode_h_bytes(d) > (size_t)WIDE_NOALLOC_SCRATCH_BYTES)
         return WIDE_ETOOLARGE;
-    float *scratch = noalloc_scratch();
-    if (!scratch)
-        return WIDE_ECUDA;
-    return ffn_decode_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d, scratch,
-                             static_cast<cudaStream_t>(stream));
+    float *scratch = nullptr;
+    uint32_t *bar = nullptr;
+    if (!noalloc_arrays(&scratch, &bar))
+        return WIDE_CUDA_FAIL();
+    return ffn_decode_run(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d, scratch, bar,
+                          static_cast<cudaStream_t>(stream));
 }

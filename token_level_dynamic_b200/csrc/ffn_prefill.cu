@@ -46,7 +46,7 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
         !make_tmap_2d(&tu, wu, I, H, H, 2, 128, 64, true) ||
         !make_tmap_2d(&th, hbuf, T, I, I, 2, kBM, 64, true) ||
         !make_tmap_2d(&td, wd, H, I, I, 2, 256, 64, true))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
 
     if ((rc = reorder_launch(mask, T, G, kBM, &wl, s)))
         return rc;

@@ -22,6 +22,15 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
                   uint64_t pitch_elems, uint32_t elem_bytes, uint32_t box_rows, uint32_t box_cols,
                   bool swizzle128);
 
+// Encodes a bf16 row-major matrix (`rows` x `cols`, row pitch `pitch_elems`,
+// cols % 64 == 0) as the 3-D tensor {64, cols / 64, rows}: a box
+// {64, box_chunks, box_rows} copies box_rows rows of 64 * box_chunks
+// consecutive elements each, landing as [box_rows][64 * box_chunks] in shared
+// memory (no swizzle).  Long rows per copy stream better than 2-D boxes of
+// short rows.
+bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                      uint64_t pitch_elems, uint32_t box_chunks, uint32_t box_rows);
+
 // Raises a kernel's dynamic shared memory limit to at least `bytes` (once
 // per kernel, device and size).
 bool raise_smem_limit(const void *kernel, size_t bytes);
@@ -30,12 +39,14 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Records "file:line: <last CUDA error>" as the calling thread's last error
+// (wide_last_error), clears the CUDA error and returns WIDE_ECUDA.
+int cuda_fail(const char *file, int line);
+#define WIDE_CUDA_FAIL() ::wide::cuda_fail(__FILE__, __LINE__)
+
 // Maps the last CUDA error to a WIDE code (and clears it).
-inline int launch_status()
-{
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? WIDE_OK : WIDE_ECUDA;
-}
+#define launch_status()                                                                            \
+    (cudaPeekAtLastError() == cudaSuccess ? WIDE_OK : WIDE_CUDA_FAIL())
 
 // Kernel ids reported by the profiler (wide_kernel_name).
 enum KernelId : int32_t {
@@ -53,6 +64,7 @@ enum KernelId : int32_t {
     KID_PREFILL_KV = 12,
     KID_PREFILL_ATTN = 13,
     KID_PREFILL_OPROJ = 14,
+    KID_DECODE_FFN_FUSED = 15,
 };
 
 // Pointers of one masked-layer call (FFN pointers unused when !ffn).
@@ -169,6 +181,31 @@ int decode_gateup_bf16(const void *x, const void *wg, const void *wu, const uint
                        float *h, int T, int H, int I, int gs, cudaStream_t s);
 int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const DownOutputs &o,
                      int T, int H, int I, int gs, cudaStream_t s);
+// Inputs of the fused decode FFN: the FFN input is either x (bf16 [T][H])
+// or x_f32 (fp32 [T][H] rows RMS-normalised with gamma and eps inside the
+// kernel, rounded to bf16 as a bf16 layer feeds its FFN).
+struct FusedInput {
+    const void *x;
+    const float *x_f32;
+    const void *gamma;
+    float eps;
+    const void *w_gate, *w_up, *w_down;
+    const uint32_t *mask;
+};
+// bf16 decode FFN of 1 <= T <= 32 tokens as one persistent cooperative
+// kernel (ffn_decode_fused.cu).  h: fp32 [T][I] scratch; bar: 2 words of
+// device memory for the grid barrier (the call zeroes bar[0] on the stream).
+bool decode_ffn_fused_supported(int T, int H, int I, int gs);
+// Whether the decode path should use it for this shape (faster there).
+bool decode_ffn_fused_preferred(int T, int H, int I, int gs);
+int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, int I, int gs,
+                     float *h, uint32_t *bar, cudaStream_t s);
+// Bytes of the fp32 h scratch of the decode path (tokens capped at 32).
+size_t ffn_decode_h_bytes(const wide_ffn_dims *d);
+// Runs the decode path with h scratch and grid-barrier words given apart.
+int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
+                   const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
+                   uint32_t *bar, cudaStream_t s);
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s);

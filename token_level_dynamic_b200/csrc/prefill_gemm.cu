@@ -692,7 +692,7 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
 {
     const int sms = num_sms();
     if (sms <= 0 || max_work < 0)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     if (max_work == 0)
         return WIDE_OK;
     const int grid = max_work < sms ? max_work : sms;
@@ -700,7 +700,7 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
                     : mode == GEMM_ROPE_Q ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROPE_Q>)
                                           : reinterpret_cast<const void *>(gather_gemm<GEMM_KV>);
     if (!raise_smem_limit(k, kSmemBytes))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     LaunchScope scope(kid, s);
     if (mode == GEMM_SWIGLU)
         gather_gemm<GEMM_SWIGLU><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
@@ -716,13 +716,13 @@ int tile_union_gemm_launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, con
 {
     const int sms = num_sms();
     if (sms <= 0)
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     const int64_t tiles = (int64_t)((a.T + kBM - 1) / kBM) * (a.N / kBN);
     if (tiles == 0)
         return WIDE_OK;
     const int grid = (int)(tiles < sms ? tiles : sms);
     if (!raise_smem_limit(reinterpret_cast<const void *>(tile_union_gemm), kSmemBytes))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     LaunchScope scope(kid, s);
     tile_union_gemm<<<grid, kThreadsDown, kSmemBytes, s>>>(tm_a, tm_b, a);
     return launch_status();

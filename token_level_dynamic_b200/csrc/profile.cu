@@ -57,7 +57,7 @@ int wide_profile_start(int32_t max_records)
     while ((int)g_pool.size() < max_records) {
         Record r{0, nullptr, nullptr};
         if (cudaEventCreate(&r.begin) != cudaSuccess || cudaEventCreate(&r.end) != cudaSuccess)
-            return WIDE_ECUDA;
+            return WIDE_CUDA_FAIL();
         g_pool.push_back(r);
     }
     g_used = 0;
@@ -79,10 +79,10 @@ int wide_profile_read(int32_t *kernel_ids, float *ms, int32_t max, int32_t *n)
     int k = 0;
     for (int i = 0; i < g_used && k < max; ++i) {
         if (cudaEventSynchronize(g_pool[i].end) != cudaSuccess)
-            return WIDE_ECUDA;
+            return WIDE_CUDA_FAIL();
         float t = 0.f;
         if (cudaEventElapsedTime(&t, g_pool[i].begin, g_pool[i].end) != cudaSuccess)
-            return WIDE_ECUDA;
+            return WIDE_CUDA_FAIL();
         kernel_ids[k] = g_pool[i].kid;
         ms[k] = t;
         ++k;
@@ -123,6 +123,8 @@ const char *wide_kernel_name(int32_t id)
         return "prefill_attention_tcgen05";
     case KID_PREFILL_OPROJ:
         return "prefill_oproj_tcgen05";
+    case KID_DECODE_FFN_FUSED:
+        return "decode_ffn_fused_gemv";
     default:
         return "?";
     }

@@ -205,7 +205,7 @@ int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
     const int tiles = (int)((T + kThreads - 1) / kThreads);
     const size_t smem = (size_t)2 * W * kThreads * sizeof(uint32_t);
     if (!raise_smem_limit(reinterpret_cast<const void *>(reorder_k1), smem))
-        return WIDE_ECUDA;
+        return WIDE_CUDA_FAIL();
     {
         LaunchScope scope(KID_REORDER_PARTITION_RANK, s);
         reorder_k1<<<(unsigned)(G + (int64_t)tiles * S), kThreads, smem, s>>>(
