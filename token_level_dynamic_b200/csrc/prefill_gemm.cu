@@ -14,8 +14,10 @@
 //              single-thread tcgen05.mma issuer
 //   warps 2-5  epilogue (warp w reads TMEM lanes 32 * (w % 4) .. +31)
 //   warps 6-7  row gather: 16-byte cp.async copies of the tile's token rows
-//              straight into the swizzled operand layout; each thread's copy
-//              completions arrive on the stage barrier
+//              straight into the swizzled operand layout, 8 consecutive lanes
+//              per 128-byte row piece so each warp instruction makes 4
+//              coalesced requests; each thread's copy completions arrive on
+//              the stage barrier
 //   modes
 //     SwiGLU  work item (g, i) of the FFN work list; B = [W_gate[g]; W_up[g]];
 //             epilogue h = silu(gate) * up, stored bf16 at the token's
@@ -62,6 +64,7 @@ struct __align__(8) Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int trow[2][kBM / 2]; // gather warp w: offsets of its rows' tokens (-1: none)
 };
 
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + sizeof(Ctl);
@@ -310,32 +313,39 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
         }
     } else if (warp >= 6) {
         // -------------------------------------------- token-row gather
-        const int p = threadIdx.x - 6 * 32;
+        // gather warp gw, lane l copies chunk l % 8 of rows 4 gw + l / 8 + 8 i
+        // (i < 16) of each stage: lanes 8j .. 8j+7 cover one 128-byte row
+        // piece.  Each warp looks up its own rows' tokens, so the two warps
+        // never wait for each other; wait results are made warp-uniform.
+        const int gw = warp - 6, lq = lane >> 3, cc = lane & 7;
+        const int lr = 4 * gw + lq;
+        int *trow = ctl->trow[gw];
         uint32_t stage = 0, phase = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
             const Work w = decode_work<MODE>(a, it);
-            const __nv_bfloat16 *src0 =
-                p < w.nrows ? a.a + (size_t)row_token<MODE>(a, w, p) * a.K : nullptr;
-            const __nv_bfloat16 *src1 =
-                p + 64 < w.nrows ? a.a + (size_t)row_token<MODE>(a, w, p + 64) * a.K : nullptr;
-            for (int kt = 0; kt < KT && ok; ++kt) {
-                if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, a.status)) {
+            __syncwarp();
+            for (int x = lane; x < kBM / 2; x += 32) {
+                const int r = (x >> 2) * 8 + 4 * gw + (x & 3);
+                trow[x] = r < w.nrows ? row_token<MODE>(a, w, r) * a.K : -1;
+            }
+            __syncwarp();
+            int off[kBM / 8];
+#pragma unroll
+            for (int i = 0; i < kBM / 8; ++i)
+                off[i] = trow[i * 4 + lq];
+            for (int kt = 0; kt < KT; ++kt) {
+                const bool got = wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, a.status);
+                if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
                 }
                 const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-                const int k0 = kt * kBK;
-                if (src0) {
+                const __nv_bfloat16 *src = a.a + kt * kBK + 8 * cc;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        cp_async16(sa + swz128(p, c), src0 + k0 + 8 * c);
-                }
-                if (src1) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        cp_async16(sa + swz128(p + 64, c), src1 + k0 + 8 * c);
-                }
+                for (int i = 0; i < kBM / 8; ++i)
+                    if (off[i] >= 0)
+                        cp_async16(sa + swz128(lr + 8 * i, cc), src + off[i]);
                 cp_async_arrive_noinc(&ctl->full[stage]);
                 if (++stage == kStages) {
                     stage = 0;
@@ -695,6 +705,8 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
         return WIDE_CUDA_FAIL();
     if (max_work == 0)
         return WIDE_OK;
+    if ((int64_t)a.T * a.K >= (int64_t)1 << 31)      // row offsets are 32-bit
+        return WIDE_EUNSUPPORTED;
     const int grid = max_work < sms ? max_work : sms;
     const void *k = mode == GEMM_SWIGLU ? reinterpret_cast<const void *>(gather_gemm<GEMM_SWIGLU>)
                     : mode == GEMM_ROPE_Q ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROPE_Q>)
