@@ -58,6 +58,7 @@ extern "C" {
 #define WIDE_DEV_BAD_MASK 0x1 /* a mask word had a bit at or above G set */
 #define WIDE_DEV_TIMEOUT 0x2  /* a bounded wait inside a kernel gave up */
 #define WIDE_DEV_BAD_ITEM 0x4 /* a work-list entry was out of range */
+#define WIDE_DEV_LAYOUT 0x8   /* a kernel's shared-memory alignment precondition failed */
 
 /* element types */
 #define WIDE_BF16 0

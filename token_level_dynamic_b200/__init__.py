@@ -21,7 +21,7 @@ from . import _native
 from ._native import (  # noqa: F401
     WIDE_OK, WIDE_EINVAL, WIDE_EUNSUPPORTED, WIDE_EWORKSPACE, WIDE_ECUDA, WIDE_ETOOLARGE,
     WIDE_NOALLOC_SCRATCH_BYTES,
-    WIDE_DEV_BAD_MASK, WIDE_DEV_TIMEOUT, WIDE_DEV_BAD_ITEM,
+    WIDE_DEV_BAD_MASK, WIDE_DEV_TIMEOUT, WIDE_DEV_BAD_ITEM, WIDE_DEV_LAYOUT,
     WIDE_BF16, WIDE_F32, WIDE_PATH_AUTO, WIDE_PATH_DECODE, WIDE_PATH_PREFILL,
     WideWorklist, WideFFNDims, WideLayerDims, WideLayerWeights,
 )

@@ -24,6 +24,7 @@ WIDE_NOALLOC_SCRATCH_BYTES = 2097152
 WIDE_DEV_BAD_MASK = 0x1
 WIDE_DEV_TIMEOUT = 0x2
 WIDE_DEV_BAD_ITEM = 0x4
+WIDE_DEV_LAYOUT = 0x8
 WIDE_BF16 = 0
 WIDE_F32 = 1
 WIDE_PATH_AUTO = 0

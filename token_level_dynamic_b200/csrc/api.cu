@@ -229,6 +229,8 @@ const char *wide_status_string(int code)
         return "device: bounded wait gave up";
     case WIDE_DEV_BAD_ITEM:
         return "device: work item out of range";
+    case WIDE_DEV_LAYOUT:
+        return "device: shared-memory alignment precondition failed";
     default:
         return code > 0 ? "device: several error bits" : "unknown status";
     }

@@ -10,15 +10,21 @@
 // range; skipped (token, group) pairs are never computed.
 //
 // prefill_attn: one CTA per (query tile, query head of the group, sequence x
-// KV head); 128 threads, thread r = query row r = TMEM lane r.  Per 128-key
-// tile up to the tile's last query position:
-//   S  = Q K^T           tcgen05, M=128 N=128 K=128, fp32 in TMEM columns 0..127
+// KV head); 128 threads, thread r = query row r = TMEM lane r; two CTAs per
+// SM (112 KB of shared memory and 256 TMEM columns each), so one CTA's
+// softmax overlaps the other's tensor-core work.  Per 64-key tile up to the
+// tile's last query position:
+//   S  = Q K^T           tcgen05, M=128 N=64 K=128, fp32 in one of two
+//                        64-column TMEM buffers; S of the next tile is issued
+//                        before this tile's softmax runs
 //   P  = online softmax of S with the causal mask (key position <= query
 //        position), exp2 domain, row max/sum and the O rescale in registers;
 //        P is written as bf16 to a 128B-swizzled K-major tile
 //   PV = P V             tcgen05, B = V read MN-major from the cache tile,
-//                        fp32 in TMEM columns 128..255, added to O (registers)
-// then O / l is written (bf16) at the token's signature-order row of the
+//                        fp32 in TMEM columns 128..255; read back (and added
+//                        to O in registers) during the next tile
+// K and V tiles are double-buffered and prefetched by TMA two tiles ahead.
+// Then O / l is written (bf16) at the token's signature-order row of the
 // o_proj input.  Tiles with no query (ragged counts) exit at once.
 #include "common.cuh"
 #include "host.h"
@@ -29,9 +35,12 @@ namespace {
 
 constexpr int kHD = 128;
 constexpr int kBQ = 128;       // queries per tile
-constexpr int kBKV = 128;      // keys per tile
-constexpr uint32_t kHalf = 128 * 128;   // one 64-column, 128-row swizzled sub-tile (16 KB)
-constexpr uint32_t kTile = 2 * kHalf;   // 128 x 128 bf16
+constexpr int kBKV = 64;       // keys per tile
+constexpr uint32_t kQHalf = 128 * 128;  // Q: one 64-column half, 128 rows (16 KB)
+constexpr uint32_t kQTile = 2 * kQHalf;
+constexpr uint32_t kKHalf = 64 * 128;   // K or V: one 64-column half, 64 rows (8 KB)
+constexpr uint32_t kKTile = 2 * kKHalf;
+constexpr uint32_t kPTile = 128 * 128;  // P: 128 rows x 64 keys (16 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnPArgs {
@@ -44,18 +53,18 @@ struct AttnPArgs {
 };
 
 struct __align__(8) ACtl {
-    uint64_t bar_q, bar_kv, bar_mma;
+    uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_pv;
     uint32_t tmem_base;
     int lo, nq, pmax;
 };
 
-constexpr size_t kAttnSmem = 1024 + 4 * kTile + sizeof(ACtl);
-
-__device__ __forceinline__ uint8_t *align1024(uint8_t *p)
-{
-    const uint32_t a = smem_u32(p);
-    return p + (((a + 1023u) & ~1023u) - a);
-}
+// Q | K[2] | V[2] | P | control.  No alignment slack: the kernel checks that
+// the dynamic shared memory starts 1024-byte aligned (it does when nothing
+// else is in shared memory) and reports WIDE_DEV_LAYOUT otherwise, so that
+// two CTAs fit one SM.
+constexpr uint32_t kOffK = kQTile, kOffV = kOffK + 2 * kKTile, kOffP = kOffV + 2 * kKTile;
+constexpr uint32_t kOffCtl = kOffP + kPTile;
+constexpr size_t kAttnSmem = kOffCtl + sizeof(ACtl);
 
 // first index i in [0, n) with v[i] >= key (v ascending)
 __device__ __forceinline__ int lower_bound(const int32_t *v, int n, int key)
@@ -71,15 +80,19 @@ __device__ __forceinline__ int lower_bound(const int32_t *v, int n, int key)
     return lo;
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
     prefill_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnPArgs a)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = align1024(smem_raw);
-    uint8_t *sq = smem, *sk = smem + kTile, *sv = smem + 2 * kTile, *sp = smem + 3 * kTile;
-    ACtl *ctl = reinterpret_cast<ACtl *>(smem + 4 * kTile);
+    extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5;
+    if (smem_u32(smem) & 1023u) {
+        if (tid == 0)
+            set_status(a.status, WIDE_DEV_LAYOUT);
+        return;
+    }
+    uint8_t *sq = smem, *sp = smem + kOffP;
+    ACtl *ctl = reinterpret_cast<ACtl *>(smem + kOffCtl);
     const int qt = blockIdx.x, hh = blockIdx.y;
     const int s = blockIdx.z / a.n_kv, j = blockIdx.z % a.n_kv;
     const int32_t *pj = a.perm + (size_t)j * a.T;
@@ -93,8 +106,12 @@ __global__ void __launch_bounds__(128, 1)
         const int last = min(hi - 1, lo + (qt + 1) * kBQ - 1);
         ctl->pmax = last >= lo ? pj[last] - s * a.seq_len : -1;
         mbar_init(&ctl->bar_q, 1);
-        mbar_init(&ctl->bar_kv, 1);
-        mbar_init(&ctl->bar_mma, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->bar_k[b], 1);
+            mbar_init(&ctl->bar_v[b], 1);
+            mbar_init(&ctl->bar_s[b], 1);
+        }
+        mbar_init(&ctl->bar_pv, 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -109,21 +126,70 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
-    const uint32_t t_s = tmem, t_pv = tmem + 128;
+    const uint32_t t_pv = tmem + 128;             // S buffers at columns 0 and 64
 
     const int nvalid = min(kBQ, nq - qt * kBQ);
-    const int idx = lo + qt * kBQ + tid;                       // row of this thread
+    const int idx = lo + qt * kBQ + tid;          // row of this thread
     const bool live = tid < nvalid;
     const int tok = live ? pj[idx] : 0;
     const int pos = live ? tok - s * a.seq_len : -1;
     const int64_t kvrow0 = ((int64_t)s * a.n_kv + j) * a.cache_cap;
     const int nkt = pmax / kBKV + 1;
+    constexpr uint32_t idesc_s = umma::idesc_bf16_f32(kBQ, kBKV);
+    constexpr uint32_t idesc_pv = umma::idesc_bf16_f32_bmn(kBQ, kHD);
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // loads and PV commits issued (thread 0), to drain them after an error
+    int nk[2] = {0, 0}, nv[2] = {0, 0}, npv = 0;
 
+    auto load_k = [&](int t) {
+        ++nk[t & 1];
+        uint8_t *dst = smem + kOffK + (t & 1) * kKTile;
+        const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
+        mbar_arrive_expect_tx(&ctl->bar_k[t & 1], kKTile);
+        tma_load_2d(dst, &tm_k, 0, krow, &ctl->bar_k[t & 1]);
+        tma_load_2d(dst + kKHalf, &tm_k, 64, krow, &ctl->bar_k[t & 1]);
+    };
+    auto load_v = [&](int t) {
+        ++nv[t & 1];
+        uint8_t *dst = smem + kOffV + (t & 1) * kKTile;
+        const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
+        mbar_arrive_expect_tx(&ctl->bar_v[t & 1], kKTile);
+        tma_load_2d(dst, &tm_v, 0, krow, &ctl->bar_v[t & 1]);
+        tma_load_2d(dst + kKHalf, &tm_v, 64, krow, &ctl->bar_v[t & 1]);
+    };
+    // S(t) = Q K(t)^T into S buffer t & 1 (one thread)
+    auto issue_s = [&](int t) {
+        umma::fence_after_sync();
+        const uint32_t q0 = smem_u32(sq), k0 = smem_u32(smem + kOffK + (t & 1) * kKTile);
+#pragma unroll
+        for (int k = 0; k < kHD / 16; ++k) {
+            const uint32_t qo = (uint32_t)(k >> 2) * kQHalf + (uint32_t)(k & 3) * 32u;
+            const uint32_t ko = (uint32_t)(k >> 2) * kKHalf + (uint32_t)(k & 3) * 32u;
+            umma::mma_bf16(tmem + (uint32_t)(t & 1) * kBKV, umma::desc_kmajor_sw128(q0 + qo),
+                           umma::desc_kmajor_sw128(k0 + ko), idesc_s, k != 0);
+        }
+        umma::commit(&ctl->bar_s[t & 1]);
+    };
+
+    bool ok = true;
     if (tid == 0) {
-        mbar_arrive_expect_tx(&ctl->bar_q, kTile);
+        mbar_arrive_expect_tx(&ctl->bar_q, kQTile);
         const int qrow = j * a.T + lo + qt * kBQ;
         tma_load_2d(sq, &tm_q, hh * kHD, qrow, &ctl->bar_q);
-        tma_load_2d(sq + kHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
+        tma_load_2d(sq + kQHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
+        for (int t = 0; t < 2 && t < nkt; ++t) {
+            load_k(t);
+            load_v(t);
+        }
+        if (!mbar_wait(&ctl->bar_q, 0) || !mbar_wait(&ctl->bar_k[0], 0))
+            ok = false;
+        else
+            issue_s(0);
+    }
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0)
+            set_status(a.status, WIDE_DEV_TIMEOUT);
+        ok = false;
     }
 
     float o[kHD];
@@ -131,74 +197,42 @@ __global__ void __launch_bounds__(128, 1)
     for (int d = 0; d < kHD; ++d)
         o[d] = 0.f;
     float m = -INFINITY, l = 0.f;
-    uint32_t mma_phase = 0, kv_phase = 0;
-    bool ok = true;
-    constexpr uint32_t idesc_s = umma::idesc_bf16_f32(kBQ, kBKV);
-    constexpr uint32_t idesc_pv = umma::idesc_bf16_f32_bmn(kBQ, kHD);
+
+    // O += PV of the previous tile (TMEM -> registers)
+    auto add_pv = [&]() {
+#pragma unroll
+        for (int c = 0; c < kHD / 32; ++c) {
+            float v[32];
+            umma::tmem_ld32(t_pv + lane_off + c * 32, v);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                o[c * 32 + e] += v[e];
+        }
+    };
 
     for (int kt = 0; kt < nkt && ok; ++kt) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&ctl->bar_kv, 2 * kTile);
-            const int krow = (int)(kvrow0 + (int64_t)kt * kBKV);
-            tma_load_2d(sk, &tm_k, 0, krow, &ctl->bar_kv);
-            tma_load_2d(sk + kHalf, &tm_k, 64, krow, &ctl->bar_kv);
-            tma_load_2d(sv, &tm_v, 0, krow, &ctl->bar_kv);
-            tma_load_2d(sv + kHalf, &tm_v, 64, krow, &ctl->bar_kv);
-        }
-        if (!mbar_wait(&ctl->bar_kv, kv_phase)) {
-            set_status(a.status, WIDE_DEV_TIMEOUT);
-            ok = false;
-        }
-        kv_phase ^= 1u;
-        if (__syncthreads_or(!ok)) {
-            ok = false;
-            break;
-        }
-        // keys past the sequence's last position may be uninitialised cache
-        // memory: clear those V rows so that 0 * garbage cannot reach P V
-        {
-            const int kmax = a.seq_len - 1 - kt * kBKV;      // last valid key row in tile
-            if (kmax < kBKV - 1) {
-                for (int rr = max(kmax + 1, 0) + warp; rr < kBKV; rr += 4)
-                    for (int c = (tid & 31); c < 16; c += 32) {
-                        const int sub = c >> 3, ch = c & 7;
-                        *reinterpret_cast<uint4 *>(sv + sub * kHalf + rr * 128 + ch * 16) =
-                            make_uint4(0u, 0u, 0u, 0u);
-                    }
-                fence_proxy_async_smem();
-                __syncthreads();
+        const int b = kt & 1;
+        const uint32_t par = (uint32_t)(kt >> 1) & 1u;
+        bool w_ok = mbar_wait(&ctl->bar_s[b], par);          // S(kt) done; K(b) free
+        if (tid == 0 && w_ok) {
+            if (kt + 1 < nkt) {
+                if (mbar_wait(&ctl->bar_k[b ^ 1], (uint32_t)((kt + 1) >> 1) & 1u))
+                    issue_s(kt + 1);
+                else
+                    w_ok = false;
             }
+            if (kt + 2 < nkt)
+                load_k(kt + 2);
         }
-        // S = Q K^T
-        if (tid == 0) {
-            if (kt == 0 && !mbar_wait(&ctl->bar_q, 0)) {
-                set_status(a.status, WIDE_DEV_TIMEOUT);
-                ok = false;
-            }
-            umma::fence_after_sync();
-            const uint32_t q0 = smem_u32(sq), k0 = smem_u32(sk);
-#pragma unroll
-            for (int k = 0; k < kHD / 16; ++k) {
-                const uint32_t off = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
-                umma::mma_bf16(t_s, umma::desc_kmajor_sw128(q0 + off),
-                               umma::desc_kmajor_sw128(k0 + off), idesc_s, k != 0);
-            }
-            umma::commit(&ctl->bar_mma);
-        }
-        if (!mbar_wait(&ctl->bar_mma, mma_phase)) {
-            set_status(a.status, WIDE_DEV_TIMEOUT);
-            ok = false;
-        }
-        mma_phase ^= 1u;
         umma::fence_after_sync();
-        // online softmax of this thread's row (two passes over TMEM: the
-        // row max, then the probabilities); P row -> swizzled smem
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // pass 1: the row max of this tile
+        const uint32_t ts = tmem + (uint32_t)b * kBKV + lane_off;
         float mt = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < kBKV / 32; ++c) {
             float v[32];
-            umma::tmem_ld32(t_s + lane_off + c * 32, v);
+            umma::tmem_ld32(ts + c * 32, v);
             umma::tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
@@ -209,11 +243,25 @@ __global__ void __launch_bounds__(128, 1)
         }
         const float mn = fmaxf(m, mt);
         const float alpha = (live && m > -INFINITY) ? exp2f(m - mn) : (live ? 0.f : 1.f);
+        // the previous tile's P V is done: add it (P and V(b^1) are free)
+        if (kt > 0) {
+            w_ok = w_ok && mbar_wait(&ctl->bar_pv, (uint32_t)(kt - 1) & 1u);
+            umma::fence_after_sync();
+            add_pv();
+            if (tid == 0 && kt + 1 < nkt)
+                load_v(kt + 1);
+        }
+        if (live) {
+#pragma unroll
+            for (int d = 0; d < kHD; ++d)
+                o[d] *= alpha;
+        }
+        // pass 2: probabilities -> P (bf16, swizzled K-major)
         float lsum = 0.f;
 #pragma unroll 1
         for (int c = 0; c < kBKV / 32; ++c) {
             float v[32];
-            umma::tmem_ld32(t_s + lane_off + c * 32, v);
+            umma::tmem_ld32(ts + c * 32, v);
             umma::tmem_ld_wait();
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
@@ -228,9 +276,7 @@ __global__ void __launch_bounds__(128, 1)
                 __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
                 __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
                 __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
-                const int chunk = c * 4 + g8;            // 16-byte chunk of the 256-byte row
-                const int sub = chunk >> 3, ch = chunk & 7;
-                *reinterpret_cast<uint4 *>(sp + sub * kHalf + swz128(tid, ch)) = make_uint4(
+                *reinterpret_cast<uint4 *>(sp + swz128(tid, c * 4 + g8)) = make_uint4(
                     *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
                     *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
             }
@@ -238,47 +284,53 @@ __global__ void __launch_bounds__(128, 1)
         if (live) {
             l = l * alpha + lsum;
             m = mn;
-#pragma unroll
-            for (int d = 0; d < kHD; ++d)
-                o[d] *= alpha;
         }
-        fence_proxy_async_smem();       // P written by threads, read by the tensor core
-        umma::fence_before_sync();
-        __syncthreads();
-        // PV = P V
-        if (tid == 0 && ok) {
-            umma::fence_after_sync();
-            const uint32_t p0 = smem_u32(sp), v0 = smem_u32(sv);
-#pragma unroll
-            for (int k = 0; k < kBKV / 16; ++k) {
-                const uint32_t aoff = (uint32_t)(k >> 2) * kHalf + (uint32_t)(k & 3) * 32u;
-                const uint32_t boff = (uint32_t)k * 16u * 128u;   // 16 key rows
-                umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
-                               umma::desc_mnmajor_sw128(v0 + boff, kHalf), idesc_pv, k != 0);
+        // V(kt) must have landed; keys past the sequence's end may be
+        // uninitialised cache memory: clear those V rows so that 0 * garbage
+        // cannot reach P V
+        w_ok = w_ok && mbar_wait(&ctl->bar_v[b], par);
+        {
+            const int kmax = a.seq_len - 1 - kt * kBKV;       // last valid key row in tile
+            if (kmax < kBKV - 1) {
+                uint8_t *sv = smem + kOffV + b * kKTile;
+                for (int rr = max(kmax + 1, 0) + warp; rr < kBKV; rr += 4)
+                    for (int c = (tid & 31); c < 16; c += 32) {
+                        const int sub = c >> 3, ch = c & 7;
+                        *reinterpret_cast<uint4 *>(sv + sub * kKHalf + rr * 128 + ch * 16) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                    }
             }
-            umma::commit(&ctl->bar_mma);
         }
-        if (!mbar_wait(&ctl->bar_mma, mma_phase)) {
-            set_status(a.status, WIDE_DEV_TIMEOUT);
-            ok = false;
-        }
-        mma_phase ^= 1u;
-        umma::fence_after_sync();
-#pragma unroll
-        for (int c = 0; c < kHD / 32; ++c) {
-            float v[32];
-            umma::tmem_ld32(t_pv + lane_off + c * 32, v);
-            umma::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-                o[c * 32 + e] += v[e];
-        }
+        fence_proxy_async_smem();       // P (and cleared V rows) written by threads
         umma::fence_before_sync();
-        // all TMEM reads are done before the next tile's MMAs; a failed wait
-        // anywhere ends the loop for every thread together
-        if (__syncthreads_or(!ok)) {
+        if (__syncthreads_or(!w_ok)) {
+            if (tid == 0)
+                set_status(a.status, WIDE_DEV_TIMEOUT);
             ok = false;
             break;
+        }
+        // PV = P V(kt)
+        if (tid == 0) {
+            umma::fence_after_sync();
+            const uint32_t p0 = smem_u32(sp), v0 = smem_u32(smem + kOffV + b * kKTile);
+#pragma unroll
+            for (int k = 0; k < kBKV / 16; ++k) {
+                const uint32_t aoff = (uint32_t)k * 32u;              // 16 keys of the P row
+                const uint32_t boff = (uint32_t)k * 16u * 128u;       // 16 key rows of V
+                umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
+                               umma::desc_mnmajor_sw128(v0 + boff, kKHalf), idesc_pv, k != 0);
+            }
+            umma::commit(&ctl->bar_pv);
+            ++npv;
+        }
+    }
+    if (ok) {
+        if (!mbar_wait(&ctl->bar_pv, (uint32_t)(nkt - 1) & 1u)) {
+            set_status(a.status, WIDE_DEV_TIMEOUT);
+            ok = false;
+        } else {
+            umma::fence_after_sync();
+            add_pv();
         }
     }
 
@@ -296,6 +348,18 @@ __global__ void __launch_bounds__(128, 1)
                 make_uint4(*reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
                            *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
         }
+    }
+    // after an error, let this CTA's copies and MMAs in flight land before
+    // the shared memory and TMEM are released
+    if (!ok && tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            if (nk[b] > 0)
+                mbar_wait(&ctl->bar_k[b], (uint32_t)(nk[b] - 1) & 1u);
+            if (nv[b] > 0)
+                mbar_wait(&ctl->bar_v[b], (uint32_t)(nv[b] - 1) & 1u);
+        }
+        umma::commit(&ctl->bar_pv);         // completes after every MMA issued so far
+        mbar_wait(&ctl->bar_pv, (uint32_t)npv & 1u);
     }
     umma::fence_before_sync();
     __syncthreads();

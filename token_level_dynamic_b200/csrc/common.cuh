@@ -79,18 +79,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (not spinning, so it
+// takes no issue slots from other warps) until the phase completes or
+// kSuspendNs elapse.
+constexpr uint32_t kSuspendNs = 1000000;   // 1 ms
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Returns false if
 // it has not completed after kWaitLimitNs (the caller then reports
-// WIDE_DEV_TIMEOUT and winds down instead of spinning for ever).
+// WIDE_DEV_TIMEOUT and winds down instead of waiting for ever).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity))
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity))
             return true;
-        if ((it & 255u) == 0 && globaltimer() - t0 > kWaitLimitNs)
+        if (globaltimer() - t0 > kWaitLimitNs)
             return false;
     }
 }

@@ -81,17 +81,15 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Ct
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity))
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity))
             return true;
-        if ((it & 255u) == 0) {
-            if (*(volatile int *)&ctl->abort)
-                return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
-                set_status(status, WIDE_DEV_TIMEOUT);
-                *(volatile int *)&ctl->abort = 1;
-                return false;
-            }
+        if (*(volatile int *)&ctl->abort)
+            return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            set_status(status, WIDE_DEV_TIMEOUT);
+            *(volatile int *)&ctl->abort = 1;
+            return false;
         }
     }
 }
