@@ -18,11 +18,15 @@
 //                        64-column TMEM buffers; S of the next tile is issued
 //                        before this tile's softmax runs
 //   P  = online softmax of S with the causal mask (key position <= query
-//        position), exp2 domain, row max/sum and the O rescale in registers;
-//        P is written as bf16 to a 128B-swizzled K-major tile
-//   PV = P V             tcgen05, B = V read MN-major from the cache tile,
-//                        fp32 in TMEM columns 128..255; read back (and added
-//                        to O in registers) during the next tile
+//        position; tiles wholly below the diagonal skip the test), exp2
+//        domain; P is written as bf16 to a 128B-swizzled K-major tile
+//   O += P V             tcgen05, B = V read MN-major from the cache tile,
+//                        O accumulated in TMEM columns 128..255 across tiles.
+//        Each row keeps its reference max m_ref: P = exp2(s - m_ref) as long
+//        as the row's running max stays within 8 (log2 units) of m_ref, so
+//        P <= 256; when it grows further the row's O and sum are rescaled
+//        (TMEM load, multiply, store) and m_ref moves up.  Rescales are rare
+//        after the first tiles, so O never passes through registers per tile.
 // K and V tiles are double-buffered and prefetched by TMA two tiles ahead.
 // Then O / l is written (bf16) at the token's signature-order row of the
 // o_proj input.  Tiles with no query (ragged counts) exit at once.
@@ -192,24 +196,8 @@ __global__ void __launch_bounds__(128, 2)
         ok = false;
     }
 
-    float o[kHD];
-#pragma unroll
-    for (int d = 0; d < kHD; ++d)
-        o[d] = 0.f;
-    float m = -INFINITY, l = 0.f;
-
-    // O += PV of the previous tile (TMEM -> registers)
-    auto add_pv = [&]() {
-#pragma unroll
-        for (int c = 0; c < kHD / 32; ++c) {
-            float v[32];
-            umma::tmem_ld32(t_pv + lane_off + c * 32, v);
-            umma::tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-                o[c * 32 + e] += v[e];
-        }
-    };
+    float m_ref = -INFINITY, l = 0.f;     // row reference max (log2 units), sum
+    const float sc = a.scale_log2;
 
     for (int kt = 0; kt < nkt && ok; ++kt) {
         const int b = kt & 1;
@@ -226,65 +214,71 @@ __global__ void __launch_bounds__(128, 2)
                 load_k(kt + 2);
         }
         umma::fence_after_sync();
-        // pass 1: the row max of this tile
+        // this row's 64 scores of the tile
         const uint32_t ts = tmem + (uint32_t)b * kBKV + lane_off;
-        float mt = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kBKV / 32; ++c) {
-            float v[32];
-            umma::tmem_ld32(ts + c * 32, v);
-            umma::tmem_ld_wait();
+        float v[kBKV];
+        umma::tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&v[0]));
+        umma::tmem_ld32(ts + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        umma::tmem_ld_wait();
+        const int k0 = kt * kBKV;
+        const bool full = live && k0 + kBKV - 1 <= pos;       // no key of the tile masked
+        if (!full) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int kp = kt * kBKV + c * 32 + e;
-                if (live && kp <= pos)
-                    mt = fmaxf(mt, v[e] * a.scale_log2);
-            }
+            for (int e = 0; e < kBKV; ++e)
+                if (!(live && k0 + e <= pos))
+                    v[e] = -INFINITY;
         }
-        const float mn = fmaxf(m, mt);
-        const float alpha = (live && m > -INFINITY) ? exp2f(m - mn) : (live ? 0.f : 1.f);
-        // the previous tile's P V is done: add it (P and V(b^1) are free)
+        float vmax = v[0];
+#pragma unroll
+        for (int e = 1; e < kBKV; ++e)
+            vmax = fmaxf(vmax, v[e]);
+        const float mt = vmax * sc;                           // -inf if no key is visible
+        // the previous tile's P V is done: P and V(b^1) are free
         if (kt > 0) {
             w_ok = w_ok && mbar_wait(&ctl->bar_pv, (uint32_t)(kt - 1) & 1u);
             umma::fence_after_sync();
-            add_pv();
             if (tid == 0 && kt + 1 < nkt)
                 load_v(kt + 1);
         }
-        if (live) {
-#pragma unroll
-            for (int d = 0; d < kHD; ++d)
-                o[d] *= alpha;
+        // move the reference max when the running max passes it by > 8
+        float alpha = 1.f;
+        if (mt > m_ref + 8.f) {
+            alpha = kt > 0 ? exp2f(m_ref - mt) : 0.f;
+            m_ref = mt;
         }
-        // pass 2: probabilities -> P (bf16, swizzled K-major)
-        float lsum = 0.f;
+        if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-        for (int c = 0; c < kBKV / 32; ++c) {
-            float v[32];
-            umma::tmem_ld32(ts + c * 32, v);
-            umma::tmem_ld_wait();
+            for (int c = 0; c < kHD / 32; ++c) {
+                float ov[32];
+                umma::tmem_ld32(t_pv + lane_off + c * 32, ov);
+                umma::tmem_ld_wait();
 #pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-                float p[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int kp = kt * kBKV + c * 32 + g8 * 8 + e;
-                    p[e] = (live && kp <= pos) ? exp2f(v[g8 * 8 + e] * a.scale_log2 - mn) : 0.f;
-                    lsum += p[e];
-                }
-                __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]);
-                __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
-                __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
-                *reinterpret_cast<uint4 *>(sp + swz128(tid, c * 4 + g8)) = make_uint4(
-                    *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
-                    *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
+                for (int e = 0; e < 32; ++e)
+                    ov[e] *= alpha;
+                umma::tmem_st32(t_pv + lane_off + c * 32, ov);
             }
+            umma::tmem_st_wait();
         }
-        if (live) {
-            l = l * alpha + lsum;
-            m = mn;
+        // probabilities -> P (bf16, swizzled K-major); masked keys give 0
+        const float mb = m_ref > -INFINITY ? m_ref : 0.f;
+        float lsum = 0.f;
+#pragma unroll
+        for (int g8 = 0; g8 < kBKV / 8; ++g8) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                p[e] = exp2f(fmaf(v[g8 * 8 + e], sc, -mb));
+                lsum += p[e];
+            }
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]);
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
+            __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
+            *reinterpret_cast<uint4 *>(sp + swz128(tid, g8)) = make_uint4(
+                *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
         }
+        l = l * alpha + lsum;
         // V(kt) must have landed; keys past the sequence's end may be
         // uninitialised cache memory: clear those V rows so that 0 * garbage
         // cannot reach P V
@@ -309,7 +303,7 @@ __global__ void __launch_bounds__(128, 2)
             ok = false;
             break;
         }
-        // PV = P V(kt)
+        // O += P V(kt)
         if (tid == 0) {
             umma::fence_after_sync();
             const uint32_t p0 = smem_u32(sp), v0 = smem_u32(smem + kOffV + b * kKTile);
@@ -318,35 +312,48 @@ __global__ void __launch_bounds__(128, 2)
                 const uint32_t aoff = (uint32_t)k * 32u;              // 16 keys of the P row
                 const uint32_t boff = (uint32_t)k * 16u * 128u;       // 16 key rows of V
                 umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
-                               umma::desc_mnmajor_sw128(v0 + boff, kKHalf), idesc_pv, k != 0);
+                               umma::desc_mnmajor_sw128(v0 + boff, kKHalf), idesc_pv,
+                               (kt | k) != 0);
             }
             umma::commit(&ctl->bar_pv);
             ++npv;
         }
     }
-    if (ok) {
-        if (!mbar_wait(&ctl->bar_pv, (uint32_t)(nkt - 1) & 1u)) {
-            set_status(a.status, WIDE_DEV_TIMEOUT);
+    if (ok) {   // ok is uniform here; keep it so (the TMEM loads below are warp-collective)
+        const bool fin = mbar_wait(&ctl->bar_pv, (uint32_t)(nkt - 1) & 1u);
+        if (__syncthreads_or(!fin)) {
+            if (tid == 0)
+                set_status(a.status, WIDE_DEV_TIMEOUT);
             ok = false;
-        } else {
-            umma::fence_after_sync();
-            add_pv();
         }
     }
+    umma::fence_after_sync();
 
-    if (live && ok) {
-        const float inv = 1.f / l;
-        __nv_bfloat16 *dst = a.o_sig + (size_t)a.sig_pos[tok] * a.ocols +
+    if (ok) {
+        // O / l, all warps (the TMEM loads are warp-collective)
+        const float inv = live ? 1.f / l : 0.f;
+        __nv_bfloat16 *dst = a.o_sig + (size_t)(live ? a.sig_pos[tok] : 0) * a.ocols +
                              (size_t)(j * a.rep + hh) * kHD;
+#pragma unroll 1
+        for (int c = 0; c < kHD / 32; ++c) {
+            float ov[32];
+            umma::tmem_ld32(t_pv + lane_off + c * 32, ov);
+            umma::tmem_ld_wait();
+            if (live) {
 #pragma unroll
-        for (int c = 0; c < kHD / 8; ++c) {
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(o[c * 8] * inv, o[c * 8 + 1] * inv);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(o[c * 8 + 2] * inv, o[c * 8 + 3] * inv);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(o[c * 8 + 4] * inv, o[c * 8 + 5] * inv);
-            __nv_bfloat162 b3 = __floats2bfloat162_rn(o[c * 8 + 6] * inv, o[c * 8 + 7] * inv);
-            reinterpret_cast<uint4 *>(dst)[c] =
-                make_uint4(*reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
-                           *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
+                for (int q = 0; q < 4; ++q) {
+                    __nv_bfloat162 b0 = __floats2bfloat162_rn(ov[q * 8] * inv, ov[q * 8 + 1] * inv);
+                    __nv_bfloat162 b1 =
+                        __floats2bfloat162_rn(ov[q * 8 + 2] * inv, ov[q * 8 + 3] * inv);
+                    __nv_bfloat162 b2 =
+                        __floats2bfloat162_rn(ov[q * 8 + 4] * inv, ov[q * 8 + 5] * inv);
+                    __nv_bfloat162 b3 =
+                        __floats2bfloat162_rn(ov[q * 8 + 6] * inv, ov[q * 8 + 7] * inv);
+                    reinterpret_cast<uint4 *>(dst + c * 32)[q] = make_uint4(
+                        *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                        *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
+                }
+            }
         }
     }
     // after an error, let this CTA's copies and MMAs in flight land before
