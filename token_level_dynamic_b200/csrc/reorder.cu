@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(kThreads)
                int32_t *status)
 {
     __shared__ int warp_act[kWarps], warp_val[kWarps];
-    extern __shared__ uint32_t dyn_keys[];  // [2][W][kThreads]
+    extern __shared__ __align__(16) uint32_t dyn_keys[];  // [2][W][kThreads], or uint4[kThreads]
     uint32_t *ukeys = dyn_keys, *tkeys = dyn_keys + W * kThreads;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
 
@@ -103,6 +103,39 @@ __global__ void __launch_bounds__(kThreads)
             set_status(status, WIDE_DEV_BAD_MASK);
     }
     int less = 0;
+    if (W <= 4) {
+        // keys of up to 128 bits: the slice's keys as uint4 in shared memory
+        // (one broadcast load per comparison), this token's key in registers,
+        // compared as two 64-bit halves (word W-1 most significant)
+        uint4 *uk4 = reinterpret_cast<uint4 *>(dyn_keys);
+        uint32_t tw[4] = {0u, 0u, 0u, 0u};
+        if (t < T)
+            for (int ww = 0; ww < W; ++ww)
+                tw[ww] = mask[(size_t)t * W + ww];
+        const uint64_t th = ((uint64_t)tw[3] << 32) | tw[2], tl = ((uint64_t)tw[1] << 32) | tw[0];
+        for (int ub = u0; ub < u1; ub += kThreads) {
+            __syncthreads();
+            {
+                const int u = ub + tid;
+                uint32_t kw[4] = {0u, 0u, 0u, 0u};
+                if (u < u1)
+                    for (int ww = 0; ww < W; ++ww)
+                        kw[ww] = mask[(size_t)u * W + ww];
+                uk4[tid] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+            }
+            __syncthreads();
+            const int n = min(kThreads, u1 - ub);
+#pragma unroll 4
+            for (int j = 0; j < n; ++j) {
+                const uint4 k = uk4[j];
+                const uint64_t uh = ((uint64_t)k.w << 32) | k.z, ul = ((uint64_t)k.y << 32) | k.x;
+                less += (uh < th) | ((uh == th) & ((ul < tl) | ((ul == tl) & (ub + j < t))));
+            }
+        }
+        if (t < T)
+            scratch[(size_t)s * T + t] = less;
+        return;
+    }
     for (int ub = u0; ub < u1; ub += kThreads) {
         __syncthreads();
         for (int idx = tid; idx < kThreads * W; idx += kThreads) {
@@ -203,7 +236,9 @@ int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
     const int W = (int)((G + 31) / 32);
     const int S = wl->scratch_splits;
     const int tiles = (int)((T + kThreads - 1) / kThreads);
-    const size_t smem = (size_t)2 * W * kThreads * sizeof(uint32_t);
+    // [2][W][kThreads] words (the keys of the generic path; the prologue
+    // writes this token's key there for every W), at least uint4[kThreads]
+    const size_t smem = (size_t)(2 * W > 4 ? 2 * W : 4) * kThreads * sizeof(uint32_t);
     if (!raise_smem_limit(reinterpret_cast<const void *>(reorder_k1), smem))
         return WIDE_CUDA_FAIL();
     {
