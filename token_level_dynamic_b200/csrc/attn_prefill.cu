@@ -10,10 +10,12 @@
 // range; skipped (token, group) pairs are never computed.
 //
 // prefill_attn: one CTA per (query tile, query head of the group, sequence x
-// KV head); 128 threads, thread r = query row r = TMEM lane r; two CTAs per
-// SM (112 KB of shared memory and 256 TMEM columns each), so one CTA's
-// softmax overlaps the other's tensor-core work.  Per 64-key tile up to the
-// tile's last query position:
+// KV head); warps 0-3 run the softmax (thread r = query row r = TMEM lane r),
+// warp 4 issues every TMA copy and tensor-core MMA; two CTAs per SM (112 KB
+// of shared memory and 256 TMEM columns each).  The warps hand work over
+// through mbarriers only (no block-wide barrier inside the loop), so the
+// softmax never waits for the issuer except for data.  Per 64-key tile up to
+// the tile's last query position:
 //   S  = Q K^T           tcgen05, M=128 N=64 K=128, fp32 in one of two
 //                        64-column TMEM buffers; S of the next tile is issued
 //                        before this tile's softmax runs
@@ -58,9 +60,14 @@ struct AttnPArgs {
 
 struct __align__(8) ACtl {
     uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_pv;
+    uint64_t s_free[2];   // softmax warps have read S buffer b (4 warp arrivals)
+    uint64_t p_full;      // softmax warps wrote P and rescaled O (4 warp arrivals)
     uint32_t tmem_base;
     int lo, nq, pmax;
+    int abort;
 };
+constexpr int kSoftWarps = 4;
+constexpr int kAttnThreads = 32 * (kSoftWarps + 1);
 
 // Q | K[2] | V[2] | P | control.  No alignment slack: the kernel checks that
 // the dynamic shared memory starts 1024-byte aligned (it does when nothing
@@ -84,12 +91,33 @@ __device__ __forceinline__ int lower_bound(const int32_t *v, int n, int key)
     return lo;
 }
 
-__global__ void __launch_bounds__(128, 2)
+// A bounded wait shared by all warps of the CTA: gives up on timeout (and
+// tells the others through ctl->abort) or when another warp gave up.
+__device__ __forceinline__ bool attn_wait(uint64_t *bar, uint32_t parity, ACtl *ctl,
+                                          int32_t *status)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity))
+            return true;
+        if (*(volatile int *)&ctl->abort)
+            return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            set_status(status, WIDE_DEV_TIMEOUT);
+            *(volatile int *)&ctl->abort = 1;
+            return false;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 2)
     prefill_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnPArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (smem_u32(smem) & 1023u) {
         if (tid == 0)
             set_status(a.status, WIDE_DEV_LAYOUT);
@@ -109,13 +137,16 @@ __global__ void __launch_bounds__(128, 2)
         ctl->nq = hi - lo;
         const int last = min(hi - 1, lo + (qt + 1) * kBQ - 1);
         ctl->pmax = last >= lo ? pj[last] - s * a.seq_len : -1;
+        ctl->abort = 0;
         mbar_init(&ctl->bar_q, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->bar_k[b], 1);
             mbar_init(&ctl->bar_v[b], 1);
             mbar_init(&ctl->bar_s[b], 1);
+            mbar_init(&ctl->s_free[b], kSoftWarps);
         }
         mbar_init(&ctl->bar_pv, 1);
+        mbar_init(&ctl->p_full, kSoftWarps);
         fence_mbar_init();
     }
     __syncthreads();
@@ -131,242 +162,256 @@ __global__ void __launch_bounds__(128, 2)
     umma::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t t_pv = tmem + 128;             // S buffers at columns 0 and 64
-
-    const int nvalid = min(kBQ, nq - qt * kBQ);
-    const int idx = lo + qt * kBQ + tid;          // row of this thread
-    const bool live = tid < nvalid;
-    const int tok = live ? pj[idx] : 0;
-    const int pos = live ? tok - s * a.seq_len : -1;
     const int64_t kvrow0 = ((int64_t)s * a.n_kv + j) * a.cache_cap;
     const int nkt = pmax / kBKV + 1;
-    constexpr uint32_t idesc_s = umma::idesc_bf16_f32(kBQ, kBKV);
-    constexpr uint32_t idesc_pv = umma::idesc_bf16_f32_bmn(kBQ, kHD);
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    // loads and PV commits issued (thread 0), to drain them after an error
-    int nk[2] = {0, 0}, nv[2] = {0, 0}, npv = 0;
 
-    auto load_k = [&](int t) {
-        ++nk[t & 1];
-        uint8_t *dst = smem + kOffK + (t & 1) * kKTile;
-        const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
-        mbar_arrive_expect_tx(&ctl->bar_k[t & 1], kKTile);
-        tma_load_2d(dst, &tm_k, 0, krow, &ctl->bar_k[t & 1]);
-        tma_load_2d(dst + kKHalf, &tm_k, 64, krow, &ctl->bar_k[t & 1]);
-    };
-    auto load_v = [&](int t) {
-        ++nv[t & 1];
-        uint8_t *dst = smem + kOffV + (t & 1) * kKTile;
-        const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
-        mbar_arrive_expect_tx(&ctl->bar_v[t & 1], kKTile);
-        tma_load_2d(dst, &tm_v, 0, krow, &ctl->bar_v[t & 1]);
-        tma_load_2d(dst + kKHalf, &tm_v, 64, krow, &ctl->bar_v[t & 1]);
-    };
-    // S(t) = Q K(t)^T into S buffer t & 1 (one thread)
-    auto issue_s = [&](int t) {
-        umma::fence_after_sync();
-        const uint32_t q0 = smem_u32(sq), k0 = smem_u32(smem + kOffK + (t & 1) * kKTile);
+    if (warp == kSoftWarps) {
+        // ---------------------------------------- TMA + MMA issuer (one lane)
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = umma::idesc_bf16_f32(kBQ, kBKV);
+            constexpr uint32_t idesc_pv = umma::idesc_bf16_f32_bmn(kBQ, kHD);
+            int nk[2] = {0, 0}, nv[2] = {0, 0}, npv = 0, ns[2] = {0, 0};
+            auto load_k = [&](int t) {
+                ++nk[t & 1];
+                uint8_t *dst = smem + kOffK + (t & 1) * kKTile;
+                const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
+                mbar_arrive_expect_tx(&ctl->bar_k[t & 1], kKTile);
+                tma_load_2d(dst, &tm_k, 0, krow, &ctl->bar_k[t & 1]);
+                tma_load_2d(dst + kKHalf, &tm_k, 64, krow, &ctl->bar_k[t & 1]);
+            };
+            auto load_v = [&](int t) {
+                ++nv[t & 1];
+                uint8_t *dst = smem + kOffV + (t & 1) * kKTile;
+                const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
+                mbar_arrive_expect_tx(&ctl->bar_v[t & 1], kKTile);
+                tma_load_2d(dst, &tm_v, 0, krow, &ctl->bar_v[t & 1]);
+                tma_load_2d(dst + kKHalf, &tm_v, 64, krow, &ctl->bar_v[t & 1]);
+            };
+            auto issue_s = [&](int t) {
+                ++ns[t & 1];
+                const uint32_t q0 = smem_u32(sq), k0 = smem_u32(smem + kOffK + (t & 1) * kKTile);
 #pragma unroll
-        for (int k = 0; k < kHD / 16; ++k) {
-            const uint32_t qo = (uint32_t)(k >> 2) * kQHalf + (uint32_t)(k & 3) * 32u;
-            const uint32_t ko = (uint32_t)(k >> 2) * kKHalf + (uint32_t)(k & 3) * 32u;
-            umma::mma_bf16(tmem + (uint32_t)(t & 1) * kBKV, umma::desc_kmajor_sw128(q0 + qo),
-                           umma::desc_kmajor_sw128(k0 + ko), idesc_s, k != 0);
-        }
-        umma::commit(&ctl->bar_s[t & 1]);
-    };
-
-    bool ok = true;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&ctl->bar_q, kQTile);
-        const int qrow = j * a.T + lo + qt * kBQ;
-        tma_load_2d(sq, &tm_q, hh * kHD, qrow, &ctl->bar_q);
-        tma_load_2d(sq + kQHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
-        for (int t = 0; t < 2 && t < nkt; ++t) {
-            load_k(t);
-            load_v(t);
-        }
-        if (!mbar_wait(&ctl->bar_q, 0) || !mbar_wait(&ctl->bar_k[0], 0))
-            ok = false;
-        else
-            issue_s(0);
-    }
-    if (__syncthreads_or(!ok)) {
-        if (tid == 0)
-            set_status(a.status, WIDE_DEV_TIMEOUT);
-        ok = false;
-    }
-
-    float m_ref = -INFINITY, l = 0.f;     // row reference max (log2 units), sum
-    const float sc = a.scale_log2;
-
-    for (int kt = 0; kt < nkt && ok; ++kt) {
-        const int b = kt & 1;
-        const uint32_t par = (uint32_t)(kt >> 1) & 1u;
-        bool w_ok = mbar_wait(&ctl->bar_s[b], par);          // S(kt) done; K(b) free
-        if (tid == 0 && w_ok) {
-            if (kt + 1 < nkt) {
-                if (mbar_wait(&ctl->bar_k[b ^ 1], (uint32_t)((kt + 1) >> 1) & 1u))
-                    issue_s(kt + 1);
-                else
-                    w_ok = false;
+                for (int k = 0; k < kHD / 16; ++k) {
+                    const uint32_t qo = (uint32_t)(k >> 2) * kQHalf + (uint32_t)(k & 3) * 32u;
+                    const uint32_t ko = (uint32_t)(k >> 2) * kKHalf + (uint32_t)(k & 3) * 32u;
+                    umma::mma_bf16(tmem + (uint32_t)(t & 1) * kBKV,
+                                   umma::desc_kmajor_sw128(q0 + qo),
+                                   umma::desc_kmajor_sw128(k0 + ko), idesc_s, k != 0);
+                }
+                umma::commit(&ctl->bar_s[t & 1]);
+            };
+            bool ok = true;
+            mbar_arrive_expect_tx(&ctl->bar_q, kQTile);
+            const int qrow = j * a.T + lo + qt * kBQ;
+            tma_load_2d(sq, &tm_q, hh * kHD, qrow, &ctl->bar_q);
+            tma_load_2d(sq + kQHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
+            for (int t = 0; t < 2 && t < nkt; ++t) {
+                load_k(t);
+                load_v(t);
             }
-            if (kt + 2 < nkt)
-                load_k(kt + 2);
-        }
-        umma::fence_after_sync();
-        // this row's 64 scores of the tile
-        const uint32_t ts = tmem + (uint32_t)b * kBKV + lane_off;
-        float v[kBKV];
-        umma::tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&v[0]));
-        umma::tmem_ld32(ts + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
-        umma::tmem_ld_wait();
-        const int k0 = kt * kBKV;
-        const bool full = live && k0 + kBKV - 1 <= pos;       // no key of the tile masked
-        if (!full) {
+            ok = attn_wait(&ctl->bar_q, 0, ctl, a.status) &&
+                 attn_wait(&ctl->bar_k[0], 0, ctl, a.status);
+            if (ok) {
+                umma::fence_after_sync();
+                issue_s(0);
+            }
+            for (int kt = 0; kt < nkt && ok; ++kt) {
+                const int b = kt & 1;
+                // S(kt+1): K(kt+1) landed and the softmax is done with S(kt-1)
+                if (kt + 1 < nkt) {
+                    ok = (kt == 0 || attn_wait(&ctl->s_free[b ^ 1], (uint32_t)((kt - 1) >> 1) & 1u,
+                                               ctl, a.status)) &&
+                         attn_wait(&ctl->bar_k[b ^ 1], (uint32_t)((kt + 1) >> 1) & 1u, ctl,
+                                   a.status);
+                    if (!ok)
+                        break;
+                    umma::fence_after_sync();
+                    issue_s(kt + 1);
+                }
+                // K(b) is free once S(kt) has completed: prefetch K(kt+2)
+                if (kt + 2 < nkt) {
+                    if (!(ok = attn_wait(&ctl->bar_s[b], (uint32_t)(kt >> 1) & 1u, ctl, a.status)))
+                        break;
+                    load_k(kt + 2);
+                }
+                // O += P(kt) V(kt) once P is written and V(kt) landed
+                ok = attn_wait(&ctl->p_full, (uint32_t)kt & 1u, ctl, a.status) &&
+                     attn_wait(&ctl->bar_v[b], (uint32_t)(kt >> 1) & 1u, ctl, a.status);
+                if (!ok)
+                    break;
+                const int kmax = a.seq_len - 1 - kt * kBKV;   // last valid key row in tile
+                if (kmax < kBKV - 1) {
+                    // keys past the sequence's end may be uninitialised cache
+                    // memory: clear those V rows so that 0 * garbage cannot
+                    // reach P V
+                    uint8_t *sv = smem + kOffV + b * kKTile;
+                    for (int rr = max(kmax + 1, 0); rr < kBKV; ++rr)
+                        for (int c = 0; c < 16; ++c)
+                            *reinterpret_cast<uint4 *>(sv + (c >> 3) * kKHalf + rr * 128 +
+                                                       (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    fence_proxy_async_smem();
+                }
+                umma::fence_after_sync();
+                const uint32_t p0 = smem_u32(sp), v0 = smem_u32(smem + kOffV + b * kKTile);
 #pragma unroll
-            for (int e = 0; e < kBKV; ++e)
-                if (!(live && k0 + e <= pos))
-                    v[e] = -INFINITY;
+                for (int k = 0; k < kBKV / 16; ++k) {
+                    const uint32_t aoff = (uint32_t)k * 32u;          // 16 keys of the P row
+                    const uint32_t boff = (uint32_t)k * 16u * 128u;   // 16 key rows of V
+                    umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
+                                   umma::desc_mnmajor_sw128(v0 + boff, kKHalf), idesc_pv,
+                                   (kt | k) != 0);
+                }
+                umma::commit(&ctl->bar_pv);
+                ++npv;
+                // V(b) is free once PV(kt) has completed: prefetch V(kt+2)
+                if (kt + 2 < nkt) {
+                    if (!(ok = attn_wait(&ctl->bar_pv, (uint32_t)kt & 1u, ctl, a.status)))
+                        break;
+                    load_v(kt + 2);
+                }
+            }
+            if (!ok) {
+                // let this CTA's copies and MMAs in flight land
+                for (int b = 0; b < 2; ++b) {
+                    if (nk[b] > 0)
+                        mbar_wait(&ctl->bar_k[b], (uint32_t)(nk[b] - 1) & 1u);
+                    if (nv[b] > 0)
+                        mbar_wait(&ctl->bar_v[b], (uint32_t)(nv[b] - 1) & 1u);
+                }
+                umma::commit(&ctl->bar_pv);
+                mbar_wait(&ctl->bar_pv, (uint32_t)npv & 1u);
+            }
+            (void)ns;
         }
-        float vmax = v[0];
-#pragma unroll
-        for (int e = 1; e < kBKV; ++e)
-            vmax = fmaxf(vmax, v[e]);
-        const float mt = vmax * sc;                           // -inf if no key is visible
-        // the previous tile's P V is done: P and V(b^1) are free
-        if (kt > 0) {
-            w_ok = w_ok && mbar_wait(&ctl->bar_pv, (uint32_t)(kt - 1) & 1u);
+    } else {
+        // ---------------------------------------- softmax warps (rows 0..127)
+        const int nvalid = min(kBQ, nq - qt * kBQ);
+        const int idx = lo + qt * kBQ + tid;          // row of this thread
+        const bool live = tid < nvalid;
+        const int tok = live ? pj[idx] : 0;
+        const int pos = live ? tok - s * a.seq_len : -1;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sc = a.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;     // row reference max (log2 units), sum
+        bool ok = true;
+        for (int kt = 0; kt < nkt; ++kt) {
+            const int b = kt & 1;
+            bool w = attn_wait(&ctl->bar_s[b], (uint32_t)(kt >> 1) & 1u, ctl, a.status);
+            if (!__all_sync(0xffffffffu, w)) {
+                ok = false;
+                break;
+            }
             umma::fence_after_sync();
-            if (tid == 0 && kt + 1 < nkt)
-                load_v(kt + 1);
+            // this row's 64 scores of the tile; then S buffer b is free
+            const uint32_t ts = tmem + (uint32_t)b * kBKV + lane_off;
+            float v[kBKV];
+            umma::tmem_ld32(ts, *reinterpret_cast<float(*)[32]>(&v[0]));
+            umma::tmem_ld32(ts + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            umma::tmem_ld_wait();
+            umma::fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ctl->s_free[b]);
+            const int k0 = kt * kBKV;
+            const bool full = live && k0 + kBKV - 1 <= pos;   // no key of the tile masked
+            if (!full) {
+#pragma unroll
+                for (int e = 0; e < kBKV; ++e)
+                    if (!(live && k0 + e <= pos))
+                        v[e] = -INFINITY;
+            }
+            float vmax = v[0];
+#pragma unroll
+            for (int e = 1; e < kBKV; ++e)
+                vmax = fmaxf(vmax, v[e]);
+            const float mt = vmax * sc;                       // -inf if no key is visible
+            // the previous tile's P V is done: P is free, O is stable
+            if (kt > 0) {
+                w = attn_wait(&ctl->bar_pv, (uint32_t)(kt - 1) & 1u, ctl, a.status);
+                if (!__all_sync(0xffffffffu, w)) {
+                    ok = false;
+                    break;
+                }
+                umma::fence_after_sync();
+            }
+            // move the reference max when the running max passes it by > 8
+            float alpha = 1.f;
+            if (mt > m_ref + 8.f) {
+                alpha = kt > 0 ? exp2f(m_ref - mt) : 0.f;
+                m_ref = mt;
+            }
+            if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                for (int c = 0; c < kHD / 32; ++c) {
+                    float ov[32];
+                    umma::tmem_ld32(t_pv + lane_off + c * 32, ov);
+                    umma::tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        ov[e] *= alpha;
+                    umma::tmem_st32(t_pv + lane_off + c * 32, ov);
+                }
+                umma::tmem_st_wait();
+            }
+            // probabilities -> P (bf16, swizzled K-major); masked keys give 0
+            const float mb = m_ref > -INFINITY ? m_ref : 0.f;
+            float lsum = 0.f;
+#pragma unroll
+            for (int g8 = 0; g8 < kBKV / 8; ++g8) {
+                float p[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    p[e] = exp2f(fmaf(v[g8 * 8 + e], sc, -mb));
+                    lsum += p[e];
+                }
+                __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]);
+                __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
+                __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
+                *reinterpret_cast<uint4 *>(sp + swz128(tid, g8)) = make_uint4(
+                    *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                    *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
+            }
+            l = l * alpha + lsum;
+            fence_proxy_async_smem();       // P written by threads, read by the tensor core
+            umma::fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&ctl->p_full);
         }
-        // move the reference max when the running max passes it by > 8
-        float alpha = 1.f;
-        if (mt > m_ref + 8.f) {
-            alpha = kt > 0 ? exp2f(m_ref - mt) : 0.f;
-            m_ref = mt;
+        if (ok) {
+            const bool w = attn_wait(&ctl->bar_pv, (uint32_t)(nkt - 1) & 1u, ctl, a.status);
+            ok = __all_sync(0xffffffffu, w);
         }
-        if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (ok) {
+            umma::fence_after_sync();
+            // O / l (the TMEM loads are warp-collective)
+            const float inv = live ? 1.f / l : 0.f;
+            __nv_bfloat16 *dst = a.o_sig + (size_t)(live ? a.sig_pos[tok] : 0) * a.ocols +
+                                 (size_t)(j * a.rep + hh) * kHD;
 #pragma unroll 1
             for (int c = 0; c < kHD / 32; ++c) {
                 float ov[32];
                 umma::tmem_ld32(t_pv + lane_off + c * 32, ov);
                 umma::tmem_ld_wait();
+                if (live) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    ov[e] *= alpha;
-                umma::tmem_st32(t_pv + lane_off + c * 32, ov);
-            }
-            umma::tmem_st_wait();
-        }
-        // probabilities -> P (bf16, swizzled K-major); masked keys give 0
-        const float mb = m_ref > -INFINITY ? m_ref : 0.f;
-        float lsum = 0.f;
-#pragma unroll
-        for (int g8 = 0; g8 < kBKV / 8; ++g8) {
-            float p[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                p[e] = exp2f(fmaf(v[g8 * 8 + e], sc, -mb));
-                lsum += p[e];
-            }
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]);
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
-            __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
-            *reinterpret_cast<uint4 *>(sp + swz128(tid, g8)) = make_uint4(
-                *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
-                *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
-        }
-        l = l * alpha + lsum;
-        // V(kt) must have landed; keys past the sequence's end may be
-        // uninitialised cache memory: clear those V rows so that 0 * garbage
-        // cannot reach P V
-        w_ok = w_ok && mbar_wait(&ctl->bar_v[b], par);
-        {
-            const int kmax = a.seq_len - 1 - kt * kBKV;       // last valid key row in tile
-            if (kmax < kBKV - 1) {
-                uint8_t *sv = smem + kOffV + b * kKTile;
-                for (int rr = max(kmax + 1, 0) + warp; rr < kBKV; rr += 4)
-                    for (int c = (tid & 31); c < 16; c += 32) {
-                        const int sub = c >> 3, ch = c & 7;
-                        *reinterpret_cast<uint4 *>(sv + sub * kKHalf + rr * 128 + ch * 16) =
-                            make_uint4(0u, 0u, 0u, 0u);
+                    for (int q = 0; q < 4; ++q) {
+                        __nv_bfloat162 b0 =
+                            __floats2bfloat162_rn(ov[q * 8] * inv, ov[q * 8 + 1] * inv);
+                        __nv_bfloat162 b1 =
+                            __floats2bfloat162_rn(ov[q * 8 + 2] * inv, ov[q * 8 + 3] * inv);
+                        __nv_bfloat162 b2 =
+                            __floats2bfloat162_rn(ov[q * 8 + 4] * inv, ov[q * 8 + 5] * inv);
+                        __nv_bfloat162 b3 =
+                            __floats2bfloat162_rn(ov[q * 8 + 6] * inv, ov[q * 8 + 7] * inv);
+                        reinterpret_cast<uint4 *>(dst + c * 32)[q] = make_uint4(
+                            *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
+                            *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
                     }
-            }
-        }
-        fence_proxy_async_smem();       // P (and cleared V rows) written by threads
-        umma::fence_before_sync();
-        if (__syncthreads_or(!w_ok)) {
-            if (tid == 0)
-                set_status(a.status, WIDE_DEV_TIMEOUT);
-            ok = false;
-            break;
-        }
-        // O += P V(kt)
-        if (tid == 0) {
-            umma::fence_after_sync();
-            const uint32_t p0 = smem_u32(sp), v0 = smem_u32(smem + kOffV + b * kKTile);
-#pragma unroll
-            for (int k = 0; k < kBKV / 16; ++k) {
-                const uint32_t aoff = (uint32_t)k * 32u;              // 16 keys of the P row
-                const uint32_t boff = (uint32_t)k * 16u * 128u;       // 16 key rows of V
-                umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
-                               umma::desc_mnmajor_sw128(v0 + boff, kKHalf), idesc_pv,
-                               (kt | k) != 0);
-            }
-            umma::commit(&ctl->bar_pv);
-            ++npv;
-        }
-    }
-    if (ok) {   // ok is uniform here; keep it so (the TMEM loads below are warp-collective)
-        const bool fin = mbar_wait(&ctl->bar_pv, (uint32_t)(nkt - 1) & 1u);
-        if (__syncthreads_or(!fin)) {
-            if (tid == 0)
-                set_status(a.status, WIDE_DEV_TIMEOUT);
-            ok = false;
-        }
-    }
-    umma::fence_after_sync();
-
-    if (ok) {
-        // O / l, all warps (the TMEM loads are warp-collective)
-        const float inv = live ? 1.f / l : 0.f;
-        __nv_bfloat16 *dst = a.o_sig + (size_t)(live ? a.sig_pos[tok] : 0) * a.ocols +
-                             (size_t)(j * a.rep + hh) * kHD;
-#pragma unroll 1
-        for (int c = 0; c < kHD / 32; ++c) {
-            float ov[32];
-            umma::tmem_ld32(t_pv + lane_off + c * 32, ov);
-            umma::tmem_ld_wait();
-            if (live) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    __nv_bfloat162 b0 = __floats2bfloat162_rn(ov[q * 8] * inv, ov[q * 8 + 1] * inv);
-                    __nv_bfloat162 b1 =
-                        __floats2bfloat162_rn(ov[q * 8 + 2] * inv, ov[q * 8 + 3] * inv);
-                    __nv_bfloat162 b2 =
-                        __floats2bfloat162_rn(ov[q * 8 + 4] * inv, ov[q * 8 + 5] * inv);
-                    __nv_bfloat162 b3 =
-                        __floats2bfloat162_rn(ov[q * 8 + 6] * inv, ov[q * 8 + 7] * inv);
-                    reinterpret_cast<uint4 *>(dst + c * 32)[q] = make_uint4(
-                        *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
-                        *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
                 }
             }
         }
-    }
-    // after an error, let this CTA's copies and MMAs in flight land before
-    // the shared memory and TMEM are released
-    if (!ok && tid == 0) {
-        for (int b = 0; b < 2; ++b) {
-            if (nk[b] > 0)
-                mbar_wait(&ctl->bar_k[b], (uint32_t)(nk[b] - 1) & 1u);
-            if (nv[b] > 0)
-                mbar_wait(&ctl->bar_v[b], (uint32_t)(nv[b] - 1) & 1u);
-        }
-        umma::commit(&ctl->bar_pv);         // completes after every MMA issued so far
-        mbar_wait(&ctl->bar_pv, (uint32_t)npv & 1u);
     }
     umma::fence_before_sync();
     __syncthreads();
@@ -512,7 +557,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
         LaunchScope scope(KID_PREFILL_ATTN, s);
         const dim3 grid((unsigned)((d->seq_len + kBQ - 1) / kBQ), (unsigned)rep,
                         (unsigned)(d->n_seq * n_kv));
-        prefill_attn<<<grid, 128, kAttnSmem, s>>>(tqc, tkc, tvc, aa);
+        prefill_attn<<<grid, kAttnThreads, kAttnSmem, s>>>(tqc, tkc, tvc, aa);
     }
     if ((rc = launch_status()))
         return rc;
