@@ -245,7 +245,7 @@ struct AttnArgs {
     const __nv_bfloat16 *k_cache;  // [n_seq][n_kv][cap][hd]
     const __nv_bfloat16 *v_cache;
     const uint32_t *head_mask;     // [T][Wh]
-    float *o;                      // [T][n_q * hd]
+    float *o;                      // [T][n_q * hd], token pairs interleaved (il2)
     int n_q, n_kv, Wh;
     int64_t nkeys, cache_cap;      // keys per sequence (cache_len + 1)
     float scale_log2;              // log2(e) / sqrt(hd)
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kHD)
         // the token skips this head group: no K/V bytes are read; its output
         // is 0 (o_proj reads 4-token blocks without per-token predication)
         if (s < rep)
-            a.o[(size_t)b * a.n_q * kHD + (size_t)(j * rep + s) * kHD + tid] = 0.f;
+            a.o[il2(b, (size_t)(j * rep + s) * kHD + tid, (size_t)a.n_q * kHD)] = 0.f;
         return;
     }
 
@@ -349,7 +349,7 @@ __global__ void __launch_bounds__(kHD)
             L += w * rml[2 * hh + 1];
             acc += w * cluster.map_shared_rank(os, q)[hh * kHD + tid];
         }
-        a.o[(size_t)b * a.n_q * kHD + (size_t)(j * rep + hh) * kHD + tid] = acc / L;
+        a.o[il2(b, (size_t)(j * rep + hh) * kHD + tid, (size_t)a.n_q * kHD)] = acc / L;
     }
     cluster.sync();
 }
@@ -397,10 +397,11 @@ DecodeWs decode_ws(const wide_layer_dims *d, void *base)
         off += align_up(bytes > 0 ? bytes : 1, 256);
         return at;
     };
+    const size_t Tp = (T + 1) / 2 * 2;                 // interleaved token pairs
     w.q = reinterpret_cast<float *>(take(T * qd * 4));
-    w.o = reinterpret_cast<float *>(take(T * qd * 4));
+    w.o = reinterpret_cast<float *>(take(Tp * qd * 4));
     w.h1 = reinterpret_cast<float *>(take(T * (size_t)d->hidden * 4));
-    w.hffn = reinterpret_cast<float *>(take(T * (size_t)d->inter * 4));
+    w.hffn = reinterpret_cast<float *>(take(Tp * (size_t)d->inter * 4));
     w.xn2 = reinterpret_cast<__nv_bfloat16 *>(take(T * (size_t)d->hidden * 2));
     w.bar = reinterpret_cast<uint32_t *>(take(256));
     w.total = off;

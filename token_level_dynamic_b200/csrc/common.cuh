@@ -167,6 +167,14 @@ __device__ __forceinline__ uint32_t swz128(uint32_t r, uint32_t j)
     return r * 128u + (((j ^ r) & 7u) << 4);
 }
 
+// Element (t, col) of a [T][ld] fp32 activation stored with token pairs
+// interleaved: row t/2 holds, for every column, the values of tokens t and
+// t+1 side by side, so a packed fp32x2 FMA can take two tokens at once.
+__host__ __device__ __forceinline__ size_t il2(int t, size_t col, size_t ld)
+{
+    return (size_t)(t >> 1) * 2 * ld + col * 2 + (size_t)(t & 1);
+}
+
 // ------------------------------------------------------------- numerics
 
 // Widens 8 bf16 values (one 16-byte chunk) to fp32 exactly.

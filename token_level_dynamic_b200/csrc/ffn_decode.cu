@@ -23,7 +23,11 @@
 //   h[t][c] * W_down[n][c] only for tokens t that execute the group.  The KS
 //   partial outputs are added through distributed shared memory.
 //
-// Tokens are processed 32 at a time (one mask bit per lane).
+// Tokens are processed 32 at a time (one mask bit per lane), two at a time
+// per packed fp32x2 FMA: x (staged in shared memory) and h (the fp32 [T][I]
+// intermediate, and the attention output that o_proj reads) are stored with
+// token pairs interleaved (il2), so one register pair holds the same column
+// of two tokens and the weight element is duplicated across the pair.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -75,55 +79,54 @@ __device__ __forceinline__ uint32_t group_token_mask(const uint32_t *mask, int T
     return __ballot_sync(0xffffffffu, a);
 }
 
-// Dot products of one weight chunk (EPC elements of two rows wa, wb) with
-// the x chunks of TB tokens (rows 0..TB-1 of xk, row stride ld): 2*TB
-// independent fp32 accumulation chains.
-template <int EPC, int TB>
-__device__ __forceinline__ void fma2_tb(const float (&wa)[EPC], const float (&wb)[EPC],
-                                        const float *xk, int ld, float *a, float *b)
+// One weight chunk (EPC elements of two rows wa, wb) times the x chunks of
+// NP token pairs (xk2: pair 0 of the chunk in the interleaved layout, pair
+// stride ld2 floats): 2*NP independent packed accumulation chains.
+template <int EPC, int NP>
+__device__ __forceinline__ void fma2_pairs(const float (&wa)[EPC], const float (&wb)[EPC],
+                                           const float *xk2, int ld2, float2 *a, float2 *b)
 {
 #pragma unroll
-    for (int e = 0; e < EPC; e += 4) {
-        float xv[TB][4];
+    for (int e = 0; e < EPC; e += 2) {
+        float4 xv[NP];
 #pragma unroll
-        for (int r = 0; r < TB; ++r) {
-            const float4 v = *reinterpret_cast<const float4 *>(xk + r * ld + e);
-            xv[r][0] = v.x;
-            xv[r][1] = v.y;
-            xv[r][2] = v.z;
-            xv[r][3] = v.w;
-        }
+        for (int p = 0; p < NP; ++p)
+            xv[p] = *reinterpret_cast<const float4 *>(xk2 + p * ld2 + e * 2);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 2; ++q) {
+            const float2 wa2 = make_float2(wa[e + q], wa[e + q]);
+            const float2 wb2 = make_float2(wb[e + q], wb[e + q]);
 #pragma unroll
-            for (int r = 0; r < TB; ++r) {
-                a[r] = fmaf(wa[e + q], xv[r][q], a[r]);
-                b[r] = fmaf(wb[e + q], xv[r][q], b[r]);
+            for (int p = 0; p < NP; ++p) {
+                const float2 xp = q == 0 ? make_float2(xv[p].x, xv[p].y)
+                                         : make_float2(xv[p].z, xv[p].w);
+                a[p] = __ffma2_rn(wa2, xp, a[p]);
+                b[p] = __ffma2_rn(wb2, xp, b[p]);
             }
+        }
     }
 }
 
-// One weight row chunk with TB token chunks: TB independent chains.
-template <int EPC, int TB>
-__device__ __forceinline__ void fma1_tb(const float (&w)[EPC], const float *xk, int ld,
-                                        float *acc)
+// One weight row chunk times the h chunks of NP token pairs.
+template <int EPC, int NP>
+__device__ __forceinline__ void fma1_pairs(const float (&w)[EPC], const float *hk2, int ld2,
+                                           float2 *acc)
 {
 #pragma unroll
-    for (int e = 0; e < EPC; e += 4) {
-        float xv[TB][4];
+    for (int e = 0; e < EPC; e += 2) {
+        float4 hv[NP];
 #pragma unroll
-        for (int r = 0; r < TB; ++r) {
-            const float4 v = *reinterpret_cast<const float4 *>(xk + r * ld + e);
-            xv[r][0] = v.x;
-            xv[r][1] = v.y;
-            xv[r][2] = v.z;
-            xv[r][3] = v.w;
+        for (int p = 0; p < NP; ++p)
+            hv[p] = *reinterpret_cast<const float4 *>(hk2 + p * ld2 + e * 2);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const float2 w2 = make_float2(w[e + q], w[e + q]);
+#pragma unroll
+            for (int p = 0; p < NP; ++p)
+                acc[p] = __ffma2_rn(w2, q == 0 ? make_float2(hv[p].x, hv[p].y)
+                                               : make_float2(hv[p].z, hv[p].w),
+                                    acc[p]);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int r = 0; r < TB; ++r)
-                acc[r] = fmaf(w[e + q], xv[r][q], acc[r]);
     }
 }
 
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(32 + 2 * GS)
         }
 #pragma unroll
         for (int e = 0; e < EPC; ++e)
-            xs[i * kslice + q * EPC + e] = f[e];
+            xs[il2(i, (size_t)q * EPC + e, kslice)] = f[e];
     }
     __syncthreads();
 
@@ -236,11 +239,11 @@ __global__ void __launch_bounds__(32 + 2 * GS)
         }
     }
 
-    float accg[kNTok], accu[kNTok];
+    float2 accg[kNTok / 2], accu[kNTok / 2];     // token pairs
 #pragma unroll
-    for (int i = 0; i < kNTok; ++i) {
-        accg[i] = 0.f;
-        accu[i] = 0.f;
+    for (int i = 0; i < kNTok / 2; ++i) {
+        accg[i] = make_float2(0.f, 0.f);
+        accu[i] = make_float2(0.f, 0.f);
     }
     if (warp > 0) {
         // ---------------------------------------------- consumers
@@ -258,12 +261,13 @@ __global__ void __launch_bounds__(32 + 2 * GS)
                 float wg[EPC], wu[EPC];
                 chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tg + swz128(c, j)), wg);
                 chunk_to_f32<TIn>(*reinterpret_cast<const uint4 *>(tu + swz128(c, j)), wu);
-                const float *xk = xs + kt * KT + j * EPC;
+                const float *xk2 = xs + (size_t)(kt * KT + j * EPC) * 2;
 #pragma unroll
                 for (int i0 = 0; i0 < kNTok; i0 += TB) {
                     if (i0 >= nactb)
                         break;
-                    fma2_tb<EPC, TB>(wg, wu, xk + i0 * kslice, kslice, &accg[i0], &accu[i0]);
+                    fma2_pairs<EPC, TB / 2>(wg, wu, xk2 + (size_t)i0 * kslice, 2 * kslice,
+                                            &accg[i0 / 2], &accu[i0 / 2]);
                 }
             }
             __syncwarp();
@@ -292,8 +296,9 @@ __global__ void __launch_bounds__(32 + 2 * GS)
         for (int i = 0; i < kNTok; ++i) {
             if (i >= nact)
                 break;
-            pg[(half * kNTok + i) * GS + c] = timeout ? 0.f : accg[i];
-            pu[(half * kNTok + i) * GS + c] = timeout ? 0.f : accu[i];
+            const float2 g2 = accg[i >> 1], u2 = accu[i >> 1];
+            pg[(half * kNTok + i) * GS + c] = timeout ? 0.f : ((i & 1) ? g2.y : g2.x);
+            pu[(half * kNTok + i) * GS + c] = timeout ? 0.f : ((i & 1) ? u2.y : u2.x);
         }
     }
     cluster.sync();
@@ -306,14 +311,14 @@ __global__ void __launch_bounds__(32 + 2 * GS)
                 gs += rg[i * GS + c] + rg[(kNTok + i) * GS + c];
                 us += ru[i * GS + c] + ru[(kNTok + i) * GS + c];
             }
-            h[(size_t)act[i] * I + (size_t)g * GS + c] = silu_f32(gs) * us;
+            h[il2(act[i], (size_t)g * GS + c, I)] = silu_f32(gs) * us;
         }
     } else if (warp > 0) {
         // tokens that skip this group get h = 0, so that the down projection
         // can run token blocks without per-token predication
         for (int t = s; t < T; t += KS)
             if (((tmask >> t) & 1u) == 0u)
-                h[(size_t)t * I + (size_t)g * GS + c] = 0.f;
+                h[il2(t, (size_t)g * GS + c, I)] = 0.f;
     }
     cluster.sync();
 }
@@ -338,8 +343,9 @@ __global__ void __launch_bounds__(32 + 2 * kDownRows)
     constexpr uint32_t kBlockMask = TB >= 32 ? 0xffffffffu : ((1u << TB) - 1u);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
-    const int TT = (T + TB - 1) / TB * TB;
-    const uint32_t hbytes = (uint32_t)T * KT * 4u;        // h tile (fp32, unswizzled)
+    const int TT = (T + TB - 1) / TB * TB;                // TB is even
+    const int TP = (T + 1) / 2;                           // token pairs TMA writes
+    const uint32_t hbytes = (uint32_t)TP * 2u * KT * 4u;  // h tile: [TP][KT][2] fp32
     const uint32_t hstride = (uint32_t)TT * KT * 4u;
     const uint32_t stage_bytes = kWBytes + ((hstride + 1023u) & ~1023u);
     uint8_t *stages = smem;
@@ -374,11 +380,12 @@ __global__ void __launch_bounds__(32 + 2 * kDownRows)
         tma_prefetch_desc(&tm_down);
         tma_prefetch_desc(&tm_h);
     }
-    // token rows T..TT-1 of every h stage stay zero (TMA writes rows < T)
-    if (TT > T) {
+    // token pairs TP..TT/2-1 of every h stage stay zero (TMA writes pairs < TP)
+    if (TT / 2 > TP) {
         for (int st = 0; st < kStages; ++st)
-            for (int i = tid; i < (TT - T) * KT; i += 32 + 2 * kDownRows)
-                reinterpret_cast<float *>(stages + st * stage_bytes + kWBytes)[T * KT + i] = 0.f;
+            for (int i = tid; i < (TT / 2 - TP) * 2 * KT; i += 32 + 2 * kDownRows)
+                reinterpret_cast<float *>(stages + st * stage_bytes + kWBytes)[TP * 2 * KT + i] =
+                    0.f;
     }
     __syncthreads();
     if (tid == 0) {
@@ -392,10 +399,10 @@ __global__ void __launch_bounds__(32 + 2 * kDownRows)
     const int ntile = n_live * TPG;
 
     bool timeout = false;
-    float acc[kNTok];
+    float2 acc[kNTok / 2];                                // token pairs
 #pragma unroll
-    for (int t = 0; t < kNTok; ++t)
-        acc[t] = 0.f;
+    for (int t = 0; t < kNTok / 2; ++t)
+        acc[t] = make_float2(0.f, 0.f);
     if (warp == 0) {
         if (lane == 0) {
             for (int kt = 0; kt < ntile; ++kt) {
@@ -409,7 +416,7 @@ __global__ void __launch_bounds__(32 + 2 * kDownRows)
                 uint8_t *dst = stages + st * stage_bytes;
                 mbar_arrive_expect_tx(&full[st], kWBytes + hbytes);
                 tma_load_2d(dst, &tm_down, col, nb * kDownRows, &full[st]);
-                tma_load_2d(dst + kWBytes, &tm_h, col, 0, &full[st]);
+                tma_load_2d(dst + kWBytes, &tm_h, 2 * col, 0, &full[st]);   // interleaved pairs
             }
         }
     } else {
@@ -433,7 +440,8 @@ __global__ void __launch_bounds__(32 + 2 * kDownRows)
                         break;
                     if (((tm >> t0) & kBlockMask) == 0u)
                         continue;
-                    fma1_tb<EPC, TB>(w, hs + t0 * KT + j * EPC, KT, &acc[t0]);
+                    fma1_pairs<EPC, TB / 2>(w, hs + (size_t)(t0 / 2) * 2 * KT + j * EPC * 2,
+                                            2 * KT, &acc[t0 / 2]);
                 }
             }
             __syncwarp();
@@ -459,7 +467,8 @@ __global__ void __launch_bounds__(32 + 2 * kDownRows)
         for (int t = 0; t < kNTok; ++t) {
             if (t >= T)
                 break;
-            part[(half * kNTok + t) * kDownRows + n] = timeout ? 0.f : acc[t];
+            part[(half * kNTok + t) * kDownRows + n] =
+                timeout ? 0.f : ((t & 1) ? acc[t >> 1].y : acc[t >> 1].x);
         }
     }
     cluster.sync();
@@ -528,18 +537,18 @@ int gateup_chunk(const TIn *x, const TIn *wg, const TIn *wu, const uint32_t *mas
     if (!make_tmap_2d(&tg, wg, I, H, H, sizeof(TIn), GS, KT, true) ||
         !make_tmap_2d(&tu, wu, I, H, H, sizeof(TIn), GS, KT, true))
         return WIDE_CUDA_FAIL();
-    const int TB = T >= 4 ? 4 : (T >= 2 ? 2 : 1);
+    const int TB = T >= 8 ? 8 : (T >= 4 ? 4 : 2);      // even: tokens go in pairs
     const size_t TT = (size_t)((T + TB - 1) / TB * TB);
     const size_t smem1 = 1024 + kStages * 2 * GS * 128 + 512 + TT * kslice * 4;
     const dim3 grid(KS, G), block(32 + 2 * GS);
 #define WIDE_GU(TBV)                                                                               \
     launch_cluster(KID_DECODE_GATEUP, ffn_decode_gateup<TIn, GS, TBV>, grid, block, smem1, KS, s, \
                    tg, tu, x, mask, h, T, H, I, W, kslice, status_ptr())
+    if (TB == 8)
+        return WIDE_GU(8);
     if (TB == 4)
         return WIDE_GU(4);
-    if (TB == 2)
-        return WIDE_GU(2);
-    return WIDE_GU(1);
+    return WIDE_GU(2);
 #undef WIDE_GU
 }
 
@@ -551,11 +560,14 @@ int down_chunk(const TIn *wd, const float *h, const uint32_t *mask, const DownOu
     constexpr int KT = 8 * EPC;
     const int G = I / GS, W = (G + 31) / 32;
     CUtensorMap td, th;
+    // h holds token pairs interleaved: [ceil(T/2)][I][2] fp32, i.e. rows of
+    // 2*I floats; a box is the KT columns of a tile for every pair
+    const int TP = (T + 1) / 2;
     if (!make_tmap_2d(&td, wd, H, I, I, sizeof(TIn), kDownRows, KT, true) ||
-        !make_tmap_2d(&th, h, T, I, I, 4, T, KT, false))
+        !make_tmap_2d(&th, h, TP, 2 * (uint64_t)I, 2 * (uint64_t)I, 4, TP, 2 * KT, false))
         return WIDE_CUDA_FAIL();
     const int KSd = G < 8 ? G : 8;
-    const int TB = T >= 8 ? 8 : (T >= 4 ? 4 : (T >= 2 ? 2 : 1));
+    const int TB = T >= 8 ? 8 : (T >= 4 ? 4 : 2);      // even: tokens go in pairs
     const size_t hb = (size_t)((T + TB - 1) / TB * TB) * KT * 4;
     const size_t stage = (size_t)kDownRows * 128 + ((hb + 1023) & ~(size_t)1023);
     const size_t smem2 = 1024 + kStages * stage + 64 + 1024 * 4 + 1024 * 4;
@@ -567,9 +579,7 @@ int down_chunk(const TIn *wd, const float *h, const uint32_t *mask, const DownOu
         return WIDE_DN(8);
     if (TB == 4)
         return WIDE_DN(4);
-    if (TB == 2)
-        return WIDE_DN(2);
-    return WIDE_DN(1);
+    return WIDE_DN(2);
 #undef WIDE_DN
 }
 
@@ -640,8 +650,10 @@ int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const
 
 size_t ffn_decode_h_bytes(const wide_ffn_dims *d)
 {
+    // h of up to 32 tokens, token pairs interleaved (an odd count rounds up)
     const int64_t T = d->tokens < kNTok ? d->tokens : kNTok;
-    return align_up((size_t)(T > 0 ? T : 1) * (size_t)d->inter * sizeof(float), 256);
+    const int64_t Tp = T > 0 ? (T + 1) / 2 * 2 : 2;
+    return align_up((size_t)Tp * (size_t)d->inter * sizeof(float), 256);
 }
 
 // h scratch, then 256 bytes holding the fused kernel's grid-barrier words.
