@@ -199,6 +199,28 @@ class FFNDevice:
         self.call(i)
         self.oh[i].copy_(self.outs[i], non_blocking=True)
 
+    def naive_gather_scatter(self, i):
+        """The naive masked FFN the pages compare against: for each group, copy
+        out the rows of the tokens that keep it (index_select, whose size
+        needs a device-to-host sync), run the three matmuls on that copy, and
+        scatter-add the result back (index_add).  torch ops only."""
+        import torch
+        import torch.nn.functional as F
+        c, x, m = self.cases[i], self.xs[i], self.ms[i]
+        gs, G = c.gs, c.I // c.gs
+        sh = torch.arange(32, device=m.device, dtype=torch.int32)
+        bits = ((m.unsqueeze(-1) >> sh) & 1).reshape(m.shape[0], -1)[:, :G].bool()
+        acc = torch.zeros(x.shape, dtype=torch.float32, device=x.device)
+        for g in range(G):
+            idx = bits[:, g].nonzero().squeeze(1)
+            if idx.numel() == 0:
+                continue
+            xg = x.index_select(0, idx)
+            sl = slice(g * gs, (g + 1) * gs)
+            h = F.silu(xg @ self.Wg[sl].T) * (xg @ self.Wu[sl].T)
+            acc.index_add_(0, idx, (h @ self.Wd[:, sl].T).float())
+        self.outs[i].copy_(acc)
+
     def dense_torch(self, i):
         import torch.nn.functional as F
         x = self.xs[i]
@@ -748,6 +770,28 @@ def run_ours(args, wl):
                        "tokens_per_s": tokens_per_step / (float(pc.sum(axis=1).mean()) / 1e3)}
     dense["masked_speedup_vs_torch_dense"] = dense["torch_cublas_bf16"]["ms_per_step"] / step_ms
     dense["masked_speedup_vs_ours_all_kept"] = dense["ours_all_groups_kept"]["ms_per_step"] / step_ms
+    if hasattr(D, "naive_gather_scatter"):
+        # the pages' naive comparator: time, and peak device memory it adds
+        # per call next to ours (our only extra memory is the workspace)
+        ng = D.naive_gather_scatter
+        timed_step(ng)
+        torch.cuda.synchronize(dev)
+        peak = 0
+        for i in range(ncalls):
+            base_mem = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            ng(i)
+            torch.cuda.synchronize(dev)
+            peak = max(peak, torch.cuda.max_memory_allocated(dev) - base_mem)
+        evs = [timed_step(ng) for _ in range(3)]
+        torch.cuda.synchronize(dev)
+        pc = ms_of(evs)
+        ng_ms = float(pc.sum(axis=1).mean())
+        dense["naive_gather_scatter_torch"] = {
+            "ms_per_step": ng_ms, "tokens_per_s": tokens_per_step / (ng_ms / 1e3),
+            "peak_extra_device_bytes_per_call": int(peak),
+            "ours_workspace_bytes": int(D.ws.numel()),
+            "masked_speedup_vs_naive": ng_ms / step_ms}
 
     # ---- end to end through the public API with host buffers
     for _ in range(3):

@@ -179,7 +179,7 @@ int wide_reorder(const uint32_t *d_mask, int64_t T, int64_t G, int32_t tile_m,
  *
  * Supported: hidden % 64 == 0; group_size in {32, 64, 128} dividing inter;
  * G <= 1024; 16-byte aligned pointers.  WIDE_PATH_PREFILL needs bf16,
- * group_size == 128 and hidden % 256 == 0.  The fp32 type runs the
+ * group_size 64 or 128 and hidden % 256 == 0.  The fp32 type runs the
  * CUDA-core path at any T.
  */
 typedef struct wide_ffn_dims {

@@ -95,3 +95,23 @@ def test_prefill_ffn_8b_full_size_sampled():
                         c.w_down, c.mask[rows])
     assert rel_l2(out[rows], _ref(sub)) <= TOL
     assert np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("T,H,I,kind,keep", [
+    (300, 256, 512, "bernoulli", 0.5),        # 8 groups of 64, ragged tails
+    (1000, 512, 2048, "prototype", 0.5),      # 32 groups of 64, prototypes
+    (513, 1024, 4352, "prototype", 0.25),     # 68 groups of 64 over three mask words
+])
+def test_prefill_group_size_64(T, H, I, kind, keep):
+    """64-channel groups: the gate/up tiles are N = 128 (gate + up rows of
+    one group) and the down projection visits one 64-column K stage per
+    union group."""
+    c = synth.ffn_case(T, H, I, 64, seed=T + 7, keep=keep, mask_kind=kind)
+    assert rel_l2(_run(c), _ref(c)) <= TOL
+
+
+def test_prefill_group_size_64_all_zero_and_dense():
+    c = synth.ffn_case(200, 256, 512, 64, seed=13, mask_kind="zeros")
+    assert not np.any(_run(c))
+    c = synth.ffn_case(260, 512, 1024, 64, seed=14, mask_kind="ones")
+    assert rel_l2(_run(c), ffn_dense(c.x, c.w_gate, c.w_up, c.w_down)) <= TOL

@@ -101,3 +101,10 @@ def test_prefill_layer_8b_full_size_sampled():
     assert rel_l2(got["ffn_out"][rows], p["ffn_out"]) <= TOL
     _kv_check(lc, got, p["k"], p["v"], rows)
     assert np.isfinite(got["out"]).all()
+
+
+def test_prefill_layer_ffn_group_size_64():
+    """The layer with 64-channel FFN groups (gate/up tiles N = 128)."""
+    lc = synth.small_layer("prefill", seed=31, n_seq=2, seq_len=256, H=512, n_q=8, n_kv=2,
+                           hd=128, I=1024, gs=64, keep_a=0.5, keep_f=0.5)
+    _check_full(lc, _run(lc))

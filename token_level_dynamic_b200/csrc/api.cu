@@ -199,7 +199,8 @@ bool ffn_shape_supported(const wide_ffn_dims *d, int path)
     if (path == WIDE_PATH_DECODE)
         return d->dtype == WIDE_BF16 ? (gs == 64 || gs == 128) : (gs == 32 || gs == 64 || gs == 128);
     // prefill: tcgen05 kernels with 128-channel groups and 256-column output blocks
-    return d->dtype == WIDE_BF16 && gs == 128 && d->hidden % 256 == 0 && d->tokens <= (1 << 24);
+    return d->dtype == WIDE_BF16 && (gs == 64 || gs == 128) && d->hidden % 256 == 0 &&
+           d->tokens <= (1 << 24);
 }
 
 }  // namespace wide

@@ -465,7 +465,8 @@ bool layer_prefill_supported(const wide_layer_dims *d)
     return d->cache_len == 0 && d->seq_len >= 1 && T >= 1 && T <= (1 << 24) &&
            d->head_dim == kHD && d->n_kv_heads >= 2 && d->n_kv_heads % 2 == 0 &&
            d->n_kv_heads <= 1024 && (rep == 2 || rep == 4) && d->hidden % 256 == 0 &&
-           d->ffn_group_size == 128 && d->inter % 128 == 0 && d->inter / 128 <= 1024 &&
+           (d->ffn_group_size == 64 || d->ffn_group_size == 128) &&
+           d->inter % d->ffn_group_size == 0 && d->inter / d->ffn_group_size <= 1024 &&
            d->cache_cap >= d->seq_len && (int64_t)d->n_kv_heads * T <= (1ll << 31) / 512;
 }
 
@@ -587,7 +588,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
     fo.res_f32 = w.h1;
     fo.out_total = static_cast<__nv_bfloat16 *>(p.out);
     return ffn_prefill_core(w.xn, p.w_gate, p.w_up, p.w_down, p.ffn_mask, fo, T, H, d->inter,
-                            w.ffn, s);
+                            d->ffn_group_size, w.ffn, s);
 }
 
 }  // namespace wide

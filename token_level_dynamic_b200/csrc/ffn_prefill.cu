@@ -17,7 +17,6 @@ namespace wide {
 
 namespace {
 constexpr int kBM = 128;
-constexpr int kGS = 128;
 }
 
 size_t ffn_prefill_workspace(const wide_ffn_dims *d)
@@ -30,9 +29,9 @@ size_t ffn_prefill_workspace(const wide_ffn_dims *d)
 
 int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *wd,
                      const uint32_t *mask, const FfnPrefillOut &o, int64_t T, int64_t H,
-                     int64_t I, void *ws, cudaStream_t s)
+                     int64_t I, int64_t gs, void *ws, cudaStream_t s)
 {
-    const int64_t G = I / kGS;
+    const int64_t G = I / gs;
     const size_t wl_bytes = wide_worklist_bytes(T, G, kBM);
     wide_worklist wl;
     int rc = wide_worklist_carve(ws, wl_bytes, T, G, kBM, &wl);
@@ -42,15 +41,15 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
         reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + align_up(wl_bytes, 1024));
 
     CUtensorMap tg, tu, th, td;
-    if (!make_tmap_2d(&tg, wg, I, H, H, 2, 128, 64, true) ||
-        !make_tmap_2d(&tu, wu, I, H, H, 2, 128, 64, true) ||
+    if (!make_tmap_2d(&tg, wg, I, H, H, 2, (uint32_t)gs, 64, true) ||
+        !make_tmap_2d(&tu, wu, I, H, H, 2, (uint32_t)gs, 64, true) ||
         !make_tmap_2d(&th, hbuf, T, I, I, 2, kBM, 64, true) ||
         !make_tmap_2d(&td, wd, H, I, I, 2, 256, 64, true))
         return WIDE_CUDA_FAIL();
 
     if ((rc = reorder_launch(mask, T, G, kBM, &wl, s)))
         return rc;
-    if ((rc = zero_dead_launch(mask, wl.sig_pos, hbuf, (int)T, (int)I, (int)G, kGS, s)))
+    if ((rc = zero_dead_launch(mask, wl.sig_pos, hbuf, (int)T, (int)I, (int)G, (int)gs, s)))
         return rc;
 
     GemmArgs ga = {};
@@ -64,6 +63,7 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
     ga.T = (int)T;
     ga.K = (int)H;
     ga.out_ld = (int)I;
+    ga.gs = (int)gs;
     ga.status = status_ptr();
     const int max_items = (int)(G * ((T + kBM - 1) / kBM));
     if ((rc = gather_gemm_launch(GEMM_SWIGLU, tg, tu, ga, max_items, KID_PREFILL_GATEUP, s)))
@@ -75,7 +75,7 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
     ua.T = (int)T;
     ua.N = (int)H;
     ua.W = (int)((G + 31) / 32);
-    ua.gs = kGS;
+    ua.gs = (int)gs;
     ua.out_sum = o.out_sum;
     ua.res_f32 = o.res_f32;
     ua.out_total = o.out_total;
@@ -89,7 +89,8 @@ int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void
 {
     FfnPrefillOut o = {};
     o.out_sum = static_cast<__nv_bfloat16 *>(out);
-    return ffn_prefill_core(x, wg, wu, wd, mask, o, d->tokens, d->hidden, d->inter, ws, s);
+    return ffn_prefill_core(x, wg, wu, wd, mask, o, d->tokens, d->hidden, d->inter,
+                            d->group_size, ws, s);
 }
 
 }  // namespace wide

@@ -114,6 +114,7 @@ struct GemmArgs {
     __nv_bfloat16 *out0, *out1;
     int T, K;
     int out_ld;          // SwiGLU: row stride of H (= inter)
+    int gs;              // SwiGLU: channels per group (64 or 128)
     int group_cols;      // RoPE-Q: columns of one head group (rep * head_dim)
     int seq_len, n_kv, kv_blocks, m_tiles;
     int64_t cache_len, cache_cap;
@@ -155,7 +156,7 @@ struct FfnPrefillOut {
 };
 int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *wd,
                      const uint32_t *mask, const FfnPrefillOut &o, int64_t T, int64_t H,
-                     int64_t I, void *ws, cudaStream_t s);
+                     int64_t I, int64_t gs, void *ws, cudaStream_t s);
 int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void *wd,
                        const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                        cudaStream_t s);

@@ -19,7 +19,8 @@
 //              coalesced requests; each thread's copy completions arrive on
 //              the stage barrier
 //   modes
-//     SwiGLU  work item (g, i) of the FFN work list; B = [W_gate[g]; W_up[g]];
+//     SwiGLU  work item (g, i) of the FFN work list; B = [W_gate[g]; W_up[g]]
+//             (N = 2 gs: 256 for 128-channel groups, 128 for 64);
 //             epilogue h = silu(gate) * up, stored bf16 at the token's
 //             signature-order row of H.
 //     RopeQ   work item (j, i) of the head-group work list, 256-column part
@@ -271,8 +272,10 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
             const Work w = decode_work<MODE>(a, it);
             const CUtensorMap *m0 = &tm0, *m1 = &tm1;
             int r0, r1;
+            uint32_t b_rows = kBN;                           // rows of the B tile
             if (MODE == GEMM_SWIGLU) {
-                r0 = r1 = w.g * 128;                         // [W_gate[g]; W_up[g]]
+                r0 = r1 = w.g * a.gs;                        // [W_gate[g]; W_up[g]]
+                b_rows = 2 * a.gs;
             } else if (MODE == GEMM_ROPE_Q) {
                 r0 = w.g * a.group_cols + w.hf * kBN;        // two query heads of group g
                 r1 = r0 + 128;
@@ -290,9 +293,9 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                         ok = false;
                     } else {
                         uint8_t *b = smem + stage * kStageBytes + kATile;
-                        mbar_arrive_expect_tx(&ctl->full[stage], kBTile);
+                        mbar_arrive_expect_tx(&ctl->full[stage], b_rows * 128u);
                         tma_load_2d(b, m0, kt * kBK, r0, &ctl->full[stage]);
-                        tma_load_2d(b + kBTile / 2, m1, kt * kBK, r1, &ctl->full[stage]);
+                        tma_load_2d(b + b_rows * 64u, m1, kt * kBK, r1, &ctl->full[stage]);
                         ++issued;
                     }
                 }
@@ -354,7 +357,9 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
         cp_async_wait_all();
     } else if (warp == 1) {
         // -------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = umma::idesc_bf16_f32(kBM, kBN);
+        // SwiGLU: N = gate rows + up rows of one group (2 gs); else 256
+        const uint32_t idesc =
+            umma::idesc_bf16_f32(kBM, MODE == GEMM_SWIGLU ? 2u * (uint32_t)a.gs : (uint32_t)kBN);
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
@@ -414,12 +419,12 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
             const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * (uint32_t)kBN;
             if (MODE == GEMM_SWIGLU) {
                 __nv_bfloat16 *dst = a.out0 + (size_t)(live ? a.sig_pos[t] : 0) * a.out_ld +
-                                     (size_t)w.g * 128;
+                                     (size_t)w.g * a.gs;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < a.gs / 32; ++c) {
                     float gv[32], uv[32];
                     umma::tmem_ld32(taddr + c * 32, gv);
-                    umma::tmem_ld32(taddr + 128 + c * 32, uv);
+                    umma::tmem_ld32(taddr + a.gs + c * 32, uv);
                     umma::tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
