@@ -573,6 +573,23 @@ def _host_cores():
     return int(_clib.lib().oracle_num_threads())
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The largest x over all ranks (the slowest rank's time); x itself
+    when no process group is up."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_step: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_step * steps / (total_ms / 1e3)
+
+
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -673,13 +690,9 @@ def run_ours(args, wl):
     if w.wide_get_device_status(stream) != 0:
         raise RuntimeError("device status set during the timed steps")
     per_call = ms_of(all_evs)                       # [K][ncalls] ms
-    total_ms = float(per_call.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(per_call.sum()), dev)
     step_ms = total_ms / args.steps
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = job_tokens_per_s(world, tokens_per_step, args.steps, total_ms)
 
     # ---- per-kernel figures from the library's launch events
     peaks = _peaks()
@@ -799,12 +812,8 @@ def run_ours(args, wl):
     barrier()
     e_evs = [timed_step(D.e2e_call) for _ in range(args.steps)]
     barrier()
-    e_ms = float(ms_of(e_evs).sum())
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e = {"value": world * tokens_per_step * args.steps / (e_ms / 1e3), "unit": "tokens/s",
+    e_ms = max_over_ranks(float(ms_of(e_evs).sum()), dev)
+    e2e = {"value": job_tokens_per_s(world, tokens_per_step, args.steps, e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": D.h2d_bytes, "d2h_bytes_per_step": D.d2h_bytes,
            "ms_per_step": e_ms / args.steps}
 
