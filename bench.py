@@ -273,11 +273,32 @@ class DecodeFFN3B:
 
 
 def _fused_decode_used(T, H, I, gs, sms=148):
-    """Mirror of the library's dispatch: the fused decode kernel runs for up
-    to 8 tokens when H % 256 == 0, gs in 64..256 and the W_down rows of one
-    CTA fit its box (ceil(H / SMs) <= 96)."""
-    return (1 <= T <= 8 and H % 256 == 0 and gs % 64 == 0 and gs <= 256 and I % gs == 0
-            and I // gs <= 1024 and -(-H // sms) <= 96)
+    """Mirror of the library's dispatch (plan_fused in ffn_decode_fused.cu):
+    the fused decode kernel runs for 1..32 tokens when H % 256 == 0, gs in
+    64..256, at most 1024 groups, and its phase-2 plan (rows of W_down per
+    CTA over at most 4 rows per thread) fits."""
+    if not (1 <= T <= 32 and H % 256 == 0 and gs % 64 == 0 and gs <= 256 and I % gs == 0):
+        return False
+    G = I // gs
+    if G > 1024 or T * (-(-G // 32)) > 1024:
+        return False
+    P = sms // -(-T // 8)
+    if P < 1:
+        return False
+    rows = -(-H // P)
+    TBP = max(2, 1 if T <= 1 else 2 if T <= 2 else 4 if T <= 4 else 8)
+    best = None
+    tpi = 32
+    while tpi <= 512:
+        nr = tpi // (gs // 8)
+        rt = -(-rows // nr)
+        ni = 512 // tpi
+        if rt <= 4:
+            cost = (rt + 2) / ni
+            if best is None or cost < best[0]:
+                best = (cost, rt, nr, ni)
+        tpi *= 2
+    return best is not None and best[3] * best[2] * best[1] * TBP <= 2048
 
 
 def _ffn_decode_bytes(case, res_bytes=0, x_bytes=None):

@@ -202,6 +202,21 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                     const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
                     void *stream);
 
+/* Kernels of the bf16 decode FFN (process-wide; the decode layer's FFN
+ * follows it too).  Both compute the same sums, in a different fp32 order:
+ *   WIDE_DECODE_AUTO   the measured faster one for the call's shape (default)
+ *   WIDE_DECODE_FUSED  the persistent fused kernel wherever its shape limits
+ *                      allow (1..32 tokens, hidden % 256 == 0, ...), else
+ *                      the GEMVs
+ *   WIDE_DECODE_GEMV   the gate/up GEMV kernel, then the down GEMV kernel
+ * Returns the previous mode, or WIDE_EINVAL for an unknown mode (the mode
+ * is then unchanged).  Not ordered with work already enqueued: it applies
+ * to calls made after it returns. */
+#define WIDE_DECODE_AUTO 0
+#define WIDE_DECODE_FUSED 1
+#define WIDE_DECODE_GEMV 2
+int wide_set_decode_ffn_path(int mode);
+
 /* --------------------------------------------------- masked attention / layer
  *
  * Section 2.A, attention half: a token that skips head group j (the
@@ -277,8 +292,9 @@ int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cac
  * channels) lives in a fixed device array inside the library of
  * WIDE_NOALLOC_SCRATCH_BYTES bytes, and the decode kernel's grid-barrier
  * words in a second one of 256 bytes, which every GPU that loads the library
- * holds until the process exits.  Limit: min(tokens, 32) * inter * 4 bytes
- * must not exceed it (inter <= 16384); larger problems return
+ * holds until the process exits.  Limit: min(tokens, 32), rounded up to
+ * an even count, * inter * 4 bytes must not exceed it (inter <= 16384 at
+ * 32 tokens); larger problems return
  * WIDE_ETOOLARGE before anything is enqueued.  The call allocates nothing.
  * Its first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream

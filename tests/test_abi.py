@@ -107,3 +107,17 @@ def test_ffn_argument_checks(native):
     # workspace too small
     assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(ok), p, 16, None) \
         == native.WIDE_EWORKSPACE
+
+
+def test_decode_path_switch_is_host_only(native):
+    """wide_set_decode_ffn_path answers on the host: returns the previous
+    mode and refuses unknown modes without changing the current one."""
+    L = native.lib()
+    prev = L.wide_set_decode_ffn_path(1)
+    try:
+        assert L.wide_set_decode_ffn_path(2) == 1
+        assert L.wide_set_decode_ffn_path(7) == -1
+        assert L.wide_set_decode_ffn_path(-1) == -1
+        assert L.wide_set_decode_ffn_path(0) == 2
+    finally:
+        L.wide_set_decode_ffn_path(prev)

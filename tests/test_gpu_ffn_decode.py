@@ -14,6 +14,20 @@ TOL_BF16 = 5e-3   # relative L2, bf16 storage / fp32 accumulation
 TOL_F32 = 1e-5    # relative L2, fp32 tiny configuration
 
 
+@pytest.fixture(params=["auto", "fused", "gemv"], autouse=True)
+def decode_kernels(request):
+    """Every case runs on the dispatcher's choice and on each of the two
+    bf16 decode implementations forced (fused persistent kernel wherever its
+    limits allow -- including token blocks of 9..32 tokens -- and the two
+    GEMV kernels)."""
+    import token_level_dynamic_b200 as w
+    mode = {"auto": w.WIDE_DECODE_AUTO, "fused": w.WIDE_DECODE_FUSED,
+            "gemv": w.WIDE_DECODE_GEMV}[request.param]
+    prev = w.wide_set_decode_ffn_path(mode)
+    yield request.param
+    w.wide_set_decode_ffn_path(prev)
+
+
 def _run(c, path=None):
     import torch
     import token_level_dynamic_b200 as w
@@ -106,11 +120,12 @@ def test_output_rows_split_unevenly_over_the_grid():
     assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
 
 
-def test_bad_mask_bit_sets_device_status():
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_bad_mask_bit_sets_device_status(dtype):
     """A bit at or above G in the decode mask sets WIDE_DEV_BAD_MASK."""
     import torch
     import token_level_dynamic_b200 as w
-    c = synth.ffn_case(2, 256, 1024, 128, seed=5)          # G = 8
+    c = synth.ffn_case(2, 256, 1024, 128, seed=5, dtype=dtype)          # G = 8
     x, wg, wu, wd, m = ffn_to_dev(c)
     m[1, 0] |= 1 << 9
     w.wide_clear_device_status()

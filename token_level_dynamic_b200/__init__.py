@@ -120,6 +120,17 @@ def wide_launch_count() -> int:
     return int(_L.wide_launch_count())
 
 
+WIDE_DECODE_AUTO, WIDE_DECODE_FUSED, WIDE_DECODE_GEMV = 0, 1, 2
+
+
+def wide_set_decode_ffn_path(mode: int) -> int:
+    """Selects the kernels of the bf16 decode FFN; returns the previous mode."""
+    rc = int(_L.wide_set_decode_ffn_path(int(mode)))
+    if rc < 0:
+        raise WideError("wide_set_decode_ffn_path", rc)
+    return rc
+
+
 # --------------------------------------------------------- mask reordering
 
 def wide_worklist_bytes(T: int, G: int, tile_m: int = 128) -> int:
@@ -205,7 +216,8 @@ def wide_ffn_masked_noalloc(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.T
     allocates nothing either).  The library keeps the kernels' scratch in a
     fixed device array of WIDE_NOALLOC_SCRATCH_BYTES bytes shared by all
     calls on a device; calls that overlap on the GPU race on it.  Raises
-    WideError (WIDE_ETOOLARGE) when min(T, 32) * I * 4 exceeds that size."""
+    WideError (WIDE_ETOOLARGE) when min(T, 32) (rounded up to
+    an even count) * I * 4 exceeds that size."""
     d = _ffn_dims(x, w_gate, group_size, WIDE_PATH_DECODE)
     _check("wide_ffn_masked_noalloc", _L.wide_ffn_masked_noalloc(
         _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),

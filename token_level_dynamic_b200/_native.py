@@ -69,6 +69,7 @@ SIGNATURES = {
     "wide_profile_read": (c_int, [c_void_p, c_void_p, c_int32, c_void_p]),
     "wide_kernel_name": (ctypes.c_char_p, [c_int32]),
     "wide_launch_count": (c_int64, []),
+    "wide_set_decode_ffn_path": (c_int, [c_int]),
     "wide_worklist_bytes": (c_size_t, [c_int64, c_int64, c_int32]),
     "wide_worklist_carve": (c_int, [c_void_p, c_size_t, c_int64, c_int64, c_int32,
                                     ctypes.POINTER(WideWorklist)]),

@@ -107,6 +107,23 @@ bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_pairs(CUtensorMap *map, const float *base, uint64_t pairs, uint64_t cols,
+                         uint32_t box_cols, uint32_t box_pairs)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || pairs == 0 || cols == 0 || cols % 16 != 0 || box_cols % 16 != 0)
+        return false;
+    const cuuint64_t dims[3] = {32, 2 * cols / 32, pairs};
+    const cuuint64_t strides[2] = {128, 2 * cols * 4};
+    const cuuint32_t box[3] = {32, box_cols / 16, box_pairs};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r =
+        fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(base), dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool raise_smem_limit(const void *kernel, size_t bytes)
 {
     // The attribute is an upper bound, so it is raised once per (kernel,

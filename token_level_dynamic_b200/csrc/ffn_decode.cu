@@ -170,6 +170,13 @@ __global__ void __launch_bounds__(32 + 2 * GS)
     const int ct = tid - 32;                    // consumer index (valid when warp > 0)
     const int c = ct % GS, half = ct / GS;
 
+    // mask bits at or above G are ignored by both kernels; one CTA reports them
+    if (g == 0 && s == 0 && (I / GS) % 32 != 0) {
+        const int G = I / GS;
+        for (int t = tid; t < T; t += 32 + 2 * GS)
+            if ((mask[(size_t)t * W + W - 1] >> (G & 31)) != 0u)
+                set_status(status, WIDE_DEV_BAD_MASK);
+    }
     const uint32_t tmask = group_token_mask(mask, T, W, g);
     if (tmask == 0u)
         return;  // block-level skip: the whole cluster leaves together

@@ -10,11 +10,11 @@
 //   Phase 1: h[t][i] = silu(x[t] . W_gate[i]) * (x[t] . W_up[i]) for every
 //     row i of the union (0 where token t skips i's group).  The union's
 //     rows, in group order, are cut into one contiguous range per CTA in
-//     units of 8 rows.  A stage holds 8 rows of W_gate and of W_up over a
-//     window of KW = 1024 columns (when H is not a multiple of 1024, KW is
-//     512 or 256 and a stage holds 1024 / KW units), fetched as one 3-D TMA copy
-//     per unit and matrix: long contiguous row pieces stream far better than
-//     2-D boxes of short rows.
+//     units of 8 rows.  A stage holds SR rows of W_gate and of W_up over a
+//     window of KW columns (16 x 512, or 32 x 256 when H is not a multiple
+//     of 512), fetched as one 3-D TMA copy of 8 rows per unit and matrix:
+//     long contiguous row pieces stream far better than 2-D boxes of short
+//     rows.
 //   Grid barrier: an arrival counter (zeroed on the stream before the
 //     launch) that the producer of every CTA polls, bounded.
 //   Phase 2: out[t][n] = sum over the union's columns i of h[t][i] *
@@ -26,35 +26,49 @@
 //
 // Warp 0 (one lane) streams every tile by TMA through an mbarrier ring.  It
 // issues phase 2's W_down tiles as soon as ring slots free up, before the
-// grid barrier; only their h tiles wait for the barrier.  Warps 1..8 compute
-// in fp32 on CUDA cores: thread (row r of 4, lane c of 8) of a warp takes
-// 16-byte column chunks c and c+8 of a 128-column piece -- in phase 1 the
-// gate and up rows of one row of a unit over two adjacent pieces, in phase 2
-// rows r + 4w + 32k of its range over each group; the 8 lanes of a row read
-// 128 contiguous bytes, and the x (or h) chunk is shared by the rows of the
-// warp (broadcast reads).  Products are formed two columns at a time with
-// packed fp32 FMAs (even and odd columns accumulate apart); the x of 4
-// tokens is loaded first and the accumulators are updated one column pair
-// at a time, so consecutive FMAs into one accumulator are far apart.  In
-// phase 1 the warps of a stage split its columns, so a unit's sums are
-// added over the 8 lanes by shuffles and over the warps in shared memory.
+// grid barrier; only their h tiles wait for the barrier.  Warps 1..16 compute
+// in fp32 on CUDA cores with packed fp32x2 FMAs over token PAIRS: one
+// register pair holds the running sums of tokens 2p and 2p+1, the x (or h)
+// operand is the pair's two values of one column and the weight operand is
+// that column's weight in both halves.  So a 16-byte weight chunk (8
+// columns of one row) read from shared memory serves every token, and a
+// 16-byte read of x serves 2 tokens x 2 columns of every row the thread
+// holds.
+//   Phase 1: a thread holds 2 rows of W_gate and the same 2 rows of W_up (4
+//     weight rows) at one 8-column chunk of the window; the 8 lanes of a
+//     quarter warp take 8 adjacent chunks of one row (128 contiguous bytes).
+//     x is staged once as bf16 token pairs [pair][column][2], its two 16-byte
+//     halves of a chunk swapped in every other group of 4 chunks, so the 8
+//     lanes of a quarter warp read 8 distinct banks.  The partial sums are
+//     added over the chunks of a row (lane shuffles that halve the values a
+//     lane carries at every step, then shared memory between the two warps
+//     of a row for 512-column windows) once per row block.
+//   Phase 2: a thread holds up to 4 rows of the CTA's W_down range at one
+//     8-column chunk of a group; several sets of whole warps ("instances")
+//     take different groups, run ahead of one another as far as the ring
+//     allows, and their sums meet in shared memory at the end.  h
+//     is written by phase 1 as fp32 token pairs and copied per group by a
+//     3-D TMA box with 128-byte swizzle, which leaves the 8 lanes of a
+//     quarter warp reading 8 distinct banks.
 #include "common.cuh"
 #include "host.h"
 
+#include <atomic>
 #include <mutex>
 
 namespace wide {
 namespace {
 
 constexpr int kFTok = 8;                    // tokens per CTA (one token block)
-constexpr int kFWarps = 8;                  // consumer warps
-constexpr int kFThreads = 32 * (kFWarps + 1);
-constexpr int kFStageCols = 1024;           // phase 1: window columns x units per stage
-constexpr uint32_t kFSlotMin = 2u * 8u * kFStageCols * 2u;   // gate + up: 32 KB
+constexpr int kFWarps = 16;                 // consumer warps
+constexpr int kFCons = 32 * kFWarps;        // consumer threads
+constexpr int kFThreads = kFCons + 32;
+constexpr int kFStageElems = 8192;          // phase 1: rows x window columns per stage
+constexpr uint32_t kFSlotMin = 2u * kFStageElems * 2u;   // gate + up: 32 KB
 constexpr int kFMaxSlots = 8;
 constexpr int kFMaxG = 1024;                // groups (union words fit one warp)
-constexpr int kFMaxR2 = 3;                  // phase 2: row sets (32 rows each) per thread
-constexpr int kFTQ = 4;                     // tokens whose x is held in registers at once
+constexpr int kFMaxRT = 4;                  // phase 2: rows per thread
+constexpr int kFRedFloats = 2048;           // cross-warp / cross-instance sums
 constexpr int kFMaxMaskWords = 1024;        // T * W
 
 struct FusedArgs {
@@ -63,16 +77,18 @@ struct FusedArgs {
     const __nv_bfloat16 *gamma;  // RMSNorm gain used with xf
     float eps;
     const uint32_t *mask;        // [T][W] packed group bits
-    float *h;                    // [T][I] fp32 scratch
+    float *h;                    // [T][I] fp32 scratch, token pairs interleaved
     uint32_t *bar;               // grid barrier arrival counter (0 at launch)
     DownOutputs o;
     int T, H, I, W, G, gs;
     int TG, P;                   // token blocks; row ranges (grid = P * TG)
-    int kw;                      // phase-1 window columns (divides H, multiple of 128)
+    int kw;                      // phase-1 window columns (512 or 256)
+    int rt, nr, ni;              // phase 2: rows per thread, row sets, instances
     int nslots;
     uint32_t slot_bytes;
     uint32_t w2_bytes;           // one W_down box (rows_box rows x gs columns)
-    uint32_t h2_bytes;           // one h box (TB tokens x gs columns, fp32)
+    uint32_t h2_bytes;           // one h box (token pairs x gs columns, fp32)
+    uint32_t h2_stride;          // h boxes' spacing in a slot (1024-byte multiple)
     uint32_t h2_off;             // offset of the h boxes inside a phase-2 slot
     int ng2;                     // groups per phase-2 stage
     int32_t *status;
@@ -93,33 +109,33 @@ __device__ __forceinline__ float4 lds128f(const uint8_t *p)
     return *reinterpret_cast<const float4 *>(p);
 }
 
-// The 8 bf16 of one chunk as 4 fp32 pairs (columns 2i, 2i+1).  Lanes whose
-// x (or h) reads start with the upper half of the chunk (sw = 1) get the
-// pairs in the matching order: 4..7 first, then 0..3.  (Lanes c and c+4
-// read x chunks 128 bytes apart; starting them on opposite halves keeps the
-// 8 distinct 16-byte reads of a warp in distinct banks.)
-__device__ __forceinline__ void widen_pairs(const uint4 v, int sw, float2 (&w)[4])
+// Word i (0..3, a compile-time index after unrolling) of a 16-byte chunk.
+__device__ __forceinline__ uint32_t word(const uint4 v, int i)
 {
-    const uint32_t a0 = sw ? v.z : v.x, a1 = sw ? v.w : v.y;
-    const uint32_t b0 = sw ? v.x : v.z, b1 = sw ? v.y : v.w;
-    w[0] = make_float2(__uint_as_float(a0 << 16), __uint_as_float(a0 & 0xffff0000u));
-    w[1] = make_float2(__uint_as_float(a1 << 16), __uint_as_float(a1 & 0xffff0000u));
-    w[2] = make_float2(__uint_as_float(b0 << 16), __uint_as_float(b0 & 0xffff0000u));
-    w[3] = make_float2(__uint_as_float(b1 << 16), __uint_as_float(b1 & 0xffff0000u));
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// The bf16 in the low / high half of w as fp32 (byte permutes: exact).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x1044)); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x3244)); }
+// ... in both halves of a register pair (the weight operand of a token
+// pair), each half written by its own byte permute
+__device__ __forceinline__ float2 dup_lo(uint32_t w)
+{
+    uint32_t a, b;
+    asm("prmt.b32 %0, %2, 0, 0x1044;\n\tprmt.b32 %1, %2, 0, 0x1044;" : "=r"(a), "=r"(b) : "r"(w));
+    return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+__device__ __forceinline__ float2 dup_hi(uint32_t w)
+{
+    uint32_t a, b;
+    asm("prmt.b32 %0, %2, 0, 0x3244;\n\tprmt.b32 %1, %2, 0, 0x3244;" : "=r"(a), "=r"(b) : "r"(w));
+    return make_float2(__uint_as_float(a), __uint_as_float(b));
 }
 
 // The two float pairs of one float4.
 __device__ __forceinline__ float2 lo2(const float4 v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(const float4 v) { return make_float2(v.z, v.w); }
-
-// Sum over the 8 lanes of a row group (lanes 8r .. 8r+7).
-__device__ __forceinline__ float sum8(float v)
-{
-    v += __shfl_xor_sync(0xffffffffu, v, 1);
-    v += __shfl_xor_sync(0xffffffffu, v, 2);
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    return v;
-}
 
 __device__ __forceinline__ void fence_proxy_async_global()
 {
@@ -127,7 +143,7 @@ __device__ __forceinline__ void fence_proxy_async_global()
 }
 __device__ __forceinline__ void consumer_sync()
 {
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kFWarps) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kFCons) : "memory");
 }
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
 {
@@ -140,116 +156,182 @@ __device__ __forceinline__ void red_add_release_gpu(uint32_t *p, uint32_t v)
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Phase 1, one stage, one thread: row `row` of its unit of W_gate (sg) and
-// W_up (su) (row stride rs bytes in the slot), chunks c and c+8 of each of
-// its two 128-column pieces (xq: x at the first piece), TB tokens.
-template <int TB>
-__device__ __forceinline__ void p1_stage(const uint8_t *sg, const uint8_t *su, const uint8_t *xq,
-                                         int H, uint32_t rs, int row, int c, int sw,
-                                         float2 (&ag)[TB], float2 (&au)[TB])
+// Halving steps of lane_reduce: as many as the lanes allow while KEEP values
+// are left per lane.
+__host__ __device__ constexpr int scatter_levels(int ratio, int lv)
 {
-    constexpr int TQ = TB < kFTQ ? TB : kFTQ;
-    const uint32_t xo1 = sw ? 16u : 0u, xo2 = 16u - xo1;
+    int s = 0;
+    while (s < lv && (2 << s) <= ratio)
+        ++s;
+    return s;
+}
+
+// Sums v[0..N) over the 2^LV lanes that differ in lane bits [0, LV).  The
+// first S = scatter_levels(N / KEEP, LV) steps halve what a lane carries
+// (a lane keeps the half its bit selects and receives its partner's copy of
+// it), the remaining LV - S steps add whole arrays.  Afterwards lane l holds
+// in v[0..N >> S) the sums of entries
+//   m = ((l >> (LV - S)) & (2^S - 1)) * (N >> S) + j.
+template <int N, int LV, int KEEP>
+__device__ __forceinline__ void lane_reduce(float (&v)[N], int lane)
+{
+    constexpr int S = scatter_levels(N / KEEP, LV);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {              // chunks c, c+8 of piece 0, then of piece 1
-        const int j = c + 8 * q;
-        float2 wg[4], wu[4];
-        widen_pairs(lds128(sg + row * rs + j * 16), sw, wg);
-        widen_pairs(lds128(su + row * rs + j * 16), sw, wu);
-        const uint8_t *xj = xq + j * 32;
+    for (int l = 0; l < S; ++l) {
+        const int o = 1 << (LV - 1 - l);
+        const bool hi = (lane & o) != 0;
+        const int n = N >> (l + 1);
 #pragma unroll
-        for (int t0 = 0; t0 < TB; t0 += TQ) {
-            float4 x1[TQ], x2[TQ];
+        for (int i = 0; i < N / 2; ++i) {
+            if (i < n) {
+                const float send = hi ? v[i] : v[i + n];
+                const float keep = hi ? v[i + n] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+    }
+    constexpr int R = N >> S;
 #pragma unroll
-            for (int t = 0; t < TQ; ++t) {
-                x1[t] = lds128f(xj + (size_t)(t0 + t) * H * 4 + xo1);
-                x2[t] = lds128f(xj + (size_t)(t0 + t) * H * 4 + xo2);
+    for (int l = S; l < LV; ++l) {
+        const int o = 1 << (LV - 1 - l);
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+    }
+}
+
+// Phase 1, one stage, one thread: rows 0 and 1 of W_gate at sg and of W_up
+// at su (row stride rs bytes), one 8-column chunk; the x half holding the
+// chunk's columns 4 h .. 4 h + 3 of token pair p at xk + p * xpair + xo[h].
+template <int NP>
+__device__ __forceinline__ void p1_stage(const uint8_t *sg, const uint8_t *su, uint32_t rs,
+                                         const uint8_t *xk, uint32_t xpair, const uint32_t (&xo)[2],
+                                         float2 (&ag)[2][NP], float2 (&au)[2][NP])
+{
+    uint4 g[2], u[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        g[i] = lds128(sg + i * rs);
+        u[i] = lds128(su + i * rs);
+    }
+#pragma unroll
+    for (int p2 = 0; p2 < 2; ++p2) {             // columns 4 p2 .. 4 p2 + 3 of the chunk
+        uint4 xr[NP];
+#pragma unroll
+        for (int tp = 0; tp < NP; ++tp)
+            xr[tp] = lds128(xk + tp * xpair + xo[p2]);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            float2 xv[NP];
+#pragma unroll
+            for (int tp = 0; tp < NP; ++tp) {
+                const uint32_t wx = word(xr[tp], cc);
+                xv[tp] = make_float2(bf_lo(wx), bf_hi(wx));
+            }
+            const int wi = 2 * p2 + (cc >> 1);    // weight word of column 4 p2 + cc
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float2 d = (cc & 1) ? dup_hi(word(g[i], wi)) : dup_lo(word(g[i], wi));
+#pragma unroll
+                for (int tp = 0; tp < NP; ++tp)
+                    ag[i][tp] = __ffma2_rn(d, xv[tp], ag[i][tp]);
             }
 #pragma unroll
-            for (int t = 0; t < TQ; ++t) {
-                ag[t0 + t] = __ffma2_rn(wg[0], lo2(x1[t]), ag[t0 + t]);
-                au[t0 + t] = __ffma2_rn(wu[0], lo2(x1[t]), au[t0 + t]);
-            }
+            for (int i = 0; i < 2; ++i) {
+                const float2 d = (cc & 1) ? dup_hi(word(u[i], wi)) : dup_lo(word(u[i], wi));
 #pragma unroll
-            for (int t = 0; t < TQ; ++t) {
-                ag[t0 + t] = __ffma2_rn(wg[1], hi2(x1[t]), ag[t0 + t]);
-                au[t0 + t] = __ffma2_rn(wu[1], hi2(x1[t]), au[t0 + t]);
-            }
-#pragma unroll
-            for (int t = 0; t < TQ; ++t) {
-                ag[t0 + t] = __ffma2_rn(wg[2], lo2(x2[t]), ag[t0 + t]);
-                au[t0 + t] = __ffma2_rn(wu[2], lo2(x2[t]), au[t0 + t]);
-            }
-#pragma unroll
-            for (int t = 0; t < TQ; ++t) {
-                ag[t0 + t] = __ffma2_rn(wg[3], hi2(x2[t]), ag[t0 + t]);
-                au[t0 + t] = __ffma2_rn(wu[3], hi2(x2[t]), au[t0 + t]);
+                for (int tp = 0; tp < NP; ++tp)
+                    au[i][tp] = __ffma2_rn(d, xv[tp], au[i][tp]);
             }
         }
     }
 }
 
-// Phase 2, one group of one stage: rows rw + 32 k (k < R2) of the range (rows
-// past the box's last row rmax read that row; their sums are discarded), the
-// gs columns of the group, TB tokens.
-template <int TB, int R2>
-__device__ __forceinline__ void p2_group(const uint8_t *wb, const uint8_t *hb, int gs, int rw,
-                                         int rmax, int c, int sw, float2 (&acc)[kFMaxR2][TB])
+// Phase 2, one group: this thread's rows of the W_down box at wb (row k at
+// wb + min(wbase + k wrs, wmax), k < RT) and the group's h box at hb, whose 16-byte unit
+// holding columns 2p, 2p+1 of this thread's chunk for token pair tp sits at
+// hb + (hoff[tp] ^ 16 p) (128-byte swizzle: the unit index within its
+// 128-byte row is XOR-ed with the row index).
+template <int NP, int RT>
+__device__ __forceinline__ void p2_group(const uint8_t *wb, uint32_t wbase, uint32_t wrs,
+                                         uint32_t wmax, const uint8_t *hb,
+                                         const uint32_t (&hoff)[NP], float2 (&acc)[kFMaxRT][NP])
 {
-    constexpr int TQ = TB < kFTQ ? TB : kFTQ;
-    const uint32_t xo1 = sw ? 16u : 0u, xo2 = 16u - xo1;
-    for (int q = 0; q < gs / 64; ++q) {
-        const int j = c + 8 * q;
-        float2 w[R2][4];
+    uint4 w[RT];
 #pragma unroll
-        for (int rr = 0; rr < R2; ++rr)
-            widen_pairs(lds128(wb + (size_t)min(rw + 32 * rr, rmax) * gs * 2 + j * 16), sw,
-                        w[rr]);
-        const uint8_t *hq = hb + j * 32;
+    for (int k = 0; k < RT; ++k)
+        w[k] = lds128(wb + min(wbase + (uint32_t)k * wrs, wmax));
 #pragma unroll
-        for (int t0 = 0; t0 < TB; t0 += TQ) {
-            float4 x1[TQ], x2[TQ];
+    for (int p = 0; p < 4; ++p) {                 // columns 2p, 2p+1 of the chunk
+        float4 hx[NP];
 #pragma unroll
-            for (int t = 0; t < TQ; ++t) {
-                x1[t] = lds128f(hq + (size_t)(t0 + t) * gs * 4 + xo1);
-                x2[t] = lds128f(hq + (size_t)(t0 + t) * gs * 4 + xo2);
+        for (int tp = 0; tp < NP; ++tp)
+            hx[tp] = lds128f(hb + (hoff[tp] ^ (uint32_t)(p << 4)));
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int k = 0; k < RT; ++k) {
+                const float2 d = e ? dup_hi(word(w[k], p)) : dup_lo(word(w[k], p));
+#pragma unroll
+                for (int tp = 0; tp < NP; ++tp)
+                    acc[k][tp] = __ffma2_rn(d, e ? hi2(hx[tp]) : lo2(hx[tp]), acc[k][tp]);
             }
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int t = 0; t < TQ; ++t)
-#pragma unroll
-                    for (int rr = 0; rr < R2; ++rr) {
-                        const float2 xv = p == 0 ? lo2(x1[t]) : p == 1 ? hi2(x1[t])
-                                        : p == 2 ? lo2(x2[t]) : hi2(x2[t]);
-                        acc[rr][t0 + t] = __ffma2_rn(w[rr][p], xv, acc[rr][t0 + t]);
-                    }
-        }
     }
 }
 
-// One CTA of 9 warps per SM.  The register file is split between the SM's
-// four sub-partitions and one of them holds 3 of the 9 warps, so a thread
-// gets at most 16384 / 96 registers; the launch bounds let ptxas apply that.
+// Phase 2's sums over the chunk lanes of a row set (2^LV = gs / 8 lanes),
+// written to red2[instance][row][token] (one writer per value).
+template <int NP, int LV>
+__device__ __forceinline__ void p2_reduce(float2 (&acc)[kFMaxRT][NP], int ch2, bool act, int gi,
+                                          int row0, int rt, int n2rows, int rstride, float *red2)
+{
+    constexpr int TBP = 2 * NP, N = kFMaxRT * TBP;
+    float v[N];
+#pragma unroll
+    for (int k = 0; k < kFMaxRT; ++k)
+#pragma unroll
+        for (int tp = 0; tp < NP; ++tp) {
+            v[k * TBP + 2 * tp] = acc[k][tp].x;
+            v[k * TBP + 2 * tp + 1] = acc[k][tp].y;
+        }
+    lane_reduce<N, LV, 1>(v, ch2);
+    constexpr int S = scatter_levels(N, LV), R = N >> S;
+    const bool owner = (ch2 & ((1 << (LV - S)) - 1)) == 0;
+    const int mb = ((ch2 >> (LV - S)) & ((1 << S) - 1)) * R;
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+        const int m = mb + j, k = m / TBP, t = m % TBP, row = row0 + k;
+        if (act && owner && k < rt && row < n2rows)
+            red2[((size_t)gi * rstride + row) * TBP + t] = v[j];
+    }
+}
+
+// One CTA of 17 warps per SM.  The register file is split between the SM's
+// four sub-partitions and one of them holds 5 of the 17 warps, so a thread
+// gets at most 16384 / 160 registers, 96 in the allocation granularity.
 template <int TB>
-__global__ void __launch_bounds__(kFThreads, 1)
+__global__ void __maxnreg__(96)
     ffn_decode_fused(const __grid_constant__ CUtensorMap tm_gate,
                      const __grid_constant__ CUtensorMap tm_up,
                      const __grid_constant__ CUtensorMap tm_down,
                      const __grid_constant__ CUtensorMap tm_h, const FusedArgs a)
 {
+    constexpr int TBP = TB < 2 ? 2 : TB;             // tokens rounded up to whole pairs
+    constexpr int NP = TBP / 2;                      // token pairs
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align1024(smem_raw);
     const int NS = a.nslots;
     uint8_t *slots = smem;
-    float *xs = reinterpret_cast<float *>(smem + (size_t)NS * a.slot_bytes);   // [TB][H]
-    float *red = xs + (size_t)TB * a.H;              // [2][4 piece pairs][8 rows][2][TB]
-    uint32_t *mall = reinterpret_cast<uint32_t *>(red + 2 * 4 * 8 * 2 * TB);  // [T][W]
+    // x as bf16 token pairs: [NP][H / 8 chunks][2 halves][4 columns][2 tokens]
+    uint8_t *xs = smem + (size_t)NS * a.slot_bytes;
+    float *red = reinterpret_cast<float *>(xs + (size_t)TBP * a.H * 2);
+    uint32_t *mall = reinterpret_cast<uint32_t *>(red + kFRedFloats);   // [T][W]
     int *live = reinterpret_cast<int *>(mall + a.T * a.W);                      // [G]
     uint64_t *full = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(live + a.G) + 7) & ~(uintptr_t)7);
     uint64_t *empty = full + NS;
     __shared__ int s_nlive, s_err;
+    __shared__ float s_rn[kFTok];
 
     const int tid = (int)threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ri = (int)blockIdx.x / a.TG, tb = (int)blockIdx.x % a.TG;
@@ -304,7 +386,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __syncthreads();
 
     const int n_live = s_nlive;
-    const int KW = a.kw, nks = KW / 128, NUS = kFStageCols / KW;
+    const int KW = a.kw, NUS = kFStageElems / 8 / KW;   // 8-row units per stage
     const int N8 = n_live * gs / 8;                      // union rows in units of 8
     const int u0 = (int)((int64_t)ri * N8 / a.P), u1 = (int)((int64_t)(ri + 1) * N8 / a.P);
     const int nRB = (u1 - u0 + NUS - 1) / NUS;           // phase-1 row blocks
@@ -326,8 +408,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 uint8_t *sb = slots + (size_t)slot * a.slot_bytes + a.h2_off;
                 const int gb = s2 * a.ng2, ge = min(n_live, gb + a.ng2);
                 for (int i = gb; i < ge; ++i)
-                    tma_load_2d(sb + (size_t)(i - gb) * a.h2_bytes, &tm_h, live[i] * gs, t0,
-                                &full[slot]);
+                    tma_load_3d(sb + (size_t)(i - gb) * a.h2_stride, &tm_h, 0, live[i] * gs / 16,
+                                t0 / 2, &full[slot]);
             };
             auto grid_done = [&]() {
                 if (!passed && ld_acquire_gpu(a.bar) >= gridDim.x) {
@@ -403,35 +485,39 @@ __global__ void __launch_bounds__(kFThreads, 1)
     } else {
         // ------------------------------------------------ consumers
         const int ct = tid - 32, cw = ct >> 5;
-        const int r = lane >> 3;                // row of 4 in the warp
-        const int c = lane & 7, sw = (c >> 2) & 1;
         bool ok = true;
-        auto wait_full = [&](int k) {
-            if (ok && !mbar_wait(&full[k % NS], (uint32_t)(k / NS) & 1u)) {
+        // ring position: slot index, its phase parity and its base address
+        int slot = 0;
+        uint32_t par = 0;
+        const uint8_t *sp = slots;
+        const uint32_t slot_bytes = a.slot_bytes;
+        auto wait_full = [&]() {
+            if (ok && !mbar_wait(&full[slot], par)) {
                 ok = false;
                 set_status(a.status, WIDE_DEV_TIMEOUT);
                 atomicExch(&s_err, 1);
             }
         };
-        auto release = [&](int k) {
+        auto release = [&]() {
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&empty[k % NS]);
+                mbar_arrive(&empty[slot]);
+            sp += slot_bytes;
+            if (++slot == NS) {
+                slot = 0;
+                par ^= 1u;
+                sp = slots;
+            }
         };
 
-        // x of this CTA's tokens, fp32 (rows bt..TB-1 zero)
+        // ---- x of this CTA's tokens as bf16 token pairs (tokens bt.. zero)
         if (a.xf) {
-            // RMSNorm fused: warp cw normalises token cw (bf16-rounded, as a
-            // bf16 layer feeds its FFN)
-            for (int t = cw; t < TB; t += kFWarps) {
-                float *xr = xs + (size_t)t * H;
-                if (t >= bt) {
-                    for (int k = lane * 4; k < H; k += 128)
-                        *reinterpret_cast<float4 *>(xr + k) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    continue;
-                }
+            // RMSNorm fused: warp cw finds 1 / rms of token cw; the values
+            // are rounded to bf16, as a bf16 layer feeds its FFN
+            for (int t = cw; t < bt; t += kFWarps) {
                 const float *src = a.xf + (size_t)(t0 + t) * H;
                 float ss = 0.f;
+#pragma unroll 8
                 for (int k = lane * 4; k < H; k += 128) {
                     const float4 v = *reinterpret_cast<const float4 *>(src + k);
                     ss = fmaf(v.x, v.x, ss);
@@ -441,105 +527,126 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 }
                 for (int off = 16; off; off >>= 1)
                     ss += __shfl_xor_sync(0xffffffffu, ss, off);
-                const float rn = 1.0f / sqrtf(ss / (float)H + a.eps);
-                for (int k = lane * 4; k < H; k += 128) {
-                    const float4 v = *reinterpret_cast<const float4 *>(src + k);
-                    const uint2 gw = *reinterpret_cast<const uint2 *>(a.gamma + k);
-                    float4 y;
-                    y.x = __bfloat162float(__float2bfloat16_rn(
-                        v.x * rn * __uint_as_float(gw.x << 16)));
-                    y.y = __bfloat162float(__float2bfloat16_rn(
-                        v.y * rn * __uint_as_float(gw.x & 0xffff0000u)));
-                    y.z = __bfloat162float(__float2bfloat16_rn(
-                        v.z * rn * __uint_as_float(gw.y << 16)));
-                    y.w = __bfloat162float(__float2bfloat16_rn(
-                        v.w * rn * __uint_as_float(gw.y & 0xffff0000u)));
-                    *reinterpret_cast<float4 *>(xr + k) = y;
-                }
+                if (lane == 0)
+                    s_rn[t] = 1.0f / sqrtf(ss / (float)H + a.eps);
             }
-        } else {
-            // all loads of a batch go out before any is used
-            constexpr int kB = 8;
-            const int cpr = H / 8, n = TB * cpr;
-            for (int i0 = ct; i0 < n; i0 += 32 * kFWarps * kB) {
-                uint4 v[kB];
+            consumer_sync();
+        }
+        {
+            // one 16-byte unit per step: 4 columns of one token pair; the
+            // global loads of kXB steps go out before any is used
+            constexpr int kXB = 8;
+            const int nu4 = H / 4, n = NP * nu4;
+            for (int i0 = ct; i0 < n; i0 += kFCons * kXB) {
+                uint2 v2[kXB][2];
 #pragma unroll
-                for (int u = 0; u < kB; ++u) {
-                    const int i = i0 + u * 32 * kFWarps;
-                    const int t = i / cpr, q = i % cpr;
-                    v[u] = (i < n && t < bt) ? *reinterpret_cast<const uint4 *>(
-                                                   a.x + (size_t)(t0 + t) * H + q * 8)
-                                             : make_uint4(0u, 0u, 0u, 0u);
+                for (int q = 0; q < kXB; ++q) {
+                    const int i = i0 + q * kFCons;
+                    const int tp = i / nu4, u4 = i % nu4;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int t = 2 * tp + e;
+                        v2[q][e] = make_uint2(0u, 0u);
+                        if (i >= n || t >= bt)
+                            continue;
+                        if (a.xf) {
+                            const float4 v = *reinterpret_cast<const float4 *>(
+                                a.xf + (size_t)(t0 + t) * H + 4 * u4);
+                            const uint2 gw = *reinterpret_cast<const uint2 *>(a.gamma + 4 * u4);
+                            const float rn = s_rn[t];
+                            const __nv_bfloat162 p0 = __floats2bfloat162_rn(
+                                v.x * rn * bf_lo(gw.x), v.y * rn * bf_hi(gw.x));
+                            const __nv_bfloat162 p1 = __floats2bfloat162_rn(
+                                v.z * rn * bf_lo(gw.y), v.w * rn * bf_hi(gw.y));
+                            v2[q][e].x = *reinterpret_cast<const uint32_t *>(&p0);
+                            v2[q][e].y = *reinterpret_cast<const uint32_t *>(&p1);
+                        } else {
+                            v2[q][e] = *reinterpret_cast<const uint2 *>(
+                                a.x + (size_t)(t0 + t) * H + 4 * u4);
+                        }
+                    }
                 }
 #pragma unroll
-                for (int u = 0; u < kB; ++u) {
-                    const int i = i0 + u * 32 * kFWarps;
-                    if (i < n) {
-                        const int t = i / cpr, q = i % cpr;
-                        float f[8];
-                        bf16x8_to_f32(v[u], f);
-                        float *d = xs + (size_t)t * H + q * 8;
-                        *reinterpret_cast<float4 *>(d) = make_float4(f[0], f[1], f[2], f[3]);
-                        *reinterpret_cast<float4 *>(d + 4) = make_float4(f[4], f[5], f[6], f[7]);
-                    }
+                for (int q = 0; q < kXB; ++q) {
+                    const int i = i0 + q * kFCons;
+                    if (i >= n)
+                        break;
+                    const int tp = i / nu4, u4 = i % nu4;
+                    uint4 o;
+                    o.x = __byte_perm(v2[q][0].x, v2[q][1].x, 0x5410);
+                    o.y = __byte_perm(v2[q][0].x, v2[q][1].x, 0x7632);
+                    o.z = __byte_perm(v2[q][0].y, v2[q][1].y, 0x5410);
+                    o.w = __byte_perm(v2[q][0].y, v2[q][1].y, 0x7632);
+                    *reinterpret_cast<uint4 *>(xs + (size_t)tp * H * 4 + (u4 >> 1) * 32 +
+                                               (((u4 & 1) ^ ((u4 >> 3) & 1)) << 4)) = o;
                 }
             }
         }
         consumer_sync();
 
         // ---- phase 1
-        // warp cw: row (cw & 1) * 4 + r of unit ui, 128-column pieces ks, ks+1
-        const int pw = cw >> 1;                    // piece pair 0..3
-        const int ui = (2 * pw) / nks, ks = (2 * pw) % nks;
-        const int row = (cw & 1) * 4 + r;
-        const int nps = nks / 2;                   // piece pairs per unit
-        const uint32_t rs = (uint32_t)KW * 2u;     // row stride of a unit in the slot
-        const uint8_t *xbase = reinterpret_cast<const uint8_t *>(xs) + ks * 512;
-        int k = 0;
+        // thread: row set rsi (rows 2 rsi, 2 rsi + 1 of a stage), chunk ch
+        const int CPR = KW / 8, NWR = CPR / 32;         // chunks per row, warps per row
+        const int rsi = ct / CPR, ch = ct % CPR;
+        const uint32_t rs = (uint32_t)KW * 2u;           // row stride in the slot
+        const uint32_t wofs = (uint32_t)rsi * 2u * rs + (uint32_t)ch * 16u;
+        const uint32_t swb = ((uint32_t)ch >> 2) & 1u;
+        const uint32_t xo[2] = {(uint32_t)ch * 32u + (swb << 4), (uint32_t)ch * 32u + ((swb ^ 1u) << 4)};
+        const uint32_t xpair = (uint32_t)H * 4u, xwin = (uint32_t)KW * 4u;
+        constexpr int S1 = scatter_levels(2 * TBP, 5);   // (gate, up) of one (row, token) left
+        float2 *red1 = reinterpret_cast<float2 *>(red);  // [2][8 row sets][32 lanes]
         for (int rb = 0; rb < nRB; ++rb) {
             const int ub = u0 + rb * NUS, nu = min(NUS, u1 - ub);
-            float2 ag[TB], au[TB];
+            const bool act = (rsi >> 2) < nu;
+            float2 ag[2][NP], au[2][NP];
 #pragma unroll
-            for (int t = 0; t < TB; ++t) {
-                ag[t] = make_float2(0.f, 0.f);
-                au[t] = make_float2(0.f, 0.f);
-            }
-            for (int kw = 0; kw < NKW; ++kw, ++k) {
-                wait_full(k);
-                if (ui < nu) {
-                    const uint8_t *sg = slots + (size_t)(k % NS) * a.slot_bytes +
-                                        (size_t)ui * box1 + ks * 256;
-                    p1_stage<TB>(sg, sg + kFSlotMin / 2, xbase + (size_t)kw * KW * 4, H, rs, row,
-                                 c, sw, ag, au);
-                }
-                release(k);
-            }
-            // lane sums, then the piece pairs of a unit through shared memory
-            float *rd = red + (rb & 1) * (4 * 8 * 2 * TB);
+            for (int i = 0; i < 2; ++i)
 #pragma unroll
-            for (int t = 0; t < TB; ++t) {
-                const float g = sum8(ag[t].x + ag[t].y);
-                const float u = sum8(au[t].x + au[t].y);
-                if (c == (t & 7)) {
-                    float *e = rd + ((pw * 8 + row) * 2) * TB + t;
-                    e[0] = g;
-                    e[TB] = u;
+                for (int tp = 0; tp < NP; ++tp) {
+                    ag[i][tp] = make_float2(0.f, 0.f);
+                    au[i][tp] = make_float2(0.f, 0.f);
+                }
+            const uint8_t *xk = xs;
+            for (int kw = 0; kw < NKW; ++kw, xk += xwin) {
+                wait_full();
+                if (act)
+                    p1_stage<NP>(sp + wofs, sp + kFSlotMin / 2 + wofs, rs, xk, xpair, xo, ag, au);
+                release();
+            }
+            // sums over the chunks of the row: lanes, then the warps of a row
+            float v[4 * TBP];
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int tp = 0; tp < NP; ++tp) {
+                    v[((i * TBP) + 2 * tp) * 2 + 0] = ag[i][tp].x;
+                    v[((i * TBP) + 2 * tp) * 2 + 1] = au[i][tp].x;
+                    v[((i * TBP) + 2 * tp + 1) * 2 + 0] = ag[i][tp].y;
+                    v[((i * TBP) + 2 * tp + 1) * 2 + 1] = au[i][tp].y;
+                }
+            lane_reduce<4 * TBP, 5, 2>(v, lane);
+            float g = v[0], u = v[1];
+            if (NWR == 2) {
+                float2 *r1 = red1 + (rb & 1) * 256 + rsi * 32 + lane;
+                if (cw & 1)
+                    *r1 = make_float2(g, u);
+                consumer_sync();
+                if (!(cw & 1)) {
+                    const float2 o = *r1;
+                    g += o.x;
+                    u += o.y;
                 }
             }
-            consumer_sync();
-            for (int i = ct; i < nu * 8 * TB; i += 32 * kFWarps) {
-                const int un = i / (8 * TB), rrow = (i / TB) % 8, t = i % TB;
-                float g = 0.f, u = 0.f;
-                for (int s = 0; s < nps; ++s) {
-                    const float *e = rd + (((un * nps + s) * 8 + rrow) * 2) * TB + t;
-                    g += e[0];
-                    u += e[TB];
-                }
+            const bool owner =
+                (NWR == 1 || !(cw & 1)) && (lane & ((1 << (5 - S1)) - 1)) == 0;
+            if (act && owner) {
+                const int combo = lane >> (5 - S1);      // row * TBP + token
+                const int r = combo / TBP, t = combo % TBP;
                 if (t < bt) {
-                    const int lr = (ub + un) * 8 + rrow;
+                    const int lr = ub * 8 + rsi * 2 + r;
                     const int grp = live[lr / gs];
                     const bool keep = (mall[(t0 + t) * W + (grp >> 5)] >> (grp & 31)) & 1u;
-                    a.h[(size_t)(t0 + t) * a.I + grp * gs + lr % gs] =
+                    a.h[il2(t0 + t, (size_t)grp * gs + lr % gs, (size_t)a.I)] =
                         keep ? silu_f32(g) * u : 0.f;
                 }
             }
@@ -554,60 +661,74 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
 
         // ---- phase 2
-        if (n2rows > 0) {
-            const int R2 = (n2rows + 31) / 32;
-            const int rw = cw * 4 + r;             // rows rw + 32 k
-            const int rmax = n2rows - 1;
-            float2 acc[kFMaxR2][TB];
+        // thread: instance gi (groups gi, gi + NI, ...), rows row0 .. row0 +
+        // RT - 1 of the range, chunk ch2 of each group
+        const int CPR2 = gs / 8, RT = a.rt, NR = a.nr, NI = a.ni, TPI = CPR2 * NR;
+        const int gi = ct / TPI, rem = ct % TPI, ch2 = rem % CPR2;
+        const int row0 = (rem / CPR2) * RT, rmax = n2rows - 1;
+        const bool act2 = gi < NI;
+        // this thread's offsets in a group's W_down box (rows past rmax read
+        // row rmax; their sums are discarded) and h box
+        const uint32_t wrs = (uint32_t)gs * 2u;
+        const uint32_t wbase = (uint32_t)row0 * wrs + (uint32_t)ch2 * 16u;
+        const uint32_t wmax = (uint32_t)rmax * wrs + (uint32_t)ch2 * 16u;
+        uint32_t hoff[NP];
 #pragma unroll
-            for (int rr = 0; rr < kFMaxR2; ++rr)
+        for (int tp = 0; tp < NP; ++tp) {
+            const uint32_t idx = (uint32_t)tp * ((uint32_t)gs / 2u) + (uint32_t)ch2 * 4u;
+            const uint32_t r = idx >> 3;
+            hoff[tp] = r * 128u + (((idx ^ r) & 7u) << 4);
+        }
+        float2 acc[kFMaxRT][NP];
 #pragma unroll
-                for (int t = 0; t < TB; ++t)
-                    acc[rr][t] = make_float2(0.f, 0.f);
-            for (int s2 = 0; s2 < n2s; ++s2, ++k) {
-                wait_full(k);
-                const uint8_t *sb = slots + (size_t)(k % NS) * a.slot_bytes;
-                const int gb = s2 * a.ng2, ge = min(n_live, gb + a.ng2);
-                for (int i = 0; i < ge - gb; ++i) {
-                    const uint8_t *wb = sb + (size_t)i * a.w2_bytes;
-                    const uint8_t *hb = sb + a.h2_off + (size_t)i * a.h2_bytes;
-                    if (R2 == 1)       // R2 <= kFMaxR2 = 3 (rows_box <= 96)
-                        p2_group<TB, 1>(wb, hb, gs, rw, rmax, c, sw, acc);
-                    else if (R2 == 2)
-                        p2_group<TB, 2>(wb, hb, gs, rw, rmax, c, sw, acc);
-                    else
-                        p2_group<TB, 3>(wb, hb, gs, rw, rmax, c, sw, acc);
+        for (int r = 0; r < kFMaxRT; ++r)
+#pragma unroll
+            for (int tp = 0; tp < NP; ++tp)
+                acc[r][tp] = make_float2(0.f, 0.f);
+        const uint32_t w2b = a.w2_bytes, h2s = a.h2_stride, h2o = a.h2_off;
+        int gnext = gi;                              // this instance's next union group
+        for (int gb = 0; gb < n_live && n2rows > 0; gb += a.ng2) {
+            const int ge = min(n_live, gb + a.ng2);
+            wait_full();
+            for (; act2 && gnext < ge; gnext += NI) {
+                const uint8_t *wb = sp + (uint32_t)(gnext - gb) * w2b;
+                const uint8_t *hb = sp + h2o + (uint32_t)(gnext - gb) * h2s;
+                switch (RT) {      // 1 <= RT <= kFMaxRT
+                case 4: p2_group<NP, 4>(wb, wbase, wrs, wmax, hb, hoff, acc); break;
+                case 3: p2_group<NP, 3>(wb, wbase, wrs, wmax, hb, hoff, acc); break;
+                case 2: p2_group<NP, 2>(wb, wbase, wrs, wmax, hb, hoff, acc); break;
+                default: p2_group<NP, 1>(wb, wbase, wrs, wmax, hb, hoff, acc); break;
                 }
-                release(k);
             }
-#pragma unroll
-            for (int rr = 0; rr < kFMaxR2; ++rr) {
-                if (rr >= R2)
-                    break;
-                const int row = rr * 32 + rw;
-#pragma unroll
-                for (int t = 0; t < TB; ++t) {
-                    const float v = sum8(acc[rr][t].x + acc[rr][t].y);
-                    if (row < n2rows && c == (t & 7) && t < bt) {
-                        const size_t at = (size_t)(t0 + t) * H + j0 + row;
-                        const DownOutputs &o = a.o;
-                        if (o.out_sum)
-                            static_cast<__nv_bfloat16 *>(o.out_sum)[at] = __float2bfloat16_rn(v);
-                        if (o.out_total || o.out_total_f32) {
-                            float tot = v;
-                            if (o.res_in)
-                                tot += __bfloat162float(
-                                    static_cast<const __nv_bfloat16 *>(o.res_in)[at]);
-                            if (o.res_f32)
-                                tot += o.res_f32[at];
-                            if (o.out_total)
-                                static_cast<__nv_bfloat16 *>(o.out_total)[at] =
-                                    __float2bfloat16_rn(tot);
-                            if (o.out_total_f32)
-                                o.out_total_f32[at] = tot;
-                        }
-                    }
-                }
+            release();
+        }
+        const int rstride = NR * RT;
+        if (CPR2 == 8)
+            p2_reduce<NP, 3>(acc, ch2, act2, gi, row0, RT, n2rows, rstride, red);
+        else if (CPR2 == 16)
+            p2_reduce<NP, 4>(acc, ch2, act2, gi, row0, RT, n2rows, rstride, red);
+        else
+            p2_reduce<NP, 5>(acc, ch2, act2, gi, row0, RT, n2rows, rstride, red);
+        consumer_sync();
+        for (int idx = ct; idx < n2rows * bt; idx += kFCons) {
+            const int row = idx % n2rows, t = idx / n2rows;
+            float v = 0.f;
+            for (int q = 0; q < NI; ++q)
+                v += red[((size_t)q * rstride + row) * TBP + t];
+            const size_t at = (size_t)(t0 + t) * H + j0 + row;
+            const DownOutputs &o = a.o;
+            if (o.out_sum)
+                static_cast<__nv_bfloat16 *>(o.out_sum)[at] = __float2bfloat16_rn(v);
+            if (o.out_total || o.out_total_f32) {
+                float tot = v;
+                if (o.res_in)
+                    tot += __bfloat162float(static_cast<const __nv_bfloat16 *>(o.res_in)[at]);
+                if (o.res_f32)
+                    tot += o.res_f32[at];
+                if (o.out_total)
+                    static_cast<__nv_bfloat16 *>(o.out_total)[at] = __float2bfloat16_rn(tot);
+                if (o.out_total_f32)
+                    o.out_total_f32[at] = tot;
             }
         }
     }
@@ -643,8 +764,8 @@ int tok_block(int T) { return T <= 1 ? 1 : (T <= 2 ? 2 : (T <= 4 ? 4 : 8)); }
 
 // Launch geometry of one call; false if the shape does not fit the kernel.
 struct FusedPlan {
-    int TB, TG, P, kw, rows_box, ng2, nslots;
-    uint32_t slot_bytes, w2_bytes, h2_bytes, h2_off;
+    int TB, TG, P, kw, rows_box, rt, nr, ni, ng2, nslots;
+    uint32_t slot_bytes, w2_bytes, h2_bytes, h2_stride, h2_off;
     size_t smem;
 };
 
@@ -659,28 +780,49 @@ bool plan_fused(int T, int H, int I, int gs, FusedPlan *p)
     if (di.sms <= 0)
         return false;
     p->TB = tok_block(T);
+    const int TBP = p->TB < 2 ? 2 : p->TB;
     p->TG = (T + kFTok - 1) / kFTok;
     p->P = di.sms / p->TG;
     if (p->P < 1)
         return false;
-    p->kw = kFStageCols;
-    while (H % p->kw != 0)
-        p->kw >>= 1;                              // 1024, 512 or 256 (two pieces per warp)
+    p->kw = H % 512 == 0 ? 512 : 256;
     p->rows_box = (H + p->P - 1) / p->P;
-    if (p->rows_box > 32 * kFMaxR2)
+    // phase 2: NI = 512 / TPI instances of TPI threads (whole warps, so no
+    // warp holds two instances that work on different groups), each NR =
+    // TPI / (gs / 8) row sets of RT = ceil(rows / NR) <= 4 rows.  Time per
+    // thread ~ (RT + 2) / NI (the 2: the h reads of a group, shared by its
+    // rows).
+    const int cpr2 = gs / 8;
+    double best = 0.0;
+    p->rt = 0;
+    for (int tpi = 32; tpi <= kFCons; tpi *= 2) {
+        const int nr = tpi / cpr2;
+        const int rt = (p->rows_box + nr - 1) / nr;
+        if (rt > kFMaxRT)
+            continue;
+        const int ni = kFCons / tpi;
+        const double cost = (double)(rt + 2) / ni;
+        if (p->rt == 0 || cost < best) {
+            best = cost;
+            p->rt = rt;
+            p->nr = nr;
+            p->ni = ni;
+        }
+    }
+    if (p->rt == 0 || p->ni * p->nr * p->rt * TBP > kFRedFloats)
         return false;
     p->w2_bytes = (uint32_t)p->rows_box * gs * 2u;
-    p->h2_bytes = (uint32_t)p->TB * gs * 4u;
-    const uint32_t per_group = p->w2_bytes + p->h2_bytes;
-    p->ng2 = (int)(kFSlotMin / per_group);
+    p->h2_bytes = (uint32_t)TBP * gs * 4u;
+    p->h2_stride = (p->h2_bytes + 1023u) & ~1023u;    // 128-byte swizzle: 1024-aligned boxes
+    p->ng2 = (int)(kFSlotMin / (p->w2_bytes + p->h2_stride));
     if (p->ng2 < 1)
         p->ng2 = 1;
-    p->h2_off = (uint32_t)p->ng2 * p->w2_bytes;
-    uint32_t slot = (uint32_t)p->ng2 * per_group;
+    p->h2_off = ((uint32_t)p->ng2 * p->w2_bytes + 1023u) & ~1023u;
+    uint32_t slot = p->h2_off + (uint32_t)p->ng2 * p->h2_stride;
     if (slot < kFSlotMin)
         slot = kFSlotMin;
     p->slot_bytes = (slot + 1023u) & ~1023u;
-    const size_t fixed = 1024 + (size_t)p->TB * H * 4 + (size_t)2 * 4 * 8 * 2 * p->TB * 4 +
+    const size_t fixed = 1024 + (size_t)TBP * H * 2 + (size_t)kFRedFloats * 4 +
                          (size_t)T * W * 4 + (size_t)G * 4 + 8 + 2 * kFMaxSlots * 8;
     if ((size_t)di.optin <= fixed + 64)
         return false;
@@ -726,12 +868,20 @@ bool decode_ffn_fused_supported(int T, int H, int I, int gs)
     return plan_fused(T, H, I, gs, &p);
 }
 
-// Measured on B200 (3B FFN, 50% keep): the fused kernel beats the two GEMV
-// kernels of ffn_decode.cu for up to 8 tokens per call (one token block);
-// for more tokens the extra h traffic of its phase 2 makes it slower.
+namespace {
+std::atomic<int> g_decode_mode{WIDE_DECODE_AUTO};
+}
+
+// Measured on B200 (3B FFN at 50% keep and 8B FFN at 72% keep, 1..32
+// tokens): the fused kernel beats the two GEMV kernels of ffn_decode.cu at
+// every token count it supports (by 1-26%), so AUTO takes it wherever its
+// shape limits allow.
 bool decode_ffn_fused_preferred(int T, int H, int I, int gs)
 {
-    return T <= kFTok && decode_ffn_fused_supported(T, H, I, gs);
+    const int mode = g_decode_mode.load(std::memory_order_relaxed);
+    if (mode == WIDE_DECODE_GEMV)
+        return false;
+    return decode_ffn_fused_supported(T, H, I, gs);
 }
 
 int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, int I, int gs,
@@ -742,10 +892,11 @@ int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, i
         return WIDE_EUNSUPPORTED;
     const int G = I / gs;
     CUtensorMap tg, tu, td, th;
+    const int TBP = pl.TB < 2 ? 2 : pl.TB;
     if (!make_tmap_rows3d(&tg, in.w_gate, I, H, H, pl.kw / 64, 8) ||
         !make_tmap_rows3d(&tu, in.w_up, I, H, H, pl.kw / 64, 8) ||
         !make_tmap_2d(&td, in.w_down, H, I, I, 2, pl.rows_box, gs, false) ||
-        !make_tmap_2d(&th, h, T, I, I, 4, pl.TB, gs, false))
+        !make_tmap_f32_pairs(&th, h, (T + 1) / 2, I, gs, TBP / 2))
         return WIDE_CUDA_FAIL();
     FusedArgs a = {};
     a.x = static_cast<const __nv_bfloat16 *>(in.x);
@@ -765,10 +916,14 @@ int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, i
     a.TG = pl.TG;
     a.P = pl.P;
     a.kw = pl.kw;
+    a.rt = pl.rt;
+    a.nr = pl.nr;
+    a.ni = pl.ni;
     a.nslots = pl.nslots;
     a.slot_bytes = pl.slot_bytes;
     a.w2_bytes = pl.w2_bytes;
     a.h2_bytes = pl.h2_bytes;
+    a.h2_stride = pl.h2_stride;
     a.h2_off = pl.h2_off;
     a.ng2 = pl.ng2;
     a.status = status_ptr();
@@ -783,3 +938,10 @@ int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, i
 }
 
 }  // namespace wide
+
+extern "C" int wide_set_decode_ffn_path(int mode)
+{
+    if (mode != WIDE_DECODE_AUTO && mode != WIDE_DECODE_FUSED && mode != WIDE_DECODE_GEMV)
+        return WIDE_EINVAL;
+    return wide::g_decode_mode.exchange(mode);
+}

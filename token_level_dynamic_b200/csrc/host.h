@@ -31,6 +31,15 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
 bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                       uint64_t pitch_elems, uint32_t box_chunks, uint32_t box_rows);
 
+// Encodes an fp32 [T][cols] activation stored with token pairs interleaved
+// (row t/2 holds 2 * cols floats: tokens t and t+1 side by side per column)
+// as the 3-D tensor {32, 2 * cols / 32, pairs} with 128-byte swizzle: a box
+// {32, box_cols / 16, box_pairs} copies box_cols columns of box_pairs token
+// pairs, landing as box_pairs x (box_cols / 16) rows of 128 bytes whose
+// 16-byte chunks are XOR-permuted by (row & 7).  cols % 16 == 0.
+bool make_tmap_f32_pairs(CUtensorMap *map, const float *base, uint64_t pairs, uint64_t cols,
+                         uint32_t box_cols, uint32_t box_pairs);
+
 // Raises a kernel's dynamic shared memory limit to at least `bytes` (once
 // per kernel, device and size).
 bool raise_smem_limit(const void *kernel, size_t bytes);
@@ -194,8 +203,9 @@ struct FusedInput {
     const uint32_t *mask;
 };
 // bf16 decode FFN of 1 <= T <= 32 tokens as one persistent cooperative
-// kernel (ffn_decode_fused.cu).  h: fp32 [T][I] scratch; bar: 2 words of
-// device memory for the grid barrier (the call zeroes bar[0] on the stream).
+// kernel (ffn_decode_fused.cu).  h: fp32 [T][I] scratch with token pairs
+// interleaved (T rounded up to even); bar: 2 words of device memory for the
+// grid barrier (the call zeroes bar[0] on the stream).
 bool decode_ffn_fused_supported(int T, int H, int I, int gs);
 // Whether the decode path should use it for this shape (faster there).
 bool decode_ffn_fused_preferred(int T, int H, int I, int gs);
