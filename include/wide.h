@@ -238,7 +238,7 @@ int wide_set_decode_ffn_path(int mode);
  *
  * Supported: bf16; head_dim == 128; decode (seq_len == 1, n_seq <= 32,
  * n_q_heads / n_kv_heads in {1, 2, 4}, hidden % 512 == 0, ffn_group_size in
- * {64, 128}).
+ * {64, 128}, cache_len < 131072).
  */
 typedef struct wide_layer_dims {
     int64_t n_seq;           /* sequences */

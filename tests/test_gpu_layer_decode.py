@@ -69,6 +69,37 @@ def test_decode_layer_ragged_cache_and_batch():
     _check(lc, _run(lc))
 
 
+@pytest.mark.parametrize("cache_len,n_q,n_kv", [(127, 8, 2), (128, 4, 4), (300, 4, 2), (1000, 8, 2)])
+def test_decode_layer_key_slices(cache_len, n_q, n_kv):
+    """Caches that span several 128-key attention slices, with a ragged last
+    slice (cache_len + 1 keys), for 4, 1 and 2 query heads per group."""
+    lc = synth.small_layer("decode", seed=cache_len, n_seq=6, cache_len=cache_len, H=512,
+                           n_q=n_q, n_kv=n_kv, hd=128, I=1024, gs=128, keep_a=0.5, keep_f=0.5)
+    _check(lc, _run(lc))
+
+
+def test_decode_layer_repeated_calls_reuse_workspace():
+    """Two calls in a row on one workspace give the same attention output
+    (the slice counters are reset between calls)."""
+    import torch
+    import token_level_dynamic_b200 as w
+    lc = synth.small_layer("decode", seed=21, n_seq=4, cache_len=400, H=512, n_q=8, n_kv=2,
+                           hd=128, I=1024, gs=128, keep_a=0.7, keep_f=0.5)
+    x, wts, kc, vc, hm, fm, cap = layer_to_dev(lc)
+    d = layer_dims(lc, cap)
+    ws = torch.full((w.wide_layer_workspace_bytes(d),), 0xAB, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        attn = torch.empty_like(x)
+        w.wide_attn_masked(x, wts, kc, vc, hm, d, attn_out=attn, workspace=ws)
+        outs.append(from_dev(attn))
+    torch.cuda.synchronize()
+    assert w.wide_get_device_status() == 0
+    np.testing.assert_array_equal(outs[0], outs[1])
+    ref, p = layer_masked(lc, ret_parts=True)
+    assert rel_l2(outs[0], p["attn_out"]) <= TOL
+
+
 def test_decode_layer_empty_cache():
     lc = synth.small_layer("decode", seed=12, n_seq=3, cache_len=0, H=512, n_q=8, n_kv=2,
                            hd=128, I=1024, gs=128)

@@ -136,6 +136,17 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// Untiled bulk copy of `bytes` contiguous bytes global -> shared, completing
+// on an mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes,
+                                          uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -176,6 +187,31 @@ __host__ __device__ __forceinline__ size_t il2(int t, size_t col, size_t ld)
 }
 
 // ------------------------------------------------------------- numerics
+
+// Word i (0..3, a compile-time index after unrolling) of a 16-byte chunk.
+__device__ __forceinline__ uint32_t word(const uint4 v, int i)
+{
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// The bf16 in the low / high half of w as fp32 (byte permutes: exact).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x1044)); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x3244)); }
+// ... in both halves of a register pair (the weight operand of a token
+// pair), each half written by its own byte permute
+__device__ __forceinline__ float2 dup_lo(uint32_t w)
+{
+    uint32_t a, b;
+    asm("prmt.b32 %0, %2, 0, 0x1044;\n\tprmt.b32 %1, %2, 0, 0x1044;" : "=r"(a), "=r"(b) : "r"(w));
+    return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+__device__ __forceinline__ float2 dup_hi(uint32_t w)
+{
+    uint32_t a, b;
+    asm("prmt.b32 %0, %2, 0, 0x3244;\n\tprmt.b32 %1, %2, 0, 0x3244;" : "=r"(a), "=r"(b) : "r"(w));
+    return make_float2(__uint_as_float(a), __uint_as_float(b));
+}
+
 
 // Widens 8 bf16 values (one 16-byte chunk) to fp32 exactly.
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&f)[8])

@@ -109,30 +109,6 @@ __device__ __forceinline__ float4 lds128f(const uint8_t *p)
     return *reinterpret_cast<const float4 *>(p);
 }
 
-// Word i (0..3, a compile-time index after unrolling) of a 16-byte chunk.
-__device__ __forceinline__ uint32_t word(const uint4 v, int i)
-{
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
-// The bf16 in the low / high half of w as fp32 (byte permutes: exact).
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x1044)); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(__byte_perm(w, 0u, 0x3244)); }
-// ... in both halves of a register pair (the weight operand of a token
-// pair), each half written by its own byte permute
-__device__ __forceinline__ float2 dup_lo(uint32_t w)
-{
-    uint32_t a, b;
-    asm("prmt.b32 %0, %2, 0, 0x1044;\n\tprmt.b32 %1, %2, 0, 0x1044;" : "=r"(a), "=r"(b) : "r"(w));
-    return make_float2(__uint_as_float(a), __uint_as_float(b));
-}
-__device__ __forceinline__ float2 dup_hi(uint32_t w)
-{
-    uint32_t a, b;
-    asm("prmt.b32 %0, %2, 0, 0x3244;\n\tprmt.b32 %1, %2, 0, 0x3244;" : "=r"(a), "=r"(b) : "r"(w));
-    return make_float2(__uint_as_float(a), __uint_as_float(b));
-}
-
 // The two float pairs of one float4.
 __device__ __forceinline__ float2 lo2(const float4 v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(const float4 v) { return make_float2(v.z, v.w); }
