@@ -790,21 +790,35 @@ bool plan_fused(int T, int H, int I, int gs, FusedPlan *p)
     p->w2_bytes = (uint32_t)p->rows_box * gs * 2u;
     p->h2_bytes = (uint32_t)TBP * gs * 4u;
     p->h2_stride = (p->h2_bytes + 1023u) & ~1023u;    // 128-byte swizzle: 1024-aligned boxes
-    p->ng2 = (int)(kFSlotMin / (p->w2_bytes + p->h2_stride));
-    if (p->ng2 < 1)
-        p->ng2 = 1;
-    p->h2_off = ((uint32_t)p->ng2 * p->w2_bytes + 1023u) & ~1023u;
-    uint32_t slot = p->h2_off + (uint32_t)p->ng2 * p->h2_stride;
-    if (slot < kFSlotMin)
-        slot = kFSlotMin;
-    p->slot_bytes = (slot + 1023u) & ~1023u;
     const size_t fixed = 1024 + (size_t)TBP * H * 2 + (size_t)kFRedFloats * 4 +
                          (size_t)T * W * 4 + (size_t)G * 4 + 8 + 2 * kFMaxSlots * 8;
     if ((size_t)di.optin <= fixed + 64)
         return false;
-    int ns = (int)(((size_t)di.optin - fixed - 64) / p->slot_bytes);
-    if (ns > kFMaxSlots)
-        ns = kFMaxSlots;
+    // ring slots for ng phase-2 groups per stage (at least a phase-1 stage)
+    auto layout = [&](int ng, uint32_t *h2_off, uint32_t *slot_bytes) {
+        *h2_off = ((uint32_t)ng * p->w2_bytes + 1023u) & ~1023u;
+        uint32_t slot = *h2_off + (uint32_t)ng * p->h2_stride;
+        if (slot < kFSlotMin)
+            slot = kFSlotMin;
+        *slot_bytes = (slot + 1023u) & ~1023u;
+        const int ns = (int)(((size_t)di.optin - fixed - 64) / *slot_bytes);
+        return ns > kFMaxSlots ? kFMaxSlots : ns;
+    };
+    p->ng2 = (int)(kFSlotMin / (p->w2_bytes + p->h2_stride));
+    if (p->ng2 < 1)
+        p->ng2 = 1;
+    int ns = layout(p->ng2, &p->h2_off, &p->slot_bytes);
+    if (p->ng2 == 1) {
+        // two groups per phase-2 stage when the larger slots cost no slot
+        uint32_t off2, sb2;
+        const int ns2 = layout(2, &off2, &sb2);
+        if (ns2 >= ns && ns2 >= 2) {
+            p->ng2 = 2;
+            p->h2_off = off2;
+            p->slot_bytes = sb2;
+            ns = ns2;
+        }
+    }
     if (ns < 2)
         return false;
     p->nslots = ns;
