@@ -78,6 +78,13 @@ def test_decode_layer_key_slices(cache_len, n_q, n_kv):
     _check(lc, _run(lc))
 
 
+def test_decode_attention_long_cache_many_slices():
+    """A 70000-entry cache: hundreds of key slices merged by the last one."""
+    lc = synth.small_layer("decode", seed=23, n_seq=2, cache_len=70000, H=512, n_q=4, n_kv=1,
+                           hd=128, I=1024, gs=128, keep_a=1.0, keep_f=0.5)
+    _check(lc, _run(lc, attn_only=True), parts=("attn_out",))
+
+
 def test_decode_layer_repeated_calls_reuse_workspace():
     """Two calls in a row on one workspace give the same attention output
     (the slice counters are reset between calls)."""

@@ -52,9 +52,9 @@ __device__ __forceinline__ uint32_t token_group_mask(const uint32_t *mask, int T
 }
 
 // ------------------------------------------------------------- decode_qkv
-// Grid (KS key slices, n_q + 2 n_kv row blocks of hd rows), clusters of KS
-// CTAs along the slices.  Row block rb is query head rb, then the K heads,
-// then the V heads; a query head whose group no token keeps exits at once.
+// Grid (KS key slices, 2 n_kv + n_q row blocks of hd rows), clusters of KS
+// CTAs along the slices.  Row blocks are the K heads, the V heads, then the
+// query heads; a query head whose group no token keeps exits at once.
 // The CTA's active tokens (those that keep the head's group; every token
 // for K and V) are compacted and staged, times gamma, as fp32 token pairs;
 // its hd x kslice weight slab streams through a TMA ring of 64-column
@@ -228,12 +228,14 @@ __global__ void __launch_bounds__(kQkvThreads, NPMAX > 8 ? 1 : 2)
 
     int kind, head;
     const CUtensorMap *map;
-    if (rb < a.n_q) {
-        kind = 0; head = rb; map = &tm_q;
-    } else if (rb < a.n_q + a.n_kv) {
-        kind = 1; head = rb - a.n_q; map = &tm_k;
+    // K and V heads first: they carry every token, so they are the longest
+    // CTAs and should not be left for the last wave
+    if (rb < a.n_kv) {
+        kind = 1; head = rb; map = &tm_k;
+    } else if (rb < 2 * a.n_kv) {
+        kind = 2; head = rb - a.n_kv; map = &tm_v;
     } else {
-        kind = 2; head = rb - a.n_q - a.n_kv; map = &tm_v;
+        kind = 0; head = rb - 2 * a.n_kv; map = &tm_q;
     }
     const uint32_t all = a.T >= 32 ? 0xffffffffu : ((1u << a.T) - 1u);
     const uint32_t tmask = kind == 0 ? token_group_mask(a.head_mask, a.T, a.Wh, head / rep) : all;
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kQkvThreads, NPMAX > 8 ? 1 : 2)
 }
 
 // ------------------------------------------------------------ decode_attn
-// One CTA per (key slice s, KV head j, sequence b).  A sequence whose token
+// One CTA per (key slice s of <= 128 keys, KV head j, sequence b).  A sequence whose token
 // skips group j reads no K/V bytes: slice 0 of the pair writes the group's
 // zero output and every slice exits.  A kept pair's CTA bulk-copies its
 // slice of the K and V slabs (contiguous rows of the [cap][hd] cache) into
@@ -421,7 +423,9 @@ __global__ void __launch_bounds__(kHD)
     const int nk = (int)max((int64_t)0, min(a.nkeys, kb + a.C) - kb);
     uint8_t *ks = sm_attn;                                        // [C][hd] bf16
     uint8_t *vs = ks + (size_t)a.C * kHD * 2;                     // [C][hd] bf16
-    float *pv = reinterpret_cast<float *>(vs + (size_t)a.C * kHD * 2);   // [C][4] scores, then P
+    // K and V, later the merge's per-slice weights: the larger of the two
+    const size_t area = max((size_t)a.C * kHD * 4, ((size_t)a.S * REP * 8 + 15) & ~(size_t)15);
+    float *pv = reinterpret_cast<float *>(ks + area);             // [C][4] scores, then P
     float *sml = pv + 4 * a.C;                                    // [REP][2]
     uint64_t *bar = reinterpret_cast<uint64_t *>(sml + 8);
     __shared__ int s_last;
@@ -546,7 +550,7 @@ __global__ void __launch_bounds__(kHD)
     if (!s_last)
         return;
     __threadfence();
-    // every slice's (max, sum) into shared memory (the K tile's space), then
+    // every slice's (max, sum) into shared memory (the K/V tiles' space), then
     // each slice's weight 2^(m_s - M) per head
     float2 *wml = reinterpret_cast<float2 *>(ks);                 // [S][REP]
     const float2 *ml = a.part_ml + pair * a.S * REP;
@@ -663,7 +667,7 @@ bool layer_decode_supported(const wide_layer_dims *d)
             (d->n_q_heads / d->n_kv_heads) * kHD == 256 ||
             (d->n_q_heads / d->n_kv_heads) * kHD == 512) &&
            d->cache_cap >= d->cache_len + 1 && d->cache_len >= 0 &&
-           d->cache_len < 131072;   // attention slices' (max, sum) fit one K tile when merged
+           d->cache_len < 131072;   // bounds the attention merge's shared memory (64 KB)
 }
 
 size_t layer_decode_workspace(const wide_layer_dims *d) { return decode_ws(d, nullptr).total; }
@@ -739,7 +743,8 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
     aa.cache_cap = d->cache_cap;
     aa.scale_log2 = kLog2e / sqrtf((float)kHD);
     aa.status = status_ptr();
-    const size_t smem_att = (size_t)w.C * kHD * 2 * 2 + (size_t)w.C * 16 + 32 + 8;
+    const size_t kv_area = (size_t)w.C * kHD * 4, merge_area = ((size_t)w.S * rep * 8 + 15) & ~15;
+    const size_t smem_att = (kv_area > merge_area ? kv_area : merge_area) + (size_t)w.C * 16 + 32 + 8;
     void (*attn)(AttnArgs) = rep == 4 ? decode_attn<4> : rep == 2 ? decode_attn<2> : decode_attn<1>;
     if (!raise_smem_limit(reinterpret_cast<const void *>(attn), smem_att))
         return WIDE_CUDA_FAIL();
