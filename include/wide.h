@@ -142,7 +142,7 @@ typedef struct wide_worklist {
     int32_t *sig_perm;
     int32_t *sig_pos;
     uint32_t *tile_union;
-    int32_t *scratch;      /* rank partial sums, owned by wide_reorder */
+    int32_t *scratch;      /* bucket histogram, member lists and rank counters, owned by wide_reorder */
     int64_t tokens, groups;
     int32_t tile_m, scratch_splits;
 } wide_worklist;

@@ -40,7 +40,7 @@ def _compare(mask_words, G, tile_m):
 @pytest.mark.parametrize("T,G,tile_m,p", [
     (1, 1, 128, 1.0), (5, 3, 64, 0.5), (37, 33, 64, 0.3), (300, 112, 128, 0.5),
     (257, 64, 128, 0.0), (257, 64, 128, 1.0), (1000, 1024, 128, 0.5), (129, 40, 64, 0.9),
-    (2049, 8, 128, 0.34),
+    (2049, 8, 128, 0.34), (9000, 40, 128, 0.5), (20000, 5, 64, 0.5), (8192, 112, 128, 0.02),
 ])
 def test_reorder_bit_exact_random(T, G, tile_m, p):
     m = np.random.default_rng(T + G).random((T, G)) < p

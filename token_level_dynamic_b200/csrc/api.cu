@@ -183,7 +183,7 @@ bool worklist_layout(int64_t T, int64_t G, int32_t tile_m, WorklistLayout *L)
     L->sig_perm = take(4 * t);
     L->sig_pos = take(4 * t);
     L->tile_union = take(4 * nt * W);
-    L->scratch = take(4 * (size_t)L->splits * t);
+    L->scratch = take(reorder_scratch_bytes(T));
     L->total = off;
     return true;
 }

@@ -153,7 +153,10 @@ int tile_union_gemm_launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, con
 // Internal entry points of the kernel files.
 int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,
                    const wide_worklist *wl, cudaStream_t s);
+// Blocks per 256-position slice of the signature-rank kernel, and the bytes
+// of reorder scratch (bucket histogram, member lists, rank counters).
 int reorder_splits(int64_t T);
+size_t reorder_scratch_bytes(int64_t T);
 
 size_t ffn_prefill_workspace(const wide_ffn_dims *d);
 // Outputs of the prefill FFN (each optional): out_sum = FFN(x); out_total =
