@@ -325,6 +325,24 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             for (int e = 1; e < kBKV; ++e)
                 vmax = fmaxf(vmax, v[e]);
             const float mt = vmax * sc;                       // -inf if no key is visible
+            // move the reference max when the running max passes it by > 8
+            float alpha = 1.f;
+            if (mt > m_ref + 8.f) {
+                alpha = kt > 0 ? exp2f(m_ref - mt) : 0.f;
+                m_ref = mt;
+            }
+            // probabilities (bf16 pairs) while the previous tile's P V may
+            // still run: only storing P and rescaling O wait for it
+            const float mb = m_ref > -INFINITY ? m_ref : 0.f;
+            float lsum = 0.f;
+            uint32_t pw[kBKV / 2];
+#pragma unroll
+            for (int e = 0; e < kBKV; e += 2) {
+                const float p0 = exp2f(fmaf(v[e], sc, -mb)), p1 = exp2f(fmaf(v[e + 1], sc, -mb));
+                lsum += p0 + p1;
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                pw[e / 2] = *reinterpret_cast<const uint32_t *>(&b2);
+            }
             // the previous tile's P V is done: P is free, O is stable
             if (kt > 0) {
                 w = attn_wait(&ctl->bar_pv, (uint32_t)(kt - 1) & 1u, ctl, a.status);
@@ -333,12 +351,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                     break;
                 }
                 umma::fence_after_sync();
-            }
-            // move the reference max when the running max passes it by > 8
-            float alpha = 1.f;
-            if (mt > m_ref + 8.f) {
-                alpha = kt > 0 ? exp2f(m_ref - mt) : 0.f;
-                m_ref = mt;
             }
             if (kt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -353,25 +365,11 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                 }
                 umma::tmem_st_wait();
             }
-            // probabilities -> P (bf16, swizzled K-major); masked keys give 0
-            const float mb = m_ref > -INFINITY ? m_ref : 0.f;
-            float lsum = 0.f;
+            // P (bf16, swizzled K-major); masked keys give 0
 #pragma unroll
-            for (int g8 = 0; g8 < kBKV / 8; ++g8) {
-                float p[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    p[e] = exp2f(fmaf(v[g8 * 8 + e], sc, -mb));
-                    lsum += p[e];
-                }
-                __nv_bfloat162 b0 = __floats2bfloat162_rn(p[0], p[1]);
-                __nv_bfloat162 b1 = __floats2bfloat162_rn(p[2], p[3]);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(p[4], p[5]);
-                __nv_bfloat162 b3 = __floats2bfloat162_rn(p[6], p[7]);
-                *reinterpret_cast<uint4 *>(sp + swz128(tid, g8)) = make_uint4(
-                    *reinterpret_cast<uint32_t *>(&b0), *reinterpret_cast<uint32_t *>(&b1),
-                    *reinterpret_cast<uint32_t *>(&b2), *reinterpret_cast<uint32_t *>(&b3));
-            }
+            for (int g8 = 0; g8 < kBKV / 8; ++g8)
+                *reinterpret_cast<uint4 *>(sp + swz128(tid, g8)) =
+                    make_uint4(pw[4 * g8], pw[4 * g8 + 1], pw[4 * g8 + 2], pw[4 * g8 + 3]);
             l = l * alpha + lsum;
             fence_proxy_async_smem();       // P written by threads, read by the tensor core
             umma::fence_before_sync();
