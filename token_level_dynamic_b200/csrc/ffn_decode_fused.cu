@@ -179,10 +179,12 @@ __device__ __forceinline__ void lane_reduce(float (&v)[N], int lane)
 // Phase 1, one stage, one thread: rows 0 and 1 of W_gate at sg and of W_up
 // at su (row stride rs bytes), one 8-column chunk; the x half holding the
 // chunk's columns 4 h .. 4 h + 3 of token pair p at xk + p * xpair + xo[h].
-template <int NP>
+// Only the first NA accumulator slots are computed: slot k holds token pair
+// (ppk >> 4k) & 15, the pairs with a token that keeps the unit's group.
+template <int NP, int NA>
 __device__ __forceinline__ void p1_stage(const uint8_t *sg, const uint8_t *su, uint32_t rs,
                                          const uint8_t *xk, uint32_t xpair, const uint32_t (&xo)[2],
-                                         float2 (&ag)[2][NP], float2 (&au)[2][NP])
+                                         uint32_t ppk, float2 (&ag)[2][NP], float2 (&au)[2][NP])
 {
     uint4 g[2], u[2];
 #pragma unroll
@@ -192,15 +194,15 @@ __device__ __forceinline__ void p1_stage(const uint8_t *sg, const uint8_t *su, u
     }
 #pragma unroll
     for (int p2 = 0; p2 < 2; ++p2) {             // columns 4 p2 .. 4 p2 + 3 of the chunk
-        uint4 xr[NP];
+        uint4 xr[NA];
 #pragma unroll
-        for (int tp = 0; tp < NP; ++tp)
-            xr[tp] = lds128(xk + tp * xpair + xo[p2]);
+        for (int tp = 0; tp < NA; ++tp)
+            xr[tp] = lds128(xk + ((ppk >> (4 * tp)) & 15u) * xpair + xo[p2]);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-            float2 xv[NP];
+            float2 xv[NA];
 #pragma unroll
-            for (int tp = 0; tp < NP; ++tp) {
+            for (int tp = 0; tp < NA; ++tp) {
                 const uint32_t wx = word(xr[tp], cc);
                 xv[tp] = make_float2(bf_lo(wx), bf_hi(wx));
             }
@@ -209,18 +211,36 @@ __device__ __forceinline__ void p1_stage(const uint8_t *sg, const uint8_t *su, u
             for (int i = 0; i < 2; ++i) {
                 const float2 d = (cc & 1) ? dup_hi(word(g[i], wi)) : dup_lo(word(g[i], wi));
 #pragma unroll
-                for (int tp = 0; tp < NP; ++tp)
+                for (int tp = 0; tp < NA; ++tp)
                     ag[i][tp] = __ffma2_rn(d, xv[tp], ag[i][tp]);
             }
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const float2 d = (cc & 1) ? dup_hi(word(u[i], wi)) : dup_lo(word(u[i], wi));
 #pragma unroll
-                for (int tp = 0; tp < NP; ++tp)
+                for (int tp = 0; tp < NA; ++tp)
                     au[i][tp] = __ffma2_rn(d, xv[tp], au[i][tp]);
             }
         }
     }
+}
+
+// p1_stage for the run-time number of active slots na (1 <= na <= NP).
+template <int NP>
+__device__ __forceinline__ void p1_dispatch(int na, const uint8_t *sg, const uint8_t *su,
+                                            uint32_t rs, const uint8_t *xk, uint32_t xpair,
+                                            const uint32_t (&xo)[2], uint32_t ppk,
+                                            float2 (&ag)[2][NP], float2 (&au)[2][NP])
+{
+    constexpr int N2 = NP < 2 ? NP : 2, N3 = NP < 3 ? NP : 3;
+    if (na >= NP)
+        p1_stage<NP, NP>(sg, su, rs, xk, xpair, xo, ppk, ag, au);
+    else if (na == 1)
+        p1_stage<NP, 1>(sg, su, rs, xk, xpair, xo, ppk, ag, au);
+    else if (na == 2)
+        p1_stage<NP, N2>(sg, su, rs, xk, xpair, xo, ppk, ag, au);
+    else if (na == 3)
+        p1_stage<NP, N3>(sg, su, rs, xk, xpair, xo, ppk, ag, au);
 }
 
 // Phase 2, one group: this thread's rows of the W_down box at wb (row k at
@@ -574,6 +594,28 @@ __global__ void __maxnreg__(96)
         for (int rb = 0; rb < nRB; ++rb) {
             const int ub = u0 + rb * NUS, nu = min(NUS, u1 - ub);
             const bool act = (rsi >> 2) < nu;
+            // token pairs with a token that keeps this unit's group first
+            // (4 bits per slot in ppk), na of them; the rest are skipped
+            uint32_t ppk = 0u;
+            int na = 0;
+            if (act) {
+                const int grp0 = live[((ub + (rsi >> 2)) * 8) / gs];
+                uint32_t dl = 0u;
+                int nd = 0;
+#pragma unroll
+                for (int tp = 0; tp < NP; ++tp) {
+                    bool k = false;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        if (2 * tp + e < bt)
+                            k |= ((mall[(t0 + 2 * tp + e) * W + (grp0 >> 5)] >> (grp0 & 31)) & 1u) != 0u;
+                    if (k)
+                        ppk |= (uint32_t)tp << (4 * na++);
+                    else
+                        dl |= (uint32_t)tp << (4 * nd++);
+                }
+                ppk |= dl << (4 * na);
+            }
             float2 ag[2][NP], au[2][NP];
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -585,8 +627,9 @@ __global__ void __maxnreg__(96)
             const uint8_t *xk = xs;
             for (int kw = 0; kw < NKW; ++kw, xk += xwin) {
                 wait_full();
-                if (act)
-                    p1_stage<NP>(sp + wofs, sp + kFSlotMin / 2 + wofs, rs, xk, xpair, xo, ag, au);
+                if (na > 0)
+                    p1_dispatch<NP>(na, sp + wofs, sp + kFSlotMin / 2 + wofs, rs, xk, xpair, xo,
+                                    ppk, ag, au);
                 release();
             }
             // sums over the chunks of the row: lanes, then the warps of a row
@@ -616,8 +659,9 @@ __global__ void __maxnreg__(96)
             const bool owner =
                 (NWR == 1 || !(cw & 1)) && (lane & ((1 << (5 - S1)) - 1)) == 0;
             if (act && owner) {
-                const int combo = lane >> (5 - S1);      // row * TBP + token
-                const int r = combo / TBP, t = combo % TBP;
+                const int combo = lane >> (5 - S1);      // row * TBP + slot token
+                const int r = combo / TBP, ts = combo % TBP;
+                const int t = 2 * (int)((ppk >> (4 * (ts >> 1))) & 15u) + (ts & 1);
                 if (t < bt) {
                     const int lr = ub * 8 + rsi * 2 + r;
                     const int grp = live[lr / gs];
