@@ -335,7 +335,14 @@ __global__ void __maxnreg__(96)
     const int bt = min(a.T - t0, TB);                // tokens of this CTA (>= 1)
     const int H = a.H, gs = a.gs, W = a.W;
 
-    // ---- the mask (one round trip), then the batch's union as a list
+    // ---- x of this CTA's tokens toward L2 (the staging below needs the
+    // union first; its loads then find x in L2), the mask (one round trip),
+    // then the batch's union as a list
+    if (!a.xf && tid >= 32) {
+        const char *xb = reinterpret_cast<const char *>(a.x + (size_t)t0 * H);
+        for (int i = tid - 32; i < bt * H * 2 / 128; i += kFCons)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(xb + (size_t)i * 128));
+    }
     for (int i = tid; i < a.T * W; i += kFThreads)
         mall[i] = a.mask[i];
     if (tid == 0) {
