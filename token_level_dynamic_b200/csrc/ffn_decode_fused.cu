@@ -39,7 +39,9 @@
 //     quarter warp take 8 adjacent chunks of one row (128 contiguous bytes).
 //     x is staged once as bf16 token pairs [pair][column][2], its two 16-byte
 //     halves of a chunk swapped in every other group of 4 chunks, so the 8
-//     lanes of a quarter warp read 8 distinct banks.  The partial sums are
+//     lanes of a quarter warp read 8 distinct banks.  A warp's rows lie in
+//     one group, so the token pairs in which neither token keeps it are
+//     left out of its FMAs (their h is written as 0).  The partial sums are
 //     added over the chunks of a row (lane shuffles that halve the values a
 //     lane carries at every step, then shared memory between the two warps
 //     of a row for 512-column windows) once per row block.
