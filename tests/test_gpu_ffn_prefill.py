@@ -115,3 +115,21 @@ def test_prefill_group_size_64_all_zero_and_dense():
     assert not np.any(_run(c))
     c = synth.ffn_case(260, 512, 1024, 64, seed=14, mask_kind="ones")
     assert rel_l2(_run(c), ffn_dense(c.x, c.w_gate, c.w_up, c.w_down)) <= TOL
+
+
+@pytest.mark.parametrize("path", ["decode", "prefill"])
+def test_empty_batch_is_a_no_op(path):
+    """Zero tokens: the call succeeds, launches nothing that fails, and
+    leaves the device status clear, on either path."""
+    import torch
+    import token_level_dynamic_b200 as w
+    c = synth.ffn_case(4, 256, 512, 128, seed=3)
+    _, wg, wu, wd, _ = ffn_to_dev(c)
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    m = torch.empty((0, 1), dtype=torch.int32, device="cuda")
+    w.wide_clear_device_status()
+    p = w.WIDE_PATH_DECODE if path == "decode" else w.WIDE_PATH_PREFILL
+    out = w.wide_ffn_masked(x, wg, wu, wd, m, 128, path=p)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 256)
+    assert w.wide_get_device_status() == 0
