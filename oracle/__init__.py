@@ -13,9 +13,10 @@ Contents
   ffn.ffn_token_loop    the same, per-token loop over kept groups (C, fp64)
   ffn.reorder           canonical mask reordering (C)
   attention.*           RMSNorm, RoPE, masked GQA attention, whole layer
+  router.*              bottleneck router -> packed group masks (section 2.A)
 
 Parity pins live in tests/test_oracle_*.py.  Nothing here is "parity
 unpinned".
 """
-from . import ffn, attention  # noqa: F401
+from . import ffn, attention, router  # noqa: F401
 from ._clib import build  # noqa: F401

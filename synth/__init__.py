@@ -11,4 +11,5 @@ from .gen import (  # noqa: F401
     bernoulli_mask, prototype_masks,
     tiny_ffn, decode_ffn, prefill_ffn, decode_layer, prefill_layer, small_layer,
     ffn_case, CONFIGS,
+    RouterCase, router_case,
 )

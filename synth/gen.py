@@ -26,6 +26,10 @@ section 2.A: GQA-aligned head groups and contiguous FFN channel groups):
 * prefill_layer: 4 sequences x 2048 tokens, 16 prototypes over (8 head groups,
           112 FFN groups) at keep k (0.25/0.5/0.75/1.0), flips p=0.1 (none at
           k=1.0).
+* router: a bottleneck router (section 2.A) with random weights: x ~ N(0,1)
+          bf16 [T][H] stands for the normalised sublayer input, W_r1 [R][H]
+          and W_r2 [G][R] ~ N(0, 0.02) bf16, optional bias ~ N(0, bias_std)
+          fp32 [G].
 
 x ~ N(0,1); weights ~ N(0, 0.02) (0.02 is the standard deviation) in the
 nn.Linear layout [out_features][in_features]; RMSNorm gains are
@@ -46,6 +50,7 @@ _STREAM = {
     "k_cache": 11, "v_cache": 12,
     "mask_f": 20, "mask_a": 21, "proto_f": 22, "proto_a": 23,
     "proto_pick": 24, "flip_f": 25, "flip_a": 26,
+    "w_r1": 30, "w_r2": 31, "b_r2": 32,
 }
 
 
@@ -363,3 +368,34 @@ CONFIGS = {
     "decode_layer_8b": "bf16 decode layer, B=16, cache 2048, head groups Bernoulli(0.34), FFN groups Bernoulli(0.72)",
     "prefill_layer_8b": "bf16 prefill layer, 4 x 2048 tokens, 16 prototypes (8 head / 112 FFN groups), keep 0.25-1.0 + 0.1 flips",
 }
+
+
+@dataclasses.dataclass
+class RouterCase:
+    """Bottleneck router inputs.  bf16 tensors are uint16 bit arrays."""
+    name: str
+    T: int
+    H: int
+    R: int
+    G: int
+    act: str                   # "relu" or "silu"
+    x: np.ndarray              # [T][H] bf16
+    w_r1: np.ndarray           # [R][H] bf16
+    w_r2: np.ndarray           # [G][R] bf16
+    b_r2: Optional[np.ndarray]  # [G] fp32 or None
+
+
+def router_case(T: int, H: int, R: int, G: int, seed: int = 0, act: str = "relu",
+                bias_std: float = 0.0, name: str = "router") -> RouterCase:
+    """Router weights depend on (seed, H, R, G) only, so decode and prefill
+    batches of one model share them."""
+    b = None
+    if bias_std > 0.0:
+        b = _rng(seed, "b_r2", G).standard_normal(G, dtype=np.float32) * np.float32(bias_std)
+    return RouterCase(
+        name, T, H, R, G, act,
+        x=_normal(seed, "x", (T, H), 1.0, True, T, H),
+        w_r1=_normal(seed, "w_r1", (R, H), 0.02, True, R, H),
+        w_r2=_normal(seed, "w_r2", (G, R), 0.02, True, G, R),
+        b_r2=b,
+    )
