@@ -571,8 +571,90 @@ class PrefillLayer8B:
         return sum(lc.attn.T for lc in samples)
 
 
+class RouterDevice:
+    """Device state of the router workload: x of each call, W_r1, W_r2 and
+    the packed mask words each call writes."""
+
+    def __init__(self, wl, cases, dev, stream):
+        import torch
+        import token_level_dynamic_b200 as w
+        from synth.torch_io import to_dev
+        self.w, self.stream, self.cases = w, stream, cases
+        base = cases[0]
+        self.W1 = to_dev(base.w_r1, "bf16", dev)
+        self.W2 = to_dev(base.w_r2, "bf16", dev)
+        self.xs = [to_dev(c.x, "bf16", dev) for c in cases]
+        self.ms = [torch.empty((c.T, (c.G + 31) // 32), dtype=torch.int32, device=dev)
+                   for c in cases]
+        self.ncalls = len(cases)
+        self.xh = [x.cpu().pin_memory() for x in self.xs]
+        self.mh = [torch.empty(m.shape, dtype=m.dtype).pin_memory() for m in self.ms]
+        self.h2d_bytes = int(sum(x.numel() * 2 for x in self.xh))
+        self.d2h_bytes = int(sum(m.numel() * 4 for m in self.mh))
+        self.ws = torch.empty(0, dtype=torch.uint8, device=dev)
+
+    def call(self, i, all_kept=False):
+        # all_kept has no meaning for the router (it produces the masks)
+        self.w.wide_route(self.xs[i], self.W1, self.W2, None, self.w.WIDE_ACT_RELU,
+                          mask_words=self.ms[i], stream=self.stream)
+
+    def e2e_call(self, i):
+        self.xs[i].copy_(self.xh[i], non_blocking=True)
+        self.call(i)
+        self.mh[i].copy_(self.ms[i], non_blocking=True)
+
+    def dense_torch(self, i):
+        """torch/cuBLAS: bf16 logits, then a dense bool [T][G] decision tensor."""
+        import torch.nn.functional as F
+        lg = F.linear(F.relu(F.linear(self.xs[i], self.W1)), self.W2)
+        self.dense_keep = lg > 0
+
+
+class Router8B:
+    name = "router_8b"
+    desc = ("router_8b: bottleneck router of the Llama-3.1-8B-shaped FFN (hidden 4096 -> "
+            "bottleneck 128, ReLU -> 112 group logits, execute iff > 0), random bf16 weights "
+            "N(0, 0.02), x ~ N(0,1); one step = 8192 tokens (the prefill layer's 4 x 2048) "
+            "plus a 16-token decode batch, packed mask words out")
+    bound = "hbm"
+    dominant = "router_tcgen05"
+    device = RouterDevice
+
+    def make_cases(self):
+        import synth
+        out = []
+        for T in (8192, 16):
+            c = synth.router_case(T, 4096, 128, 112, seed=0)
+            c.name = f"router_8b_t{T}"
+            out.append(c)
+        return out
+
+    @staticmethod
+    def units(case):
+        """Algorithmic bytes per call: x, W_r1 and W_r2 read once, the mask
+        words written once."""
+        b = (case.T * case.H * 2 + case.R * case.H * 2 + case.G * case.R * 2
+             + case.T * ((case.G + 31) // 32) * 4)
+        return {"router_tcgen05": b, "total": b}
+
+    def reference_sample(self, cases):
+        out = []
+        for c in cases:
+            s = type(c)(**{**c.__dict__})
+            s.x, s.T = c.x[:64], min(64, c.T)
+            out.append(s)
+        return out, "per step: the first 64 tokens of the 8192-token call and 16 of the decode call"
+
+    @staticmethod
+    def reference_step(samples):
+        import oracle
+        for c in samples:
+            oracle.router.route_mask(c.x, c.w_r1, c.w_r2, c.b_r2, c.act)
+        return sum(c.T for c in samples)
+
+
 WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B(), DecodeLayer8B(),
-                                 PrefillLayer8B())}
+                                 PrefillLayer8B(), Router8B())}
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -785,7 +867,7 @@ def run_ours(args, wl):
                           "frac_of_bf16_peak_whole_call":
                               units[i]["total"] / (t / 1e3) / 1e12 / peaks["bf16_tflops"],
                           "kept_fraction_of_dense": units[i]["total"] / units[i]["dense_flops"]})
-            per_call_out[wl.name] = d
+            per_call_out[getattr(c, "name", wl.name)] = d
             continue
         t = float(per_call[:, i].mean())
         d = {"tokens": c.T, "us_per_call": 1e3 * t, "tokens_per_s": c.T / (t / 1e3)}

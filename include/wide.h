@@ -307,6 +307,47 @@ int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, const void *d
                             const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
                             const wide_ffn_dims *d, void *stream);
 
+/* ------------------------------------------------------------------ router
+ *
+ * Technical summary section 2.A, "router architecture": a light bottleneck
+ * router maps a block's input activations to one binary decision per group,
+ * execute or skip (Gumbel-Softmax relaxes that decision in training only).
+ * The pages give no formula; this call computes, for every token t,
+ *     z[t]        = act(x[t] W_r1^T)                      [rn]
+ *     logit[t][g] = z[t] . W_r2[g] + b_r2[g]              (b_r2 = 0 if NULL)
+ *     execute     = logit[t][g] > 0                       (0 skips)
+ * and writes the decisions straight into the packed mask words that
+ * wide_reorder, wide_ffn_masked and wide_layer_masked read, so no dense
+ * per-(token, group) byte or float mask exists on the device.
+ *
+ *   d_x       bf16 [tokens][hidden], the sublayer's (normalised) input
+ *   d_w_r1    bf16 [bottleneck][hidden]          (nn.Linear layout)
+ *   d_w_r2    bf16 [groups][bottleneck]
+ *   d_b_r2    fp32 [groups] or NULL
+ *   d_mask    out: uint32 [tokens][ceil(groups / 32)]; every word written,
+ *             bits at or above groups zero
+ *   d_logits  out: fp32 [tokens][groups] (the values the decisions were
+ *             taken on), or NULL
+ * Arithmetic: x W_r1^T on tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation in tensor memory), activation and W_r2 products in fp32 on
+ * CUDA cores; no intermediate is rounded to bf16.
+ * Supported: hidden a multiple of 64; bottleneck a multiple of 32 in
+ * [32, 256]; groups in [1, 1024]; tokens * hidden < 2^31; d_x, d_w_r1 and
+ * d_w_r2 16-byte aligned (else WIDE_EUNSUPPORTED).  tokens == 0 enqueues
+ * nothing.  No workspace; nothing is allocated. */
+#define WIDE_ACT_RELU 0
+#define WIDE_ACT_SILU 1
+typedef struct wide_router_dims {
+    int64_t tokens;
+    int64_t hidden;
+    int64_t bottleneck;
+    int64_t groups;
+    int32_t act; /* WIDE_ACT_RELU or WIDE_ACT_SILU */
+} wide_router_dims;
+
+int wide_route(const void *d_x, const void *d_w_r1, const void *d_w_r2, const float *d_b_r2,
+               uint32_t *d_mask, float *d_logits, const wide_router_dims *d, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

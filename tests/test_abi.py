@@ -121,3 +121,31 @@ def test_decode_path_switch_is_host_only(native):
         assert L.wide_set_decode_ffn_path(0) == 2
     finally:
         L.wide_set_decode_ffn_path(prev)
+
+
+def test_route_argument_checks(native):
+    """wide_route refuses bad dims, shapes and alignment on the host."""
+    L = native.lib()
+    D = native.WideRouterDims
+    p = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    for bad in (D(-1, 4096, 128, 112, 0), D(8, 0, 128, 112, 0), D(8, 4096, 0, 112, 0),
+                D(8, 4096, 128, 0, 0), D(8, 4096, 128, 112, 2)):
+        assert L.wide_route(p, p, p, None, p, None, ctypes.byref(bad), None) == native.WIDE_EINVAL
+    assert L.wide_route(None, None, None, None, None, None, None, None) == native.WIDE_EINVAL
+    ok = D(8, 4096, 128, 112, native.WIDE_ACT_RELU)
+    assert L.wide_route(None, p, p, None, p, None, ctypes.byref(ok), None) == native.WIDE_EINVAL
+    assert L.wide_route(p, p, p, None, None, None, ctypes.byref(ok), None) == native.WIDE_EINVAL
+    # zero tokens is a no-op
+    assert L.wide_route(None, None, None, None, None, None, ctypes.byref(D(0, 4096, 128, 112, 0)),
+                        None) == native.WIDE_OK
+    for unsup in (D(8, 4000, 128, 112, 0), D(8, 4096, 100, 112, 0), D(8, 4096, 288, 112, 0),
+                  D(8, 4096, 128, 1025, 0), D(1 << 20, 4096, 128, 112, 0)):
+        assert L.wide_route(p, p, p, None, p, None, ctypes.byref(unsup), None) \
+            == native.WIDE_EUNSUPPORTED
+    assert L.wide_route(mis, p, p, None, p, None, ctypes.byref(ok), None) \
+        == native.WIDE_EUNSUPPORTED
+    assert L.wide_route(p, p, mis, None, p, None, ctypes.byref(ok), None) \
+        == native.WIDE_EUNSUPPORTED
+    assert L.wide_route(p, p, p, ctypes.c_void_p((1 << 20) + 2), p, None, ctypes.byref(ok),
+                        None) == native.WIDE_EUNSUPPORTED

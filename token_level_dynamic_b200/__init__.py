@@ -23,7 +23,8 @@ from ._native import (  # noqa: F401
     WIDE_NOALLOC_SCRATCH_BYTES,
     WIDE_DEV_BAD_MASK, WIDE_DEV_TIMEOUT, WIDE_DEV_BAD_ITEM, WIDE_DEV_LAYOUT,
     WIDE_BF16, WIDE_F32, WIDE_PATH_AUTO, WIDE_PATH_DECODE, WIDE_PATH_PREFILL,
-    WideWorklist, WideFFNDims, WideLayerDims, WideLayerWeights,
+    WIDE_ACT_RELU, WIDE_ACT_SILU,
+    WideWorklist, WideFFNDims, WideLayerDims, WideLayerWeights, WideRouterDims,
 )
 
 _L = _native.lib()
@@ -291,3 +292,26 @@ def wide_attn_masked(x: torch.Tensor, weights: dict, k_cache: torch.Tensor,
         _dev_ptr(attn_out, "attn_out"), ctypes.byref(d), workspace.data_ptr(), workspace.numel(),
         _stream(stream, x.device)))
     return attn_out
+
+
+# ------------------------------------------------------------------ router
+
+def wide_route(x: torch.Tensor, w_r1: torch.Tensor, w_r2: torch.Tensor,
+               b_r2: torch.Tensor = None, act: int = WIDE_ACT_RELU,
+               mask_words: torch.Tensor = None, logits: torch.Tensor = None,
+               stream=None) -> torch.Tensor:
+    """Bottleneck router (section 2.A): execute bits of act(x W_r1^T) W_r2^T
+    + b_r2 > 0, packed.  x bf16 [T][H]; W_r1 bf16 [R][H]; W_r2 bf16 [G][R];
+    b_r2 fp32 [G] or None; returns int32 mask words [T][ceil(G/32)].  If
+    `logits` (fp32 [T][G]) is given, the logits are written there too."""
+    T, H = x.shape
+    R, G = w_r1.shape[0], w_r2.shape[0]
+    if mask_words is None:
+        mask_words = torch.empty((T, (G + 31) // 32), dtype=torch.int32, device=x.device)
+    d = WideRouterDims(T, H, R, G, act)
+    _check("wide_route", _L.wide_route(
+        _dev_ptr(x, "x"), _dev_ptr(w_r1, "w_r1"), _dev_ptr(w_r2, "w_r2"),
+        None if b_r2 is None else _dev_ptr(b_r2, "b_r2"), _dev_ptr(mask_words, "mask_words"),
+        None if logits is None else _dev_ptr(logits, "logits"), ctypes.byref(d),
+        _stream(stream, x.device)))
+    return mask_words

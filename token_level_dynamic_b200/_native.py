@@ -30,6 +30,8 @@ WIDE_F32 = 1
 WIDE_PATH_AUTO = 0
 WIDE_PATH_DECODE = 1
 WIDE_PATH_PREFILL = 2
+WIDE_ACT_RELU = 0
+WIDE_ACT_SILU = 1
 
 
 class WideWorklist(ctypes.Structure):
@@ -55,6 +57,11 @@ class WideLayerDims(ctypes.Structure):
 class WideLayerWeights(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in ("gamma1", "wq", "wk", "wv", "wo",
                                         "gamma2", "w_gate", "w_up", "w_down")]
+
+
+class WideRouterDims(ctypes.Structure):
+    _fields_ = [("tokens", c_int64), ("hidden", c_int64), ("bottleneck", c_int64),
+                ("groups", c_int64), ("act", c_int32)]
 
 
 # name -> (restype, argtypes); every symbol include/wide.h declares
@@ -87,6 +94,8 @@ SIGNATURES = {
     "wide_attn_masked": (c_int, [c_void_p, ctypes.POINTER(WideLayerWeights), c_void_p, c_void_p,
                                  c_void_p, c_void_p, ctypes.POINTER(WideLayerDims), c_void_p,
                                  c_size_t, c_void_p]),
+    "wide_route": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                           ctypes.POINTER(WideRouterDims), c_void_p]),
 }
 
 _lib = None

@@ -74,6 +74,7 @@ enum KernelId : int32_t {
     KID_PREFILL_ATTN = 13,
     KID_PREFILL_OPROJ = 14,
     KID_DECODE_FFN_FUSED = 15,
+    KID_ROUTER = 16,
 };
 
 // Pointers of one masked-layer call (FFN pointers unused when !ffn).
@@ -115,7 +116,7 @@ struct DownOutputs {
 };
 
 // ---- tcgen05 grouped GEMMs of the prefill path (prefill_gemm.cu)
-enum GemmMode : int { GEMM_SWIGLU = 0, GEMM_ROPE_Q = 1, GEMM_KV = 2 };
+enum GemmMode : int { GEMM_SWIGLU = 0, GEMM_ROPE_Q = 1, GEMM_KV = 2, GEMM_ROUTER = 3 };
 
 struct GemmArgs {
     const __nv_bfloat16 *a;                   // [T][K] activation rows
@@ -128,6 +129,13 @@ struct GemmArgs {
     int seq_len, n_kv, kv_blocks, m_tiles;
     int64_t cache_len, cache_cap;
     float log2_theta;
+    // Router: B = W_r1 [rn][K]; the epilogue computes act(z) W_r2^T + b_r2
+    // for the tile's tokens and writes the packed execute bits.
+    const __nv_bfloat16 *w_r2;   // [G][rn]
+    const float *b_r2;           // [G] or null
+    uint32_t *mask_out;          // [T][ceil(G/32)]
+    float *logits_out;           // [T][G] or null
+    int rn, n_groups, act;
     int32_t *status;
 };
 
@@ -149,6 +157,8 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
                        const GemmArgs &a, int max_work, int32_t kid, cudaStream_t s);
 int tile_union_gemm_launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const UnionArgs &a,
                            int32_t kid, cudaStream_t s);
+int route_launch(const void *x, const void *w_r1, const void *w_r2, const float *b_r2,
+                 uint32_t *mask, float *logits, const wide_router_dims *d, cudaStream_t s);
 
 // Internal entry points of the kernel files.
 int reorder_launch(const uint32_t *mask, int64_t T, int64_t G, int32_t tile_m,

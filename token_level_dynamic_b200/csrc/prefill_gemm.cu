@@ -185,6 +185,68 @@ __global__ void __launch_bounds__(128)
     }
 }
 
+// Router epilogue for one token row (TMEM lane) of a tile: z = act(the
+// row's rn accumulator columns), logit[g] = b_r2[g] + z . W_r2[g], execute
+// bit = logit > 0.  Each thread produces its token's mask words itself, 32
+// groups at a time; the z chunks are re-read from TMEM for every word.
+// W_r2 is read through L1 at addresses shared by the whole warp.  Called by
+// whole warps (tcgen05.ld is warp-collective); only live rows store.
+__device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t taddr, int t,
+                                                bool live)
+{
+    const int G = a.n_groups, nw = (G + 31) >> 5, rn = a.rn;
+#pragma unroll 1
+    for (int wd = 0; wd < nw; ++wd) {
+        const int g0 = wd * 32;
+        const int ng = min(32, G - g0);
+        float lg[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            lg[j] = (a.b_r2 && j < ng) ? __ldg(a.b_r2 + g0 + j) : 0.f;
+#pragma unroll 1
+        for (int c = 0; c < rn / 32; ++c) {
+            float z[32];
+            umma::tmem_ld32(taddr + c * 32, z);
+            umma::tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                z[e] = a.act == WIDE_ACT_SILU ? silu_f32(z[e]) : fmaxf(z[e], 0.f);
+            const __nv_bfloat16 *w2 = a.w_r2 + (size_t)g0 * rn + c * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (j < ng) {
+                    const uint4 *wp = reinterpret_cast<const uint4 *>(w2 + (size_t)j * rn);
+                    float acc = lg[j];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float wv[8];
+                        bf16x8_to_f32(__ldg(wp + q), wv);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            acc = fmaf(z[8 * q + k], wv[k], acc);
+                    }
+                    lg[j] = acc;
+                }
+            }
+        }
+        uint32_t bits = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < ng && lg[j] > 0.f)
+                bits |= 1u << j;
+        if (live) {
+            a.mask_out[(size_t)t * nw + wd] = bits;
+            if (a.logits_out) {
+                float *lo = a.logits_out + (size_t)t * G + g0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j < ng)
+                        lo[j] = lg[j];
+            }
+        }
+    }
+}
+
 // --------------------------------------------------------- gather_gemm
 struct Work {
     int g, base, nrows, hf, nb;
@@ -197,6 +259,8 @@ __device__ __forceinline__ int n_work(const GemmArgs &a, int n_items)
         return n_items;
     if (MODE == GEMM_ROPE_Q)
         return (a.group_cols / kBN) * n_items;    // 256-column parts per group
+    if (MODE == GEMM_ROUTER)
+        return a.m_tiles;
     return a.kv_blocks * a.m_tiles;
 }
 
@@ -206,7 +270,7 @@ __device__ __forceinline__ Work decode_work(const GemmArgs &a, int it)
     Work w;
     w.hf = 0;
     w.nb = 0;
-    if (MODE == GEMM_KV) {
+    if (MODE == GEMM_KV || MODE == GEMM_ROUTER) {
         w.nb = it / a.m_tiles;
         const int ti = it % a.m_tiles;
         w.g = 0;
@@ -230,7 +294,7 @@ __device__ __forceinline__ Work decode_work(const GemmArgs &a, int it)
 template <int MODE>
 __device__ __forceinline__ int row_token(const GemmArgs &a, const Work &w, int r)
 {
-    if (MODE == GEMM_KV)
+    if (MODE == GEMM_KV || MODE == GEMM_ROUTER)
         return w.base + r;
     return a.perm[(size_t)w.g * a.T + w.base + r];
 }
@@ -244,7 +308,7 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
     uint8_t *smem = align1024(smem_raw);
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + kStages * kStageBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = (MODE == GEMM_KV) ? 0 : *a.n_items_p;
+    const int n_items = (MODE == GEMM_KV || MODE == GEMM_ROUTER) ? 0 : *a.n_items_p;
     const int nw = n_work<MODE>(a, n_items);
     const int KT = a.K / kBK;
 
@@ -280,6 +344,11 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                 r0 = w.g * a.group_cols + w.hf * kBN;        // two query heads of group g
                 r1 = r0 + 128;
                 m1 = &tm0;
+            } else if (MODE == GEMM_ROUTER) {
+                r0 = 0;                                      // all of W_r1, two halves
+                r1 = a.rn / 2;
+                m1 = &tm0;
+                b_rows = a.rn;
             } else {
                 const int half = a.kv_blocks / 2;            // first half: Wk, then Wv
                 const bool is_k = w.nb < half;
@@ -357,9 +426,12 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
         cp_async_wait_all();
     } else if (warp == 1) {
         // -------------------------------------------- MMA issuer
-        // SwiGLU: N = gate rows + up rows of one group (2 gs); else 256
-        const uint32_t idesc =
-            umma::idesc_bf16_f32(kBM, MODE == GEMM_SWIGLU ? 2u * (uint32_t)a.gs : (uint32_t)kBN);
+        // SwiGLU: N = gate rows + up rows of one group (2 gs); router: the
+        // bottleneck width; else 256
+        const uint32_t idesc = umma::idesc_bf16_f32(
+            kBM, MODE == GEMM_SWIGLU   ? 2u * (uint32_t)a.gs
+                 : MODE == GEMM_ROUTER ? (uint32_t)a.rn
+                                       : (uint32_t)kBN);
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
@@ -432,6 +504,9 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                     if (live)
                         store_bf16x32(dst + c * 32, gv);
                 }
+            } else if (MODE == GEMM_ROUTER) {
+                if (__any_sync(0xffffffffu, live))
+                    router_epilogue(a, taddr, t, live);
             } else if (MODE == GEMM_ROPE_Q) {
                 const int pos = (int)(t % a.seq_len + a.cache_len);
                 __nv_bfloat16 *dst = a.out0 + ((size_t)w.g * a.T + w.base + r) * a.group_cols +
@@ -711,8 +786,9 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
     if ((int64_t)a.T * a.K >= (int64_t)1 << 31)      // row offsets are 32-bit
         return WIDE_EUNSUPPORTED;
     const int grid = max_work < sms ? max_work : sms;
-    const void *k = mode == GEMM_SWIGLU ? reinterpret_cast<const void *>(gather_gemm<GEMM_SWIGLU>)
+    const void *k = mode == GEMM_SWIGLU   ? reinterpret_cast<const void *>(gather_gemm<GEMM_SWIGLU>)
                     : mode == GEMM_ROPE_Q ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROPE_Q>)
+                    : mode == GEMM_ROUTER ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROUTER>)
                                           : reinterpret_cast<const void *>(gather_gemm<GEMM_KV>);
     if (!raise_smem_limit(k, kSmemBytes))
         return WIDE_CUDA_FAIL();
@@ -721,6 +797,8 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
         gather_gemm<GEMM_SWIGLU><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
     else if (mode == GEMM_ROPE_Q)
         gather_gemm<GEMM_ROPE_Q><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
+    else if (mode == GEMM_ROUTER)
+        gather_gemm<GEMM_ROUTER><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
     else
         gather_gemm<GEMM_KV><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
     return launch_status();

@@ -125,6 +125,8 @@ const char *wide_kernel_name(int32_t id)
         return "prefill_oproj_tcgen05";
     case KID_DECODE_FFN_FUSED:
         return "decode_ffn_fused_gemv";
+    case KID_ROUTER:
+        return "router_tcgen05";
     default:
         return "?";
     }
