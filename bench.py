@@ -635,7 +635,8 @@ class Router8B:
         words written once."""
         b = (case.T * case.H * 2 + case.R * case.H * 2 + case.G * case.R * 2
              + case.T * ((case.G + 31) // 32) * 4)
-        return {"router_tcgen05": b, "total": b}
+        kernel = "router_small_gemv" if case.T <= 32 else "router_tcgen05"
+        return {kernel: b, "total": b}
 
     def reference_sample(self, cases):
         out = []

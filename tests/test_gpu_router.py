@@ -1,5 +1,7 @@
 """Bottleneck router (WIDE, technical summary section 2.A, router
-architecture) on the GPU against the fp64 oracle, through the C ABI.
+architecture) on the GPU against the fp64 oracle, through the C ABI.  Both
+kernels are covered: the cluster kernel on CUDA cores (up to 32 tokens) and
+the tcgen05 kernel (more tokens).
 
 The logits are floating point: relative L2 <= 1e-4 against the oracle (the
 kernel keeps every intermediate in fp32; bf16 appears only in the stored
@@ -70,8 +72,13 @@ def _check(rc, m, lg):
 
 
 @pytest.mark.parametrize("T,H,R,G,act,bias", [
+    # up to 32 tokens: the cluster kernel (CUDA cores)
     (1, 256, 32, 8, "silu", 0.0),          # one token, one word
+    (5, 1024, 256, 1024, "silu", 0.05),    # partial cluster, widest shapes
     (16, 4096, 128, 8, "relu", 0.0),       # decode batch, head-group router
+    (32, 4096, 128, 112, "relu", 0.02),    # largest batch of the cluster kernel
+    # more than 32 tokens: tcgen05
+    (33, 4096, 128, 112, "relu", 0.02),    # one partial tile
     (127, 512, 64, 33, "relu", 0.05),      # one partial tile, two words
     (300, 256, 64, 40, "relu", 0.05),      # three tiles, ragged tail
     (384, 192, 96, 200, "silu", 0.02),     # three full tiles, 7 words
@@ -82,6 +89,21 @@ def test_router_matches_oracle(T, H, R, G, act, bias):
     rc = synth.router_case(T, H, R, G, seed=11, act=act, bias_std=bias)
     m, lg = _route(rc)
     _check(rc, m, lg)
+
+
+def test_router_paths_agree_at_the_boundary():
+    """Tokens 0..31 routed as a batch of 32 (cluster kernel) and as the first
+    rows of a batch of 33 (tcgen05 kernel): same decisions away from the
+    margin, logits within the tolerance of each other."""
+    rc33 = synth.router_case(33, 2048, 64, 40, seed=14, bias_std=0.02)
+    rc32 = synth.RouterCase(**{**rc33.__dict__})
+    rc32.x, rc32.T = rc33.x[:32], 32
+    m33, lg33 = _route(rc33)
+    m32, lg32 = _route(rc32)
+    assert rel_l2(lg32, lg33[:32]) <= TOL_LOGITS
+    rms = float(np.sqrt(np.mean(lg33 * lg33)))
+    clear = np.abs(lg33[:32]) > MARGIN * rms
+    np.testing.assert_array_equal(mask_bool(m32, 40)[clear], mask_bool(m33[:32], 40)[clear])
 
 
 def test_router_without_logits_output():

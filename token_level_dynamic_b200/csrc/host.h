@@ -75,6 +75,7 @@ enum KernelId : int32_t {
     KID_PREFILL_OPROJ = 14,
     KID_DECODE_FFN_FUSED = 15,
     KID_ROUTER = 16,
+    KID_ROUTER_SMALL = 17,
 };
 
 // Pointers of one masked-layer call (FFN pointers unused when !ffn).

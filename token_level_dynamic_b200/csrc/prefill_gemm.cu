@@ -185,55 +185,93 @@ __global__ void __launch_bounds__(128)
     }
 }
 
-// Router epilogue for one token row (TMEM lane) of a tile: z = act(the
-// row's rn accumulator columns), logit[g] = b_r2[g] + z . W_r2[g], execute
-// bit = logit > 0.  Each thread produces its token's mask words itself, 32
-// groups at a time; the z chunks are re-read from TMEM for every word.
-// W_r2 is read through L1 at addresses shared by the whole warp.  Called by
-// whole warps (tcgen05.ld is warp-collective); only live rows store.
-__device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t taddr, int t,
-                                                bool live)
+// Router epilogue.  A W_r2 block is 32 groups x 32 bottleneck units; lane l
+// of a warp loads group (32 wd + l)'s 64 bytes of chunk c (zeros past G).
+__device__ __forceinline__ void w2_block_load(const GemmArgs &a, int wd, int c, int lane,
+                                              uint4 (&v)[4])
 {
-    const int G = a.n_groups, nw = (G + 31) >> 5, rn = a.rn;
+    const int g = wd * 32 + lane;
+    if (g < a.n_groups) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(a.w_r2 + (size_t)g * a.rn + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            v[q] = __ldg(p + q);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            v[q] = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+// One token row (TMEM lane) per thread: z = act(the row's rn accumulator
+// columns), logit[g] = b_r2[g] + z . W_r2[g], execute bit = logit > 0.  Each
+// thread builds its token's mask words itself, 32 groups at a time; the z
+// chunks are re-read from TMEM for every word.  W_r2 goes through this
+// warp's own fp32 block in shared memory (rows of kRW2Stride floats, so the
+// lanes' row stores hit distinct banks; the FMA loop reads it as broadcasts),
+// and the next block is fetched into registers while this one is used.
+// Packed fp32x2 FMAs keep even and odd bottleneck units in two partial sums.
+// Called by whole warps (tcgen05.ld is warp-collective); only live rows store.
+constexpr int kRW2Stride = 36;
+constexpr uint32_t kRouterScratch = 4u * 32u * kRW2Stride * 4u + 16u;
+static_assert(kSmemBytes + kRouterScratch <= 232448, "router mode exceeds 227 KB of shared memory");
+
+__device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t taddr, int t,
+                                                bool live, float *ws, int lane)
+{
+    const int G = a.n_groups, nw = (G + 31) >> 5, nc = a.rn >> 5, nblk = nw * nc;
+    uint4 nx[4];
+    w2_block_load(a, 0, 0, lane, nx);
 #pragma unroll 1
     for (int wd = 0; wd < nw; ++wd) {
         const int g0 = wd * 32;
         const int ng = min(32, G - g0);
-        float lg[32];
+        float2 acc[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-            lg[j] = (a.b_r2 && j < ng) ? __ldg(a.b_r2 + g0 + j) : 0.f;
+            acc[j] = make_float2((a.b_r2 && j < ng) ? __ldg(a.b_r2 + g0 + j) : 0.f, 0.f);
 #pragma unroll 1
-        for (int c = 0; c < rn / 32; ++c) {
+        for (int c = 0; c < nc; ++c) {
+            __syncwarp();
+            float *row = ws + lane * kRW2Stride;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float f[8];
+                bf16x8_to_f32(nx[q], f);
+                *reinterpret_cast<float4 *>(row + 8 * q) = make_float4(f[0], f[1], f[2], f[3]);
+                *reinterpret_cast<float4 *>(row + 8 * q + 4) = make_float4(f[4], f[5], f[6], f[7]);
+            }
+            __syncwarp();
+            const int nb = wd * nc + c + 1;
+            if (nb < nblk)
+                w2_block_load(a, nb / nc, nb % nc, lane, nx);
             float z[32];
             umma::tmem_ld32(taddr + c * 32, z);
             umma::tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e)
                 z[e] = a.act == WIDE_ACT_SILU ? silu_f32(z[e]) : fmaxf(z[e], 0.f);
-            const __nv_bfloat16 *w2 = a.w_r2 + (size_t)g0 * rn + c * 32;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                if (j < ng) {
-                    const uint4 *wp = reinterpret_cast<const uint4 *>(w2 + (size_t)j * rn);
-                    float acc = lg[j];
+                const float4 *wr = reinterpret_cast<const float4 *>(ws + j * kRW2Stride);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float wv[8];
-                        bf16x8_to_f32(__ldg(wp + q), wv);
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            acc = fmaf(z[8 * q + k], wv[k], acc);
-                    }
-                    lg[j] = acc;
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 w = wr[e4];
+                    acc[j] = __ffma2_rn(make_float2(z[4 * e4], z[4 * e4 + 1]),
+                                        make_float2(w.x, w.y), acc[j]);
+                    acc[j] = __ffma2_rn(make_float2(z[4 * e4 + 2], z[4 * e4 + 3]),
+                                        make_float2(w.z, w.w), acc[j]);
                 }
             }
         }
         uint32_t bits = 0;
+        float lg[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < 32; ++j) {
+            lg[j] = acc[j].x + acc[j].y;
             if (j < ng && lg[j] > 0.f)
                 bits |= 1u << j;
+        }
         if (live) {
             a.mask_out[(size_t)t * nw + wd] = bits;
             if (a.logits_out) {
@@ -505,8 +543,12 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                         store_bf16x32(dst + c * 32, gv);
                 }
             } else if (MODE == GEMM_ROUTER) {
+                // this warp's W_r2 block in shared memory, after the Ctl block
+                float *ws = reinterpret_cast<float *>(
+                                smem + ((kStages * kStageBytes + sizeof(Ctl) + 15) & ~(size_t)15)) +
+                            q * 32 * kRW2Stride;
                 if (__any_sync(0xffffffffu, live))
-                    router_epilogue(a, taddr, t, live);
+                    router_epilogue(a, taddr, t, live, ws, lane);
             } else if (MODE == GEMM_ROPE_Q) {
                 const int pos = (int)(t % a.seq_len + a.cache_len);
                 __nv_bfloat16 *dst = a.out0 + ((size_t)w.g * a.T + w.base + r) * a.group_cols +
@@ -790,7 +832,8 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
                     : mode == GEMM_ROPE_Q ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROPE_Q>)
                     : mode == GEMM_ROUTER ? reinterpret_cast<const void *>(gather_gemm<GEMM_ROUTER>)
                                           : reinterpret_cast<const void *>(gather_gemm<GEMM_KV>);
-    if (!raise_smem_limit(k, kSmemBytes))
+    const size_t smem = mode == GEMM_ROUTER ? kSmemBytes + kRouterScratch : kSmemBytes;
+    if (!raise_smem_limit(k, smem))
         return WIDE_CUDA_FAIL();
     LaunchScope scope(kid, s);
     if (mode == GEMM_SWIGLU)
@@ -798,7 +841,7 @@ int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
     else if (mode == GEMM_ROPE_Q)
         gather_gemm<GEMM_ROPE_Q><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
     else if (mode == GEMM_ROUTER)
-        gather_gemm<GEMM_ROUTER><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
+        gather_gemm<GEMM_ROUTER><<<grid, kThreadsGather, smem, s>>>(tm0, tm1, a);
     else
         gather_gemm<GEMM_KV><<<grid, kThreadsGather, kSmemBytes, s>>>(tm0, tm1, a);
     return launch_status();

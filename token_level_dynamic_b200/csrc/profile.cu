@@ -127,6 +127,8 @@ const char *wide_kernel_name(int32_t id)
         return "decode_ffn_fused_gemv";
     case KID_ROUTER:
         return "router_tcgen05";
+    case KID_ROUTER_SMALL:
+        return "router_small_gemv";
     default:
         return "?";
     }

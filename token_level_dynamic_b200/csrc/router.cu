@@ -6,23 +6,177 @@
 // execute = logit > 0, written as the packed token-major mask words that
 // every masked kernel reads.
 //
-// One launch of gather_gemm in router mode (prefill_gemm.cu): every 128-token
-// tile of x times all of W_r1 (N = bottleneck width) on tcgen05, fp32 in
-// tensor memory; its epilogue applies the activation and the W_r2 products on
-// CUDA cores, one token per thread, and stores the mask words directly.
+// More than 32 tokens: one launch of gather_gemm in router mode
+// (prefill_gemm.cu): every 128-token tile of x times all of W_r1 (N =
+// bottleneck width) on tcgen05, fp32 in tensor memory; its epilogue applies
+// the activation and the W_r2 products on CUDA cores, one token per thread,
+// and stores the mask words directly.
+//
+// Up to 32 tokens (decode): route_small, CUDA cores, clusters of 8 CTAs.  A
+// cluster takes 4 tokens; CTA k of it takes bottleneck units
+// [k R/8, (k+1) R/8): it streams those rows of W_r1 once (16-byte loads, x
+// staged in shared memory), forms z for its units, and multiplies them by
+// the matching columns of W_r2 into partial logits [4][G] in its shared
+// memory.  After a cluster barrier every CTA sums the 8 partials of its
+// share of the (token, mask word) items through distributed shared memory,
+// adds the bias and takes the decisions with a warp ballot (lane j = group
+// 32 w + j).  W_r1 is read from HBM once per call (the clusters of a batch
+// share it through L2).
 #include "common.cuh"
 #include "host.h"
 
+#include <cooperative_groups.h>
+
 namespace wide {
+
+namespace cg = cooperative_groups;
 
 namespace {
 constexpr int kBM = 128;
+constexpr int kRTok = 4;         // tokens per cluster
+constexpr int kRCluster = 8;     // CTAs per cluster
+constexpr int kRThreads = 256;
+constexpr int kRMaxTokens = 32;  // route_small's range
+
+__device__ __forceinline__ float router_act(float v, int act)
+{
+    return act == WIDE_ACT_SILU ? silu_f32(v) : fmaxf(v, 0.f);
 }
+
+// Shared memory: x rows [kRTok][H] bf16, z [kRTok][R/8] fp32, partial
+// logits [kRTok][G] fp32.
+__global__ void __launch_bounds__(kRThreads, 1)
+    route_small(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w1,
+                const __nv_bfloat16 *__restrict__ w2, const float *__restrict__ b2,
+                uint32_t *__restrict__ mask, float *__restrict__ logits, int T, int H, int R,
+                int G, int act)
+{
+    extern __shared__ __align__(16) uint8_t sm[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int k = (int)cluster.block_rank();
+    const int t0 = (int)(blockIdx.x / kRCluster) * kRTok;
+    const int nt = min(kRTok, T - t0);
+    const int RB = R / kRCluster, r0 = k * RB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(sm);
+    float *zs = reinterpret_cast<float *>(sm + (size_t)kRTok * H * 2);
+    float *ps = zs + kRTok * RB;
+
+    // x rows of this cluster's tokens (rows past T are zeros)
+    const int hc = H / 8;
+    for (int i = threadIdx.x; i < kRTok * hc; i += kRThreads) {
+        const int tt = i / hc, ch = i - tt * hc;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (tt < nt)
+            v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H) + ch);
+        reinterpret_cast<uint4 *>(xs)[i] = v;
+    }
+    __syncthreads();
+
+    // z[tt][rr] = act(x[t0 + tt] . W_r1[r0 + rr]): one warp per unit
+    for (int rr = warp; rr < RB; rr += kRThreads / 32) {
+        const uint4 *wr = reinterpret_cast<const uint4 *>(w1 + (size_t)(r0 + rr) * H);
+        float acc[kRTok] = {};
+#pragma unroll 4
+        for (int ch = lane; ch < hc; ch += 32) {
+            float wv[8];
+            bf16x8_to_f32(__ldg(wr + ch), wv);
+#pragma unroll
+            for (int tt = 0; tt < kRTok; ++tt) {
+                float xv[8];
+                bf16x8_to_f32(reinterpret_cast<const uint4 *>(xs + (size_t)tt * H)[ch], xv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[tt] = fmaf(wv[e], xv[e], acc[tt]);
+            }
+        }
+#pragma unroll
+        for (int tt = 0; tt < kRTok; ++tt) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], o);
+        }
+        if (lane < kRTok)
+            zs[lane * RB + rr] = router_act(acc[lane], act);
+    }
+    __syncthreads();
+
+    // partial logits of this CTA's units: ps[tt][g] = z[tt] . W_r2[g][r0 : r0 + RB]
+    for (int i = threadIdx.x; i < kRTok * G; i += kRThreads) {
+        const int tt = i / G, g = i - tt * G;
+        const __nv_bfloat162 *wg = reinterpret_cast<const __nv_bfloat162 *>(w2 + (size_t)g * R + r0);
+        float acc = 0.f;
+        for (int rr = 0; rr < RB; rr += 2) {
+            const float2 wv = __bfloat1622float2(wg[rr / 2]);
+            acc = fmaf(zs[tt * RB + rr], wv.x, acc);
+            acc = fmaf(zs[tt * RB + rr + 1], wv.y, acc);
+        }
+        ps[i] = acc;
+    }
+    cluster.sync();
+
+    // sum the 8 partials: item (tt, wd) to warp (item - k*8) of rank k
+    const int nw = (G + 31) >> 5;
+    for (int it = k * (kRThreads / 32) + warp; it < nt * nw; it += kRCluster * (kRThreads / 32)) {
+        const int tt = it / nw, wd = it - tt * nw;
+        const int g = wd * 32 + lane;
+        float lg = 0.f;
+        if (g < G) {
+            lg = b2 ? b2[g] : 0.f;
+#pragma unroll
+            for (int q = 0; q < kRCluster; ++q)
+                lg += cluster.map_shared_rank(ps, q)[tt * G + g];
+        }
+        const uint32_t bits = __ballot_sync(0xffffffffu, g < G && lg > 0.f);
+        if (lane == 0)
+            mask[(size_t)(t0 + tt) * nw + wd] = bits;
+        if (logits && g < G)
+            logits[(size_t)(t0 + tt) * G + g] = lg;
+    }
+    cluster.sync();  // no CTA leaves while another still reads its partials
+}
+
+size_t route_small_smem(int H, int R, int G)
+{
+    return (size_t)kRTok * H * 2 + (size_t)kRTok * (R / kRCluster) * 4 + (size_t)kRTok * G * 4;
+}
+
+int route_small_launch(const void *x, const void *w1, const void *w2, const float *b2,
+                       uint32_t *mask, float *logits, int T, int H, int R, int G, int act,
+                       cudaStream_t s)
+{
+    const size_t smem = route_small_smem(H, R, G);
+    if (!raise_smem_limit(reinterpret_cast<const void *>(route_small), smem))
+        return WIDE_CUDA_FAIL();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(((T + kRTok - 1) / kRTok) * kRCluster));
+    cfg.blockDim = dim3(kRThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kRCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope scope(KID_ROUTER_SMALL, s);
+    if (cudaLaunchKernelEx(&cfg, route_small, static_cast<const __nv_bfloat16 *>(x),
+                           static_cast<const __nv_bfloat16 *>(w1),
+                           static_cast<const __nv_bfloat16 *>(w2), b2, mask, logits, T, H, R, G,
+                           act) != cudaSuccess)
+        return WIDE_CUDA_FAIL();
+    return WIDE_OK;
+}
+}  // namespace
 
 int route_launch(const void *x, const void *w_r1, const void *w_r2, const float *b_r2,
                  uint32_t *mask, float *logits, const wide_router_dims *d, cudaStream_t s)
 {
     const int64_t T = d->tokens, H = d->hidden, R = d->bottleneck, G = d->groups;
+    if (T <= kRMaxTokens && route_small_smem((int)H, (int)R, (int)G) <= 227u * 1024u)
+        return route_small_launch(x, w_r1, w_r2, b_r2, mask, logits, (int)T, (int)H, (int)R,
+                                  (int)G, d->act, s);
     CUtensorMap tw;
     // W_r1 in two boxes of R/2 rows x 64 columns (128-byte swizzle)
     if (!make_tmap_2d(&tw, w_r1, (uint64_t)R, (uint64_t)H, (uint64_t)H, 2, (uint32_t)(R / 2), 64,
