@@ -13,10 +13,11 @@
 // and stores the mask words directly.
 //
 // Up to 32 tokens (decode): route_small, CUDA cores, clusters of 8 CTAs.  A
-// cluster takes 4 tokens; CTA k of it takes bottleneck units
-// [k R/8, (k+1) R/8): it streams those rows of W_r1 once (16-byte loads, x
-// staged in shared memory), forms z for its units, and multiplies them by
-// the matching columns of W_r2 into partial logits [4][G] in its shared
+// cluster takes 2 tokens; CTA k of it takes bottleneck units
+// [k R/8, (k+1) R/8).  One thread bulk-copies those rows of W_r1 into
+// shared memory (all in flight at once, one mbarrier) while the others stage
+// x as fp32 and the matching columns of W_r2; then each warp forms z for its
+// units and each thread partial logits [2][G] for its share, in shared
 // memory.  After a cluster barrier every CTA sums the 8 partials of its
 // share of the (token, mask word) items through distributed shared memory,
 // adds the bias and takes the decisions with a warp ballot (lane j = group
@@ -33,7 +34,7 @@ namespace cg = cooperative_groups;
 
 namespace {
 constexpr int kBM = 128;
-constexpr int kRTok = 4;         // tokens per cluster
+constexpr int kRTok = 2;         // tokens per cluster
 constexpr int kRCluster = 8;     // CTAs per cluster
 constexpr int kRThreads = 256;
 constexpr int kRMaxTokens = 32;  // route_small's range
@@ -43,13 +44,21 @@ __device__ __forceinline__ float router_act(float v, int act)
     return act == WIDE_ACT_SILU ? silu_f32(v) : fmaxf(v, 0.f);
 }
 
-// Shared memory: x rows [kRTok][H] bf16, z [kRTok][R/8] fp32, partial
-// logits [kRTok][G] fp32.
+// Shared memory, in order: mbarrier (16 bytes), W_r1 rows [R/8][H] bf16,
+// x [kRTok][H] fp32, W_r2 columns [G][R/8] fp32, z [kRTok][R/8] fp32,
+// partial logits [kRTok][G] fp32.
+size_t route_small_smem(int H, int R, int G)
+{
+    const size_t RB = (size_t)(R / kRCluster);
+    return 16 + RB * H * 2 + (size_t)kRTok * H * 4 + (size_t)G * RB * 4 + kRTok * RB * 4 +
+           (size_t)kRTok * G * 4;
+}
+
 __global__ void __launch_bounds__(kRThreads, 1)
     route_small(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ w1,
                 const __nv_bfloat16 *__restrict__ w2, const float *__restrict__ b2,
                 uint32_t *__restrict__ mask, float *__restrict__ logits, int T, int H, int R,
-                int G, int act)
+                int G, int act, int32_t *status)
 {
     extern __shared__ __align__(16) uint8_t sm[];
     cg::cluster_group cluster = cg::this_cluster();
@@ -58,36 +67,64 @@ __global__ void __launch_bounds__(kRThreads, 1)
     const int nt = min(kRTok, T - t0);
     const int RB = R / kRCluster, r0 = k * RB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __nv_bfloat16 *xs = reinterpret_cast<__nv_bfloat16 *>(sm);
-    float *zs = reinterpret_cast<float *>(sm + (size_t)kRTok * H * 2);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm);
+    __nv_bfloat16 *w1s = reinterpret_cast<__nv_bfloat16 *>(sm + 16);
+    float *xs = reinterpret_cast<float *>(sm + 16 + (size_t)RB * H * 2);
+    float *w2s = xs + kRTok * H;
+    float *zs = w2s + G * RB;
     float *ps = zs + kRTok * RB;
 
-    // x rows of this cluster's tokens (rows past T are zeros)
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        const uint32_t row_bytes = (uint32_t)H * 2u;
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)RB);
+        for (int rr = 0; rr < RB; ++rr)
+            bulk_load(w1s + (size_t)rr * H, w1 + (size_t)(r0 + rr) * H, row_bytes, bar);
+    }
+    // x rows of this cluster's tokens as fp32 (rows past T are zeros)
     const int hc = H / 8;
     for (int i = threadIdx.x; i < kRTok * hc; i += kRThreads) {
         const int tt = i / hc, ch = i - tt * hc;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        float f[8] = {};
         if (tt < nt)
-            v = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H) + ch);
-        reinterpret_cast<uint4 *>(xs)[i] = v;
+            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H) + ch), f);
+        float4 *d = reinterpret_cast<float4 *>(xs + (size_t)tt * H + 8 * ch);
+        d[0] = make_float4(f[0], f[1], f[2], f[3]);
+        d[1] = make_float4(f[4], f[5], f[6], f[7]);
     }
-    __syncthreads();
+    // this CTA's columns of W_r2 as fp32, [g][rr]
+    for (int i = threadIdx.x; i < G * (RB / 2); i += kRThreads) {
+        const int g = i / (RB / 2), p = i - g * (RB / 2);
+        const float2 v = __bfloat1622float2(
+            reinterpret_cast<const __nv_bfloat162 *>(w2 + (size_t)g * R + r0)[p]);
+        w2s[g * RB + 2 * p] = v.x;
+        w2s[g * RB + 2 * p + 1] = v.y;
+    }
+    __syncthreads();  // barrier initialised, x and W_r2 staged
+    if (!mbar_wait(bar, 0))
+        set_status(status, WIDE_DEV_TIMEOUT);
 
     // z[tt][rr] = act(x[t0 + tt] . W_r1[r0 + rr]): one warp per unit
     for (int rr = warp; rr < RB; rr += kRThreads / 32) {
-        const uint4 *wr = reinterpret_cast<const uint4 *>(w1 + (size_t)(r0 + rr) * H);
+        const uint4 *wr = reinterpret_cast<const uint4 *>(w1s + (size_t)rr * H);
         float acc[kRTok] = {};
 #pragma unroll 4
         for (int ch = lane; ch < hc; ch += 32) {
             float wv[8];
-            bf16x8_to_f32(__ldg(wr + ch), wv);
+            bf16x8_to_f32(wr[ch], wv);
 #pragma unroll
             for (int tt = 0; tt < kRTok; ++tt) {
-                float xv[8];
-                bf16x8_to_f32(reinterpret_cast<const uint4 *>(xs + (size_t)tt * H)[ch], xv);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    acc[tt] = fmaf(wv[e], xv[e], acc[tt]);
+                const float4 *xp = reinterpret_cast<const float4 *>(xs + (size_t)tt * H + 8 * ch);
+                const float4 a = xp[0], b = xp[1];
+                acc[tt] = fmaf(wv[0], a.x, acc[tt]);
+                acc[tt] = fmaf(wv[1], a.y, acc[tt]);
+                acc[tt] = fmaf(wv[2], a.z, acc[tt]);
+                acc[tt] = fmaf(wv[3], a.w, acc[tt]);
+                acc[tt] = fmaf(wv[4], b.x, acc[tt]);
+                acc[tt] = fmaf(wv[5], b.y, acc[tt]);
+                acc[tt] = fmaf(wv[6], b.z, acc[tt]);
+                acc[tt] = fmaf(wv[7], b.w, acc[tt]);
             }
         }
 #pragma unroll
@@ -104,18 +141,16 @@ __global__ void __launch_bounds__(kRThreads, 1)
     // partial logits of this CTA's units: ps[tt][g] = z[tt] . W_r2[g][r0 : r0 + RB]
     for (int i = threadIdx.x; i < kRTok * G; i += kRThreads) {
         const int tt = i / G, g = i - tt * G;
-        const __nv_bfloat162 *wg = reinterpret_cast<const __nv_bfloat162 *>(w2 + (size_t)g * R + r0);
+        const float *wg = w2s + g * RB;
+        const float *z = zs + tt * RB;
         float acc = 0.f;
-        for (int rr = 0; rr < RB; rr += 2) {
-            const float2 wv = __bfloat1622float2(wg[rr / 2]);
-            acc = fmaf(zs[tt * RB + rr], wv.x, acc);
-            acc = fmaf(zs[tt * RB + rr + 1], wv.y, acc);
-        }
+        for (int rr = 0; rr < RB; ++rr)
+            acc = fmaf(z[rr], wg[rr], acc);
         ps[i] = acc;
     }
     cluster.sync();
 
-    // sum the 8 partials: item (tt, wd) to warp (item - k*8) of rank k
+    // sum the 8 partials of item (tt, wd), items dealt round-robin to warps
     const int nw = (G + 31) >> 5;
     for (int it = k * (kRThreads / 32) + warp; it < nt * nw; it += kRCluster * (kRThreads / 32)) {
         const int tt = it / nw, wd = it - tt * nw;
@@ -134,11 +169,6 @@ __global__ void __launch_bounds__(kRThreads, 1)
             logits[(size_t)(t0 + tt) * G + g] = lg;
     }
     cluster.sync();  // no CTA leaves while another still reads its partials
-}
-
-size_t route_small_smem(int H, int R, int G)
-{
-    return (size_t)kRTok * H * 2 + (size_t)kRTok * (R / kRCluster) * 4 + (size_t)kRTok * G * 4;
 }
 
 int route_small_launch(const void *x, const void *w1, const void *w2, const float *b2,
@@ -164,7 +194,7 @@ int route_small_launch(const void *x, const void *w1, const void *w2, const floa
     if (cudaLaunchKernelEx(&cfg, route_small, static_cast<const __nv_bfloat16 *>(x),
                            static_cast<const __nv_bfloat16 *>(w1),
                            static_cast<const __nv_bfloat16 *>(w2), b2, mask, logits, T, H, R, G,
-                           act) != cudaSuccess)
+                           act, status_ptr()) != cudaSuccess)
         return WIDE_CUDA_FAIL();
     return WIDE_OK;
 }
