@@ -19,6 +19,10 @@
 //              coalesced requests; each thread's copy completions arrive on
 //              the stage barrier
 //   modes
+//     Router  dense: every 128-token tile of x (one TMA box per K stage;
+//             the gather warps only arrive) times all of W_r1 (N = the
+//             bottleneck width); epilogue: activation, W_r2 products and
+//             the packed execute bits (router_epilogue)
 //     SwiGLU  work item (g, i) of the FFN work list; B = [W_gate[g]; W_up[g]]
 //             (N = 2 gs: 256 for 128-channel groups, 128 for 64);
 //             epilogue h = silu(gate) * up, stored bf16 at the token's
@@ -400,7 +404,13 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                         ok = false;
                     } else {
                         uint8_t *b = smem + stage * kStageBytes + kATile;
-                        mbar_arrive_expect_tx(&ctl->full[stage], b_rows * 128u);
+                        // router: the token rows are contiguous, so the A tile
+                        // is one TMA box of x as well (rows past T read zeros)
+                        mbar_arrive_expect_tx(&ctl->full[stage],
+                                              b_rows * 128u + (MODE == GEMM_ROUTER ? kATile : 0u));
+                        if (MODE == GEMM_ROUTER)
+                            tma_load_2d(smem + stage * kStageBytes, &tm1, kt * kBK, w.base,
+                                        &ctl->full[stage]);
                         tma_load_2d(b, m0, kt * kBK, r0, &ctl->full[stage]);
                         tma_load_2d(b + b_rows * 64u, m1, kt * kBK, r1, &ctl->full[stage]);
                         ++issued;
@@ -435,7 +445,9 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
             __syncwarp();
             for (int x = lane; x < kBM / 2; x += 32) {
                 const int r = (x >> 2) * 8 + 4 * gw + (x & 3);
-                trow[x] = r < w.nrows ? row_token<MODE>(a, w, r) * a.K : -1;
+                // router: A arrives by TMA; these warps only arrive per stage
+                trow[x] = (MODE != GEMM_ROUTER && r < w.nrows) ? row_token<MODE>(a, w, r) * a.K
+                                                                : -1;
             }
             __syncwarp();
             int off[kBM / 8];

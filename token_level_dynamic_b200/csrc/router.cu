@@ -7,7 +7,7 @@
 // every masked kernel reads.
 //
 // More than 32 tokens: one launch of gather_gemm in router mode
-// (prefill_gemm.cu): every 128-token tile of x times all of W_r1 (N =
+// (prefill_gemm.cu): every 128-token tile of x (TMA) times all of W_r1 (N =
 // bottleneck width) on tcgen05, fp32 in tensor memory; its epilogue applies
 // the activation and the W_r2 products on CUDA cores, one token per thread,
 // and stores the mask words directly.
@@ -83,23 +83,51 @@ __global__ void __launch_bounds__(kRThreads, 1)
             bulk_load(w1s + (size_t)rr * H, w1 + (size_t)(r0 + rr) * H, row_bytes, bar);
     }
     // x rows of this cluster's tokens as fp32 (rows past T are zeros)
+    // (loads issued in batches of 8 per thread before their stores, so a
+    // thread has 8 requests in flight instead of one)
     const int hc = H / 8;
-    for (int i = threadIdx.x; i < kRTok * hc; i += kRThreads) {
-        const int tt = i / hc, ch = i - tt * hc;
-        float f[8] = {};
-        if (tt < nt)
-            bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H) + ch), f);
-        float4 *d = reinterpret_cast<float4 *>(xs + (size_t)tt * H + 8 * ch);
-        d[0] = make_float4(f[0], f[1], f[2], f[3]);
-        d[1] = make_float4(f[4], f[5], f[6], f[7]);
+    for (int i0 = threadIdx.x; i0 < kRTok * hc; i0 += 8 * kRThreads) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRThreads;
+            const int tt = i / hc, ch = i - tt * hc;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < kRTok * hc && tt < nt)
+                v[u] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H) + ch);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRThreads;
+            if (i < kRTok * hc) {
+                float f[8];
+                bf16x8_to_f32(v[u], f);
+                float4 *d = reinterpret_cast<float4 *>(xs + 8 * (size_t)i);
+                d[0] = make_float4(f[0], f[1], f[2], f[3]);
+                d[1] = make_float4(f[4], f[5], f[6], f[7]);
+            }
+        }
     }
     // this CTA's columns of W_r2 as fp32, [g][rr]
-    for (int i = threadIdx.x; i < G * (RB / 2); i += kRThreads) {
-        const int g = i / (RB / 2), p = i - g * (RB / 2);
-        const float2 v = __bfloat1622float2(
-            reinterpret_cast<const __nv_bfloat162 *>(w2 + (size_t)g * R + r0)[p]);
-        w2s[g * RB + 2 * p] = v.x;
-        w2s[g * RB + 2 * p + 1] = v.y;
+    const int np = G * (RB / 2);
+    for (int i0 = threadIdx.x; i0 < np; i0 += 8 * kRThreads) {
+        __nv_bfloat162 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRThreads;
+            const int g = i / (RB / 2), p = i - g * (RB / 2);
+            if (i < np)
+                v[u] = reinterpret_cast<const __nv_bfloat162 *>(w2 + (size_t)g * R + r0)[p];
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kRThreads;
+            if (i < np) {
+                const float2 f = __bfloat1622float2(v[u]);
+                w2s[2 * i] = f.x;
+                w2s[2 * i + 1] = f.y;
+            }
+        }
     }
     __syncthreads();  // barrier initialised, x and W_r2 staged
     if (!mbar_wait(bar, 0))
@@ -207,10 +235,12 @@ int route_launch(const void *x, const void *w_r1, const void *w_r2, const float 
     if (T <= kRMaxTokens && route_small_smem((int)H, (int)R, (int)G) <= 227u * 1024u)
         return route_small_launch(x, w_r1, w_r2, b_r2, mask, logits, (int)T, (int)H, (int)R,
                                   (int)G, d->act, s);
-    CUtensorMap tw;
-    // W_r1 in two boxes of R/2 rows x 64 columns (128-byte swizzle)
+    CUtensorMap tw, tx;
+    // W_r1 in two boxes of R/2 rows x 64 columns, x in boxes of 128 rows x 64
+    // columns (128-byte swizzle, the tensor cores' operand layout)
     if (!make_tmap_2d(&tw, w_r1, (uint64_t)R, (uint64_t)H, (uint64_t)H, 2, (uint32_t)(R / 2), 64,
-                      true))
+                      true) ||
+        !make_tmap_2d(&tx, x, (uint64_t)T, (uint64_t)H, (uint64_t)H, 2, kBM, 64, true))
         return WIDE_CUDA_FAIL();
     GemmArgs ga = {};
     ga.a = static_cast<const __nv_bfloat16 *>(x);
@@ -225,7 +255,7 @@ int route_launch(const void *x, const void *w_r1, const void *w_r2, const float 
     ga.n_groups = (int)G;
     ga.act = d->act;
     ga.status = status_ptr();
-    return gather_gemm_launch(GEMM_ROUTER, tw, tw, ga, ga.m_tiles, KID_ROUTER, s);
+    return gather_gemm_launch(GEMM_ROUTER, tw, tx, ga, ga.m_tiles, KID_ROUTER, s);
 }
 
 }  // namespace wide
