@@ -55,6 +55,12 @@ constexpr int kStages = 4;
 constexpr uint32_t kATile = kBM * 128;
 constexpr uint32_t kBTile = kBN * 128;
 constexpr uint32_t kStageBytes = kATile + kBTile;
+// The router with a bottleneck of at most 128 rows splits the same ring bytes
+// into 6 slots of 32 KB (A tile + 128-row B tile): more bytes in flight.
+constexpr int kRouterStages = 6;
+constexpr uint32_t kRouterStageBytes = kATile + 128u * 128u;
+constexpr int kMaxStages = 6;
+static_assert(kRouterStages * kRouterStageBytes <= kStages * kStageBytes, "router ring");
 constexpr int kThreadsDown = 192;
 constexpr int kThreadsGather = 256;
 constexpr int kGatherThreads = 64;
@@ -62,8 +68,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kHD = 128;
 
 struct __align__(8) Ctl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -115,7 +121,7 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&
 
 __device__ __forceinline__ void init_ctl(Ctl *ctl, uint32_t full_count)
 {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
         mbar_init(&ctl->full[s], full_count);
         mbar_init(&ctl->empty[s], 1);
     }
@@ -353,6 +359,10 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
     const int n_items = (MODE == GEMM_KV || MODE == GEMM_ROUTER) ? 0 : *a.n_items_p;
     const int nw = n_work<MODE>(a, n_items);
     const int KT = a.K / kBK;
+    // ring: kStages slots of kStageBytes, or the router's 6 smaller slots
+    const bool small_slots = MODE == GEMM_ROUTER && a.rn <= 128;
+    const uint32_t nst = small_slots ? (uint32_t)kRouterStages : (uint32_t)kStages;
+    const uint32_t sbytes = small_slots ? kRouterStageBytes : kStageBytes;
 
     if (threadIdx.x == 0) {
         // one arrive (with the weight bytes) from the producer plus one
@@ -403,13 +413,13 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                     if (!wait_or_abort(&ctl->empty[stage], phase ^ 1u, ctl, a.status)) {
                         ok = false;
                     } else {
-                        uint8_t *b = smem + stage * kStageBytes + kATile;
+                        uint8_t *b = smem + stage * sbytes + kATile;
                         // router: the token rows are contiguous, so the A tile
                         // is one TMA box of x as well (rows past T read zeros)
                         mbar_arrive_expect_tx(&ctl->full[stage],
                                               b_rows * 128u + (MODE == GEMM_ROUTER ? kATile : 0u));
                         if (MODE == GEMM_ROUTER)
-                            tma_load_2d(smem + stage * kStageBytes, &tm1, kt * kBK, w.base,
+                            tma_load_2d(smem + stage * sbytes, &tm1, kt * kBK, w.base,
                                         &ctl->full[stage]);
                         tma_load_2d(b, m0, kt * kBK, r0, &ctl->full[stage]);
                         tma_load_2d(b + b_rows * 64u, m1, kt * kBK, r1, &ctl->full[stage]);
@@ -417,15 +427,15 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                     }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (++stage == kStages) {
+                if (++stage == nst) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
         }
         if (!ok && lane == 0) {
-            for (uint32_t s = 0; s < kStages && s < issued; ++s) {
-                const uint32_t uses = (issued - s + kStages - 1) / kStages;
+            for (uint32_t s = 0; s < nst && s < issued; ++s) {
+                const uint32_t uses = (issued - s + nst - 1) / nst;
                 mbar_wait(&ctl->full[s], (uses - 1u) & 1u);
             }
         }
@@ -460,14 +470,14 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                     ok = false;
                     break;
                 }
-                const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                const uint32_t sa = smem_u32(smem + stage * sbytes);
                 const __nv_bfloat16 *src = a.a + kt * kBK + 8 * cc;
 #pragma unroll
                 for (int i = 0; i < kBM / 8; ++i)
                     if (off[i] >= 0)
                         cp_async16(sa + swz128(lr + 8 * i, cc), src + off[i]);
                 cp_async_arrive_noinc(&ctl->full[stage]);
-                if (++stage == kStages) {
+                if (++stage == nst) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -499,7 +509,7 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                     // is read by the tensor core (async proxy)
                     fence_proxy_async_smem();
                     umma::fence_after_sync();
-                    const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                    const uint32_t sa = smem_u32(smem + stage * sbytes);
                     const uint32_t sb = sa + kATile;
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
@@ -507,7 +517,7 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                                        umma::desc_kmajor_sw128(sb + 32u * k), idesc,
                                        (kt | k) != 0);
                     umma::commit(&ctl->empty[stage]);
-                    if (++stage == kStages) {
+                    if (++stage == nst) {
                         stage = 0;
                         phase ^= 1u;
                     }

@@ -14,11 +14,11 @@
 //
 // Up to 32 tokens (decode): route_small, CUDA cores, clusters of 8 CTAs.  A
 // cluster takes 2 tokens; CTA k of it takes bottleneck units
-// [k R/8, (k+1) R/8).  One thread bulk-copies those rows of W_r1 into
-// shared memory (all in flight at once, one mbarrier) while the others stage
-// x as fp32 and the matching columns of W_r2; then each warp forms z for its
-// units and each thread partial logits [2][G] for its share, in shared
-// memory.  After a cluster barrier every CTA sums the 8 partials of its
+// [k R/8, (k+1) R/8).  One thread bulk-copies those rows of W_r1 and the
+// cluster's x rows into shared memory (all in flight at once, one mbarrier)
+// while the others stage the matching columns of W_r2 as fp32; then each
+// warp forms z for its units and each thread partial logits [2][G] for its
+// share, in shared memory.  After a cluster barrier every CTA sums the 8 partials of its
 // share of the (token, mask word) items through distributed shared memory,
 // adds the bias and takes the decisions with a warp ballot (lane j = group
 // 32 w + j).  W_r1 is read from HBM once per call (the clusters of a batch
@@ -45,12 +45,12 @@ __device__ __forceinline__ float router_act(float v, int act)
 }
 
 // Shared memory, in order: mbarrier (16 bytes), W_r1 rows [R/8][H] bf16,
-// x [kRTok][H] fp32, W_r2 columns [G][R/8] fp32, z [kRTok][R/8] fp32,
+// x [kRTok][H] bf16, W_r2 columns [G][R/8] fp32, z [kRTok][R/8] fp32,
 // partial logits [kRTok][G] fp32.
 size_t route_small_smem(int H, int R, int G)
 {
     const size_t RB = (size_t)(R / kRCluster);
-    return 16 + RB * H * 2 + (size_t)kRTok * H * 4 + (size_t)G * RB * 4 + kRTok * RB * 4 +
+    return 16 + RB * H * 2 + (size_t)kRTok * H * 2 + (size_t)G * RB * 4 + kRTok * RB * 4 +
            (size_t)kRTok * G * 4;
 }
 
@@ -69,8 +69,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm);
     __nv_bfloat16 *w1s = reinterpret_cast<__nv_bfloat16 *>(sm + 16);
-    float *xs = reinterpret_cast<float *>(sm + 16 + (size_t)RB * H * 2);
-    float *w2s = xs + kRTok * H;
+    __nv_bfloat16 *xs = w1s + (size_t)RB * H;
+    float *w2s = reinterpret_cast<float *>(xs + (size_t)kRTok * H);
     float *zs = w2s + G * RB;
     float *ps = zs + kRTok * RB;
 
@@ -78,36 +78,18 @@ __global__ void __launch_bounds__(kRThreads, 1)
         mbar_init(bar, 1);
         fence_mbar_init();
         const uint32_t row_bytes = (uint32_t)H * 2u;
-        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)RB);
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)(RB + nt));
         for (int rr = 0; rr < RB; ++rr)
             bulk_load(w1s + (size_t)rr * H, w1 + (size_t)(r0 + rr) * H, row_bytes, bar);
+        for (int tt = 0; tt < nt; ++tt)
+            bulk_load(xs + (size_t)tt * H, x + (size_t)(t0 + tt) * H, row_bytes, bar);
     }
-    // x rows of this cluster's tokens as fp32 (rows past T are zeros)
-    // (loads issued in batches of 8 per thread before their stores, so a
-    // thread has 8 requests in flight instead of one)
+    // x rows past T are zeros
     const int hc = H / 8;
-    for (int i0 = threadIdx.x; i0 < kRTok * hc; i0 += 8 * kRThreads) {
-        uint4 v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kRThreads;
-            const int tt = i / hc, ch = i - tt * hc;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (i < kRTok * hc && tt < nt)
-                v[u] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(t0 + tt) * H) + ch);
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int i = i0 + u * kRThreads;
-            if (i < kRTok * hc) {
-                float f[8];
-                bf16x8_to_f32(v[u], f);
-                float4 *d = reinterpret_cast<float4 *>(xs + 8 * (size_t)i);
-                d[0] = make_float4(f[0], f[1], f[2], f[3]);
-                d[1] = make_float4(f[4], f[5], f[6], f[7]);
-            }
-        }
-    }
+    for (int i = nt * hc + threadIdx.x; i < kRTok * hc; i += kRThreads)
+        reinterpret_cast<uint4 *>(xs)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // (W_r2 loads issued in batches of 8 per thread before their stores, so
+    // a thread has 8 requests in flight instead of one)
     // this CTA's columns of W_r2 as fp32, [g][rr]
     const int np = G * (RB / 2);
     for (int i0 = threadIdx.x; i0 < np; i0 += 8 * kRThreads) {
@@ -129,7 +111,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
             }
         }
     }
-    __syncthreads();  // barrier initialised, x and W_r2 staged
+    __syncthreads();  // barrier initialised, W_r2 staged
     if (!mbar_wait(bar, 0))
         set_status(status, WIDE_DEV_TIMEOUT);
 
@@ -143,16 +125,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
             bf16x8_to_f32(wr[ch], wv);
 #pragma unroll
             for (int tt = 0; tt < kRTok; ++tt) {
-                const float4 *xp = reinterpret_cast<const float4 *>(xs + (size_t)tt * H + 8 * ch);
-                const float4 a = xp[0], b = xp[1];
-                acc[tt] = fmaf(wv[0], a.x, acc[tt]);
-                acc[tt] = fmaf(wv[1], a.y, acc[tt]);
-                acc[tt] = fmaf(wv[2], a.z, acc[tt]);
-                acc[tt] = fmaf(wv[3], a.w, acc[tt]);
-                acc[tt] = fmaf(wv[4], b.x, acc[tt]);
-                acc[tt] = fmaf(wv[5], b.y, acc[tt]);
-                acc[tt] = fmaf(wv[6], b.z, acc[tt]);
-                acc[tt] = fmaf(wv[7], b.w, acc[tt]);
+                float xv[8];
+                bf16x8_to_f32(reinterpret_cast<const uint4 *>(xs + (size_t)tt * H)[ch], xv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[tt] = fmaf(wv[e], xv[e], acc[tt]);
             }
         }
 #pragma unroll
