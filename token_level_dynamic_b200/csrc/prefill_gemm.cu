@@ -55,11 +55,12 @@ constexpr int kStages = 4;
 constexpr uint32_t kATile = kBM * 128;
 constexpr uint32_t kBTile = kBN * 128;
 constexpr uint32_t kStageBytes = kATile + kBTile;
-// The router with a bottleneck of at most 128 rows uses slots of 32 KB (A
-// tile + 128-row B tile); the 64 KB of ring this leaves free hold W_r2 as
-// fp32 when it fits (kRouterW2Cache bytes).
+// The router with a bottleneck of at most 128 rows splits the same ring bytes
+// into 6 slots of 32 KB (A tile + 128-row B tile): more bytes in flight.
+constexpr int kRouterStages = 6;
 constexpr uint32_t kRouterStageBytes = kATile + 128u * 128u;
-constexpr uint32_t kRouterW2Cache = kStages * (kStageBytes - kRouterStageBytes);
+constexpr int kMaxStages = 6;
+static_assert(kRouterStages * kRouterStageBytes <= kStages * kStageBytes, "router ring");
 constexpr int kThreadsDown = 192;
 constexpr int kThreadsGather = 256;
 constexpr int kGatherThreads = 64;
@@ -67,8 +68,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kHD = 128;
 
 struct __align__(8) Ctl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -120,7 +121,7 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16 *dst, const float (&
 
 __device__ __forceinline__ void init_ctl(Ctl *ctl, uint32_t full_count)
 {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
         mbar_init(&ctl->full[s], full_count);
         mbar_init(&ctl->empty[s], 1);
     }
@@ -225,43 +226,12 @@ constexpr int kRW2Stride = 36;
 constexpr uint32_t kRouterScratch = 4u * 32u * kRW2Stride * 4u + 16u;
 static_assert(kSmemBytes + kRouterScratch <= 232448, "router mode exceeds 227 KB of shared memory");
 
-// All of W_r2 as fp32 rows of rn floats, groups padded with zero rows to a
-// multiple of 32, by the 128 epilogue threads (tid 0..127); loads in batches
-// of 4 per thread before their stores.
-__device__ __forceinline__ void router_w2_cache(const GemmArgs &a, float *c, int tid)
-{
-    const int rn = a.rn, n8 = ((a.n_groups + 31) & ~31) * rn / 8;
-    for (int i0 = tid; i0 < n8; i0 += 4 * 128) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * 128;
-            const int g = (i * 8) / rn, col = (i * 8) % rn;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
-            if (i < n8 && g < a.n_groups)
-                v[u] = __ldg(reinterpret_cast<const uint4 *>(a.w_r2 + (size_t)g * rn + col));
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u * 128;
-            if (i < n8) {
-                float f[8];
-                bf16x8_to_f32(v[u], f);
-                float4 *d = reinterpret_cast<float4 *>(c + (size_t)i * 8);
-                d[0] = make_float4(f[0], f[1], f[2], f[3]);
-                d[1] = make_float4(f[4], f[5], f[6], f[7]);
-            }
-        }
-    }
-}
-
 __device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t taddr, int t,
-                                                bool live, float *ws, const float *w2c, int lane)
+                                                bool live, float *ws, int lane)
 {
     const int G = a.n_groups, nw = (G + 31) >> 5, nc = a.rn >> 5, nblk = nw * nc;
     uint4 nx[4];
-    if (!w2c)
-        w2_block_load(a, 0, 0, lane, nx);
+    w2_block_load(a, 0, 0, lane, nx);
 #pragma unroll 1
     for (int wd = 0; wd < nw; ++wd) {
         const int g0 = wd * 32;
@@ -272,30 +242,19 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t tadd
             acc[j] = make_float2((a.b_r2 && j < ng) ? __ldg(a.b_r2 + g0 + j) : 0.f, 0.f);
 #pragma unroll 1
         for (int c = 0; c < nc; ++c) {
-            // W_r2 block: rows of the cache, or this warp's staged copy
-            const float *wb;
-            int wstride;
-            if (w2c) {
-                wb = w2c + (size_t)g0 * a.rn + c * 32;
-                wstride = a.rn;
-            } else {
-                __syncwarp();
-                float *row = ws + lane * kRW2Stride;
+            __syncwarp();
+            float *row = ws + lane * kRW2Stride;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float f[8];
-                    bf16x8_to_f32(nx[q], f);
-                    *reinterpret_cast<float4 *>(row + 8 * q) = make_float4(f[0], f[1], f[2], f[3]);
-                    *reinterpret_cast<float4 *>(row + 8 * q + 4) =
-                        make_float4(f[4], f[5], f[6], f[7]);
-                }
-                __syncwarp();
-                const int nb = wd * nc + c + 1;
-                if (nb < nblk)
-                    w2_block_load(a, nb / nc, nb % nc, lane, nx);
-                wb = ws;
-                wstride = kRW2Stride;
+            for (int q = 0; q < 4; ++q) {
+                float f[8];
+                bf16x8_to_f32(nx[q], f);
+                *reinterpret_cast<float4 *>(row + 8 * q) = make_float4(f[0], f[1], f[2], f[3]);
+                *reinterpret_cast<float4 *>(row + 8 * q + 4) = make_float4(f[4], f[5], f[6], f[7]);
             }
+            __syncwarp();
+            const int nb = wd * nc + c + 1;
+            if (nb < nblk)
+                w2_block_load(a, nb / nc, nb % nc, lane, nx);
             float z[32];
             umma::tmem_ld32(taddr + c * 32, z);
             umma::tmem_ld_wait();
@@ -304,7 +263,7 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t tadd
                 z[e] = a.act == WIDE_ACT_SILU ? silu_f32(z[e]) : fmaxf(z[e], 0.f);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float4 *wr = reinterpret_cast<const float4 *>(wb + j * wstride);
+                const float4 *wr = reinterpret_cast<const float4 *>(ws + j * kRW2Stride);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     const float4 w = wr[e4];
@@ -400,10 +359,9 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
     const int n_items = (MODE == GEMM_KV || MODE == GEMM_ROUTER) ? 0 : *a.n_items_p;
     const int nw = n_work<MODE>(a, n_items);
     const int KT = a.K / kBK;
-    // ring: kStages slots of kStageBytes, or of kRouterStageBytes for the
-    // router with a bottleneck of at most 128 rows
+    // ring: kStages slots of kStageBytes, or the router's 6 smaller slots
     const bool small_slots = MODE == GEMM_ROUTER && a.rn <= 128;
-    const uint32_t nst = (uint32_t)kStages;
+    const uint32_t nst = small_slots ? (uint32_t)kRouterStages : (uint32_t)kStages;
     const uint32_t sbytes = small_slots ? kRouterStageBytes : kStageBytes;
 
     if (threadIdx.x == 0) {
@@ -583,16 +541,6 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
         const int q = warp & 3;
         const int r = q * 32 + lane;          // tile row = TMEM lane
         uint32_t acc = 0, acc_phase = 0;
-        // router: all of W_r2 as fp32 [32 ceil(G/32)][rn] in the ring bytes the
-        // small slots leave free, loaded while the first tile's K loop runs
-        const float *w2c = nullptr;
-        if (MODE == GEMM_ROUTER && small_slots &&
-            (uint32_t)((a.n_groups + 31) & ~31) * (uint32_t)a.rn * 4u <= kRouterW2Cache) {
-            float *c = reinterpret_cast<float *>(smem + kStages * kRouterStageBytes);
-            router_w2_cache(a, c, threadIdx.x - 64);
-            asm volatile("bar.sync 2, 128;" ::: "memory");
-            w2c = c;
-        }
         for (int it = blockIdx.x; it < nw; it += gridDim.x) {
             const Work w = decode_work<MODE>(a, it);
             const bool live = r < w.nrows;
@@ -622,7 +570,7 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
                                 smem + ((kStages * kStageBytes + sizeof(Ctl) + 15) & ~(size_t)15)) +
                             q * 32 * kRW2Stride;
                 if (__any_sync(0xffffffffu, live))
-                    router_epilogue(a, taddr, t, live, ws, w2c, lane);
+                    router_epilogue(a, taddr, t, live, ws, lane);
             } else if (MODE == GEMM_ROPE_Q) {
                 const int pos = (int)(t % a.seq_len + a.cache_len);
                 __nv_bfloat16 *dst = a.out0 + ((size_t)w.g * a.T + w.base + r) * a.group_cols +
