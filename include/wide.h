@@ -328,9 +328,12 @@ int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, const void *d
  *             bits at or above groups zero
  *   d_logits  out: fp32 [tokens][groups] (the values the decisions were
  *             taken on), or NULL
- * Arithmetic: x W_r1^T on tcgen05 tensor cores (bf16 operands, fp32
- * accumulation in tensor memory), activation and W_r2 products in fp32 on
- * CUDA cores; no intermediate is rounded to bf16.
+ * Arithmetic: for more than 32 tokens x W_r1^T runs on tcgen05 tensor
+ * cores (bf16 operands, fp32 accumulation in tensor memory), for up to 32
+ * on CUDA cores (fp32); the activation and the W_r2 products are fp32 on
+ * CUDA cores; no intermediate is rounded to bf16.  A decision can differ
+ * between the two kernels, or from an fp64 evaluation, only where the logit
+ * is within fp32 rounding of 0.
  * Supported: hidden a multiple of 64; bottleneck a multiple of 32 in
  * [32, 256]; groups in [1, 1024]; tokens * hidden < 2^31; d_x, d_w_r1 and
  * d_w_r2 16-byte aligned (else WIDE_EUNSUPPORTED).  tokens == 0 enqueues

@@ -261,17 +261,16 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs &a, uint32_t tadd
 #pragma unroll
             for (int e = 0; e < 32; ++e)
                 z[e] = a.act == WIDE_ACT_SILU ? silu_f32(z[e]) : fmaxf(z[e], 0.f);
-            // units outer, groups inner: consecutive FMAs update different
-            // accumulators (each still sums its units in ascending order)
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                const float2 z01 = make_float2(z[4 * e4], z[4 * e4 + 1]);
-                const float2 z23 = make_float2(z[4 * e4 + 2], z[4 * e4 + 3]);
+            for (int j = 0; j < 32; ++j) {
+                const float4 *wr = reinterpret_cast<const float4 *>(ws + j * kRW2Stride);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float4 w = reinterpret_cast<const float4 *>(ws + j * kRW2Stride)[e4];
-                    acc[j] = __ffma2_rn(z01, make_float2(w.x, w.y), acc[j]);
-                    acc[j] = __ffma2_rn(z23, make_float2(w.z, w.w), acc[j]);
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 w = wr[e4];
+                    acc[j] = __ffma2_rn(make_float2(z[4 * e4], z[4 * e4 + 1]),
+                                        make_float2(w.x, w.y), acc[j]);
+                    acc[j] = __ffma2_rn(make_float2(z[4 * e4 + 2], z[4 * e4 + 3]),
+                                        make_float2(w.z, w.w), acc[j]);
                 }
             }
         }

@@ -18,11 +18,11 @@
 // cluster's x rows into shared memory (all in flight at once, one mbarrier)
 // while the others stage the matching columns of W_r2 as fp32; then each
 // warp forms z for its units and each thread partial logits [2][G] for its
-// share, in shared memory.  After a cluster barrier every CTA sums the 8 partials of its
-// share of the (token, mask word) items through distributed shared memory,
-// adds the bias and takes the decisions with a warp ballot (lane j = group
-// 32 w + j).  W_r1 is read from HBM once per call (the clusters of a batch
-// share it through L2).
+// share, in shared memory.  After a cluster barrier every CTA sums the 8
+// partials of its share of the (token, mask word) items through distributed
+// shared memory, adds the bias and takes the decisions with a warp ballot
+// (lane j = group 32 w + j).  W_r1 is read from HBM once per call (the
+// clusters of a batch share it through L2).
 #include "common.cuh"
 #include "host.h"
 
