@@ -1,0 +1,48 @@
+"""bench.py's host side on CPU: the reference arm's JSON line, and the
+algorithmic units the router workload divides by (no GPU needed)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.parametrize("workload", ["decode_ffn_3b", "router_8b"])
+def test_reference_arm_line(workload):
+    """Rank 0 of the reference arm times the oracle on the host cores and
+    prints one JSON line with the contract's keys."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", workload, "--steps", "1", "--warmup", "3"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 3
+    assert d["config"]["workload"].startswith(workload)
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_router_units():
+    """Algorithmic bytes of one router call: x, W_r1 and W_r2 read once,
+    the packed mask words written once; the kernel name follows the size
+    split of the library (cluster kernel up to 32 tokens, tcgen05 above)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = bench.WORKLOADS["router_8b"]
+    cases = wl.make_cases()
+    assert [c.T for c in cases] == [8192, 16]
+    u_big, u_small = (wl.units(c) for c in cases)
+    assert u_big == {"router_tcgen05": 8192 * 4096 * 2 + 128 * 4096 * 2 + 112 * 128 * 2
+                     + 8192 * 4 * 4, "total": u_big["total"]}
+    assert u_small == {"router_small_gemv": 16 * 4096 * 2 + 128 * 4096 * 2 + 112 * 128 * 2
+                       + 16 * 4 * 4, "total": u_small["total"]}
+    assert u_big["total"] == u_big["router_tcgen05"]
