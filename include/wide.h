@@ -330,8 +330,11 @@ int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, const void *d
  *             taken on), or NULL
  * Arithmetic: for more than 32 tokens x W_r1^T runs on tcgen05 tensor
  * cores (bf16 operands, fp32 accumulation in tensor memory), for up to 32
- * on CUDA cores (fp32); the activation and the W_r2 products are fp32 on
- * CUDA cores; no intermediate is rounded to bf16.  A decision can differ
+ * on CUDA cores in fp32 (when that kernel's shared memory, about
+ * (bottleneck / 4 + 4) * hidden + 4 * groups * (bottleneck / 8 + 2) bytes,
+ * fits in 227 KB; otherwise on the tensor-core kernel too); the activation
+ * and the W_r2 products are fp32 on CUDA cores; no intermediate is rounded
+ * to bf16.  A decision can differ
  * between the two kernels, or from an fp64 evaluation, only where the logit
  * is within fp32 rounding of 0.
  * Supported: hidden a multiple of 64; bottleneck a multiple of 32 in

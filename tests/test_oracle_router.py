@@ -135,3 +135,16 @@ def test_packing_layout():
     m = route_mask(rc.x, rc.w_r1, rc.w_r2, rc.b_r2)
     assert np.all(m[:, 1] >> np.uint32(45 - 32) == 0)
     np.testing.assert_array_equal(m, synth.pack_mask(synth.unpack_mask(m, rc.G)))
+
+
+def test_router_case_weights_independent_of_batch():
+    """The seeded router weights depend on (seed, H, R, G) only, so a decode
+    batch and a prefill batch of one model share them; x depends on T."""
+    a = synth.router_case(T=3, H=64, R=32, G=10, seed=4, bias_std=0.1)
+    b = synth.router_case(T=9, H=64, R=32, G=10, seed=4, bias_std=0.1)
+    np.testing.assert_array_equal(a.w_r1, b.w_r1)
+    np.testing.assert_array_equal(a.w_r2, b.w_r2)
+    np.testing.assert_array_equal(a.b_r2, b.b_r2)
+    assert a.x.shape == (3, 64) and b.x.shape == (9, 64)
+    c = synth.router_case(T=3, H=64, R=32, G=10, seed=5, bias_std=0.1)
+    assert not np.array_equal(a.w_r1, c.w_r1)
