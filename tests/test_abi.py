@@ -149,3 +149,40 @@ def test_route_argument_checks(native):
         == native.WIDE_EUNSUPPORTED
     assert L.wide_route(p, p, p, ctypes.c_void_p((1 << 20) + 2), p, None, ctypes.byref(ok),
                         None) == native.WIDE_EUNSUPPORTED
+
+
+def test_layer_argument_checks(native):
+    """wide_layer_masked / wide_attn_masked / wide_layer_workspace_bytes
+    answer on the host for bad dims, missing or misaligned pointers and a
+    short workspace, before anything is enqueued."""
+    L = native.lib()
+    D, Wt = native.WideLayerDims, native.WideLayerWeights
+    dec = D(16, 1, 2048, 2049, 4096, 14336, 128, 32, 8, 128, 5e5, 1e-5)
+    pre = D(4, 2048, 0, 2048, 4096, 14336, 128, 32, 8, 128, 5e5, 1e-5)
+    ws_dec = L.wide_layer_workspace_bytes(ctypes.byref(dec))
+    ws_pre = L.wide_layer_workspace_bytes(ctypes.byref(pre))
+    assert ws_dec > 16 * 14336 * 4
+    assert ws_pre > 8192 * 14336 * 2
+    for bad in (D(16, 1, 2048, 2049, 4096, 14336, 128, 32, 7, 128, 5e5, 1e-5),     # 32 % 7
+                D(16, 1, 2048, 2048, 4096, 14336, 128, 32, 8, 128, 5e5, 1e-5),     # no room
+                D(16, 1, 2048, 2049, 4096, 14336, 128, 32, 8, 128, 5e5, -1.0),     # eps < 0
+                D(16, 1, 2048, 2049, 4096, 14336, 128, 32, 8, 128, 0.0, 1e-5),     # theta 0
+                D(16, 1, 2048, 2049, 4096, 14336, 100, 32, 8, 128, 5e5, 1e-5),     # gs does not divide I
+                D(16, 1, 2048, 2049, 4096, 14336, 128, 32, 8, 64, 5e5, 1e-5),      # head_dim 64
+                D(16, 1, 131072, 131073, 4096, 14336, 128, 32, 8, 128, 5e5, 1e-5)):  # cache too long
+        assert L.wide_layer_workspace_bytes(ctypes.byref(bad)) == 0
+    p = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    full = Wt(*([p] * 9))
+    empty = Wt(*([None] * 9))
+    args = lambda x, w, ws_bytes, d: (x, ctypes.byref(w), p, p, p, p, p, p, p, ctypes.byref(d),
+                                      p, ws_bytes, None)
+    assert L.wide_layer_masked(p, None, p, p, p, p, p, p, p, ctypes.byref(dec), p, ws_dec,
+                               None) == native.WIDE_EINVAL
+    assert L.wide_layer_masked(*args(p, empty, ws_dec, dec)) == native.WIDE_EINVAL
+    assert L.wide_layer_masked(*args(mis, full, ws_dec, dec)) == native.WIDE_EUNSUPPORTED
+    assert L.wide_layer_masked(*args(p, full, ws_dec - 1, dec)) == native.WIDE_EWORKSPACE
+    assert L.wide_layer_masked(*args(p, full, ws_pre - 1, pre)) == native.WIDE_EWORKSPACE
+    # the attention half alone needs its output pointer
+    assert L.wide_attn_masked(p, ctypes.byref(full), p, p, p, None, ctypes.byref(dec), p,
+                              ws_dec, None) == native.WIDE_EINVAL
