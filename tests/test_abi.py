@@ -186,3 +186,27 @@ def test_layer_argument_checks(native):
     # the attention half alone needs its output pointer
     assert L.wide_attn_masked(p, ctypes.byref(full), p, p, p, None, ctypes.byref(dec), p,
                               ws_dec, None) == native.WIDE_EINVAL
+
+
+def test_route_binding_checks_dtypes_and_shapes():
+    """The Python binding refuses tensors the C ABI cannot check (dtype and
+    shape) before touching the device."""
+    import torch
+    import token_level_dynamic_b200 as w
+    bf = torch.bfloat16
+    x, w1, w2 = torch.zeros(4, 64, dtype=bf), torch.zeros(32, 64, dtype=bf), torch.zeros(8, 32, dtype=bf)
+    with pytest.raises(TypeError):
+        w.wide_route(x.float(), w1, w2)
+    with pytest.raises(ValueError):
+        w.wide_route(x, torch.zeros(32, 32, dtype=bf), w2)          # W_r1 width != H
+    with pytest.raises(ValueError):
+        w.wide_route(x, w1, torch.zeros(8, 16, dtype=bf))           # W_r2 width != R
+    with pytest.raises(ValueError):
+        w.wide_route(x, w1, w2, b_r2=torch.zeros(8, dtype=torch.float64))
+    with pytest.raises(ValueError):
+        w.wide_route(x, w1, w2, mask_words=torch.zeros(4, 2, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        w.wide_route(x, w1, w2, logits=torch.zeros(4, 9))
+    # well-formed CPU tensors get past these checks and stop at the device check
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        w.wide_route(x, w1, w2, mask_words=torch.zeros(4, 1, dtype=torch.int32))

@@ -306,6 +306,19 @@ def wide_route(x: torch.Tensor, w_r1: torch.Tensor, w_r2: torch.Tensor,
     `logits` (fp32 [T][G]) is given, the logits are written there too."""
     T, H = x.shape
     R, G = w_r1.shape[0], w_r2.shape[0]
+    for name, t in (("x", x), ("w_r1", w_r1), ("w_r2", w_r2)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if tuple(w_r1.shape) != (R, H) or tuple(w_r2.shape) != (G, R):
+        raise ValueError(f"w_r1 {tuple(w_r1.shape)} / w_r2 {tuple(w_r2.shape)} do not fit "
+                         f"x [{T}][{H}]: expected [R][{H}] and [G][R]")
+    if b_r2 is not None and (b_r2.dtype != torch.float32 or tuple(b_r2.shape) != (G,)):
+        raise ValueError(f"b_r2 must be float32 [{G}]")
+    if mask_words is not None and (mask_words.dtype != torch.int32 or
+                                   tuple(mask_words.shape) != (T, (G + 31) // 32)):
+        raise ValueError(f"mask_words must be int32 [{T}][{(G + 31) // 32}]")
+    if logits is not None and (logits.dtype != torch.float32 or tuple(logits.shape) != (T, G)):
+        raise ValueError(f"logits must be float32 [{T}][{G}]")
     if mask_words is None:
         mask_words = torch.empty((T, (G + 31) // 32), dtype=torch.int32, device=x.device)
     d = WideRouterDims(T, H, R, G, act)
