@@ -210,3 +210,28 @@ def test_route_binding_checks_dtypes_and_shapes():
     # well-formed CPU tensors get past these checks and stop at the device check
     with pytest.raises(ValueError, match="CUDA tensor"):
         w.wide_route(x, w1, w2, mask_words=torch.zeros(4, 1, dtype=torch.int32))
+
+
+def test_ffn_binding_checks_dtypes_and_shapes():
+    """The FFN bindings refuse mismatched dtypes and shapes before the C call."""
+    import torch
+    import token_level_dynamic_b200 as w
+    bf = torch.bfloat16
+    x = torch.zeros(4, 64, dtype=bf)
+    wg, wu, wd = torch.zeros(256, 64, dtype=bf), torch.zeros(256, 64, dtype=bf), torch.zeros(64, 256, dtype=bf)
+    m = torch.zeros(4, 1, dtype=torch.int32)                     # G = 256 / 64 = 4
+    for f in (lambda *a, **k: w.wide_ffn_masked(*a, **k),
+              lambda *a, **k: w.wide_ffn_masked_noalloc(*a, out=k.pop("out", torch.zeros(4, 64, dtype=bf)), **k)):
+        with pytest.raises(TypeError):
+            f(x, wg.float(), wu, wd, m, 64)
+        with pytest.raises(ValueError):
+            f(x, wg, wu, wd.t().contiguous(), m, 64)             # W_down transposed
+        with pytest.raises(ValueError):
+            f(x, wg, wu, wd, torch.zeros(4, 2, dtype=torch.int32), 64)
+        with pytest.raises(ValueError):
+            f(x, wg, wu, wd, m.to(torch.int64), 64)
+        with pytest.raises(ValueError):
+            f(x, wg, wu, wd, m, 64, out=torch.zeros(4, 64))       # fp32 out for bf16 x
+        # well-formed CPU tensors pass these checks and stop at the device check
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            f(x, wg, wu, wd, m, 64)

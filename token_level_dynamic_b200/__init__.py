@@ -178,6 +178,27 @@ def wide_reorder(mask_words: torch.Tensor, G: int, tile_m: int = 128, buf: torch
 
 # -------------------------------------------------------------- masked FFN
 
+def _check_ffn(x, w_gate, w_up, w_down, mask_words, group_size, out) -> None:
+    """Dtypes and shapes the C ABI cannot see (it takes raw pointers)."""
+    T, H = x.shape
+    I = w_gate.shape[0]
+    for name, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} is {t.dtype}, x is {x.dtype}")
+    if tuple(w_gate.shape) != (I, H) or tuple(w_up.shape) != (I, H) or \
+            tuple(w_down.shape) != (H, I):
+        raise ValueError(f"weights {tuple(w_gate.shape)}, {tuple(w_up.shape)}, "
+                         f"{tuple(w_down.shape)} do not fit x [{T}][{H}]: expected "
+                         f"W_gate, W_up [I][{H}] and W_down [{H}][I]")
+    if group_size > 0 and I % group_size == 0:
+        W = (I // group_size + 31) // 32
+        if mask_words.dtype != torch.int32 or tuple(mask_words.shape) != (T, W):
+            raise ValueError(f"mask_words must be int32 [{T}][{W}], got {mask_words.dtype} "
+                             f"{tuple(mask_words.shape)}")
+    if out is not None and (out.dtype != x.dtype or tuple(out.shape) != (T, H)):
+        raise ValueError(f"out must be {x.dtype} [{T}][{H}]")
+
+
 def _ffn_dims(x, w_gate, group_size, path) -> WideFFNDims:
     T, H = x.shape
     I = w_gate.shape[0]
@@ -196,6 +217,7 @@ def wide_ffn_masked(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
                     path: int = WIDE_PATH_AUTO, stream=None) -> torch.Tensor:
     """Masked SwiGLU FFN (section 2.A).  x[T][H]; W_gate/W_up[I][H];
     W_down[H][I]; mask_words int32 [T][ceil(G/32)]; returns out[T][H]."""
+    _check_ffn(x, w_gate, w_up, w_down, mask_words, group_size, out)
     d = _ffn_dims(x, w_gate, group_size, path)
     if out is None:
         out = torch.empty_like(x)
@@ -219,6 +241,7 @@ def wide_ffn_masked_noalloc(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.T
     calls on a device; calls that overlap on the GPU race on it.  Raises
     WideError (WIDE_ETOOLARGE) when min(T, 32) (rounded up to
     an even count) * I * 4 exceeds that size."""
+    _check_ffn(x, w_gate, w_up, w_down, mask_words, group_size, out)
     d = _ffn_dims(x, w_gate, group_size, WIDE_PATH_DECODE)
     _check("wide_ffn_masked_noalloc", _L.wide_ffn_masked_noalloc(
         _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
