@@ -46,3 +46,47 @@ def test_router_units():
     assert u_small == {"router_small_gemv": 16 * 4096 * 2 + 128 * 4096 * 2 + 112 * 128 * 2
                        + 16 * 4 * 4, "total": u_small["total"]}
     assert u_big["total"] == u_big["router_tcgen05"]
+
+
+def test_clock_sampler_against_a_fake_nvml(monkeypatch):
+    """The clock record: median SM clock, max clock and the throttle reasons
+    seen while sampling, read through NVML (a fake one here; read-only)."""
+    import time
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    calls = {"n": 0}
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlClocksEventReasonSwPowerCap=0x4, nvmlClocksEventReasonHwSlowdown=0x8,
+        nvmlClocksEventReasonSwThermalSlowdown=0x20,
+        nvmlClocksEventReasonHwThermalSlowdown=0x40,
+        nvmlClocksEventReasonHwPowerBrakeSlowdown=0x80,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("dev", i),
+        nvmlDeviceGetHandleByUUID=lambda u: ("dev", u),
+        nvmlDeviceGetMaxClockInfo=lambda h, k: 1965,
+    )
+
+    def clock(h, k):
+        calls["n"] += 1
+        return (1965, 1800, 1965)[calls["n"] % 3]
+    fake.nvmlDeviceGetClockInfo = clock
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4 if calls["n"] % 2 else 0
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    with bench.ClockSampler(0, period=0.001) as c:
+        time.sleep(0.05)
+    s = c.summary()
+    assert s["source"] == "nvml" and s["sm_max_mhz"] == 1965
+    assert s["samples"] >= 5 and s["sm_mhz"] in (1800, 1965)
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvml(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setitem(sys.modules, "pynvml", None)      # import fails
+    with bench.ClockSampler(0) as c:
+        pass
+    assert c.summary()["source"] == "unavailable"
