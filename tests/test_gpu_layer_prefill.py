@@ -82,12 +82,14 @@ def test_prefill_all_groups_kept():
     _check_full(lc, _run(lc))
 
 
-def test_prefill_layer_8b_full_size_sampled():
+@pytest.mark.parametrize("keep", [0.25, 0.5, 0.75, 1.0])
+def test_prefill_layer_8b_full_size_sampled(keep):
     """The Llama-3.1-8B-shaped prefill layer (4 sequences x 2048 tokens,
-    16 prototypes at keep 0.5 + 0.1 flips), checked on 24 sampled tokens
-    (first, last and random positions of every sequence) and on the K/V the
-    layer wrote for them."""
-    lc = synth.prefill_layer(keep=0.5)
+    16 prototypes + 0.1 flips) at every keep rate the benchmark sweeps
+    (1.0: every group kept, no flips), checked on 24 sampled tokens (first,
+    last and random positions of every sequence) and on the K/V the layer
+    wrote for them."""
+    lc = synth.prefill_layer(keep=keep)
     got = _run(lc)
     S = lc.attn.seq_len
     rng = np.random.default_rng(1)
