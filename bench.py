@@ -274,47 +274,36 @@ class DecodeFFN3B:
     reference_step = staticmethod(lambda samples: _ffn_oracle_step(samples))
 
 
-def _fused_decode_used(T, H, I, gs, sms=148):
-    """Mirror of the library's dispatch (plan_fused in ffn_decode_fused.cu):
-    the fused decode kernel runs for 1..32 tokens when H % 256 == 0, gs in
-    64..256, at most 1024 groups, and its phase-2 plan (rows of W_down per
-    CTA over at most 4 rows per thread) fits."""
-    if not (1 <= T <= 32 and H % 256 == 0 and gs % 64 == 0 and gs <= 256 and I % gs == 0):
+def _split_decode_used(T, H, I, gs, sms=148):
+    """Mirror of the library's dispatch (plan_split in ffn_decode_split.cu):
+    the channel-split decode kernel runs launches of up to 16 tokens when
+    H % 256 == 0, the group size is a multiple of 8 in 8..256 dividing I, there
+    are at most 1024 groups (at most 8 whole groups per CTA), and its fp32
+    [T][H] accumulator plus counter fits the decode path's h scratch."""
+    T1 = min(T, 16)
+    if not (T1 >= 1 and H % 256 == 0 and gs % 8 == 0 and 8 <= gs <= 256 and I % gs == 0):
         return False
     G = I // gs
-    if G > 1024 or T * (-(-G // 32)) > 1024:
+    if G > 1024 or T1 * (-(-G // 32)) > 1024 or -(-G // sms) > 8:
         return False
-    P = sms // -(-T // 8)
-    if P < 1:
-        return False
-    rows = -(-H // P)
-    TBP = max(2, 1 if T <= 1 else 2 if T <= 2 else 4 if T <= 4 else 8)
-    best = None
-    tpi = 32
-    while tpi <= 512:
-        nr = tpi // (gs // 8)
-        rt = -(-rows // nr)
-        ni = 512 // tpi
-        if rt <= 4:
-            cost = (rt + 2) / ni
-            if best is None or cost < best[0]:
-                best = (cost, rt, nr, ni)
-        tpi *= 2
-    return best is not None and best[3] * best[2] * best[1] * TBP <= 2048
+    Tp = (min(T, 32) + 1) // 2 * 2
+    h_bytes = -(-(Tp * I * 4) // 256) * 256
+    acc = -(-(T1 * H * 4) // 256) * 256 + 256
+    return acc <= h_bytes
 
 
 def _ffn_decode_bytes(case, res_bytes=0, x_bytes=None):
     """Algorithmic bytes per kernel of one decode FFN call: every weight byte
     of the batch's union of groups once, plus activations in and out (h of
     the two-kernel path goes through memory; the fused kernel keeps it in
-    L2)."""
+    L2; its fp32 accumulator is not counted: it lives in L2)."""
     B, H, I, gs = case.T, case.H, case.I, case.gs
     U = int(case.mask.any(axis=0).sum())
     m = case.mask_words.nbytes
     xb = B * H * 2 if x_bytes is None else x_bytes
-    if _fused_decode_used(B, H, I, gs):
+    if _split_decode_used(B, H, I, gs):
         fused = 3 * U * gs * H * 2 + xb + m + B * H * 2 + res_bytes
-        return {"decode_ffn_fused_gemv": fused, "total": fused, "union_groups": U}
+        return {"decode_ffn_split_gemv": fused, "total": fused, "union_groups": U}
     pairs = int(case.mask.sum())
     h = pairs * gs * 4
     gateup = 2 * U * gs * H * 2 + xb + m + h
@@ -473,9 +462,11 @@ class DecodeLayer8B:
         attn = kept_pairs * 2 * keys * hd * 2 + kept_pairs * rep * hd * 4 * 2
         oproj = H * Ua * rep * hd * 2 + kept_pairs * rep * hd * 4 + T * H * 2 * 2 + T * H * 4
         out = {"decode_qkv_rope_gemv": qkv, "decode_attention": attn}
-        if _fused_decode_used(T, H, f.I, f.gs):
-            # FFN with its input norm: h1 (fp32) and gamma2 in, ffn_out and out back
-            ffn = _ffn_decode_bytes(f, res_bytes=T * H * 2, x_bytes=T * H * 4 + H * 2)
+        if _split_decode_used(T, H, f.I, f.gs):
+            # FFN input norm (h1 fp32 in, bf16 out), then the FFN: bf16 x and
+            # h1 in (residual), ffn_out and out back
+            out["rmsnorm"] = T * H * 4 + T * H * 2 + H * 2
+            ffn = _ffn_decode_bytes(f, res_bytes=T * H * 4 + T * H * 2)
             out["decode_down_gemv"] = oproj
         else:
             norm = T * H * 4 + T * H * 2 + H * 2

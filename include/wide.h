@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define WIDE_ABI_VERSION 1
+#define WIDE_ABI_VERSION 2
 
 /* host-side status codes */
 #define WIDE_OK 0
@@ -196,11 +196,26 @@ size_t wide_ffn_workspace_bytes(const wide_ffn_dims *d);
 
 /* Masked SwiGLU FFN.  d_workspace: device, >= wide_ffn_workspace_bytes(d)
  * bytes, 256-byte aligned, contents need not be initialised and are
- * clobbered.  Calls that share a workspace must be ordered on one stream. */
+ * clobbered.  Calls that share a workspace must be ordered on one stream.
+ *
+ * wl (host struct of device pointers, optional): a work list that
+ * wide_reorder already built from this same d_group_mask with
+ * tile_m == 128 and G = inter / group_size, so a caller that routes once
+ * can reuse one reordering across calls (section 2.B: the reordering is a
+ * function of the mask alone).  NULL: the prefill path reorders inside the
+ * workspace.  With a work list the prefill path reads it and does not
+ * reorder; the caller must have enqueued that wide_reorder on `stream` (or
+ * ordered it before this call) and must not change the mask in between --
+ * a work list built from another mask gives wrong results, not an error.
+ * The work list's arrays are only read.  A work list whose tokens, groups
+ * or tile_m do not match returns WIDE_EINVAL.  The decode path computes the
+ * batch's union of groups inside its kernel and reads no work list; wl is
+ * checked the same way there and otherwise ignored.  The workspace size
+ * does not depend on wl. */
 int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                     const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
-                    const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
-                    void *stream);
+                    const wide_ffn_dims *d, const wide_worklist *wl, void *d_workspace,
+                    size_t workspace_bytes, void *stream);
 
 /* Kernels of the bf16 decode FFN (process-wide; the decode layer's FFN
  * follows it too).  Both compute the same sums, in a different fp32 order:
@@ -297,10 +312,12 @@ int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cac
  * 32 tokens); larger problems return
  * WIDE_ETOOLARGE before anything is enqueued.  The call allocates nothing.
  * Its first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls on a device share the array, which keeps the last
- * call's contents (nothing in it needs to start at zero); calls that overlap
- * on the GPU -- on streams not ordered with each other -- race on it.
+ * device and CUDA context, with that device current: after a
+ * cudaDeviceReset the next call looks it up again); make that first call
+ * before any stream capture.  All calls on a device share the array, which
+ * keeps the last call's contents (no call depends on them: what a kernel
+ * needs zeroed it zeroes on the stream first); calls that overlap on the GPU
+ * -- on streams not ordered with each other -- race on it.
  * d->path must be WIDE_PATH_AUTO or WIDE_PATH_DECODE. */
 #define WIDE_NOALLOC_SCRATCH_BYTES 2097152
 int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, const void *d_w_up,

@@ -47,7 +47,7 @@ def test_constants_match_header(native):
 
 def test_version_and_status_strings(native):
     L = native.lib()
-    assert L.wide_abi_version() == 1
+    assert L.wide_abi_version() == 2
     for code in (0, -1, -2, -3, -4, 1, 2, 4):
         assert L.wide_status_string(code)
 
@@ -82,31 +82,80 @@ def test_ffn_argument_checks(native):
                 D(8, 3072, 8192, 128, 5, 1), D(8, 3072, 8192, 128, 0, 7),
                 D(8, 3072, 128 * 2000, 128, 0, 1)):
         assert L.wide_ffn_workspace_bytes(ctypes.byref(bad)) == 0
-        assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(bad),
+        assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(bad), None,
                                  None, 0, None) == native.WIDE_EINVAL
     # null pointers with valid dims
-    assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(ok), None, 0,
+    assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(ok), None, None, 0,
                              None) == native.WIDE_EINVAL
     # zero tokens is a no-op
     z = D(0, 3072, 8192, 128, 0, 1)
-    assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(z), None, 0,
+    assert L.wide_ffn_masked(None, None, None, None, None, None, ctypes.byref(z), None, None, 0,
                              None) == native.WIDE_OK
     # an unsupported shape is refused on the host (hidden not a multiple of 128)
     p = ctypes.c_void_p(1 << 20)
     odd = D(8, 3000, 8192, 128, 0, 1)
-    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(odd), p, 1 << 30, None) \
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(odd), None, p, 1 << 30, None) \
         == native.WIDE_EUNSUPPORTED
-    # bf16 group size 32 is not built on the decode path
-    g32 = D(8, 3072, 8192, 32, 0, 1)
-    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(g32), p, 1 << 30, None) \
+    # group size 16 is not built on the bf16 decode path
+    g16 = D(8, 3072, 8192, 16, 0, 1)
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(g16), None, p, 1 << 30, None) \
         == native.WIDE_EUNSUPPORTED
     # misaligned pointer
     mis = ctypes.c_void_p((1 << 20) + 8)
-    assert L.wide_ffn_masked(mis, p, p, p, p, p, ctypes.byref(ok), p, 1 << 30, None) \
+    assert L.wide_ffn_masked(mis, p, p, p, p, p, ctypes.byref(ok), None, p, 1 << 30, None) \
         == native.WIDE_EUNSUPPORTED
     # workspace too small
-    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(ok), p, 16, None) \
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(ok), None, p, 16, None) \
         == native.WIDE_EWORKSPACE
+
+
+def test_ffn_worklist_argument_checks(native):
+    """A caller work list must match the call's (T, G, tile_m = 128): a
+    mismatch or a null array is refused on the host before anything runs."""
+    L = native.lib()
+    D = native.WideFFNDims
+    T, H, I, gs = 300, 4096, 8192, 128
+    G = I // gs
+    base = ctypes.c_void_p(1 << 24)                     # never dereferenced
+    p = ctypes.c_void_p(1 << 20)
+    nbytes = L.wide_worklist_bytes(T, G, 128)
+    wl = native.WideWorklist()
+    assert L.wide_worklist_carve(base, nbytes, T, G, 128, ctypes.byref(wl)) == native.WIDE_OK
+    d = D(T, H, I, gs, native.WIDE_BF16, native.WIDE_PATH_PREFILL)
+    # a matching work list passes the check (the tiny workspace then stops the call)
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(d), ctypes.byref(wl), p, 16,
+                             None) == native.WIDE_EWORKSPACE
+    for dims in (D(T + 1, H, I, gs, 0, 2), D(T, H, I, 64, 0, 2), D(T, H, I // 2, gs, 0, 2)):
+        assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(dims), ctypes.byref(wl), p,
+                                 1 << 30, None) == native.WIDE_EINVAL
+    wl64 = native.WideWorklist()
+    assert L.wide_worklist_carve(base, L.wide_worklist_bytes(T, G, 64), T, G, 64,
+                                 ctypes.byref(wl64)) == native.WIDE_OK
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(d), ctypes.byref(wl64), p,
+                             1 << 30, None) == native.WIDE_EINVAL
+    wl.sig_pos = None
+    assert L.wide_ffn_masked(p, p, p, p, p, p, ctypes.byref(d), ctypes.byref(wl), p, 1 << 30,
+                             None) == native.WIDE_EINVAL
+
+
+def test_binding_refuses_operands_on_two_devices():
+    """The binding launches on the operands' device and refuses operands on
+    different devices (or off the GPU) before any C call."""
+    import types
+    import torch
+    pkg = pytest.importorskip("token_level_dynamic_b200")
+    cuda0, cuda1 = torch.device("cuda", 0), torch.device("cuda", 1)
+
+    def fake(dev):
+        return types.SimpleNamespace(is_cuda=dev.type == "cuda", device=dev)
+
+    assert pkg._one_device("f", x=fake(cuda1), w=fake(cuda1), out=None) == cuda1
+    with pytest.raises(ValueError, match="every operand must be on one device"):
+        pkg._one_device("f", x=fake(cuda0), w=fake(cuda1))
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        pkg._one_device("f", x=fake(cuda0), mask=fake(torch.device("cpu")))
+    with pytest.raises(ValueError, match="no tensor operand"):
+        pkg._one_device("f", x=None)
 
 
 def test_decode_path_switch_is_host_only(native):

@@ -17,9 +17,10 @@ TOL_F32 = 1e-5    # relative L2, fp32 tiny configuration
 @pytest.fixture(params=["auto", "fused", "gemv"], autouse=True)
 def decode_kernels(request):
     """Every case runs on the dispatcher's choice and on each of the two
-    bf16 decode implementations forced (fused persistent kernel wherever its
-    limits allow -- including token blocks of 9..32 tokens -- and the two
-    GEMV kernels)."""
+    bf16 decode implementations forced: the persistent channel-split kernel
+    wherever its limits allow (1..32 tokens per launch, hidden % 256 == 0),
+    and the two GEMV kernels.  bf16 group size 32 exists on the channel-
+    split kernel only and runs there in every mode."""
     import token_level_dynamic_b200 as w
     mode = {"auto": w.WIDE_DECODE_AUTO, "fused": w.WIDE_DECODE_FUSED,
             "gemv": w.WIDE_DECODE_GEMV}[request.param]
@@ -89,17 +90,41 @@ def test_single_token_single_group():
     assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
 
 
-def test_repeatable_bitwise():
+def test_repeatable(decode_kernels):
+    """The GEMV kernels are bitwise repeatable.  The channel-split kernel
+    adds its CTAs' fp32 partial sums with atomics, in an order that varies
+    from call to call, so two calls agree to within one bf16 rounding step
+    per element."""
     c = synth.decode_ffn(8)
     a, b = _run(c), _run(c)
-    np.testing.assert_array_equal(a, b)
+    if decode_kernels == "gemv":
+        np.testing.assert_array_equal(a, b)
+    else:
+        assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)))
 
 
 @pytest.mark.parametrize("T", [9, 17, 24, 31])
-def test_token_blocks_share_weight_tiles(T):
-    """Batches of more than 8 tokens run as blocks of 8 tokens whose CTAs
-    read the same weight rows; a ragged last block included."""
+def test_odd_and_mid_token_counts(T):
+    """Token counts between the kernel's pair templates, odd ones included
+    (the last pair of a group then has one padding slot)."""
     c = synth.ffn_case(T, 1024, 4096, 128, seed=40 + T)
+    assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("T,H,I,gs", [
+    (2, 512, 2048, 128),       # one token pair
+    (7, 768, 3072, 64),        # odd count, 48 groups of 64
+    (32, 512, 4096, 32),       # bf16 group size 32, 128 groups
+    (31, 512, 2048, 32),       # group size 32, odd count
+    (8, 512, 16384, 64),       # ~256 live groups: more groups than CTAs
+    (13, 256, 32768, 32),      # 1024 groups of 32: several whole groups per CTA
+    (20, 1280, 2560, 128),     # hidden 1280: a partial last 1024-row block
+])
+def test_channel_split_shapes(T, H, I, gs):
+    """Shapes that exercise the channel-split kernel's work split: items
+    cut from one group over several CTAs, several whole groups per CTA, a
+    W_down row block cut short by the hidden size, group sizes 32 to 128."""
+    c = synth.ffn_case(T, H, I, gs, seed=T + H, keep=0.5)
     assert rel_l2(_run(c), _ref(c)) <= TOL_BF16
 
 

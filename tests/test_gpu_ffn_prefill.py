@@ -133,3 +133,40 @@ def test_empty_batch_is_a_no_op(path):
     torch.cuda.synchronize()
     assert out.shape == (0, 256)
     assert w.wide_get_device_status() == 0
+
+
+def test_prefill_caller_worklist_reused():
+    """A work list built once by wide_reorder from the mask and passed to
+    wide_ffn_masked twice (and for a second input x) gives the oracle's
+    result each time; the call does not reorder again."""
+    import torch
+    import token_level_dynamic_b200 as w
+    c = synth.ffn_case(700, 512, 1024, 128, seed=21, mask_kind="prototype")
+    x, wg, wu, wd, m = ffn_to_dev(c)
+    wl = w.wide_reorder(m, c.G, 128)
+    w.wide_clear_device_status()
+    n0 = w.wide_launch_count()
+    a = from_dev(w.wide_ffn_masked(x, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_PREFILL,
+                                   worklist=wl))
+    per_call = w.wide_launch_count() - n0
+    b = from_dev(w.wide_ffn_masked(x, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_PREFILL,
+                                   worklist=wl))
+    x2 = torch.flip(x, dims=[1]).contiguous()
+    c2 = synth.FFNCase("flipped", c.T, c.H, c.I, c.gs, "bf16", c.x[:, ::-1].copy(), c.w_gate,
+                       c.w_up, c.w_down, c.mask)
+    d = from_dev(w.wide_ffn_masked(x2, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_PREFILL,
+                                   worklist=wl))
+    torch.cuda.synchronize()
+    assert w.wide_get_device_status() == 0
+    ref = _ref(c)
+    assert rel_l2(a, ref) <= TOL
+    np.testing.assert_array_equal(a, b)
+    assert rel_l2(d, _ref(c2)) <= TOL
+    # the internal path launches the reorder kernels on top of the GEMMs
+    n1 = w.wide_launch_count()
+    w.wide_ffn_masked(x, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_PREFILL)
+    assert w.wide_launch_count() - n1 > per_call
+    # a work list for another shape is refused before any launch
+    wl_other = w.wide_reorder(m[:-1].contiguous(), c.G, 128)
+    with pytest.raises(ValueError, match="worklist was built for"):
+        w.wide_ffn_masked(x, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_PREFILL, worklist=wl_other)

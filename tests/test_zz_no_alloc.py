@@ -53,9 +53,43 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(make, tol):
         torch.cuda.synchronize()
         outs.append(from_dev(out))
     assert w.wide_get_device_status() == 0
+    from oracle.ffn import ffn_masked
+    oracle = ffn_masked(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs, c.dtype)
     for o in outs:
         assert np.isfinite(o).all()
         assert rel_l2(o, ref) <= tol
+        assert rel_l2(o, oracle) <= tol
+
+
+def test_noalloc_token_counts_after_other_shapes():
+    """Odd and multi-launch token counts (1, 33 = 32 + 1, 40 = 32 + 8) on the
+    3B FFN shape, each called right after a call of another shape, so the
+    fixed array holds an earlier call's unrelated data: the result equals
+    the workspace entry point's and the oracle's, and is finite."""
+    import torch
+    import token_level_dynamic_b200 as w
+    from oracle.ffn import ffn_masked
+    stream = torch.cuda.current_stream().cuda_stream
+    other = synth.ffn_case(24, 1024, 4096, 64, seed=77)       # a different shape
+    ox, owg, owu, owd, om = ffn_to_dev(other)
+    base = synth.decode_ffn(1)
+    for T in (1, 33, 40):
+        c = synth.decode_ffn(T, weights=False) if T > 1 else base
+        c.w_gate, c.w_up, c.w_down = base.w_gate, base.w_up, base.w_down
+        x, wg, wu, wd, m = ffn_to_dev(c)
+        w.wide_clear_device_status()
+        oo = torch.empty_like(ox)
+        assert _noalloc_c_call(ox, owg, owu, owd, om, oo, other.gs, stream) == w.WIDE_OK
+        out = torch.full_like(x, float("nan"))
+        assert _noalloc_c_call(x, wg, wu, wd, m, out, c.gs, stream) == w.WIDE_OK
+        ref = from_dev(w.wide_ffn_masked(x, wg, wu, wd, m, c.gs, path=w.WIDE_PATH_DECODE))
+        torch.cuda.synchronize()
+        assert w.wide_get_device_status() == 0
+        got = from_dev(out)
+        assert np.isfinite(got).all()
+        assert rel_l2(got, ref) <= TOL_BF16
+        assert rel_l2(got, ffn_masked(c.x, c.w_gate, c.w_up, c.w_down, c.mask_words, c.gs,
+                                      c.dtype)) <= TOL_BF16
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():

@@ -66,6 +66,28 @@ def _dev_ptr(t: torch.Tensor, name: str) -> int:
     return t.data_ptr()
 
 
+def _one_device(fn: str, **tensors) -> torch.device:
+    """The CUDA device every given tensor is on.  The library launches on the
+    current device and takes raw pointers, so operands on another device
+    would be handed to kernels that cannot address them: refuse that here
+    (ValueError).  None entries are skipped."""
+    dev = None
+    first = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{fn}: {name} must be a CUDA tensor (is on {t.device})")
+        if dev is None:
+            dev, first = t.device, name
+        elif t.device != dev:
+            raise ValueError(f"{fn}: {name} is on {t.device} but {first} is on {dev}; "
+                             "every operand must be on one device")
+    if dev is None:
+        raise ValueError(f"{fn}: no tensor operand")
+    return dev
+
+
 # ------------------------------------------------------------------ status
 
 def wide_status_string(code: int) -> str:
@@ -149,14 +171,16 @@ def wide_reorder(mask_words: torch.Tensor, G: int, tile_m: int = 128, buf: torch
     nbytes = wide_worklist_bytes(T, G, tile_m)
     if nbytes == 0:
         raise WideError("wide_worklist_bytes", WIDE_EINVAL)
-    dev = mask_words.device
+    dev = _one_device("wide_reorder", mask_words=mask_words, buf=buf)
     if buf is None:
         buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     wl = WideWorklist()
     _check("wide_worklist_carve", _L.wide_worklist_carve(
         buf.data_ptr(), buf.numel(), T, G, tile_m, ctypes.byref(wl)))
-    _check("wide_reorder", _L.wide_reorder(
-        _dev_ptr(mask_words, "mask_words"), T, G, tile_m, ctypes.byref(wl), _stream(stream, dev)))
+    with torch.cuda.device(dev):
+        _check("wide_reorder", _L.wide_reorder(
+            _dev_ptr(mask_words, "mask_words"), T, G, tile_m, ctypes.byref(wl),
+            _stream(stream, dev)))
     base = buf.data_ptr()
     nt = (T + tile_m - 1) // tile_m
 
@@ -173,6 +197,8 @@ def wide_reorder(mask_words: torch.Tensor, G: int, tile_m: int = 128, buf: torch
         "sig_pos": view(wl.sig_pos, T),
         "tile_union": view(wl.tile_union, nt * W).view(nt, W),
         "_buf": buf,
+        "_wl": wl,
+        "_key": (T, G, tile_m),
     }
 
 
@@ -214,20 +240,34 @@ def wide_ffn_workspace_bytes(T: int, H: int, I: int, group_size: int, dtype=torc
 def wide_ffn_masked(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.Tensor,
                     w_down: torch.Tensor, mask_words: torch.Tensor, group_size: int,
                     out: torch.Tensor = None, workspace: torch.Tensor = None,
-                    path: int = WIDE_PATH_AUTO, stream=None) -> torch.Tensor:
+                    path: int = WIDE_PATH_AUTO, stream=None, worklist: dict = None) -> torch.Tensor:
     """Masked SwiGLU FFN (section 2.A).  x[T][H]; W_gate/W_up[I][H];
-    W_down[H][I]; mask_words int32 [T][ceil(G/32)]; returns out[T][H]."""
+    W_down[H][I]; mask_words int32 [T][ceil(G/32)]; returns out[T][H].
+    ``worklist``: the dict wide_reorder returned for this same mask
+    (tile_m 128), to reuse that reordering instead of reordering again."""
     _check_ffn(x, w_gate, w_up, w_down, mask_words, group_size, out)
+    dev = _one_device("wide_ffn_masked", x=x, w_gate=w_gate, w_up=w_up, w_down=w_down,
+                      mask_words=mask_words, out=out, workspace=workspace,
+                      worklist=None if worklist is None else worklist["_buf"])
     d = _ffn_dims(x, w_gate, group_size, path)
+    wl = None
+    if worklist is not None:
+        T, I = x.shape[0], w_gate.shape[0]
+        if worklist["_key"] != (T, I // group_size if group_size > 0 else -1, 128):
+            raise ValueError(f"worklist was built for (T, G, tile_m) = {worklist['_key']}, "
+                             f"this call needs ({T}, {I // max(group_size, 1)}, 128)")
+        wl = ctypes.byref(worklist["_wl"])
     if out is None:
         out = torch.empty_like(x)
     need = int(_L.wide_ffn_workspace_bytes(ctypes.byref(d)))
     if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
-    _check("wide_ffn_masked", _L.wide_ffn_masked(
-        _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
-        _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"), _dev_ptr(out, "out"),
-        ctypes.byref(d), workspace.data_ptr(), workspace.numel(), _stream(stream, x.device)))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("wide_ffn_masked", _L.wide_ffn_masked(
+            _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
+            _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"),
+            _dev_ptr(out, "out"), ctypes.byref(d), wl, workspace.data_ptr(), workspace.numel(),
+            _stream(stream, dev)))
     return out
 
 
@@ -242,11 +282,14 @@ def wide_ffn_masked_noalloc(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.T
     WideError (WIDE_ETOOLARGE) when min(T, 32) (rounded up to
     an even count) * I * 4 exceeds that size."""
     _check_ffn(x, w_gate, w_up, w_down, mask_words, group_size, out)
+    dev = _one_device("wide_ffn_masked_noalloc", x=x, w_gate=w_gate, w_up=w_up, w_down=w_down,
+                      mask_words=mask_words, out=out)
     d = _ffn_dims(x, w_gate, group_size, WIDE_PATH_DECODE)
-    _check("wide_ffn_masked_noalloc", _L.wide_ffn_masked_noalloc(
-        _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
-        _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"), _dev_ptr(out, "out"),
-        ctypes.byref(d), _stream(stream, x.device)))
+    with torch.cuda.device(dev):
+        _check("wide_ffn_masked_noalloc", _L.wide_ffn_masked_noalloc(
+            _dev_ptr(x, "x"), _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"),
+            _dev_ptr(w_down, "w_down"), _dev_ptr(mask_words, "mask_words"),
+            _dev_ptr(out, "out"), ctypes.byref(d), _stream(stream, dev)))
     return out
 
 
@@ -282,19 +325,24 @@ def wide_layer_masked(x: torch.Tensor, weights: dict, k_cache: torch.Tensor,
                       stream=None) -> torch.Tensor:
     """The masked layer (pre-norm block); appends K/V to the caches.
     weights: dict with gamma1, wq, wk, wv, wo, gamma2, w_gate, w_up, w_down."""
+    dev = _one_device("wide_layer_masked", x=x, k_cache=k_cache, v_cache=v_cache,
+                      head_mask=head_mask, ffn_mask=ffn_mask, out=out, attn_out=attn_out,
+                      ffn_out=ffn_out, workspace=workspace,
+                      **{n: weights.get(n) for n in LAYER_WEIGHT_NAMES})
     if out is None:
         out = torch.empty_like(x)
     need = wide_layer_workspace_bytes(d)
     if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     w = _weights(weights)
-    _check("wide_layer_masked", _L.wide_layer_masked(
-        _dev_ptr(x, "x"), ctypes.byref(w), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache"), _dev_ptr(head_mask, "head_mask"),
-        _dev_ptr(ffn_mask, "ffn_mask"), _dev_ptr(out, "out"),
-        None if attn_out is None else _dev_ptr(attn_out, "attn_out"),
-        None if ffn_out is None else _dev_ptr(ffn_out, "ffn_out"),
-        ctypes.byref(d), workspace.data_ptr(), workspace.numel(), _stream(stream, x.device)))
+    with torch.cuda.device(dev):
+        _check("wide_layer_masked", _L.wide_layer_masked(
+            _dev_ptr(x, "x"), ctypes.byref(w), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"), _dev_ptr(head_mask, "head_mask"),
+            _dev_ptr(ffn_mask, "ffn_mask"), _dev_ptr(out, "out"),
+            None if attn_out is None else _dev_ptr(attn_out, "attn_out"),
+            None if ffn_out is None else _dev_ptr(ffn_out, "ffn_out"),
+            ctypes.byref(d), workspace.data_ptr(), workspace.numel(), _stream(stream, dev)))
     return out
 
 
@@ -303,17 +351,22 @@ def wide_attn_masked(x: torch.Tensor, weights: dict, k_cache: torch.Tensor,
                      attn_out: torch.Tensor = None, workspace: torch.Tensor = None,
                      stream=None) -> torch.Tensor:
     """The masked attention half: attn_out = o_proj(attn(RMSNorm(x) * gamma1))."""
+    names = ("gamma1", "wq", "wk", "wv", "wo")
+    dev = _one_device("wide_attn_masked", x=x, k_cache=k_cache, v_cache=v_cache,
+                      head_mask=head_mask, attn_out=attn_out, workspace=workspace,
+                      **{n: weights.get(n) for n in names})
     if attn_out is None:
         attn_out = torch.empty_like(x)
     need = wide_layer_workspace_bytes(d)
     if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
-    w = _weights(weights, names=("gamma1", "wq", "wk", "wv", "wo"))
-    _check("wide_attn_masked", _L.wide_attn_masked(
-        _dev_ptr(x, "x"), ctypes.byref(w), _dev_ptr(k_cache, "k_cache"),
-        _dev_ptr(v_cache, "v_cache"), _dev_ptr(head_mask, "head_mask"),
-        _dev_ptr(attn_out, "attn_out"), ctypes.byref(d), workspace.data_ptr(), workspace.numel(),
-        _stream(stream, x.device)))
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    w = _weights(weights, names=names)
+    with torch.cuda.device(dev):
+        _check("wide_attn_masked", _L.wide_attn_masked(
+            _dev_ptr(x, "x"), ctypes.byref(w), _dev_ptr(k_cache, "k_cache"),
+            _dev_ptr(v_cache, "v_cache"), _dev_ptr(head_mask, "head_mask"),
+            _dev_ptr(attn_out, "attn_out"), ctypes.byref(d), workspace.data_ptr(),
+            workspace.numel(), _stream(stream, dev)))
     return attn_out
 
 
@@ -342,12 +395,16 @@ def wide_route(x: torch.Tensor, w_r1: torch.Tensor, w_r2: torch.Tensor,
         raise ValueError(f"mask_words must be int32 [{T}][{(G + 31) // 32}]")
     if logits is not None and (logits.dtype != torch.float32 or tuple(logits.shape) != (T, G)):
         raise ValueError(f"logits must be float32 [{T}][{G}]")
+    dev = _one_device("wide_route", x=x, w_r1=w_r1, w_r2=w_r2, b_r2=b_r2,
+                      mask_words=mask_words, logits=logits)
     if mask_words is None:
-        mask_words = torch.empty((T, (G + 31) // 32), dtype=torch.int32, device=x.device)
+        mask_words = torch.empty((T, (G + 31) // 32), dtype=torch.int32, device=dev)
     d = WideRouterDims(T, H, R, G, act)
-    _check("wide_route", _L.wide_route(
-        _dev_ptr(x, "x"), _dev_ptr(w_r1, "w_r1"), _dev_ptr(w_r2, "w_r2"),
-        None if b_r2 is None else _dev_ptr(b_r2, "b_r2"), _dev_ptr(mask_words, "mask_words"),
-        None if logits is None else _dev_ptr(logits, "logits"), ctypes.byref(d),
-        _stream(stream, x.device)))
+    with torch.cuda.device(dev):
+        _check("wide_route", _L.wide_route(
+            _dev_ptr(x, "x"), _dev_ptr(w_r1, "w_r1"), _dev_ptr(w_r2, "w_r2"),
+            None if b_r2 is None else _dev_ptr(b_r2, "b_r2"),
+            _dev_ptr(mask_words, "mask_words"),
+            None if logits is None else _dev_ptr(logits, "logits"), ctypes.byref(d),
+            _stream(stream, dev)))
     return mask_words

@@ -84,7 +84,8 @@ SIGNATURES = {
                              ctypes.POINTER(WideWorklist), c_void_p]),
     "wide_ffn_workspace_bytes": (c_size_t, [ctypes.POINTER(WideFFNDims)]),
     "wide_ffn_masked": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                                ctypes.POINTER(WideFFNDims), c_void_p, c_size_t, c_void_p]),
+                                ctypes.POINTER(WideFFNDims), ctypes.POINTER(WideWorklist),
+                                c_void_p, c_size_t, c_void_p]),
     "wide_ffn_masked_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, ctypes.POINTER(WideFFNDims), c_void_p]),
     "wide_layer_workspace_bytes": (c_size_t, [ctypes.POINTER(WideLayerDims)]),

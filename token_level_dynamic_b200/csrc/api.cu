@@ -31,18 +31,58 @@ int cuda_fail(const char *file, int line)
     return WIDE_ECUDA;
 }
 
-int32_t *status_ptr()
+namespace {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+}  // namespace
+
+unsigned long long current_context_id()
 {
-    static int32_t *ptrs[64] = {};
+    static CtxGetCurrentFn get_cur = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr, *q = nullptr;
+        cudaDriverEntryPointQueryResult r1, r2;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault,
+                                             &r1) == cudaSuccess &&
+            r1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPointByVersion("cuCtxGetId", &q, 12000, cudaEnableDefault, &r2) ==
+                cudaSuccess &&
+            r2 == cudaDriverEntryPointSuccess) {
+            get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+            get_id = reinterpret_cast<CtxGetIdFn>(q);
+        }
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+void *device_symbol_address(DeviceSymbolCache &cache, const void *symbol)
+{
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return nullptr;
-    if (!ptrs[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_wide_status) == cudaSuccess)
-            ptrs[dev] = static_cast<int32_t *>(p);
-    }
-    return ptrs[dev];
+    std::lock_guard<std::mutex> lock(cache.mu);
+    const unsigned long long id = current_context_id();
+    if (cache.ptr[dev] && id != 0 && cache.ctx[dev] == id)
+        return cache.ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess)
+        return nullptr;
+    cache.ptr[dev] = p;
+    cache.ctx[dev] = current_context_id();
+    return p;
+}
+
+int32_t *status_ptr()
+{
+    static DeviceSymbolCache cache;
+    return static_cast<int32_t *>(device_symbol_address(cache, &g_wide_status));
 }
 
 namespace {
@@ -104,6 +144,25 @@ bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_
         fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap *map, const void *base, const uint64_t (&dims)[3],
+                  const uint64_t (&strides)[2], const uint32_t (&box)[3], uint32_t elem_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const CUtensorMapDataType dt =
+        elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    const cuuint64_t st[2] = {strides[0], strides[1]};
+    const cuuint32_t b[3] = {box[0], box[1], box[2]};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r =
+        fn(map, dt, 3, const_cast<void *>(base), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -190,6 +249,18 @@ bool worklist_layout(int64_t T, int64_t G, int32_t tile_m, WorklistLayout *L)
 
 }  // namespace
 
+bool worklist_matches(const wide_worklist *wl, int64_t T, int64_t G, int32_t tile_m)
+{
+    WorklistLayout L;
+    if (!wl || !worklist_layout(T, G, tile_m, &L))
+        return false;
+    if (wl->tokens != T || wl->groups != G || wl->tile_m != tile_m ||
+        wl->scratch_splits != L.splits)
+        return false;
+    return wl->count && wl->perm && wl->items && wl->n_items && wl->sig_perm && wl->sig_pos &&
+           wl->tile_union && wl->scratch;
+}
+
 bool ffn_dims_ok(const wide_ffn_dims *d)
 {
     if (!d || d->tokens < 0 || d->hidden <= 0 || d->inter <= 0 || d->group_size <= 0)
@@ -213,8 +284,15 @@ bool ffn_shape_supported(const wide_ffn_dims *d, int path)
     if (d->hidden % 128 != 0 || d->hidden > (1 << 20) || d->inter > (1 << 22))
         return false;
     const int64_t gs = d->group_size;
-    if (path == WIDE_PATH_DECODE)
-        return d->dtype == WIDE_BF16 ? (gs == 64 || gs == 128) : (gs == 32 || gs == 64 || gs == 128);
+    if (path == WIDE_PATH_DECODE) {
+        if (d->dtype != WIDE_BF16)
+            return gs == 32 || gs == 64 || gs == 128;
+        // bf16 group size 32 runs on the channel-split kernel only
+        const int T1 = (int)(d->tokens < kSplitMaxTok ? (d->tokens > 0 ? d->tokens : 1)
+                                                      : kSplitMaxTok);
+        return gs == 64 || gs == 128 ||
+               (gs == 32 && decode_ffn_split_supported(T1, (int)d->hidden, (int)d->inter, 32));
+    }
     // prefill: tcgen05 kernels with 128-channel groups and 256-column output blocks
     return d->dtype == WIDE_BF16 && (gs == 64 || gs == 128) && d->hidden % 256 == 0 &&
            d->tokens <= (1 << 24);
@@ -315,14 +393,7 @@ int wide_worklist_carve(void *d_base, size_t bytes, int64_t T, int64_t G, int32_
 int wide_reorder(const uint32_t *d_mask, int64_t T, int64_t G, int32_t tile_m,
                  const wide_worklist *wl, void *stream)
 {
-    WorklistLayout L;
-    if (!wl || !worklist_layout(T, G, tile_m, &L))
-        return WIDE_EINVAL;
-    if (wl->tokens != T || wl->groups != G || wl->tile_m != tile_m ||
-        wl->scratch_splits != L.splits)
-        return WIDE_EINVAL;
-    if ((T > 0 && !d_mask) || !wl->count || !wl->perm || !wl->items || !wl->n_items ||
-        !wl->sig_perm || !wl->sig_pos || !wl->tile_union || !wl->scratch)
+    if (!worklist_matches(wl, T, G, tile_m) || (T > 0 && !d_mask))
         return WIDE_EINVAL;
     return reorder_launch(d_mask, T, G, tile_m, wl, static_cast<cudaStream_t>(stream));
 }
@@ -339,10 +410,12 @@ size_t wide_ffn_workspace_bytes(const wide_ffn_dims *d)
 
 int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                     const void *d_w_down, const uint32_t *d_group_mask, void *d_out,
-                    const wide_ffn_dims *d, void *d_workspace, size_t workspace_bytes,
-                    void *stream)
+                    const wide_ffn_dims *d, const wide_worklist *wl, void *d_workspace,
+                    size_t workspace_bytes, void *stream)
 {
     if (!ffn_dims_ok(d))
+        return WIDE_EINVAL;
+    if (wl && !worklist_matches(wl, d->tokens, d->inter / d->group_size, 128))
         return WIDE_EINVAL;
     if (d->tokens == 0)
         return WIDE_OK;
@@ -360,7 +433,7 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
     if (path == WIDE_PATH_DECODE)
         return ffn_decode_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d,
                                  d_workspace, s);
-    return ffn_prefill_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d,
+    return ffn_prefill_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d, wl,
                               d_workspace, s);
 }
 

@@ -586,7 +586,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
     fo.res_f32 = w.h1;
     fo.out_total = static_cast<__nv_bfloat16 *>(p.out);
     return ffn_prefill_core(w.xn, p.w_gate, p.w_up, p.w_down, p.ffn_mask, fo, T, H, d->inter,
-                            d->ffn_group_size, w.ffn, s);
+                            d->ffn_group_size, nullptr, w.ffn, s);
 }
 
 }  // namespace wide

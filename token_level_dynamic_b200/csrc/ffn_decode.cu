@@ -668,7 +668,7 @@ size_t ffn_decode_workspace(const wide_ffn_dims *d) { return ffn_decode_h_bytes(
 
 int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
                    const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
-                   uint32_t *bar, cudaStream_t s)
+                   size_t h_cap, uint32_t *bar, cudaStream_t s)
 {
     if (d->tokens == 0)
         return WIDE_OK;
@@ -677,7 +677,26 @@ int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd
         const int H = (int)d->hidden, I = (int)d->inter;
         const int64_t T = d->tokens;
         const int W = (int)((I / gs + 31) / 32);
-        if (decode_ffn_fused_preferred((int)(T < kNTok ? T : kNTok), H, I, (int)gs)) {
+        const int T1 = (int)(T < kNTok ? T : kNTok);
+        const int TS = (int)(T < kSplitMaxTok ? T : kSplitMaxTok);
+        // group size 32 has no GEMV kernel: the channel-split kernel runs it
+        // whatever the path mode
+        const bool split = decode_ffn_split_preferred(TS, H, I, (int)gs) ||
+                           (gs == 32 && decode_ffn_split_supported(TS, H, I, (int)gs));
+        if (split && decode_ffn_split_scratch(TS, H) <= h_cap) {
+            for (int64_t t0 = 0; t0 < T; t0 += kSplitMaxTok) {
+                const int Tc = (int)(T - t0 < kSplitMaxTok ? T - t0 : kSplitMaxTok);
+                DownOutputs o = {};
+                o.out_sum = static_cast<__nv_bfloat16 *>(out) + t0 * H;
+                const int rc = decode_ffn_split(static_cast<const __nv_bfloat16 *>(x) + t0 * H,
+                                                wg, wu, wd, mask + t0 * W, o, Tc, H, I, (int)gs,
+                                                h, s);
+                if (rc)
+                    return rc;
+            }
+            return WIDE_OK;
+        }
+        if (decode_ffn_fused_preferred(T1, H, I, (int)gs)) {
             for (int64_t t0 = 0; t0 < T; t0 += kNTok) {
                 const int Tc = (int)(T - t0 < kNTok ? T - t0 : kNTok);
                 FusedInput in = {};
@@ -713,8 +732,11 @@ int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void 
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s)
 {
+    // h, then the 256 bytes of the barrier words: ffn_decode_h_bytes + 256
+    // contiguous bytes
     char *base = static_cast<char *>(ws);
     return ffn_decode_run(x, wg, wu, wd, mask, out, d, reinterpret_cast<float *>(base),
+                          ffn_decode_h_bytes(d) + 256,
                           reinterpret_cast<uint32_t *>(base + ffn_decode_h_bytes(d)), s);
 }
 

@@ -927,6 +927,8 @@ bool decode_ffn_fused_preferred(int T, int H, int I, int gs)
     return decode_ffn_fused_supported(T, H, I, gs);
 }
 
+int wide_get_decode_ffn_path_mode() { return g_decode_mode.load(std::memory_order_relaxed); }
+
 int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, int I, int gs,
                      float *h, uint32_t *bar, cudaStream_t s)
 {
@@ -984,7 +986,8 @@ int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, i
 
 extern "C" int wide_set_decode_ffn_path(int mode)
 {
-    if (mode != WIDE_DECODE_AUTO && mode != WIDE_DECODE_FUSED && mode != WIDE_DECODE_GEMV)
+    if (mode != WIDE_DECODE_AUTO && mode != WIDE_DECODE_FUSED && mode != WIDE_DECODE_GEMV &&
+        mode != wide::kDecodeFusedOld)
         return WIDE_EINVAL;
     return wide::g_decode_mode.exchange(mode);
 }

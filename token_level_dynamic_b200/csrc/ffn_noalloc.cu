@@ -5,17 +5,29 @@
 // owns the whole device memory pool and hands out no workspace, or a
 // latency-critical loop where cudaMalloc/cudaFree would synchronise the
 // device.  This entry point runs the same decode kernels as
-// wide_ffn_masked's decode path, but keeps their scratch -- the fp32
-// intermediate h = silu(gate) * up of up to 32 tokens, and the two words of
-// the fused kernel's grid barrier -- in the file-scope device arrays below
-// instead of a caller workspace.
+// wide_ffn_masked's decode path, but keeps their scratch in the file-scope
+// device arrays below instead of a caller workspace: for the channel-split
+// kernel (bf16, the usual case) its fp32 [T][hidden] accumulator and arrival
+// counter, for the GEMV kernels (fp32, and bf16 shapes outside the split
+// kernel's limits) the fp32 intermediate h = silu(gate) * up of up to 32
+// tokens; the earlier fused kernel's grid-barrier words sit in the second
+// array.
 //
-// The array is a module global: every GPU that loads the library holds
-// WIDE_NOALLOC_SCRATCH_BYTES of device memory for it until the process exits.
-// All calls on a device share it and it keeps the last call's contents.  The
-// kernels write every entry they later read (kept (token, group) pairs only),
-// so nothing in it needs clearing between calls; but two calls whose work
-// overlaps on the GPU (different streams without ordering) race on it.
+// The arrays are module globals: every GPU that loads the library holds
+// WIDE_NOALLOC_SCRATCH_BYTES (+ 256) bytes of device memory for them until
+// the process exits.  All calls on a device share them and they keep the
+// last call's contents.  No call depends on those contents: the split
+// kernel's launch zeroes, on the stream, the accumulator and counter it is
+// about to use, and the GEMV kernels read h only at the (token, group) pairs
+// the same call wrote.  Two calls whose work overlaps on the GPU (different
+// streams without ordering) race on the arrays.
+//
+// In host code the arrays' names are host-side stand-ins, not device
+// addresses: the addresses are looked up with cudaGetSymbolAddress, with the
+// device current, once per device and CUDA context (device_symbol_address),
+// so after a cudaDeviceReset the next call looks them up again.  The first
+// call on a device (or in a new context) does that lookup; make it before
+// any stream capture.
 #include <cuda_runtime.h>
 #include <mutex>
 
@@ -29,28 +41,13 @@ namespace wide {
 namespace {
 
 // Device addresses of this device's copies of g_noalloc_scratch and
-// g_noalloc_bar.  In host code the arrays' names are only host-side
-// stand-ins, so the addresses are looked up with cudaGetSymbolAddress once
-// per device, with that device current.
+// g_noalloc_bar (see device_symbol_address).
 bool noalloc_arrays(float **scratch, uint32_t **bar)
 {
-    static std::mutex mu;
-    static void *ptrs[64][2] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
-        return false;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev][0]) {
-        void *p = nullptr, *q = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess ||
-            cudaGetSymbolAddress(&q, g_noalloc_bar) != cudaSuccess)
-            return false;
-        ptrs[dev][0] = p;
-        ptrs[dev][1] = q;
-    }
-    *scratch = static_cast<float *>(ptrs[dev][0]);
-    *bar = static_cast<uint32_t *>(ptrs[dev][1]);
-    return true;
+    static DeviceSymbolCache cs, cb;
+    *scratch = static_cast<float *>(device_symbol_address(cs, &g_noalloc_scratch));
+    *bar = static_cast<uint32_t *>(device_symbol_address(cb, &g_noalloc_bar));
+    return *scratch && *bar;
 }
 
 }  // namespace
@@ -81,6 +78,6 @@ extern "C" int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, co
     uint32_t *bar = nullptr;
     if (!noalloc_arrays(&scratch, &bar))
         return WIDE_CUDA_FAIL();
-    return ffn_decode_run(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d, scratch, bar,
-                          static_cast<cudaStream_t>(stream));
+    return ffn_decode_run(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d, scratch,
+                          WIDE_NOALLOC_SCRATCH_BYTES, bar, static_cast<cudaStream_t>(stream));
 }

@@ -29,13 +29,16 @@ size_t ffn_prefill_workspace(const wide_ffn_dims *d)
 
 int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *wd,
                      const uint32_t *mask, const FfnPrefillOut &o, int64_t T, int64_t H,
-                     int64_t I, int64_t gs, void *ws, cudaStream_t s)
+                     int64_t I, int64_t gs, const wide_worklist *ext_wl, void *ws,
+                     cudaStream_t s)
 {
     const int64_t G = I / gs;
     const size_t wl_bytes = wide_worklist_bytes(T, G, kBM);
     wide_worklist wl;
-    int rc = wide_worklist_carve(ws, wl_bytes, T, G, kBM, &wl);
-    if (rc)
+    int rc = WIDE_OK;
+    if (ext_wl)
+        wl = *ext_wl;
+    else if ((rc = wide_worklist_carve(ws, wl_bytes, T, G, kBM, &wl)))
         return rc;
     __nv_bfloat16 *hbuf =
         reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + align_up(wl_bytes, 1024));
@@ -47,7 +50,7 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
         !make_tmap_2d(&td, wd, H, I, I, 2, 256, 64, true))
         return WIDE_CUDA_FAIL();
 
-    if ((rc = reorder_launch(mask, T, G, kBM, &wl, s)))
+    if (!ext_wl && (rc = reorder_launch(mask, T, G, kBM, &wl, s)))
         return rc;
     if ((rc = zero_dead_launch(mask, wl.sig_pos, hbuf, (int)T, (int)I, (int)G, (int)gs, s)))
         return rc;
@@ -84,13 +87,13 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
 }
 
 int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void *wd,
-                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
-                       cudaStream_t s)
+                       const uint32_t *mask, void *out, const wide_ffn_dims *d,
+                       const wide_worklist *ext_wl, void *ws, cudaStream_t s)
 {
     FfnPrefillOut o = {};
     o.out_sum = static_cast<__nv_bfloat16 *>(out);
     return ffn_prefill_core(x, wg, wu, wd, mask, o, d->tokens, d->hidden, d->inter,
-                            d->group_size, ws, s);
+                            d->group_size, ext_wl, ws, s);
 }
 
 }  // namespace wide

@@ -7,12 +7,30 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "wide.h"
 
 namespace wide {
 
-// Device address of this device's status word (looked up once per device).
+// Device address of this device's status word (looked up once per device
+// and context).
 int32_t *status_ptr();
+
+// The device address of a module-scope __device__ variable on the current
+// device.  In host code such a variable's name is only a host-side stand-in;
+// its device address is looked up with cudaGetSymbolAddress, with the device
+// current, once per (device, context): a cudaDeviceReset ends the context and
+// the module's memory with it, and the next call looks the address up again
+// in the new context.  Returns null if the lookup fails.
+struct DeviceSymbolCache {
+    std::mutex mu;
+    void *ptr[64] = {};
+    unsigned long long ctx[64] = {};
+};
+void *device_symbol_address(DeviceSymbolCache &cache, const void *symbol);
+// Unique id of the current CUDA context (cuCtxGetId), 0 if there is none.
+unsigned long long current_context_id();
 
 // Encodes a 2-D row-major tensor map: `rows` x `cols` elements of
 // `elem_bytes` bytes, row pitch `pitch_elems`, box `box_rows` x `box_cols`,
@@ -30,6 +48,11 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
 // short rows.
 bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                       uint64_t pitch_elems, uint32_t box_chunks, uint32_t box_rows);
+
+// Encodes a 3-D tensor: dims (innermost first), byte strides of dims 1 and
+// 2, box extents, no swizzle; bf16 (elem_bytes 2) or fp32 (4).
+bool make_tmap_3d(CUtensorMap *map, const void *base, const uint64_t (&dims)[3],
+                  const uint64_t (&strides)[2], const uint32_t (&box)[3], uint32_t elem_bytes);
 
 // Encodes an fp32 [T][cols] activation stored with token pairs interleaved
 // (row t/2 holds 2 * cols floats: tokens t and t+1 side by side per column)
@@ -76,6 +99,7 @@ enum KernelId : int32_t {
     KID_DECODE_FFN_FUSED = 15,
     KID_ROUTER = 16,
     KID_ROUTER_SMALL = 17,
+    KID_DECODE_FFN_SPLIT = 18,
 };
 
 // Pointers of one masked-layer call (FFN pointers unused when !ffn).
@@ -98,6 +122,9 @@ class LaunchScope {
     int slot_;
     cudaStream_t s_;
 };
+
+// Whether *wl is a carved work list for (T, G, tile_m) with every array set.
+bool worklist_matches(const wide_worklist *wl, int64_t T, int64_t G, int32_t tile_m);
 
 // FFN argument checks shared by the FFN entry points (api.cu).
 bool ffn_dims_ok(const wide_ffn_dims *d);
@@ -177,12 +204,15 @@ struct FfnPrefillOut {
     const float *res_f32;
     __nv_bfloat16 *out_total;
 };
+// ext_wl: a caller-built work list of the same mask (tile_m 128), or null
+// to reorder inside ws.
 int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *wd,
                      const uint32_t *mask, const FfnPrefillOut &o, int64_t T, int64_t H,
-                     int64_t I, int64_t gs, void *ws, cudaStream_t s);
+                     int64_t I, int64_t gs, const wide_worklist *ext_wl, void *ws,
+                     cudaStream_t s);
 int ffn_prefill_launch(const void *x, const void *wg, const void *wu, const void *wd,
-                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
-                       cudaStream_t s);
+                       const uint32_t *mask, void *out, const wide_ffn_dims *d,
+                       const wide_worklist *ext_wl, void *ws, cudaStream_t s);
 
 bool layer_prefill_supported(const wide_layer_dims *d);
 size_t layer_prefill_workspace(const wide_layer_dims *d);
@@ -225,12 +255,30 @@ bool decode_ffn_fused_supported(int T, int H, int I, int gs);
 bool decode_ffn_fused_preferred(int T, int H, int I, int gs);
 int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, int I, int gs,
                      float *h, uint32_t *bar, cudaStream_t s);
+// bf16 decode FFN of 1 <= T <= kSplitMaxTok tokens as one persistent
+// cooperative kernel in which every CTA owns a slice of the batch's kept
+// channels
+// (ffn_decode_split.cu).  x: bf16 [T][H].  scratch: device memory of at
+// least decode_ffn_split_scratch(T, H) bytes (an fp32 [T][H] accumulator and
+// an arrival counter, zeroed on the stream by the call).
+constexpr int kSplitMaxTok = 16;   // tokens per launch of the split kernel
+size_t decode_ffn_split_scratch(int T, int H);
+bool decode_ffn_split_supported(int T, int H, int I, int gs);
+bool decode_ffn_split_preferred(int T, int H, int I, int gs);
+// Current wide_set_decode_ffn_path mode; kDecodeFusedOld selects the
+// earlier fused kernel (ffn_decode_fused.cu) for comparison runs.
+int wide_get_decode_ffn_path_mode();
+constexpr int kDecodeFusedOld = 3;
+int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *wd,
+                     const uint32_t *mask, const DownOutputs &o, int T, int H, int I, int gs,
+                     void *scratch, cudaStream_t s);
 // Bytes of the fp32 h scratch of the decode path (tokens capped at 32).
 size_t ffn_decode_h_bytes(const wide_ffn_dims *d);
-// Runs the decode path with h scratch and grid-barrier words given apart.
+// Runs the decode path with h scratch (h_cap contiguous bytes at h, at
+// least ffn_decode_h_bytes(d)) and grid-barrier words given apart.
 int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
                    const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
-                   uint32_t *bar, cudaStream_t s);
+                   size_t h_cap, uint32_t *bar, cudaStream_t s);
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s);

@@ -129,6 +129,8 @@ const char *wide_kernel_name(int32_t id)
         return "router_tcgen05";
     case KID_ROUTER_SMALL:
         return "router_small_gemv";
+    case KID_DECODE_FFN_SPLIT:
+        return "decode_ffn_split_gemv";
     default:
         return "?";
     }
