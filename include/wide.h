@@ -177,10 +177,11 @@ int wide_reorder(const uint32_t *d_mask, int64_t T, int64_t G, int32_t tile_m,
  * W_down[hidden][inter], group_mask[T][W] with G = inter / group_size,
  * out[T][hidden]; element type `dtype` for x, weights and out.  All device.
  *
- * Supported: hidden % 64 == 0; group_size in {32, 64, 128} dividing inter;
- * G <= 1024; 16-byte aligned pointers.  WIDE_PATH_PREFILL needs bf16,
- * group_size 64 or 128 and hidden % 256 == 0.  The fp32 type runs the
- * CUDA-core path at any T.
+ * Supported: hidden % 128 == 0; group_size in {32, 64, 128} dividing inter;
+ * G <= 1024; 16-byte aligned pointers.  The bf16 decode path with
+ * group_size 32 needs hidden % 256 == 0 (it runs on the channel-split
+ * kernel only).  WIDE_PATH_PREFILL needs bf16, group_size 64 or 128 and
+ * hidden % 256 == 0.  The fp32 type runs the CUDA-core path at any T.
  */
 typedef struct wide_ffn_dims {
     int64_t tokens;        /* T */
@@ -219,11 +220,18 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
 
 /* Kernels of the bf16 decode FFN (process-wide; the decode layer's FFN
  * follows it too).  Both compute the same sums, in a different fp32 order:
- *   WIDE_DECODE_AUTO   the measured faster one for the call's shape (default)
- *   WIDE_DECODE_FUSED  the persistent fused kernel wherever its shape limits
- *                      allow (1..32 tokens, hidden % 256 == 0, ...), else
- *                      the GEMVs
+ *   WIDE_DECODE_AUTO   the channel-split kernel wherever its shape limits
+ *                      allow, else the GEMVs (default)
+ *   WIDE_DECODE_FUSED  the same: one persistent kernel per launch of up to
+ *                      16 tokens (hidden % 256 == 0, group size a multiple
+ *                      of 8 up to 256); each CTA owns one group's channel
+ *                      range, computes gate/up for the tokens that keep the
+ *                      group and adds its share of the down projection into
+ *                      an fp32 accumulator with atomics, so two calls can
+ *                      differ in the last fp32 bits
  *   WIDE_DECODE_GEMV   the gate/up GEMV kernel, then the down GEMV kernel
+ *                      (bitwise repeatable); bf16 group size 32 exists on
+ *                      the channel-split kernel only and runs there
  * Returns the previous mode, or WIDE_EINVAL for an unknown mode (the mode
  * is then unchanged).  Not ordered with work already enqueued: it applies
  * to calls made after it returns. */

@@ -792,18 +792,6 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
         }
         return WIDE_OK;
     }
-    if (decode_ffn_fused_preferred(T, H, I, gsf)) {
-        // one persistent kernel: the norm is applied while x is staged
-        FusedInput in = {};
-        in.x_f32 = w.h1;
-        in.gamma = p.gamma2;
-        in.eps = d->eps;
-        in.w_gate = p.w_gate;
-        in.w_up = p.w_up;
-        in.w_down = p.w_down;
-        in.mask = p.ffn_mask;
-        return decode_ffn_fused(in, fo, T, H, I, gsf, w.hffn, w.bar, s);
-    }
     if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
         return rc;
     rc = decode_gateup_bf16(w.xn2, p.w_gate, p.w_up, p.ffn_mask, w.hffn, T, H, I, gsf, s);

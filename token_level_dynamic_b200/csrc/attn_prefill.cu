@@ -533,9 +533,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
     if ((rc = gather_gemm_launch(GEMM_KV, tk, tv, gk, n_kv * m_tiles, KID_PREFILL_KV, s)))
         return rc;
 
-    // 5. attention on compacted queries -> o_sig (zeros at skipped pairs)
-    if ((rc = zero_dead_launch(p.head_mask, wl.sig_pos, w.o_sig, (int)T, qd, n_kv, qcols, s)))
-        return rc;
+    // 5. attention on compacted queries -> o_sig (rows of kept pairs only)
     AttnPArgs aa;
     aa.count = wl.count;
     aa.perm = wl.perm;
@@ -565,10 +563,13 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
     UnionArgs ua = {};
     ua.tile_union = wl.tile_union;
     ua.sig_perm = wl.sig_perm;
+    ua.mask = p.head_mask;
+    ua.h = w.o_sig;
     ua.T = (int)T;
     ua.N = (int)H;
     ua.W = (n_kv + 31) / 32;
     ua.gs = qcols;
+    ua.ld = qd;
     ua.out_sum = static_cast<__nv_bfloat16 *>(p.attn_out);
     if (p.ffn) {
         ua.res_in = static_cast<const __nv_bfloat16 *>(p.x);

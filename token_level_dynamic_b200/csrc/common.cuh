@@ -159,6 +159,16 @@ __device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gsrc)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gsrc)
                  : "memory");
 }
+// As cp_async16, but copies src_bytes (0 or 16) bytes and fills the rest of
+// the 16 with zeros: with 0, nothing is read from global memory (src must
+// still be a valid address) and the destination is zeroed.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t smem_dst, const void *gsrc,
+                                                 uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_dst), "l"(gsrc),
+                 "r"(src_bytes)
+                 : "memory");
+}
 // Arrive on the mbarrier once every cp.async this thread issued so far has
 // completed; the barrier's expected count already includes this arrive.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)

@@ -677,7 +677,6 @@ int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd
         const int H = (int)d->hidden, I = (int)d->inter;
         const int64_t T = d->tokens;
         const int W = (int)((I / gs + 31) / 32);
-        const int T1 = (int)(T < kNTok ? T : kNTok);
         const int TS = (int)(T < kSplitMaxTok ? T : kSplitMaxTok);
         // group size 32 has no GEMV kernel: the channel-split kernel runs it
         // whatever the path mode
@@ -691,23 +690,6 @@ int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd
                 const int rc = decode_ffn_split(static_cast<const __nv_bfloat16 *>(x) + t0 * H,
                                                 wg, wu, wd, mask + t0 * W, o, Tc, H, I, (int)gs,
                                                 h, s);
-                if (rc)
-                    return rc;
-            }
-            return WIDE_OK;
-        }
-        if (decode_ffn_fused_preferred(T1, H, I, (int)gs)) {
-            for (int64_t t0 = 0; t0 < T; t0 += kNTok) {
-                const int Tc = (int)(T - t0 < kNTok ? T - t0 : kNTok);
-                FusedInput in = {};
-                in.x = static_cast<const __nv_bfloat16 *>(x) + t0 * H;
-                in.w_gate = wg;
-                in.w_up = wu;
-                in.w_down = wd;
-                in.mask = mask + t0 * W;
-                DownOutputs o = {};
-                o.out_sum = static_cast<__nv_bfloat16 *>(out) + t0 * H;
-                const int rc = decode_ffn_fused(in, o, Tc, H, I, (int)gs, h, bar, s);
                 if (rc)
                     return rc;
             }

@@ -58,11 +58,21 @@
 namespace wide {
 namespace {
 
-constexpr int kSWarps = 8;                    // consumer warps
+// Consumer warps and the weight rows each consumer thread owns (the gate
+// and up rows of kSRows / 2 channels in phase A, kSRows output rows in phase
+// B): 8 x 4 or 16 x 2.  A CTA is the consumers plus 3 warps; with 8
+// consumer warps a sub-partition holds 3 warps, so a thread may use 168
+// registers, with 16 it holds 5 (96 registers).
+#ifndef WIDE_SPLIT_WARPS
+#define WIDE_SPLIT_WARPS 8
+#endif
+constexpr int kSWarps = WIDE_SPLIT_WARPS;     // consumer warps
+constexpr int kSRows = 32 / kSWarps;          // weight rows per consumer thread
+constexpr int kSMaxReg = kSWarps == 8 ? 168 : 96;
 constexpr int kSCons = 32 * kSWarps;          // consumer threads
 constexpr int kSThreads = kSCons + 96;        // + the TMA producer and two x converter warps
 constexpr int kSMaxTok = kSplitMaxTok;        // tokens per launch (a larger batch: several)
-constexpr int kSRowBlk = 1024;                // phase-B rows per block (4 per consumer thread)
+constexpr int kSRowBlk = kSCons * kSRows;     // phase-B rows per block (1024)
 constexpr int kSDownBox = 256;                // rows per W_down TMA box
 constexpr int kSMaxSlots = 8;
 constexpr int kSMaxG = 1024;
@@ -183,39 +193,40 @@ __device__ __forceinline__ void lane_reduce2(float2 (&v)[N], int lane)
 // updates of one accumulator are 4 * NA FMAs apart (no stall on the
 // previous result).
 template <int NP, int NA, int QS>
-__device__ __forceinline__ void rows4(const uint4 (&w)[4], const uint8_t *ob, uint32_t pstride,
-                                      float2 (&acc)[4 * NP])
+__device__ __forceinline__ void rows4(const uint4 (&w)[kSRows], const uint8_t *ob,
+                                      uint32_t pstride, float2 (&acc)[kSRows * NP])
 {
+    constexpr int R = kSRows;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         float4 v[NA];
 #pragma unroll
         for (int p = 0; p < NA; ++p)
             v[p] = lds128f(ob + p * pstride + q * QS);
-        float2 d[4];
+        float2 d[R];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < R; ++r)
             d[r] = dup_lo(word(w[r], q));
 #pragma unroll
         for (int p = 0; p < NA; ++p)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                acc[4 * p + r] = __ffma2_rn(d[r], lo2(v[p]), acc[4 * p + r]);
+            for (int r = 0; r < R; ++r)
+                acc[R * p + r] = __ffma2_rn(d[r], lo2(v[p]), acc[R * p + r]);
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < R; ++r)
             d[r] = dup_hi(word(w[r], q));
 #pragma unroll
         for (int p = 0; p < NA; ++p)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                acc[4 * p + r] = __ffma2_rn(d[r], hi2(v[p]), acc[4 * p + r]);
+            for (int r = 0; r < R; ++r)
+                acc[R * p + r] = __ffma2_rn(d[r], hi2(v[p]), acc[R * p + r]);
     }
 }
 
 // rows4 for the run-time pair count np (1 <= np <= NP).
 template <int NP, int QS>
-__device__ __forceinline__ void rows4_np(int np, const uint4 (&w)[4], const uint8_t *ob,
-                                         uint32_t pstride, float2 (&acc)[4 * NP])
+__device__ __forceinline__ void rows4_np(int np, const uint4 (&w)[kSRows], const uint8_t *ob,
+                                         uint32_t pstride, float2 (&acc)[kSRows * NP])
 {
 #define WIDE_ROWS4_CASE(n)                                                                          \
     case n:                                                                                        \
@@ -231,47 +242,39 @@ __device__ __forceinline__ void rows4_np(int np, const uint4 (&w)[4], const uint
 #undef WIDE_ROWS4_CASE
 }
 
-// Phase A for up to 8 tokens, column-pair form: four weight rows' 8 columns
-// (w[0..3]: gate and up of two channels) against the n active tokens' bf16 x
-// rows (token i's row at xw + xr[i]).  The packed FMA takes two adjacent
-// columns: a weight word widens into one register pair (one byte permute per
-// element), the token's two x values into another, and acc[4i + r] collects
-// token i's row-r sums over even and odd columns (added at the end of the
-// pass).
+// Phase A for up to 8 tokens, column-pair form: the thread's weight rows' 8
+// columns (w[r]: gate and up of its channels) against the n active tokens'
+// fp32 x (token i's 8 columns: 16 bytes at xw + xr[i], 16 more 1 KB
+// further).  The packed FMA takes two adjacent columns: a weight word widens
+// into one register pair (one byte permute per element), the token's two x
+// values are a register pair already, and acc[R i + r] collects token i's
+// row-r sums over even and odd columns (added at the end of the pass).
 template <int NT, int NA>
-__device__ __forceinline__ void colpair4(const uint4 (&w)[4], const uint8_t *xw,
-                                         const uint32_t (&xr)[NT], float2 (&acc)[4 * NT])
+__device__ __forceinline__ void colpair4(const uint4 (&w)[kSRows], const uint8_t *xw,
+                                         const uint32_t (&xr)[NT], float2 (&acc)[kSRows * NT])
 {
-    float2 wv[4][4];
+    constexpr int R = kSRows;
+    float2 wv[R][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < R; ++r)
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             wv[r][q] = make_float2(bf_lo(word(w[r], q)), bf_hi(word(w[r], q)));
-    // two tokens per step: 8 independent accumulators per column pair
 #pragma unroll
-    for (int i = 0; i < NA; i += 2) {
-        const uint4 xv0 = lds128(xw + xr[i]);
-        const uint4 xv1 = i + 1 < NA ? lds128(xw + xr[i + 1]) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < NA; ++i) {
+        const float4 a = lds128f(xw + xr[i]), b = lds128f(xw + xr[i] + 1024);
+        const float2 x2[4] = {lo2(a), hi2(a), lo2(b), hi2(b)};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float2 x0 = make_float2(bf_lo(word(xv0, q)), bf_hi(word(xv0, q)));
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-                acc[4 * i + r] = __ffma2_rn(wv[r][q], x0, acc[4 * i + r]);
-            if (i + 1 < NA) {
-                const float2 x1 = make_float2(bf_lo(word(xv1, q)), bf_hi(word(xv1, q)));
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    acc[4 * (i + 1) + r] = __ffma2_rn(wv[r][q], x1, acc[4 * (i + 1) + r]);
-            }
-        }
+            for (int r = 0; r < R; ++r)
+                acc[R * i + r] = __ffma2_rn(wv[r][q], x2[q], acc[R * i + r]);
     }
 }
 
 template <int NT>
-__device__ __forceinline__ void colpair4_n(int n, const uint4 (&w)[4], const uint8_t *xw,
-                                           const uint32_t (&xr)[NT], float2 (&acc)[4 * NT])
+__device__ __forceinline__ void colpair4_n(int n, const uint4 (&w)[kSRows], const uint8_t *xw,
+                                           const uint32_t (&xr)[NT], float2 (&acc)[kSRows * NT])
 {
 #define WIDE_COLPAIR_CASE(m)                                                                       \
     case m:                                                                                        \
@@ -293,8 +296,8 @@ __device__ __forceinline__ void colpair4_n(int n, const uint4 (&w)[4], const uin
 //   NP <= 4 (up to 8 tokens; the weight stream sets the pace): 512-column
 //     windows (1 KB of every weight row per copy: long row pieces stream far
 //     better than 256-byte ones), one warp per channel pair (each lane two
-//     8-column chunks), 16 channels per pass, the column-pair form straight
-//     from the bf16 x window (no x32, no converters).
+//     8-column chunks), 16 channels per pass, the column-pair form on the
+//     window's x widened to fp32 per token by the converters.
 //   NP == 8 (9..16 tokens; the multiplies set the pace): 128-column windows
 //     (the x32 area of a window grows with NP), a half warp per channel
 //     pair, 32 channels per pass, token pairs from x32.
@@ -304,7 +307,7 @@ template <int NP> struct SplitCfg {
     static constexpr int CL = kWide ? 32 : 16;        // chunk lanes per channel
     static constexpr int LV = kWide ? 5 : 4;          // log2(CL)
     static constexpr int CPL = KW / (8 * CL);         // chunks per lane per window
-    static constexpr int S = 2 * kSCons / CL;         // channels per pass
+    static constexpr int S = kSCons / CL * kSRows / 2; // channels per pass
     static constexpr int WB = 2 * S * KW * 2;         // weight bytes per phase-A stage
 };
 
@@ -315,15 +318,30 @@ struct Item {
 };
 
 // The items of CTA c of P for U live groups of gs channels; returns their
-// count (0..kSMaxItems).
-__device__ __forceinline__ int cta_items(int c, int P, int U, int gs, Item (&it)[kSMaxItems])
+// count (0..kSMaxItems).  cw[0..U] are the live groups' cumulative work
+// weights (cw[0] = 0).  With at least as many CTAs as groups, every group
+// gets one CTA and the other P - U are dealt out in proportion to the
+// weights (group i: K(i + 1) - K(i) CTAs, K(i) = i + floor((P - U) cw[i] /
+// cw[U])); its units are then cut evenly over its CTAs.
+__device__ __forceinline__ int cta_items(int c, int P, int U, int gs, const int *cw,
+                                         Item (&it)[kSMaxItems])
 {
     if (U <= 0)
         return 0;
     const int units = gs / 8;
     if (P >= U) {
-        const int i = (int)(((int64_t)(c + 1) * U + P - 1) / P) - 1;
-        const int f = (int)((int64_t)i * P / U), e = (int)((int64_t)(i + 1) * P / U);
+        const int64_t R = P - U, Wt = cw[U] > 0 ? cw[U] : 1;
+        auto K = [&](int i) { return i + (int)(R * cw[i] / Wt); };
+        int lo = 0, hi = U - 1;                    // the last i with K(i) <= c
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (K(mid) <= c)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int i = lo;
+        const int f = K(i), e = K(i + 1);
         const int k = e - f, j = c - f;
         it[0].li = i;
         it[0].u0 = j * units / k;
@@ -345,7 +363,7 @@ __device__ __forceinline__ int cta_items(int c, int P, int U, int gs, Item (&it)
 // 16384 / 96 registers, 168 in the allocation granularity: room for the
 // accumulators of 4 rows x 8 token pairs without spilling.
 template <int NP>
-__global__ void __maxnreg__(168)
+__global__ void __maxnreg__(kSMaxReg)
     ffn_decode_split(const __grid_constant__ CUtensorMap tm_gate,
                      const __grid_constant__ CUtensorMap tm_up,
                      const __grid_constant__ CUtensorMap tm_gate8,
@@ -364,7 +382,8 @@ __global__ void __maxnreg__(168)
     float *hs = reinterpret_cast<float *>(smem + (size_t)NS * a.slot_bytes);   // [NP][gs][2]
     uint32_t *mall = reinterpret_cast<uint32_t *>(hs + (size_t)NP * gs * 2);   // [T][W]
     int *live = reinterpret_cast<int *>(mall + T * W);                         // [G]
-    int *toks = live + a.G;                                                    // [items][32]
+    int *cw = live + a.G;                                                      // [G + 1]
+    int *toks = cw + a.G + 1;                                                  // [items][32]
     uint64_t *full = reinterpret_cast<uint64_t *>(
         (reinterpret_cast<uintptr_t>(toks + kSMaxItems * kSMaxTok) + 7) & ~(uintptr_t)7);
     uint64_t *empty = full + NS;
@@ -422,11 +441,46 @@ __global__ void __maxnreg__(168)
             s_nlive = total;
     }
     __syncthreads();
+    // work weight of every live group: 16 + its active tokens (the weight
+    // stream costs a group the same whatever its tokens; each token adds
+    // about a sixteenth in multiplies), then the cumulative sums (warp 0)
+    {
+        const int U = s_nlive;
+        for (int li = tid; li < U; li += kSThreads) {
+            const int g = live[li];
+            int n = 0;
+            for (int t = 0; t < T; ++t)
+                n += (mall[t * W + (g >> 5)] >> (g & 31)) & 1u;
+            cw[li + 1] = 16 + n;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const int per = (U + 31) / 32, b0 = min(U, lane * per), b1 = min(U, b0 + per);
+            int sum = 0;
+            for (int i = b0; i < b1; ++i)
+                sum += cw[i + 1];
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off)
+                    incl += v;
+            }
+            int run = incl - sum;
+            for (int i = b0; i < b1; ++i) {
+                run += cw[i + 1];
+                cw[i + 1] = run;
+            }
+            if (lane == 0)
+                cw[0] = 0;
+        }
+    }
+    __syncthreads();
     // this CTA's items and each item's active tokens, ascending (warp 1:
     // one ballot per item)
     if (warp == 1) {
         Item its[kSMaxItems];
-        const int n_it = cta_items(c, P, s_nlive, gs, its);
+        const int n_it = cta_items(c, P, s_nlive, gs, cw, its);
         if (lane == 0) {
             s_nitems = n_it;
             for (int k = 0; k < n_it; ++k)
@@ -515,7 +569,7 @@ __global__ void __maxnreg__(168)
         // bytes], the 16 bytes holding columns 8 * chunk + 2q, + 1 of the
         // pair (the chunk lanes of a channel then read contiguous bytes).
         // Every stage (phase B too) is handed on through xready.
-        if constexpr (!C::kWide) {
+        {
             const int cv = warp - 1;
             bool ok = true;
             int k = 0;
@@ -539,7 +593,24 @@ __global__ void __maxnreg__(168)
                 const int nB = NRB * (((it.u1 - it.u0) * 8 + a.bch - 1) / a.bch);
                 for (int kA = 0; kA < nA; ++kA, ++k) {
                     wait_full(k);
-                    if (ok) {
+                    if (ok && C::kWide) {
+                        // every token's 512 columns in fp32: [t][half][64
+                        // chunks][16 bytes], half 0 the chunk's first 4
+                        // columns (the lanes of a warp then read 512
+                        // contiguous bytes); one (token, chunk) per lane and
+                        // step: a 16-byte read, two 16-byte writes
+                        const uint8_t *xb = slot_of(k) + a.xb_off;
+                        uint8_t *x32 = slot_of(k) + a.x32_off;
+                        for (int u = cv * 32 + lane; u < T * (KW / 8); u += 64) {
+                            const int t = u / (KW / 8), l = u % (KW / 8);
+                            const uint4 xv = lds128(xb + (size_t)t * KW * 2 + l * 16);
+                            uint8_t *dst = x32 + (size_t)t * KW * 4 + l * 16;
+                            *reinterpret_cast<float4 *>(dst) =
+                                make_float4(bf_lo(xv.x), bf_hi(xv.x), bf_lo(xv.y), bf_hi(xv.y));
+                            *reinterpret_cast<float4 *>(dst + KW * 2) =
+                                make_float4(bf_lo(xv.z), bf_hi(xv.z), bf_lo(xv.w), bf_hi(xv.w));
+                        }
+                    } else if (ok) {
                         // one (pair, 8-column chunk) per lane and step: two
                         // 16-byte reads, four 16-byte writes
                         const uint8_t *xb = slot_of(k) + a.xb_off;
@@ -570,9 +641,7 @@ __global__ void __maxnreg__(168)
         // ------------------------------------------------ consumers
         const int ct = tid - 96;
         bool ok = true;
-        // the token-pair variant waits for its converters, the column-pair
-        // variant for the copies themselves
-        uint64_t *ready = C::kWide ? full : xready;
+        uint64_t *ready = xready;                  // the converters hand every stage on
         auto wait_ready = [&](int kk) {
             if (ok && !mbar_wait(&ready[kk % NS], par_of(kk))) {
                 ok = false;
@@ -586,8 +655,9 @@ __global__ void __maxnreg__(168)
                 mbar_arrive(&empty[kk % NS]);
         };
 
-        const int sp = ct / CL, cl = ct % CL;      // phase A: channel pair of the pass, chunk lane
-        float2 acc[4 * NP];
+        constexpr int R = kSRows, RC = kSRows / 2;   // rows, channels per thread
+        const int sp = ct / CL, cl = ct % CL;      // phase A: channel set of the pass, chunk lane
+        float2 acc[R * NP];
         int k = 0;
         for (int ii = 0; ii < n_items; ++ii) {
             const Item it = items[ii];
@@ -597,20 +667,20 @@ __global__ void __maxnreg__(168)
             // ---- phase A
             for (int ps = 0; ps * S < nch; ++ps) {
                 const int ns = min(S, nch - ps * S);
-                const bool act = 2 * sp < ns;        // ns is a multiple of 8
+                const bool act = RC * sp < ns;       // ns is a multiple of 8
 #pragma unroll
-                for (int e = 0; e < 4 * NP; ++e)
+                for (int e = 0; e < R * NP; ++e)
                     acc[e] = make_float2(0.f, 0.f);
                 if constexpr (C::kWide) {
                     constexpr int NT = 2 * NP;      // tokens of a group, at most
-                    float2 acw[4 * NT];
+                    float2 acw[R * NT];
 #pragma unroll
-                    for (int e = 0; e < 4 * NT; ++e)
+                    for (int e = 0; e < R * NT; ++e)
                         acw[e] = make_float2(0.f, 0.f);
                     uint32_t xr[NT];
 #pragma unroll
                     for (int i = 0; i < NT; ++i)
-                        xr[i] = (uint32_t)(i < n ? tk[i] : 0) * KW * 2u;
+                        xr[i] = (uint32_t)(i < n ? tk[i] : 0) * KW * 4u;
                     for (int w = 0; w < NW; ++w, ++k) {
                         wait_ready(k);
                         if (ok && act) {
@@ -618,35 +688,39 @@ __global__ void __maxnreg__(168)
 #pragma unroll
                             for (int h = 0; h < C::CPL; ++h) {
                                 const int ch = cl + h * CL;
-                                const size_t r0 = (size_t)(2 * sp) * KW * 2 + ch * 16;
-                                const uint4 wr[4] = {lds128(sb + r0), lds128(sb + WB / 2 + r0),
-                                                     lds128(sb + r0 + KW * 2),
-                                                     lds128(sb + WB / 2 + r0 + KW * 2)};
-                                colpair4_n<NT>(n, wr, sb + a.xb_off + ch * 16, xr, acw);
+                                const size_t r0 = (size_t)(RC * sp) * KW * 2 + ch * 16;
+                                uint4 wr[R];
+#pragma unroll
+                                for (int c2 = 0; c2 < RC; ++c2) {
+                                    wr[2 * c2] = lds128(sb + r0 + c2 * KW * 2);
+                                    wr[2 * c2 + 1] = lds128(sb + WB / 2 + r0 + c2 * KW * 2);
+                                }
+                                colpair4_n<NT>(n, wr, sb + a.x32_off + ch * 16, xr, acw);
                             }
                         }
                         release(k);
                     }
-                    // token i's (gate, up) sums of channel c (acc[4i + 2c],
-                    // acc[4i + 2c + 1], each over even and odd columns) over
+                    // token i's (gate, up) sums of channel c (acw[R i + 2c],
+                    // acw[R i + 2c + 1], each over even and odd columns) over
                     // the chunk lanes; the owners write h (token i is slot
                     // i & 1 of pair i / 2)
-                    float2 gu[2 * NT];
+                    float2 gu[RC * NT];
 #pragma unroll
                     for (int i = 0; i < NT; ++i)
 #pragma unroll
-                        for (int cc = 0; cc < 2; ++cc)
-                            gu[2 * i + cc] = make_float2(acw[4 * i + 2 * cc].x + acw[4 * i + 2 * cc].y,
-                                                         acw[4 * i + 2 * cc + 1].x +
-                                                             acw[4 * i + 2 * cc + 1].y);
-                    lane_reduce2<2 * NT, C::LV, 1>(gu, lane);
-                    constexpr int LV = C::LV, Sl = scatter_levels(2 * NT, LV), R = (2 * NT) >> Sl;
+                        for (int cc = 0; cc < RC; ++cc)
+                            gu[RC * i + cc] = make_float2(acw[R * i + 2 * cc].x + acw[R * i + 2 * cc].y,
+                                                          acw[R * i + 2 * cc + 1].x +
+                                                              acw[R * i + 2 * cc + 1].y);
+                    lane_reduce2<RC * NT, C::LV, 1>(gu, lane);
+                    constexpr int LV = C::LV, Sl = scatter_levels(RC * NT, LV),
+                                  RR = (RC * NT) >> Sl;
                     if (act && (cl & ((1 << (LV - Sl)) - 1)) == 0) {
-                        const int mb = ((cl >> (LV - Sl)) & ((1 << Sl) - 1)) * R;
+                        const int mb = ((cl >> (LV - Sl)) & ((1 << Sl) - 1)) * RR;
 #pragma unroll
-                        for (int e = 0; e < R; ++e) {
-                            const int m = mb + e, i = m >> 1;
-                            const int chl = ps * S + 2 * sp + (m & 1);
+                        for (int e = 0; e < RR; ++e) {
+                            const int m = mb + e, i = m / RC;
+                            const int chl = ps * S + RC * sp + m % RC;
                             if (i < n)
                                 hs[((size_t)(i >> 1) * nch + chl) * 2 + (i & 1)] =
                                     silu_f32(gu[e].x) * gu[e].y;
@@ -657,28 +731,31 @@ __global__ void __maxnreg__(168)
                         wait_ready(k);
                         if (ok && act) {
                             const uint8_t *sb = slot_of(k);
-                            const size_t r0 = (size_t)(2 * sp) * KW * 2 + cl * 16;
-                            const uint4 wr[4] = {lds128(sb + r0), lds128(sb + WB / 2 + r0),
-                                                 lds128(sb + r0 + KW * 2),
-                                                 lds128(sb + WB / 2 + r0 + KW * 2)};
+                            const size_t r0 = (size_t)(RC * sp) * KW * 2 + cl * 16;
+                            uint4 wr[R];
+#pragma unroll
+                            for (int c2 = 0; c2 < RC; ++c2) {
+                                wr[2 * c2] = lds128(sb + r0 + c2 * KW * 2);
+                                wr[2 * c2 + 1] = lds128(sb + WB / 2 + r0 + c2 * KW * 2);
+                            }
                             rows4_np<NP, KW * 2>(np, wr, sb + a.x32_off + cl * 16,
                                                  (uint32_t)KW * 8u, acc);
                         }
                         release(k);
                     }
-                    // sums over the chunk lanes, in place: acc[4p + 2c] is
-                    // pair p's gate sums of channel c, acc[4p + 2c + 1] its up
-                    // sums (each: the pair's two token slots); the owners
+                    // sums over the chunk lanes, in place: acc[R p + 2c] is
+                    // pair p's gate sums of channel c, acc[R p + 2c + 1] its
+                    // up sums (each: the pair's two token slots); the owners
                     // write h for this pass's channels
-                    constexpr int N = 4 * NP, LV = C::LV;
+                    constexpr int N = R * NP, LV = C::LV;
                     lane_reduce2<N, LV, 2>(acc, lane);
-                    constexpr int Sl = scatter_levels(N / 2, LV), R = N >> Sl;
+                    constexpr int Sl = scatter_levels(N / 2, LV), RR = N >> Sl;
                     if (act && (cl & ((1 << (LV - Sl)) - 1)) == 0) {
-                        const int mb = ((cl >> (LV - Sl)) & ((1 << Sl) - 1)) * R;
+                        const int mb = ((cl >> (LV - Sl)) & ((1 << Sl) - 1)) * RR;
 #pragma unroll
-                        for (int e = 0; e < R; e += 2) {
-                            const int m = mb + e, p = m >> 2;
-                            const int chl = ps * S + 2 * sp + ((m >> 1) & 1);
+                        for (int e = 0; e < RR; e += 2) {
+                            const int m = mb + e, p = m / R;
+                            const int chl = ps * S + RC * sp + (m % R) / 2;
                             if (p < np)
                                 *reinterpret_cast<float2 *>(hs + ((size_t)p * nch + chl) * 2) =
                                     make_float2(silu_f32(acc[e].x) * acc[e + 1].x,
@@ -692,7 +769,7 @@ __global__ void __maxnreg__(168)
             const int BC = a.bch, nbs = (nch + BC - 1) / BC;
             for (int rb = 0; rb < NRB; ++rb) {
 #pragma unroll
-                for (int e = 0; e < 4 * NP; ++e)
+                for (int e = 0; e < R * NP; ++e)
                     acc[e] = make_float2(0.f, 0.f);
                 for (int cc = 0; cc < nbs; ++cc, ++k) {
                     wait_ready(k);
@@ -711,9 +788,9 @@ __global__ void __maxnreg__(168)
                             const int c8 = cc * BC + half * 8;     // channel within the item
                             if (c8 >= nch)
                                 continue;
-                            uint4 wr[4];
+                            uint4 wr[R];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j)
+                            for (int j = 0; j < R; ++j)
                                 wr[j] = lds128(sb + (size_t)(ct + kSCons * j) * BC * 2 + half * 16);
                             rows4_np<NP, 16>(np, wr, reinterpret_cast<const uint8_t *>(hs) + c8 * 8,
                                              (uint32_t)nch * 8u, acc);
@@ -730,12 +807,12 @@ __global__ void __maxnreg__(168)
                             break;
                         const int ta = tk[2 * p], tb = 2 * p + 1 < n ? tk[2 * p + 1] : -1;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
+                        for (int j = 0; j < R; ++j) {
                             const int r = rb * kSRowBlk + ct + kSCons * j;
                             if (r < H) {
-                                red_add_f32(a.acc + (size_t)ta * H + r, acc[4 * p + j].x);
+                                red_add_f32(a.acc + (size_t)ta * H + r, acc[R * p + j].x);
                                 if (tb >= 0)
-                                    red_add_f32(a.acc + (size_t)tb * H + r, acc[4 * p + j].y);
+                                    red_add_f32(a.acc + (size_t)tb * H + r, acc[R * p + j].y);
                             }
                         }
                     }
@@ -889,12 +966,15 @@ bool plan_split(int T, int H, int I, int gs, SplitPlan *p)
     const uint32_t xb = ((uint32_t)T * KW * 2u + 1023u) & ~1023u;
     p->xb_off = (uint32_t)WB;
     p->x32_off = (uint32_t)WB + xb;
-    uint32_t slot = p->x32_off + (p->NP <= 4 ? 0u : (uint32_t)p->NP * KW * 8u);
-    // a phase-B stage of 16 channels (32 bytes of every W_down row) when the
-    // slot holds its 32 KB, else 8
-    p->bch = slot >= (uint32_t)kSRowBlk * 32u ? 16 : 8;
+    uint32_t slot = p->x32_off + (p->NP <= 4 ? (uint32_t)T * KW * 4u : (uint32_t)p->NP * KW * 8u);
+    // phase-B stages of 16 channels (32 bytes of every W_down row: 1024 row
+    // pieces of 16 bytes take about as long to copy as 1024 of 32), so a
+    // slot holds at least 32 KB
+    p->bch = 16;
+    if (slot < (uint32_t)kSRowBlk * 32u)
+        slot = (uint32_t)kSRowBlk * 32u;
     p->slot_bytes = (slot + 1023u) & ~1023u;
-    const size_t fixed = 1024 + (size_t)p->NP * gs * 8 + (size_t)T * W * 4 + (size_t)G * 4 +
+    const size_t fixed = 1024 + (size_t)p->NP * gs * 8 + (size_t)T * W * 4 + (size_t)G * 8 + 4 +
                          (size_t)kSMaxItems * kSMaxTok * 4 + 8 + 3 * kSMaxSlots * 8;
     if ((size_t)di.optin <= fixed + 64)
         return false;
@@ -948,10 +1028,15 @@ bool decode_ffn_split_supported(int T, int H, int I, int gs)
     return plan_split(T, H, I, gs, &p);
 }
 
+namespace {
+std::atomic<int> g_decode_mode{WIDE_DECODE_AUTO};
+}
+
+// AUTO takes the channel-split kernel wherever its shape limits allow (on
+// B200 it is at least as fast as the two GEMV kernels at every token count).
 bool decode_ffn_split_preferred(int T, int H, int I, int gs)
 {
-    const int mode = wide_get_decode_ffn_path_mode();
-    if (mode == WIDE_DECODE_GEMV || mode == kDecodeFusedOld)
+    if (g_decode_mode.load(std::memory_order_relaxed) == WIDE_DECODE_GEMV)
         return false;
     return decode_ffn_split_supported(T, H, I, gs);
 }
@@ -972,7 +1057,8 @@ int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *
     const uint32_t dbox[3] = {(uint32_t)pl.bch, kSDownBox, kSRowBlk / kSDownBox};
     // W_gate / W_up rows and x rows as {64, cols / 64, rows}: a box copies
     // whole KW-column pieces of rows (1 KB each in the 512-column variant)
-    const uint32_t kwc = (uint32_t)pl.kw / 64, S = (uint32_t)(2 * kSCons / (pl.kw == 512 ? 32 : 16));
+    const uint32_t kwc = (uint32_t)pl.kw / 64,
+                   S = (uint32_t)(kSCons / (pl.kw == 512 ? 32 : 16) * kSRows / 2);
     if (!make_tmap_rows3d(&m.gate, wg, I, H, H, kwc, S) ||
         !make_tmap_rows3d(&m.up, wu, I, H, H, kwc, S) ||
         !make_tmap_rows3d(&m.gate8, wg, I, H, H, kwc, 8) ||
@@ -1009,3 +1095,10 @@ int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *
 }
 
 }  // namespace wide
+
+extern "C" int wide_set_decode_ffn_path(int mode)
+{
+    if (mode != WIDE_DECODE_AUTO && mode != WIDE_DECODE_FUSED && mode != WIDE_DECODE_GEMV)
+        return WIDE_EINVAL;
+    return wide::g_decode_mode.exchange(mode);
+}

@@ -10,8 +10,8 @@
 // kernel (bf16, the usual case) its fp32 [T][hidden] accumulator and arrival
 // counter, for the GEMV kernels (fp32, and bf16 shapes outside the split
 // kernel's limits) the fp32 intermediate h = silu(gate) * up of up to 32
-// tokens; the earlier fused kernel's grid-barrier words sit in the second
-// array.
+// tokens.  The second array holds the barrier words the decode path's
+// interface carries (unused by the current kernels).
 //
 // The arrays are module globals: every GPU that loads the library holds
 // WIDE_NOALLOC_SCRATCH_BYTES (+ 256) bytes of device memory for them until

@@ -2,13 +2,16 @@
 //
 // WIDE, technical summary sections 2.B and 2.C.  After wide_reorder (per
 // group stable partition, signature order, per-tile unions; no host sync):
-//   zero_dead        zeros in H at (token, group) pairs the token skips
 //   gather_gemm      SwiGLU mode: each (group, row tile) work item gathers
 //                    its active token rows and multiplies them by the
 //                    group's [W_gate; W_up] slab on tcgen05; the epilogue
 //                    writes silu(gate) * up into H at signature-order rows
+//                    (only kept (token, group) pairs are ever written)
 //   tile_union_gemm  out = H W_down^T over each signature tile's union of
-//                    kept groups, written at the tokens' own rows
+//                    kept groups, written at the tokens' own rows; a row
+//                    whose token skips a group enters that group's K steps
+//                    as zeros (set in shared memory; H there is never
+//                    written)
 // The kernels live in prefill_gemm.cu.
 #include "common.cuh"
 #include "host.h"
@@ -52,8 +55,6 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
 
     if (!ext_wl && (rc = reorder_launch(mask, T, G, kBM, &wl, s)))
         return rc;
-    if ((rc = zero_dead_launch(mask, wl.sig_pos, hbuf, (int)T, (int)I, (int)G, (int)gs, s)))
-        return rc;
 
     GemmArgs ga = {};
     ga.a = static_cast<const __nv_bfloat16 *>(x);
@@ -75,10 +76,13 @@ int ffn_prefill_core(const void *x, const void *wg, const void *wu, const void *
     UnionArgs ua = {};
     ua.tile_union = wl.tile_union;
     ua.sig_perm = wl.sig_perm;
+    ua.mask = mask;
+    ua.h = hbuf;
     ua.T = (int)T;
     ua.N = (int)H;
     ua.W = (int)((G + 31) / 32);
     ua.gs = (int)gs;
+    ua.ld = (int)I;
     ua.out_sum = o.out_sum;
     ua.res_f32 = o.res_f32;
     ua.out_total = o.out_total;

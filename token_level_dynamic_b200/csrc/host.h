@@ -86,7 +86,6 @@ enum KernelId : int32_t {
     KID_REORDER_FINISH = 2,
     KID_DECODE_GATEUP = 3,
     KID_DECODE_DOWN = 4,
-    KID_PREFILL_ZERO = 5,
     KID_PREFILL_GATEUP = 6,
     KID_PREFILL_DOWN = 7,
     KID_DECODE_QKV = 8,
@@ -96,7 +95,6 @@ enum KernelId : int32_t {
     KID_PREFILL_KV = 12,
     KID_PREFILL_ATTN = 13,
     KID_PREFILL_OPROJ = 14,
-    KID_DECODE_FFN_FUSED = 15,
     KID_ROUTER = 16,
     KID_ROUTER_SMALL = 17,
     KID_DECODE_FFN_SPLIT = 18,
@@ -170,7 +168,9 @@ struct GemmArgs {
 struct UnionArgs {
     const uint32_t *tile_union;
     const int32_t *sig_perm;
-    int T, N, W, gs;
+    const uint32_t *mask;            // [T][W] group bits of the tokens (token order)
+    const __nv_bfloat16 *h;          // A: [T][ld] rows in signature order (loaded by tm_a)
+    int T, N, W, gs, ld;
     __nv_bfloat16 *out_sum;          // projection (optional)
     const __nv_bfloat16 *res_in;     // residual, bf16 (optional)
     const float *res_f32;            // residual, fp32 (optional)
@@ -179,8 +179,6 @@ struct UnionArgs {
     int32_t *status;
 };
 
-int zero_dead_launch(const uint32_t *mask, const int32_t *sig_pos, void *buf, int T, int ld,
-                     int G, int gs, cudaStream_t s);
 int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
                        const GemmArgs &a, int max_work, int32_t kid, cudaStream_t s);
 int tile_union_gemm_launch(const CUtensorMap &tm_a, const CUtensorMap &tm_b, const UnionArgs &a,
@@ -235,26 +233,6 @@ int decode_gateup_bf16(const void *x, const void *wg, const void *wu, const uint
                        float *h, int T, int H, int I, int gs, cudaStream_t s);
 int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const DownOutputs &o,
                      int T, int H, int I, int gs, cudaStream_t s);
-// Inputs of the fused decode FFN: the FFN input is either x (bf16 [T][H])
-// or x_f32 (fp32 [T][H] rows RMS-normalised with gamma and eps inside the
-// kernel, rounded to bf16 as a bf16 layer feeds its FFN).
-struct FusedInput {
-    const void *x;
-    const float *x_f32;
-    const void *gamma;
-    float eps;
-    const void *w_gate, *w_up, *w_down;
-    const uint32_t *mask;
-};
-// bf16 decode FFN of 1 <= T <= 32 tokens as one persistent cooperative
-// kernel (ffn_decode_fused.cu).  h: fp32 [T][I] scratch with token pairs
-// interleaved (T rounded up to even); bar: 2 words of device memory for the
-// grid barrier (the call zeroes bar[0] on the stream).
-bool decode_ffn_fused_supported(int T, int H, int I, int gs);
-// Whether the decode path should use it for this shape (faster there).
-bool decode_ffn_fused_preferred(int T, int H, int I, int gs);
-int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, int I, int gs,
-                     float *h, uint32_t *bar, cudaStream_t s);
 // bf16 decode FFN of 1 <= T <= kSplitMaxTok tokens as one persistent
 // cooperative kernel in which every CTA owns a slice of the batch's kept
 // channels
@@ -264,11 +242,9 @@ int decode_ffn_fused(const FusedInput &in, const DownOutputs &o, int T, int H, i
 constexpr int kSplitMaxTok = 16;   // tokens per launch of the split kernel
 size_t decode_ffn_split_scratch(int T, int H);
 bool decode_ffn_split_supported(int T, int H, int I, int gs);
+// Whether the decode path should use it for this shape (the
+// wide_set_decode_ffn_path mode allows it and the shape fits).
 bool decode_ffn_split_preferred(int T, int H, int I, int gs);
-// Current wide_set_decode_ffn_path mode; kDecodeFusedOld selects the
-// earlier fused kernel (ffn_decode_fused.cu) for comparison runs.
-int wide_get_decode_ffn_path_mode();
-constexpr int kDecodeFusedOld = 3;
 int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *wd,
                      const uint32_t *mask, const DownOutputs &o, int T, int H, int I, int gs,
                      void *scratch, cudaStream_t s);

@@ -35,9 +35,17 @@
 //             RoPE in the epilogue) or Wv; stored into the caches.
 // tile_union_gemm: persistent, M=128 tokens of one signature tile x N=256
 //   outputs; the K loop visits only the groups (gs columns each) in the
-//   tile's union of kept groups; inactive rows inside a visited group read
-//   the zeros written by zero_dead.  Epilogue: projection and/or projection
-//   plus residuals (bf16 and fp32), written at the tokens' own rows.
+//   tile's union of kept groups (block-level skip).  Warp 0 loads the A tile
+//   (the tokens' rows of H, stored in signature order) and the weight tile
+//   (B) by TMA; warps 6-7 then overwrite, in shared memory, the rows whose
+//   token skips the group with zeros before the stage goes to the MMA, so
+//   those rows contribute nothing and H entries of skipped pairs are never
+//   written (no zeroing pass over H in HBM).  Gathering only the active rows
+//   with 16-byte cp.async copies instead (source size 0 for a skipped row)
+//   measured 1.8x slower on the 8B FFN: H streams from DRAM, and per-thread
+//   copies behind a 4-stage ring do not cover that latency the way TMA
+//   boxes do.  Epilogue: projection and/or projection plus residuals (bf16
+//   and fp32), written at the tokens' own rows.
 //
 // Every mbarrier wait is bounded; on expiry the kernel records
 // WIDE_DEV_TIMEOUT, drains what it issued (bounded), frees TMEM and returns.
@@ -62,7 +70,7 @@ constexpr int kRouterStages = 6;
 constexpr uint32_t kRouterStageBytes = kATile + 128u * 128u;
 constexpr int kMaxStages = 6;
 static_assert(kRouterStages * kRouterStageBytes <= kStages * kStageBytes, "router ring");
-constexpr int kThreadsDown = 192;
+constexpr int kThreadsDown = 256;
 constexpr int kThreadsGather = 256;
 constexpr int kGatherThreads = 64;
 constexpr uint32_t kTmemCols = 512;
@@ -74,6 +82,7 @@ struct __align__(8) Ctl {
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
+    uint64_t fixed[kMaxStages];   // tile_union_gemm: skipped rows zeroed
     uint32_t tmem_base;
     int abort;
     int trow[2][kBM / 2]; // gather warp w: offsets of its rows' tokens (-1: none)
@@ -173,26 +182,6 @@ __device__ __forceinline__ void copy_head_store(uint32_t taddr, __nv_bfloat16 *d
         umma::tmem_ld_wait();
         if (store)
             store_bf16x32(dst + cc * 32, v);
-    }
-}
-
-// ------------------------------------------------------------- zero_dead
-// One block per token: clears the gs-column slice of every group the token
-// skips, in row sig_pos[t] of a [T][ld] bf16 buffer.
-__global__ void __launch_bounds__(128)
-    zero_dead(const uint32_t *__restrict__ mask, const int32_t *__restrict__ sig_pos,
-              __nv_bfloat16 *__restrict__ buf, int T, int ld, int G, int W, int gs)
-{
-    const int t = blockIdx.x;
-    if (t >= T)
-        return;
-    const size_t row = (size_t)sig_pos[t] * ld;
-    const int per = gs / 8;                      // 16-byte chunks per group slice
-    for (int idx = threadIdx.x; idx < G * per; idx += 128) {
-        const int g = idx / per, q = idx % per;
-        if ((mask[(size_t)t * W + (g >> 5)] >> (g & 31)) & 1u)
-            continue;
-        reinterpret_cast<uint4 *>(buf + row + (size_t)g * gs)[q] = make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
@@ -626,7 +615,12 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
     const int spg = a.gs / kBK;            // K stages per group
 
     if (threadIdx.x == 0) {
+        // full: the producer's arrive with the A and B bytes; fixed: one
+        // arrive per zero-filling thread once its rows of the stage are done
         init_ctl(ctl, 1);
+        for (int st = 0; st < kStages; ++st)
+            mbar_init(&ctl->fixed[st], kGatherThreads);
+        fence_mbar_init();
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
     }
@@ -648,6 +642,7 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
     auto uword = [&](int s, int w) { return a.tile_union[(size_t)s * a.W + w]; };
 
     if (warp == 0) {
+        // -------------------------------------------- weight producer
         uint32_t stage = 0, phase = 0, issued = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
@@ -668,10 +663,10 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
                                 const int col = g * a.gs + sub * kBK;
                                 tma_load_2d(sa, &tm_a, col, s * kBM, &ctl->full[stage]);
                                 tma_load_2d(sa + kATile, &tm_b, col, nb * kBN, &ctl->full[stage]);
+                                ++issued;
                             }
                         }
                         ok = __shfl_sync(0xffffffffu, ok, 0);
-                        issued += ok ? 1u : 0u;
                         if (++stage == kStages) {
                             stage = 0;
                             phase ^= 1u;
@@ -684,6 +679,62 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
             for (uint32_t s = 0; s < kStages && s < issued; ++s) {
                 const uint32_t uses = (issued - s + kStages - 1) / kStages;
                 mbar_wait(&ctl->full[s], (uses - 1u) & 1u);
+            }
+        }
+    } else if (warp >= 6) {
+        // -------------------------------------------- skipped rows to zero
+        // warp gw, lane l handles chunk l % 8 of rows 4 gw + l / 8 + 8 i
+        // (i < 16) of each stage (lanes 8j .. 8j+7 cover one 128-byte row
+        // piece).  Row r of signature tile s is H row s * 128 + r; its token
+        // sig_perm[s * 128 + r] decides, per group, whether the loaded row
+        // stays or is overwritten with zeros (rows past T too: the TMA box
+        // already read zeros there).
+        const int gw = warp - 6, lq = lane >> 3, cc = lane & 7;
+        const int lr = 4 * gw + lq;
+        uint32_t stage = 0, phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            int s, nb;
+            coords(tile, s, nb);
+            int tok[kBM / 8];
+#pragma unroll
+            for (int i = 0; i < kBM / 8; ++i) {
+                const int sr = s * kBM + lr + 8 * i;
+                tok[i] = sr < a.T ? a.sig_perm[sr] : -1;
+            }
+            for (int w = 0; w < a.W && ok; ++w) {
+                uint32_t bits = uword(s, w);
+                if (!bits)
+                    continue;
+                uint32_t mw[kBM / 8];
+#pragma unroll
+                for (int i = 0; i < kBM / 8; ++i)
+                    mw[i] = tok[i] >= 0 ? a.mask[(size_t)tok[i] * a.W + w] : 0u;
+                while (bits && ok) {
+                    const int gb = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    for (int sub = 0; sub < spg; ++sub) {
+                        const bool got = wait_or_abort(&ctl->full[stage], phase, ctl, a.status);
+                        if (!__all_sync(0xffffffffu, got)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *sa = smem + stage * kStageBytes;
+#pragma unroll
+                        for (int i = 0; i < kBM / 8; ++i)
+                            if (!((mw[i] >> gb) & 1u))
+                                *reinterpret_cast<uint4 *>(sa + swz128(lr + 8 * i, cc)) =
+                                    make_uint4(0u, 0u, 0u, 0u);
+                        // the zeros are written by the generic proxy and read
+                        // by the tensor core (async proxy)
+                        fence_proxy_async_smem();
+                        mbar_arrive(&ctl->fixed[stage]);
+                        if (++stage == kStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
             }
         }
     } else if (warp == 1) {
@@ -702,7 +753,9 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
                 for (int w = 0; w < a.W && ok; ++w) {
                     const int nsteps = __popc(uword(s, w)) * spg;
                     for (int n = 0; n < nsteps && ok; ++n) {
-                        if (!wait_or_abort(&ctl->full[stage], phase, ctl, a.status)) {
+                        // fixed completes once the zero-filling warps (which
+                        // waited for full) are done with the stage
+                        if (!wait_or_abort(&ctl->fixed[stage], phase, ctl, a.status)) {
                             ok = false;
                             break;
                         }
@@ -828,17 +881,6 @@ int num_sms()
 }
 
 }  // namespace
-
-int zero_dead_launch(const uint32_t *mask, const int32_t *sig_pos, void *buf, int T, int ld,
-                     int G, int gs, cudaStream_t s)
-{
-    if (T <= 0)
-        return WIDE_OK;
-    LaunchScope scope(KID_PREFILL_ZERO, s);
-    zero_dead<<<(unsigned)T, 128, 0, s>>>(mask, sig_pos, static_cast<__nv_bfloat16 *>(buf), T, ld,
-                                          G, (G + 31) / 32, gs);
-    return launch_status();
-}
 
 int gather_gemm_launch(int mode, const CUtensorMap &tm0, const CUtensorMap &tm1,
                        const GemmArgs &a, int max_work, int32_t kid, cudaStream_t s)

@@ -103,8 +103,6 @@ const char *wide_kernel_name(int32_t id)
         return "decode_gateup_gemv";
     case KID_DECODE_DOWN:
         return "decode_down_gemv";
-    case KID_PREFILL_ZERO:
-        return "prefill_zero_fill";
     case KID_PREFILL_GATEUP:
         return "prefill_gateup_tcgen05";
     case KID_PREFILL_DOWN:
@@ -123,8 +121,6 @@ const char *wide_kernel_name(int32_t id)
         return "prefill_attention_tcgen05";
     case KID_PREFILL_OPROJ:
         return "prefill_oproj_tcgen05";
-    case KID_DECODE_FFN_FUSED:
-        return "decode_ffn_fused_gemv";
     case KID_ROUTER:
         return "router_tcgen05";
     case KID_ROUTER_SMALL:
