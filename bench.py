@@ -264,12 +264,13 @@ class DecodeFFN3B:
         return _ffn_decode_bytes(case)
 
     def reference_sample(self, cases):
-        out = []
-        for c in cases:
-            s = type(c)(**{**c.__dict__})
-            s.x, s.mask, s.T = c.x[:1], c.mask[:1], 1
-            out.append(s)
-        return out, "per step: token 0 of each of batches 1, 8, 32 (3 tokens)"
+        # one call of n tokens (the oracle's token loop runs one token per
+        # OpenMP thread, so n = the host threads, at most the batch of 32)
+        c = cases[-1]
+        n = max(1, min(c.T, _host_cores()))
+        s = type(c)(**{**c.__dict__})
+        s.x, s.mask, s.T = c.x[:n], c.mask[:n], n
+        return [s], f"per step: the first {n} tokens of the batch-32 call, in one oracle call"
 
     reference_step = staticmethod(lambda samples: _ffn_oracle_step(samples))
 
@@ -347,9 +348,10 @@ class PrefillFFN8B:
 
     def reference_sample(self, cases):
         c = cases[0]
+        n = max(8, min(32, _host_cores()))
         s = type(c)(**{**c.__dict__})
-        s.x, s.mask, s.T = c.x[:8], c.mask[:8], 8
-        return [s], "per step: the first 8 tokens of the 4096-token batch"
+        s.x, s.mask, s.T = c.x[:n], c.mask[:n], n
+        return [s], f"per step: the first {n} tokens of the 4096-token batch, in one oracle call"
 
     reference_step = staticmethod(lambda samples: _ffn_oracle_step(samples))
 
@@ -651,23 +653,38 @@ WORKLOADS = {w.name: w for w in (DecodeFFN3B(), PrefillFFN8B(), DecodeLayer8B(),
 
 # ------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_baseline(wl, samples, seconds: float):
-    """Times the oracle on the host cores, repeating the sample until
-    `seconds` have passed."""
-    from oracle import _clib
-    tokens, t0, reps = 0, time.perf_counter(), 0
-    while True:
-        tokens += wl.reference_step(samples)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    return tokens / el, _host_cores(), reps, el
+def cpu_oracle_baseline(wl, samples, seconds: float, threads=None):
+    """Times the oracle, repeating the sample until `seconds` have passed.
+    `threads` caps the OpenMP and BLAS thread pools the oracle runs on
+    (None: every host thread).  Returns (tokens/s, threads used, reps, s)."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        used = _host_cores()
+        tokens, t0, reps = 0, time.perf_counter(), 0
+        while True:
+            tokens += wl.reference_step(samples)
+            reps += 1
+            el = time.perf_counter() - t0
+            if el >= seconds:
+                break
+    return tokens / el, used, reps, el
 
 
 def _host_cores():
+    """OpenMP threads the oracle's C loops run on (BLAS uses as many)."""
     from oracle import _clib
     return int(_clib.lib().oracle_num_threads())
+
+
+def cpu_baseline_record(wl, cases, seconds: float):
+    """The oracle on every host thread and on one, same sample."""
+    samples, what = wl.reference_sample(cases)
+    v, cores, reps, el = cpu_oracle_baseline(wl, samples, seconds)
+    v1, _, reps1, el1 = cpu_oracle_baseline(wl, samples, seconds, threads=1)
+    return {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{what}; repeated {reps}x over {el:.1f} s (fp64 oracle)",
+            "one_core": {"value": v1, "unit": "tokens/s", "cores": 1,
+                         "sample": f"the same; repeated {reps1}x over {el1:.1f} s"}}
 
 
 def max_over_ranks(x: float, device) -> float:
@@ -716,8 +733,10 @@ def run_reference(args, wl):
 
 # ------------------------------------------------------------------- ours
 
+EXTRA_WORKLOADS = ("prefill_layer_8b", "decode_layer_8b")
+
+
 def run_ours(args, wl):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -732,6 +751,39 @@ def run_ours(args, wl):
     dev = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
     torch.cuda.set_device(dev)
 
+    line = measure(args, wl, dev, world, rank, args.steps,
+                   cpu_leg=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    # The default run also times the two whole-layer workloads (prefill at
+    # keep 0.5, decode), one GPU only, without a CPU leg; each entry carries
+    # the same fields as the main line.
+    extra = {}
+    if world == 1 and args.workload == "decode_ffn_3b" and not args.no_extra_workloads:
+        for name in EXTRA_WORKLOADS:
+            torch.cuda.empty_cache()
+            ewl = PrefillLayer8B(0.5) if name == "prefill_layer_8b" else WORKLOADS[name]
+            e = measure(args, ewl, dev, world, rank, min(args.steps, 50), cpu_leg=False)
+            for k in ("n_gpus", "warmup", "higher_is_better", "scaling", "vs_baseline", "dtype",
+                      "data", "kernel_timing", "cpu_baseline"):
+                e.pop(k, None)
+            extra[name] = e
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    if extra:
+        line["extra_workloads"] = extra
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure(args, wl, dev, world, rank, steps, cpu_leg):
+    """Times `steps` steps of workload `wl` on `dev` (after args.warmup
+    untimed ones) and returns the bench line's fields as a dict."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
     import token_level_dynamic_b200 as w
 
     cases = wl.make_cases()
@@ -778,7 +830,7 @@ def run_ours(args, wl):
     n0 = w.wide_launch_count()
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         barrier()
-        all_evs = [timed_step(call) for _ in range(args.steps)]
+        all_evs = [timed_step(call) for _ in range(steps)]
         barrier()
     launches = w.wide_launch_count() - n0
     if w.wide_get_device_status(stream) != 0:
@@ -790,14 +842,14 @@ def run_ours(args, wl):
     # region above runs without them)
     w.wide_profile_start(65536)
     barrier()
-    for _ in range(args.steps):
+    for _ in range(steps):
         timed_step(call)
     barrier()
     w.wide_profile_stop()
     recs = w.wide_profile_read()
     total_ms = max_over_ranks(float(per_call.sum()), dev)
-    step_ms = total_ms / args.steps
-    value = job_tokens_per_s(world, tokens_per_step, args.steps, total_ms)
+    step_ms = total_ms / steps
+    value = job_tokens_per_s(world, tokens_per_step, steps, total_ms)
 
     # ---- per-kernel figures from the library's launch events
     peaks = _peaks()
@@ -806,7 +858,7 @@ def run_ours(args, wl):
         kern.setdefault(name, []).append(t)
     kernels = {}
     for name, ts in kern.items():
-        t_step = sum(ts) / args.steps
+        t_step = sum(ts) / steps
         entry = {"launches": len(ts), "avg_us": 1e3 * statistics.mean(ts),
                  "us_per_step": 1e3 * t_step}
         if any(name in u for u in units):
@@ -876,7 +928,7 @@ def run_ours(args, wl):
 
     # ---- dense baselines: torch/cuBLAS bf16 and our kernels with every group kept
     dense = {}
-    nd = max(3, min(args.steps, 20))
+    nd = max(3, min(steps, 20))
     for name, fn in (("torch_cublas_bf16", D.dense_torch),
                      ("ours_all_groups_kept", lambda i: D.call(i, all_kept=True))):
         for _ in range(3):
@@ -915,28 +967,18 @@ def run_ours(args, wl):
     for _ in range(3):
         timed_step(D.e2e_call)
     barrier()
-    e_evs = [timed_step(D.e2e_call) for _ in range(args.steps)]
+    e_evs = [timed_step(D.e2e_call) for _ in range(steps)]
     barrier()
     e_ms = max_over_ranks(float(ms_of(e_evs).sum()), dev)
-    e2e = {"value": job_tokens_per_s(world, tokens_per_step, args.steps, e_ms), "unit": "tokens/s",
+    e2e = {"value": job_tokens_per_s(world, tokens_per_step, steps, e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": D.h2d_bytes, "d2h_bytes_per_step": D.d2h_bytes,
-           "ms_per_step": e_ms / args.steps}
+           "ms_per_step": e_ms / steps}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        samples, what = wl.reference_sample(cases)
-        v, cores, reps, el = cpu_oracle_baseline(wl, samples, args.cpu_seconds)
-        cpu = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": f"{what}; repeated {reps}x over {el:.1f} s (fp64 oracle)"}
+    cpu = cpu_baseline_record(wl, cases, args.cpu_seconds) if cpu_leg else None
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return 0
-    line = {
+    return {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; shapes of the pages' Llama workloads)",
         "config": {"workload": wl.desc, "global_batch": world * tokens_per_step,
@@ -950,8 +992,6 @@ def run_ours(args, wl):
         "dense_baseline": dense, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": int(launches), "clocks": clk.summary(),
     }
-    print(json.dumps(line), flush=True)
-    return 0
 
 
 def main():
@@ -962,6 +1002,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_ffn_3b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="time only --workload (the default run also times "
+                         "prefill_layer_8b at keep 0.5 and decode_layer_8b)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--keep", type=float, default=0.5,
                     help="keep rate of the prefill_layer_8b masks (0.25, 0.5, 0.75, 1.0)")

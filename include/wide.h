@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define WIDE_ABI_VERSION 2
+#define WIDE_ABI_VERSION 3
 
 /* host-side status codes */
 #define WIDE_OK 0
@@ -219,26 +219,74 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                     size_t workspace_bytes, void *stream);
 
 /* Kernels of the bf16 decode FFN (process-wide; the decode layer's FFN
- * follows it too).  Both compute the same sums, in a different fp32 order:
- *   WIDE_DECODE_AUTO   the channel-split kernel wherever its shape limits
- *                      allow, else the GEMVs (default)
- *   WIDE_DECODE_FUSED  the same: one persistent kernel per launch of up to
+ * follows it too).  All compute the same sums, in a different fp32 order:
+ *   WIDE_DECODE_AUTO   the channel-split kernel for up to 8 tokens, the
+ *                      tensor-core kernel above, each where its shape
+ *                      limits allow, else the GEMVs (default)
+ *   WIDE_DECODE_TC     the tensor-core kernel: one persistent kernel per launch of
+ *                      up to 32 tokens (hidden % 128 == 0, group size a
+ *                      multiple of 16 up to 256); each CTA owns a slice of
+ *                      the union's channels, runs gate/up and its share of
+ *                      the down projection as tcgen05 MMAs (h rounded to
+ *                      bf16 between them) and adds that share into an fp32
+ *                      accumulator with atomics, so two calls can differ in
+ *                      the last fp32 bits
+ *   WIDE_DECODE_FUSED  the channel-split CUDA-core kernel, launches of up to
  *                      16 tokens (hidden % 256 == 0, group size a multiple
- *                      of 8 up to 256); each CTA owns one group's channel
- *                      range, computes gate/up for the tokens that keep the
- *                      group and adds its share of the down projection into
- *                      an fp32 accumulator with atomics, so two calls can
- *                      differ in the last fp32 bits
+ *                      of 8 up to 256), atomics as above
  *   WIDE_DECODE_GEMV   the gate/up GEMV kernel, then the down GEMV kernel
- *                      (bitwise repeatable); bf16 group size 32 exists on
- *                      the channel-split kernel only and runs there
+ *                      (bitwise repeatable); bf16 group size 32 has no GEMV
+ *                      kernel and runs on a persistent kernel
  * Returns the previous mode, or WIDE_EINVAL for an unknown mode (the mode
  * is then unchanged).  Not ordered with work already enqueued: it applies
  * to calls made after it returns. */
 #define WIDE_DECODE_AUTO 0
 #define WIDE_DECODE_FUSED 1
 #define WIDE_DECODE_GEMV 2
+#define WIDE_DECODE_TC 3
 int wide_set_decode_ffn_path(int mode);
+
+/* ------------------------------------------------- packed decode weights
+ *
+ * The decode FFN reads every kept weight byte once per call, so it runs at
+ * the speed HBM delivers the union's weights.  The tensor cores take a
+ * K-major bf16 operand from shared memory in atoms of 8 rows x 128 bytes;
+ * from the nn.Linear layout such a tile is 128-byte pieces of rows that lie
+ * kilobytes apart, which B200 HBM serves at about half its bandwidth.  A
+ * packed copy holds the same weights with every tile the decode kernel loads
+ * stored as one contiguous run:
+ *   W_gate, W_up  interleaved, [inter / 64][hidden / 64][4][2][16][64]:
+ *                 64-channel panels, K-step-major, inside each K step four
+ *                 16-channel groups of 16 W_gate rows then the same 16 W_up
+ *                 rows (element [p][k][q][s][r][e] = (s ? W_up : W_gate)
+ *                 [64p + 16q + r][64k + e]);
+ *   W_down        [inter / 16][hidden][16] (element [c][n][e] =
+ *                 W_down[n][16c + e]),
+ * in that order in one buffer.  The values are copied bitwise, so results
+ * equal those of the nn.Linear weights up to the fp32 summation order.
+ * Pack once when the weights are loaded; the copy costs as much device
+ * memory as the FFN weights.  Supported: hidden % 128 == 0, inter % 64 == 0.
+ */
+
+/* Bytes of the packed copy (3 * hidden * inter * 2), or 0 if unsupported. */
+size_t wide_ffn_packed_bytes(int64_t hidden, int64_t inter);
+
+/* Writes the packed copy of W_gate, W_up [inter][hidden] and W_down
+ * [hidden][inter] (device, bf16, 16-byte aligned) into d_packed (device,
+ * >= wide_ffn_packed_bytes, 256-byte aligned).  Enqueued on `stream`. */
+int wide_ffn_pack(const void *d_w_gate, const void *d_w_up, const void *d_w_down, int64_t hidden,
+                  int64_t inter, void *d_packed, size_t packed_bytes, void *stream);
+
+/* The masked FFN of wide_ffn_masked, decode path, reading the packed copy:
+ * the tensor-core kernel in launches of up to 32 tokens (any token count).
+ * bf16 only; d->path WIDE_PATH_AUTO or WIDE_PATH_DECODE (PREFILL:
+ * WIDE_EUNSUPPORTED); group size a multiple of 16 up to 256; the same
+ * workspace as wide_ffn_masked's decode path (wide_ffn_workspace_bytes with
+ * path WIDE_PATH_DECODE).  Atomics order the fp32 sums differently from
+ * call to call (see WIDE_DECODE_TC). */
+int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const uint32_t *d_group_mask,
+                           void *d_out, const wide_ffn_dims *d, void *d_workspace,
+                           size_t workspace_bytes, void *stream);
 
 /* --------------------------------------------------- masked attention / layer
  *
@@ -259,9 +307,20 @@ int wide_set_decode_ffn_path(int mode);
  * already hold (post-RoPE) keys and values.  Masks: head_mask [T][W] over
  * n_kv_heads groups; ffn_mask [T][W] over inter / ffn_group_size groups.
  *
- * Supported: bf16; head_dim == 128; decode (seq_len == 1, n_seq <= 32,
- * n_q_heads / n_kv_heads in {1, 2, 4}, hidden % 512 == 0, ffn_group_size in
- * {64, 128}, cache_len < 131072).
+ * Supported: bf16; head_dim == 128; ffn_group_size in {64, 128} dividing
+ * inter; and one of two forms:
+ *   decode  (seq_len == 1): n_seq <= 32, n_q_heads / n_kv_heads in
+ *           {1, 2, 4}, n_kv_heads <= 1024, hidden % 512 == 0,
+ *           cache_len < 131072, cache_cap >= cache_len + 1;
+ *   prefill (seq_len >= 1 with cache_len == 0, i.e. no earlier context):
+ *           n_kv_heads even, 2..1024, n_q_heads / n_kv_heads in {2, 4},
+ *           hidden % 256 == 0, inter / ffn_group_size <= 1024,
+ *           cache_cap >= seq_len, n_seq * seq_len <= 2^24 and
+ *           n_kv_heads * n_seq * seq_len <= 2^22.
+ * Dims that both forms accept (seq_len == 1, cache_len == 0) run the decode
+ * form.  Anything else
+ * (a prefill chunk after cached context, other head ratios) returns
+ * WIDE_EUNSUPPORTED.
  */
 typedef struct wide_layer_dims {
     int64_t n_seq;           /* sequences */
@@ -279,6 +338,9 @@ typedef struct wide_layer_dims {
 typedef struct wide_layer_weights {
     const void *gamma1, *wq, *wk, *wv, *wo;       /* attention half (device) */
     const void *gamma2, *w_gate, *w_up, *w_down;  /* FFN half (device) */
+    const void *ffn_packed;   /* optional wide_ffn_pack copy of the FFN weights
+                                 (NULL: none); the decode layer's FFN reads it
+                                 where the tensor-core kernel takes the shape */
 } wide_layer_weights;
 
 /* Device workspace bytes for wide_layer_masked / wide_attn_masked (0 on

@@ -47,7 +47,7 @@ def test_constants_match_header(native):
 
 def test_version_and_status_strings(native):
     L = native.lib()
-    assert L.wide_abi_version() == 2
+    assert L.wide_abi_version() == 3
     for code in (0, -1, -2, -3, -4, 1, 2, 4):
         assert L.wide_status_string(code)
 
@@ -138,6 +138,35 @@ def test_ffn_worklist_argument_checks(native):
                              None) == native.WIDE_EINVAL
 
 
+def test_packed_weight_entry_points_check_on_the_host(native):
+    """The packed decode layout: its size, and the argument checks of
+    wide_ffn_pack and wide_ffn_masked_packed, all answered before anything
+    is enqueued (no GPU needed)."""
+    L = native.lib()
+    assert L.wide_ffn_packed_bytes(3072, 8192) == 3 * 3072 * 8192 * 2
+    assert L.wide_ffn_packed_bytes(3072 + 64, 8192) == 0      # hidden % 128
+    assert L.wide_ffn_packed_bytes(3072, 8192 + 32) == 0      # inter % 64
+    assert L.wide_ffn_packed_bytes(0, 8192) == 0
+    p = ctypes.c_void_p(1 << 20)
+    need = L.wide_ffn_packed_bytes(256, 512)
+    assert L.wide_ffn_pack(None, p, p, 256, 512, p, need, None) == native.WIDE_EINVAL
+    assert L.wide_ffn_pack(p, p, p, 256, 512 + 32, p, need, None) == native.WIDE_EUNSUPPORTED
+    assert L.wide_ffn_pack(p, p, p, 256, 512, p, need - 1, None) == native.WIDE_EWORKSPACE
+    assert L.wide_ffn_pack(p, p, p, 256, 512, ctypes.c_void_p((1 << 20) + 16), need,
+                           None) == native.WIDE_EUNSUPPORTED       # packed not 256-aligned
+    D = native.WideFFNDims
+    d = D(8, 256, 512, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)
+    assert L.wide_ffn_masked_packed(None, p, p, p, ctypes.byref(d), p, 1 << 30,
+                                    None) == native.WIDE_EINVAL
+    for bad in (D(8, 256, 512, 128, native.WIDE_BF16, native.WIDE_PATH_PREFILL),
+                D(8, 256, 512, 128, native.WIDE_F32, native.WIDE_PATH_DECODE),
+                D(8, 256 + 64, 512, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)):
+        assert L.wide_ffn_masked_packed(p, p, p, p, ctypes.byref(bad), p, 1 << 30,
+                                        None) == native.WIDE_EUNSUPPORTED
+    z = D(0, 256, 512, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)
+    assert L.wide_ffn_masked_packed(p, p, p, p, ctypes.byref(z), p, 0, None) == native.WIDE_OK
+
+
 def test_binding_refuses_operands_on_two_devices():
     """The binding launches on the operands' device and refuses operands on
     different devices (or off the GPU) before any C call."""
@@ -165,6 +194,8 @@ def test_decode_path_switch_is_host_only(native):
     prev = L.wide_set_decode_ffn_path(1)
     try:
         assert L.wide_set_decode_ffn_path(2) == 1
+        assert L.wide_set_decode_ffn_path(3) == 2
+        assert L.wide_set_decode_ffn_path(2) == 3
         assert L.wide_set_decode_ffn_path(7) == -1
         assert L.wide_set_decode_ffn_path(-1) == -1
         assert L.wide_set_decode_ffn_path(0) == 2

@@ -31,6 +31,23 @@ def test_reference_arm_line(workload):
                         "d2h_bytes_per_step": 0}
 
 
+def test_cpu_baseline_on_all_threads_and_on_one():
+    """The CPU leg times the oracle twice on the same sample: with every
+    host thread (the decode sample is one oracle call of as many tokens as
+    threads, so the token loop has work for each) and capped at one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    wl = bench.WORKLOADS["decode_ffn_3b"]
+    cases = wl.make_cases()
+    samples, _ = wl.reference_sample(cases)
+    assert len(samples) == 1 and samples[0].T == min(32, bench._host_cores())
+    rec = bench.cpu_baseline_record(wl, cases, 0.01)
+    assert rec["kind"] == "oracle" and rec["cores"] == bench._host_cores() and rec["value"] > 0
+    assert rec["one_core"]["cores"] == 1 and rec["one_core"]["value"] > 0
+    # the cap is lifted again afterwards
+    assert bench._host_cores() == rec["cores"]
+
+
 def test_router_units():
     """Algorithmic bytes of one router call: x, W_r1 and W_r2 read once,
     the packed mask words written once; the kernel name follows the size

@@ -14,15 +14,17 @@ TOL_BF16 = 5e-3   # relative L2, bf16 storage / fp32 accumulation
 TOL_F32 = 1e-5    # relative L2, fp32 tiny configuration
 
 
-@pytest.fixture(params=["auto", "fused", "gemv"], autouse=True)
+@pytest.fixture(params=["auto", "tc", "fused", "gemv"], autouse=True)
 def decode_kernels(request):
-    """Every case runs on the dispatcher's choice and on each of the two
-    bf16 decode implementations forced: the persistent channel-split kernel
-    wherever its limits allow (1..32 tokens per launch, hidden % 256 == 0),
-    and the two GEMV kernels.  bf16 group size 32 exists on the channel-
-    split kernel only and runs there in every mode."""
+    """Every case runs on the dispatcher's choice and on each bf16 decode
+    implementation forced: the tensor-core kernel (launches of up to 32
+    tokens, hidden % 128 == 0, group size a multiple of 16), the channel-
+    split CUDA-core kernel (launches of up to 16 tokens, hidden % 256 ==
+    0) and the two GEMV kernels, each wherever its limits allow (else the
+    dispatcher's next choice).  bf16 group size 32 has no GEMV kernel and
+    runs on a persistent kernel in every mode."""
     import token_level_dynamic_b200 as w
-    mode = {"auto": w.WIDE_DECODE_AUTO, "fused": w.WIDE_DECODE_FUSED,
+    mode = {"auto": w.WIDE_DECODE_AUTO, "tc": w.WIDE_DECODE_TC, "fused": w.WIDE_DECODE_FUSED,
             "gemv": w.WIDE_DECODE_GEMV}[request.param]
     prev = w.wide_set_decode_ffn_path(mode)
     yield request.param
@@ -91,16 +93,22 @@ def test_single_token_single_group():
 
 
 def test_repeatable(decode_kernels):
-    """The GEMV kernels are bitwise repeatable.  The channel-split kernel
-    adds its CTAs' fp32 partial sums with atomics, in an order that varies
-    from call to call, so two calls agree to within one bf16 rounding step
-    per element."""
+    """The GEMV kernels are bitwise repeatable.  The persistent kernels add
+    their CTAs' fp32 partial sums with atomics, in an order that varies from
+    call to call, so two calls agree to within one bf16 rounding step of the
+    element plus the fp32 summation noise (an element whose terms nearly
+    cancel can land on either side of a bf16 step of its own small size):
+    1e-5 of the output's rms, far below any real error."""
     c = synth.decode_ffn(8)
     a, b = _run(c), _run(c)
     if decode_kernels == "gemv":
         np.testing.assert_array_equal(a, b)
     else:
-        assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)))
+        rms = float(np.sqrt(np.mean(a.astype(np.float64) ** 2)))
+        lim = 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 1e-5 * rms
+        bad = np.abs(a - b) > lim
+        i = np.unravel_index(np.argmax(np.abs(a - b) - lim), a.shape)
+        assert not bad.any(), (int(bad.sum()), i, float(a[i]), float(b[i]), rms)
 
 
 @pytest.mark.parametrize("T", [9, 17, 24, 31])

@@ -143,7 +143,7 @@ def wide_launch_count() -> int:
     return int(_L.wide_launch_count())
 
 
-WIDE_DECODE_AUTO, WIDE_DECODE_FUSED, WIDE_DECODE_GEMV = 0, 1, 2
+WIDE_DECODE_AUTO, WIDE_DECODE_FUSED, WIDE_DECODE_GEMV, WIDE_DECODE_TC = 0, 1, 2, 3
 
 
 def wide_set_decode_ffn_path(mode: int) -> int:
@@ -293,9 +293,68 @@ def wide_ffn_masked_noalloc(x: torch.Tensor, w_gate: torch.Tensor, w_up: torch.T
     return out
 
 
+def wide_ffn_packed_bytes(hidden: int, inter: int) -> int:
+    return int(_L.wide_ffn_packed_bytes(hidden, inter))
+
+
+def wide_ffn_pack(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor,
+                  packed: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """The decode kernel's packed copy of W_gate, W_up [I][H] and W_down
+    [H][I] (bf16) as a uint8 device tensor of wide_ffn_packed_bytes(H, I)."""
+    I, H = w_gate.shape
+    for name, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} is {t.dtype}; the packed layout is bf16")
+    if tuple(w_up.shape) != (I, H) or tuple(w_down.shape) != (H, I):
+        raise ValueError(f"weights {tuple(w_gate.shape)}, {tuple(w_up.shape)}, "
+                         f"{tuple(w_down.shape)}: expected W_gate, W_up [I][H], W_down [H][I]")
+    dev = _one_device("wide_ffn_pack", w_gate=w_gate, w_up=w_up, w_down=w_down, packed=packed)
+    need = wide_ffn_packed_bytes(H, I)
+    if need == 0:
+        raise WideError("wide_ffn_pack", WIDE_EUNSUPPORTED)
+    if packed is None:
+        packed = torch.empty(need, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("wide_ffn_pack", _L.wide_ffn_pack(
+            _dev_ptr(w_gate, "w_gate"), _dev_ptr(w_up, "w_up"), _dev_ptr(w_down, "w_down"), H, I,
+            _dev_ptr(packed, "packed"), packed.numel(), _stream(stream, dev)))
+    return packed
+
+
+def wide_ffn_masked_packed(x: torch.Tensor, packed: torch.Tensor, mask_words: torch.Tensor,
+                           group_size: int, inter: int, out: torch.Tensor = None,
+                           workspace: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """The decode-path masked FFN on a wide_ffn_pack copy of the weights."""
+    T, H = x.shape
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"x is {x.dtype}; the packed decode FFN is bf16")
+    if packed.dtype != torch.uint8 or packed.numel() < wide_ffn_packed_bytes(H, inter):
+        raise ValueError("packed must be the uint8 tensor wide_ffn_pack returned for these sizes")
+    if group_size > 0 and inter % group_size == 0:
+        W = (inter // group_size + 31) // 32
+        if mask_words.dtype != torch.int32 or tuple(mask_words.shape) != (T, W):
+            raise ValueError(f"mask_words must be int32 [{T}][{W}], got {mask_words.dtype} "
+                             f"{tuple(mask_words.shape)}")
+    dev = _one_device("wide_ffn_masked_packed", x=x, packed=packed, mask_words=mask_words, out=out,
+                      workspace=workspace)
+    d = WideFFNDims(T, H, inter, group_size, WIDE_BF16, WIDE_PATH_DECODE)
+    if out is None:
+        out = torch.empty_like(x)
+    need = int(_L.wide_ffn_workspace_bytes(ctypes.byref(d)))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("wide_ffn_masked_packed", _L.wide_ffn_masked_packed(
+            _dev_ptr(x, "x"), _dev_ptr(packed, "packed"), _dev_ptr(mask_words, "mask_words"),
+            _dev_ptr(out, "out"), ctypes.byref(d), workspace.data_ptr(), workspace.numel(),
+            _stream(stream, dev)))
+    return out
+
+
 # ----------------------------------------------------------- masked layer
 
-LAYER_WEIGHT_NAMES = ("gamma1", "wq", "wk", "wv", "wo", "gamma2", "w_gate", "w_up", "w_down")
+LAYER_WEIGHT_NAMES = ("gamma1", "wq", "wk", "wv", "wo", "gamma2", "w_gate", "w_up", "w_down",
+                      "ffn_packed")
 
 
 def wide_layer_dims(n_seq: int, seq_len: int, cache_len: int, cache_cap: int, hidden: int,
@@ -324,7 +383,9 @@ def wide_layer_masked(x: torch.Tensor, weights: dict, k_cache: torch.Tensor,
                       ffn_out: torch.Tensor = None, workspace: torch.Tensor = None,
                       stream=None) -> torch.Tensor:
     """The masked layer (pre-norm block); appends K/V to the caches.
-    weights: dict with gamma1, wq, wk, wv, wo, gamma2, w_gate, w_up, w_down."""
+    weights: dict with gamma1, wq, wk, wv, wo, gamma2, w_gate, w_up, w_down,
+    and optionally ffn_packed (wide_ffn_pack of the FFN weights), which the
+    decode layer's FFN then reads."""
     dev = _one_device("wide_layer_masked", x=x, k_cache=k_cache, v_cache=v_cache,
                       head_mask=head_mask, ffn_mask=ffn_mask, out=out, attn_out=attn_out,
                       ffn_out=ffn_out, workspace=workspace,

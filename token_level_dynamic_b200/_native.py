@@ -56,7 +56,7 @@ class WideLayerDims(ctypes.Structure):
 
 class WideLayerWeights(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in ("gamma1", "wq", "wk", "wv", "wo",
-                                        "gamma2", "w_gate", "w_up", "w_down")]
+                                        "gamma2", "w_gate", "w_up", "w_down", "ffn_packed")]
 
 
 class WideRouterDims(ctypes.Structure):
@@ -86,6 +86,11 @@ SIGNATURES = {
     "wide_ffn_masked": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 ctypes.POINTER(WideFFNDims), ctypes.POINTER(WideWorklist),
                                 c_void_p, c_size_t, c_void_p]),
+    "wide_ffn_packed_bytes": (c_size_t, [c_int64, c_int64]),
+    "wide_ffn_pack": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_size_t,
+                              c_void_p]),
+    "wide_ffn_masked_packed": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p,
+                                       ctypes.POINTER(WideFFNDims), c_void_p, c_size_t, c_void_p]),
     "wide_ffn_masked_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, ctypes.POINTER(WideFFNDims), c_void_p]),
     "wide_layer_workspace_bytes": (c_size_t, [ctypes.POINTER(WideLayerDims)]),

@@ -130,6 +130,69 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
     return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_swz(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                      uint64_t pitch_elems, uint32_t box_rows, uint32_t box_cols,
+                      uint32_t swizzle_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || rows == 0 || cols == 0 || box_cols * 2 > (swizzle_bytes ? swizzle_bytes : 512))
+        return false;
+    const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                        : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch_elems * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d_swz(CUtensorMap *map, const void *base, const uint64_t (&dims)[3],
+                      const uint64_t (&strides)[2], const uint32_t (&box)[3],
+                      uint32_t swizzle_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || box[0] * 2 > (swizzle_bytes ? swizzle_bytes : 512))
+        return false;
+    const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                        : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    const cuuint64_t st[2] = {strides[0], strides[1]};
+    const cuuint32_t b[3] = {box[0], box[1], box[2]};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), d,
+                          st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_4d_swz(CUtensorMap *map, const void *base, const uint64_t (&dims)[4],
+                      const uint64_t (&strides)[3], const uint32_t (&box)[4],
+                      uint32_t swizzle_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || box[0] * 2 > (swizzle_bytes ? swizzle_bytes : 512))
+        return false;
+    const CUtensorMapSwizzle sw = swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                  : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                        : CU_TENSOR_MAP_SWIZZLE_NONE;
+    const cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+    const cuuint64_t st[3] = {strides[0], strides[1], strides[2]};
+    const cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), d,
+                          st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                       uint64_t pitch_elems, uint32_t box_chunks, uint32_t box_rows)
 {
@@ -287,11 +350,13 @@ bool ffn_shape_supported(const wide_ffn_dims *d, int path)
     if (path == WIDE_PATH_DECODE) {
         if (d->dtype != WIDE_BF16)
             return gs == 32 || gs == 64 || gs == 128;
-        // bf16 group size 32 runs on the channel-split kernel only
+        // bf16 group size 32 runs on the persistent kernels only
         const int T1 = (int)(d->tokens < kSplitMaxTok ? (d->tokens > 0 ? d->tokens : 1)
                                                       : kSplitMaxTok);
+        const int H = (int)d->hidden, I = (int)d->inter;
         return gs == 64 || gs == 128 ||
-               (gs == 32 && decode_ffn_split_supported(T1, (int)d->hidden, (int)d->inter, 32));
+               (gs == 32 && (decode_ffn_split_supported(T1, H, I, 32) ||
+                             decode_ffn_tc_supported(T1, H, I, 32)));
     }
     // prefill: tcgen05 kernels with 128-channel groups and 256-column output blocks
     return d->dtype == WIDE_BF16 && (gs == 64 || gs == 128) && d->hidden % 256 == 0 &&
@@ -437,6 +502,61 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
                               d_workspace, s);
 }
 
+size_t wide_ffn_packed_bytes(int64_t hidden, int64_t inter)
+{
+    return ffn_packed_bytes(hidden, inter);
+}
+
+int wide_ffn_pack(const void *d_w_gate, const void *d_w_up, const void *d_w_down, int64_t hidden,
+                  int64_t inter, void *d_packed, size_t packed_bytes, void *stream)
+{
+    if (!d_w_gate || !d_w_up || !d_w_down || !d_packed || hidden <= 0 || inter <= 0)
+        return WIDE_EINVAL;
+    const size_t need = ffn_packed_bytes(hidden, inter);
+    if (need == 0 || hidden > (1 << 20) || inter > (1 << 22))
+        return WIDE_EUNSUPPORTED;
+    if (packed_bytes < need)
+        return WIDE_EWORKSPACE;
+    if (!aligned16(d_w_gate) || !aligned16(d_w_up) || !aligned16(d_w_down) ||
+        (reinterpret_cast<uintptr_t>(d_packed) & 255u) != 0)
+        return WIDE_EUNSUPPORTED;
+    return ffn_pack_launch(d_w_gate, d_w_up, d_w_down, hidden, inter, d_packed,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const uint32_t *d_group_mask,
+                           void *d_out, const wide_ffn_dims *d, void *d_workspace,
+                           size_t workspace_bytes, void *stream)
+{
+    if (!ffn_dims_ok(d))
+        return WIDE_EINVAL;
+    if (d->tokens == 0)
+        return WIDE_OK;
+    if (!d_x || !d_packed || !d_group_mask || !d_out || !d_workspace)
+        return WIDE_EINVAL;
+    if (d->dtype != WIDE_BF16 || d->path == WIDE_PATH_PREFILL ||
+        ffn_packed_bytes(d->hidden, d->inter) == 0 || d->hidden > (1 << 20) ||
+        d->inter > (1 << 22))
+        return WIDE_EUNSUPPORTED;
+    const int H = (int)d->hidden, I = (int)d->inter, gs = (int)d->group_size;
+    const int T1 = (int)(d->tokens < kTcMaxTok ? d->tokens : kTcMaxTok);
+    if (!decode_ffn_tc_packed_supported(T1, H, I, gs))
+        return WIDE_EUNSUPPORTED;
+    if (!aligned16(d_x) || !aligned16(d_out) || (reinterpret_cast<uintptr_t>(d_packed) & 255u) ||
+        (reinterpret_cast<uintptr_t>(d_workspace) & 255u) != 0)
+        return WIDE_EUNSUPPORTED;
+    wide_ffn_dims dd = *d;
+    dd.path = WIDE_PATH_DECODE;
+    const size_t need = wide_ffn_workspace_bytes(&dd);
+    if (workspace_bytes < need)
+        return WIDE_EWORKSPACE;
+    DownOutputs o = {};
+    o.out_sum = d_out;
+    return decode_ffn_persistent(d_x, nullptr, nullptr, nullptr, d_group_mask, o, d->tokens, H, I,
+                                 gs, d_workspace, need, static_cast<cudaStream_t>(stream),
+                                 d_packed);
+}
+
 static bool layer_dims_ok(const wide_layer_dims *d, bool ffn)
 {
     if (!d || d->n_seq < 1 || d->seq_len < 1 || d->cache_len < 0 || d->hidden <= 0 ||
@@ -511,7 +631,9 @@ int wide_layer_masked(const void *d_x, const wide_layer_weights *w, void *d_k_ca
         return WIDE_EINVAL;
     LayerPtrs p = {d_x, w->gamma1, w->wq, w->wk, w->wv, w->wo, w->gamma2, w->w_gate, w->w_up,
                    w->w_down, d_k_cache, d_v_cache, d_head_mask, d_ffn_mask, d_out, d_attn_out,
-                   d_ffn_out, true};
+                   d_ffn_out, true, w->ffn_packed};
+    if (w->ffn_packed && !aligned16(w->ffn_packed))
+        return WIDE_EUNSUPPORTED;
     return layer_call(p, d, d_workspace, workspace_bytes, stream);
 }
 
@@ -525,7 +647,7 @@ int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cac
     const wide_layer_dims a = attn_only_dims(d);
     LayerPtrs p = {d_x, w->gamma1, w->wq, w->wk, w->wv, w->wo, nullptr, nullptr, nullptr,
                    nullptr, d_k_cache, d_v_cache, d_head_mask, nullptr, nullptr, d_attn_out,
-                   nullptr, false};
+                   nullptr, false, nullptr};
     return layer_call(p, &a, d_workspace, workspace_bytes, stream);
 }
 

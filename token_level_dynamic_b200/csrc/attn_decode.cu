@@ -772,25 +772,18 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
     fo.out_sum = p.ffn_out;
     fo.res_f32 = w.h1;
     fo.out_total = p.out;
-    const int TS = T < kSplitMaxTok ? T : kSplitMaxTok;
-    if (decode_ffn_split_preferred(TS, H, I, gsf) &&
-        decode_ffn_split_scratch(TS, H) <= align_up((size_t)(T + 1) / 2 * 2 * I * 4, 256)) {
+    const size_t hcap = align_up((size_t)(T + 1) / 2 * 2 * I * 4, 256);
+    // the packed copy where the tensor-core kernel takes this shape, else
+    // the nn.Linear weights
+    const void *pk = p.ffn_packed && decode_ffn_persistent_available(T, H, I, gsf, hcap,
+                                                                     p.ffn_packed)
+                         ? p.ffn_packed
+                         : nullptr;
+    if (decode_ffn_persistent_available(T, H, I, gsf, hcap, pk)) {
         if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
             return rc;
-        const int Wf = (I / gsf + 31) / 32;
-        for (int t0 = 0; t0 < T; t0 += kSplitMaxTok) {
-            const int Tc = T - t0 < kSplitMaxTok ? T - t0 : kSplitMaxTok;
-            DownOutputs fc = {};
-            fc.out_sum = p.ffn_out ? static_cast<__nv_bfloat16 *>(p.ffn_out) + (size_t)t0 * H
-                                   : nullptr;
-            fc.res_f32 = w.h1 + (size_t)t0 * H;
-            fc.out_total = static_cast<__nv_bfloat16 *>(p.out) + (size_t)t0 * H;
-            if ((rc = decode_ffn_split(w.xn2 + (size_t)t0 * H, p.w_gate, p.w_up, p.w_down,
-                                       p.ffn_mask + (size_t)t0 * Wf, fc, Tc, H, I, gsf, w.hffn,
-                                       s)))
-                return rc;
-        }
-        return WIDE_OK;
+        return decode_ffn_persistent(w.xn2, p.w_gate, p.w_up, p.w_down, p.ffn_mask, fo, T, H, I,
+                                     gsf, w.hffn, hcap, s, pk);
     }
     if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
         return rc;

@@ -657,10 +657,13 @@ int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const
 
 size_t ffn_decode_h_bytes(const wide_ffn_dims *d)
 {
-    // h of up to 32 tokens, token pairs interleaved (an odd count rounds up)
+    // h of up to 32 tokens, token pairs interleaved (an odd count rounds
+    // up); at least the persistent kernels' fp32 [T][H] accumulator
     const int64_t T = d->tokens < kNTok ? d->tokens : kNTok;
     const int64_t Tp = T > 0 ? (T + 1) / 2 * 2 : 2;
-    return align_up((size_t)Tp * (size_t)d->inter * sizeof(float), 256);
+    const size_t T4 = (size_t)(T > 0 ? T + 3 : 4) / 4 * 4;    // the tensor-core kernel's [H][T4]
+    const size_t h = (size_t)Tp * (size_t)d->inter, acc = T4 * d->hidden;
+    return align_up((h > acc ? h : acc) * sizeof(float), 256);
 }
 
 // h scratch, then 256 bytes holding the fused kernel's grid-barrier words.
@@ -676,24 +679,10 @@ int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd
     if (d->dtype == WIDE_BF16) {
         const int H = (int)d->hidden, I = (int)d->inter;
         const int64_t T = d->tokens;
-        const int W = (int)((I / gs + 31) / 32);
-        const int TS = (int)(T < kSplitMaxTok ? T : kSplitMaxTok);
-        // group size 32 has no GEMV kernel: the channel-split kernel runs it
-        // whatever the path mode
-        const bool split = decode_ffn_split_preferred(TS, H, I, (int)gs) ||
-                           (gs == 32 && decode_ffn_split_supported(TS, H, I, (int)gs));
-        if (split && decode_ffn_split_scratch(TS, H) <= h_cap) {
-            for (int64_t t0 = 0; t0 < T; t0 += kSplitMaxTok) {
-                const int Tc = (int)(T - t0 < kSplitMaxTok ? T - t0 : kSplitMaxTok);
-                DownOutputs o = {};
-                o.out_sum = static_cast<__nv_bfloat16 *>(out) + t0 * H;
-                const int rc = decode_ffn_split(static_cast<const __nv_bfloat16 *>(x) + t0 * H,
-                                                wg, wu, wd, mask + t0 * W, o, Tc, H, I, (int)gs,
-                                                h, s);
-                if (rc)
-                    return rc;
-            }
-            return WIDE_OK;
+        if (decode_ffn_persistent_available(T, H, I, (int)gs, h_cap)) {
+            DownOutputs o = {};
+            o.out_sum = out;
+            return decode_ffn_persistent(x, wg, wu, wd, mask, o, T, H, I, (int)gs, h, h_cap, s);
         }
         if (gs == 128)
             return decode_all<__nv_bfloat16, 128>(x, wg, wu, wd, mask, out, d, h, s);

@@ -1030,15 +1030,80 @@ bool decode_ffn_split_supported(int T, int H, int I, int gs)
 
 namespace {
 std::atomic<int> g_decode_mode{WIDE_DECODE_AUTO};
+
+// Which persistent kernel runs a bf16 decode FFN of T tokens (launches of
+// at most kTcMaxTok or kSplitMaxTok tokens) with `cap` bytes of scratch:
+// 2 the tensor-core kernel, 1 the channel-split kernel, 0 neither (the
+// GEMV kernels run).  AUTO and TC take the tensor-core kernel wherever it
+// applies (on B200 it is the fastest at every token count), FUSED the
+// channel-split kernel, GEMV neither except for group size 32, which has no
+// GEMV kernel.
+int persistent_choice(int64_t T, int H, int I, int gs, size_t cap, const void *packed)
+{
+    const int mode = g_decode_mode.load(std::memory_order_relaxed);
+    const int Ttc = (int)(T < kTcMaxTok ? T : kTcMaxTok);
+    const int Tsp = (int)(T < kSplitMaxTok ? T : kSplitMaxTok);
+    if (packed)
+        return Ttc >= 1 && decode_ffn_tc_packed_supported(Ttc, H, I, gs) &&
+                       decode_ffn_tc_scratch(Ttc, H) <= cap
+                   ? 2
+                   : 0;
+    const bool tc = Ttc >= 1 && decode_ffn_tc_supported(Ttc, H, I, gs) &&
+                    decode_ffn_tc_scratch(Ttc, H) <= cap;
+    const bool sp = Tsp >= 1 && decode_ffn_split_supported(Tsp, H, I, gs) &&
+                    decode_ffn_split_scratch(Tsp, H) <= cap;
+    if (mode == WIDE_DECODE_FUSED)
+        return sp ? 1 : tc && gs == 32 ? 2 : 0;
+    if (mode == WIDE_DECODE_GEMV && gs != 32)
+        return 0;
+    if (mode == WIDE_DECODE_TC)
+        return tc ? 2 : sp ? 1 : 0;
+    // AUTO on nn.Linear weights: the channel-split kernel up to 8 tokens per
+    // launch (there it streams the row-strided tiles faster), the tensor-core
+    // kernel above
+    if (sp && T <= 8)
+        return 1;
+    return tc ? 2 : sp ? 1 : 0;
+}
+}  // namespace
+
+bool decode_ffn_persistent_available(int64_t T, int H, int I, int gs, size_t cap,
+                                     const void *packed)
+{
+    return persistent_choice(T, H, I, gs, cap, packed) != 0;
 }
 
-// AUTO takes the channel-split kernel wherever its shape limits allow (on
-// B200 it is at least as fast as the two GEMV kernels at every token count).
-bool decode_ffn_split_preferred(int T, int H, int I, int gs)
+int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const void *wd,
+                          const uint32_t *mask, const DownOutputs &o, int64_t T, int H, int I,
+                          int gs, void *scratch, size_t cap, cudaStream_t s, const void *packed)
 {
-    if (g_decode_mode.load(std::memory_order_relaxed) == WIDE_DECODE_GEMV)
-        return false;
-    return decode_ffn_split_supported(T, H, I, gs);
+    const int which = persistent_choice(T, H, I, gs, cap, packed);
+    if (which == 0)
+        return WIDE_EUNSUPPORTED;
+    const int per = which == 2 ? kTcMaxTok : kSplitMaxTok;
+    const int W = (I / gs + 31) / 32;
+    auto at = [](const void *p, int64_t off, size_t elem) -> const char * {
+        return p ? static_cast<const char *>(p) + off * (int64_t)elem : nullptr;
+    };
+    for (int64_t t0 = 0; t0 < T; t0 += per) {
+        const int Tc = (int)(T - t0 < per ? T - t0 : per);
+        const int64_t e = t0 * H;
+        DownOutputs c = {};
+        c.out_sum = const_cast<char *>(at(o.out_sum, e, 2));
+        c.res_in = at(o.res_in, e, 2);
+        c.res_f32 = reinterpret_cast<const float *>(at(o.res_f32, e, 4));
+        c.out_total = const_cast<char *>(at(o.out_total, e, 2));
+        c.out_total_f32 = reinterpret_cast<float *>(const_cast<char *>(at(o.out_total_f32, e, 4)));
+        const void *xc = at(x, e, 2);
+        const int rc = which == 2
+                           ? decode_ffn_tc(xc, wg, wu, wd, packed, mask + t0 * W, c, Tc, H, I, gs,
+                                           scratch, s)
+                           : decode_ffn_split(xc, wg, wu, wd, mask + t0 * W, c, Tc, H, I, gs,
+                                             scratch, s);
+        if (rc)
+            return rc;
+    }
+    return WIDE_OK;
 }
 
 int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *wd,
@@ -1098,7 +1163,8 @@ int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *
 
 extern "C" int wide_set_decode_ffn_path(int mode)
 {
-    if (mode != WIDE_DECODE_AUTO && mode != WIDE_DECODE_FUSED && mode != WIDE_DECODE_GEMV)
+    if (mode != WIDE_DECODE_AUTO && mode != WIDE_DECODE_FUSED && mode != WIDE_DECODE_GEMV &&
+        mode != WIDE_DECODE_TC)
         return WIDE_EINVAL;
     return wide::g_decode_mode.exchange(mode);
 }

@@ -46,6 +46,23 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t co
 // consecutive elements each, landing as [box_rows][64 * box_chunks] in shared
 // memory (no swizzle).  Long rows per copy stream better than 2-D boxes of
 // short rows.
+// As make_tmap_2d for bf16, with the shared-memory swizzle of the given
+// width in bytes (0, 32, 64 or 128; the box's row must not be wider).
+bool make_tmap_2d_swz(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
+                      uint64_t pitch_elems, uint32_t box_rows, uint32_t box_cols,
+                      uint32_t swizzle_bytes);
+
+// A bf16 3-D tensor (dims innermost first, byte strides of dims 1 and 2 in
+// any order) with the given shared-memory swizzle (0, 32, 64 or 128 bytes).
+bool make_tmap_3d_swz(CUtensorMap *map, const void *base, const uint64_t (&dims)[3],
+                      const uint64_t (&strides)[2], const uint32_t (&box)[3],
+                      uint32_t swizzle_bytes);
+
+// The same for a 4-D tensor (byte strides of dims 1..3).
+bool make_tmap_4d_swz(CUtensorMap *map, const void *base, const uint64_t (&dims)[4],
+                      const uint64_t (&strides)[3], const uint32_t (&box)[4],
+                      uint32_t swizzle_bytes);
+
 bool make_tmap_rows3d(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
                       uint64_t pitch_elems, uint32_t box_chunks, uint32_t box_rows);
 
@@ -98,6 +115,8 @@ enum KernelId : int32_t {
     KID_ROUTER = 16,
     KID_ROUTER_SMALL = 17,
     KID_DECODE_FFN_SPLIT = 18,
+    KID_DECODE_FFN_TC = 19,
+    KID_FFN_PACK = 20,
 };
 
 // Pointers of one masked-layer call (FFN pointers unused when !ffn).
@@ -107,6 +126,7 @@ struct LayerPtrs {
     const uint32_t *head_mask, *ffn_mask;
     void *out, *attn_out, *ffn_out;
     bool ffn;
+    const void *ffn_packed;   // wide_ffn_pack copy of the FFN weights, or NULL
 };
 
 // Brackets one kernel launch: counts it and, while profiling is on, records
@@ -242,12 +262,39 @@ int decode_down_bf16(const void *wd, const float *h, const uint32_t *mask, const
 constexpr int kSplitMaxTok = 16;   // tokens per launch of the split kernel
 size_t decode_ffn_split_scratch(int T, int H);
 bool decode_ffn_split_supported(int T, int H, int I, int gs);
-// Whether the decode path should use it for this shape (the
-// wide_set_decode_ffn_path mode allows it and the shape fits).
-bool decode_ffn_split_preferred(int T, int H, int I, int gs);
 int decode_ffn_split(const void *x, const void *wg, const void *wu, const void *wd,
                      const uint32_t *mask, const DownOutputs &o, int T, int H, int I, int gs,
                      void *scratch, cudaStream_t s);
+// bf16 decode FFN of 1 <= T <= kTcMaxTok tokens on the tensor cores, one
+// persistent cooperative kernel (ffn_decode_tc.cu); arguments and scratch
+// as for decode_ffn_split.
+constexpr int kTcMaxTok = 32;
+size_t decode_ffn_tc_scratch(int T, int H);
+bool decode_ffn_tc_supported(int T, int H, int I, int gs);
+// `packed` (the wide_ffn_pack layout; NULL: the nn.Linear weights wg, wu,
+// wd) selects where the weights are read from.
+int decode_ffn_tc(const void *x, const void *wg, const void *wu, const void *wd,
+                  const void *packed, const uint32_t *mask, const DownOutputs &o, int T, int H,
+                  int I, int gs, void *scratch, cudaStream_t s);
+bool decode_ffn_tc_packed_supported(int T, int H, int I, int gs);
+// Packed decode weights (ffn_pack.cu): W_gate and W_up in 64-row panels,
+// each panel K-step-major ([I/64][H/64][64][64]), then W_down in 16-channel
+// column panels ([I/16][H][16]); 3 * I * H bf16 in all.
+size_t ffn_packed_bytes(int64_t H, int64_t I);
+int ffn_pack_launch(const void *wg, const void *wu, const void *wd, int64_t H, int64_t I,
+                    void *packed, cudaStream_t s);
+// The bf16 decode FFN of any T >= 1 on whichever persistent kernel the
+// wide_set_decode_ffn_path mode and the shape allow, in launches of up to 32
+// (tensor-core kernel) or 16 (channel-split kernel) tokens, with `cap` bytes
+// of scratch.  WIDE_EUNSUPPORTED, with nothing enqueued, when neither
+// applies: the caller then runs the GEMV kernels.
+// With `packed` non-NULL only the tensor-core kernel applies (any mode).
+bool decode_ffn_persistent_available(int64_t T, int H, int I, int gs, size_t cap,
+                                     const void *packed = nullptr);
+int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const void *wd,
+                          const uint32_t *mask, const DownOutputs &o, int64_t T, int H, int I,
+                          int gs, void *scratch, size_t cap, cudaStream_t s,
+                          const void *packed = nullptr);
 // Bytes of the fp32 h scratch of the decode path (tokens capped at 32).
 size_t ffn_decode_h_bytes(const wide_ffn_dims *d);
 // Runs the decode path with h scratch (h_cap contiguous bytes at h, at

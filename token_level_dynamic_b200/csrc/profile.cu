@@ -127,6 +127,10 @@ const char *wide_kernel_name(int32_t id)
         return "router_small_gemv";
     case KID_DECODE_FFN_SPLIT:
         return "decode_ffn_split_gemv";
+    case KID_DECODE_FFN_TC:
+        return "decode_ffn_tcgen05";
+    case KID_FFN_PACK:
+        return "ffn_pack";
     default:
         return "?";
     }
