@@ -182,6 +182,11 @@ class FFNDevice:
         self.ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         self.ones = [_all_ones(m, base.I // base.gs) for m in self.ms]
         self.ncalls = len(cases)
+        # decode: the weights' packed copy, made once like loading the weights
+        # (outside every timed region); each call then hands the library
+        # both copies and it picks the kernel per launch
+        self.packed = (w.wide_ffn_pack(self.Wg, self.Wu, self.Wd)
+                       if self.path == w.WIDE_PATH_DECODE else None)
         # e2e: pinned host copies of each call's inputs and output
         self.xh = [x.cpu().pin_memory() for x in self.xs]
         self.mh = [m.cpu().pin_memory() for m in self.ms]
@@ -190,8 +195,13 @@ class FFNDevice:
         self.d2h_bytes = int(sum(o.numel() * 2 for o in self.oh))
 
     def call(self, i, all_kept=False):
-        self.w.wide_ffn_masked(self.xs[i], self.Wg, self.Wu, self.Wd,
-                               self.ones[i] if all_kept else self.ms[i], self.cases[i].gs,
+        m = self.ones[i] if all_kept else self.ms[i]
+        if self.packed is not None:
+            self.w.wide_ffn_masked_packed(self.xs[i], self.packed, m, self.cases[i].gs,
+                                          self.cases[i].I, out=self.outs[i], workspace=self.ws,
+                                          stream=self.stream, weights=(self.Wg, self.Wu, self.Wd))
+            return
+        self.w.wide_ffn_masked(self.xs[i], self.Wg, self.Wu, self.Wd, m, self.cases[i].gs,
                                out=self.outs[i], workspace=self.ws, path=self.path,
                                stream=self.stream)
 
@@ -241,7 +251,9 @@ class DecodeFFN3B:
     name = "decode_ffn_3b"
     desc = ("decode_ffn_3b: Llama-3.2-3B-shaped masked SwiGLU FFN decode, hidden 3072, "
             "intermediate 8192 = 64 groups x 128, bf16, Bernoulli(0.5) masks; one step = "
-            "batches 1, 8 and 32 (41 tokens)")
+            "batches 1, 8 and 32 (41 tokens); weights also packed once (wide_ffn_pack, outside "
+            "timing) and passed with the nn.Linear copy, so the library picks the kernel per "
+            "launch")
     bound = "hbm"
     dominant = None          # the kernel with the largest share of the step
     path_name = "WIDE_PATH_DECODE"
@@ -276,41 +288,64 @@ class DecodeFFN3B:
 
 
 def _split_decode_used(T, H, I, gs, sms=148):
-    """Mirror of the library's dispatch (plan_split in ffn_decode_split.cu):
-    the channel-split decode kernel runs launches of up to 16 tokens when
-    H % 256 == 0, the group size is a multiple of 8 in 8..256 dividing I, there
-    are at most 1024 groups (at most 8 whole groups per CTA), and its fp32
-    [T][H] accumulator plus counter fits the decode path's h scratch."""
+    """Mirror of the library's limits of the channel-split decode kernel
+    (plan_split in ffn_decode_split.cu): launches of up to 16 tokens,
+    H % 256 == 0, the group size a multiple of 8 in 8..256 dividing I, at
+    most 1024 groups (at most 8 whole groups per CTA)."""
     T1 = min(T, 16)
     if not (T1 >= 1 and H % 256 == 0 and gs % 8 == 0 and 8 <= gs <= 256 and I % gs == 0):
         return False
     G = I // gs
-    if G > 1024 or T1 * (-(-G // 32)) > 1024 or -(-G // sms) > 8:
-        return False
-    Tp = (min(T, 32) + 1) // 2 * 2
-    h_bytes = -(-(Tp * I * 4) // 256) * 256
-    acc = -(-(T1 * H * 4) // 256) * 256 + 256
-    return acc <= h_bytes
+    return not (G > 1024 or T1 * (-(-G // 32)) > 1024 or -(-G // sms) > 8)
+
+
+def _tc_decode_used(T, H, I, gs, sms=148):
+    """Mirror of the tensor-core decode kernel's limits (plan_tc in
+    ffn_decode_tc.cu): launches of up to 32 tokens, H % 128 == 0, group size
+    a multiple of 16 up to 256, at most 1024 groups and 16 chunks of 16
+    channels per CTA."""
+    G = I // gs if gs else 0
+    return (H % 128 == 0 and gs % 16 == 0 and 16 <= gs <= 256 and I % gs == 0 and G <= 1024 and
+            -(-(I // 16) // sms) <= 16)
 
 
 def _ffn_decode_bytes(case, res_bytes=0, x_bytes=None):
-    """Algorithmic bytes per kernel of one decode FFN call: every weight byte
-    of the batch's union of groups once, plus activations in and out (h of
-    the two-kernel path goes through memory; the fused kernel keeps it in
-    L2; its fp32 accumulator is not counted: it lives in L2)."""
+    """Algorithmic bytes per kernel of one decode FFN call, following the
+    library's choice per launch (AUTO): the channel-split kernel for up to 8
+    tokens, the tensor-core kernel (launches of up to 32 tokens) above.  Per
+    launch, every weight byte of that launch's union of groups once, plus
+    activations in and out; the fp32 accumulators are not counted (they live
+    in L2).  The GEMV path (neither kernel applies): h goes through memory."""
     B, H, I, gs = case.T, case.H, case.I, case.gs
     U = int(case.mask.any(axis=0).sum())
     m = case.mask_words.nbytes
     xb = B * H * 2 if x_bytes is None else x_bytes
-    if _split_decode_used(B, H, I, gs):
-        fused = 3 * U * gs * H * 2 + xb + m + B * H * 2 + res_bytes
-        return {"decode_ffn_split_gemv": fused, "total": fused, "union_groups": U}
-    pairs = int(case.mask.sum())
-    h = pairs * gs * 4
-    gateup = 2 * U * gs * H * 2 + xb + m + h
-    down = H * U * gs * 2 + h + m + B * H * 2 + res_bytes
-    return {"decode_gateup_gemv": gateup, "decode_down_gemv": down,
-            "total": gateup + down, "union_groups": U}
+    io = xb + m + B * H * 2 + res_bytes
+    split_ok, tc_ok = _split_decode_used(B, H, I, gs), _tc_decode_used(B, H, I, gs)
+    if not (split_ok or tc_ok):
+        pairs = int(case.mask.sum())
+        h = pairs * gs * 4
+        gateup = 2 * U * gs * H * 2 + xb + m + h
+        down = H * U * gs * 2 + h + m + B * H * 2 + res_bytes
+        return {"decode_gateup_gemv": gateup, "decode_down_gemv": down,
+                "total": gateup + down, "union_groups": U}
+    out, t0 = {}, 0
+    while t0 < B:
+        rem = B - t0
+        if split_ok and (rem <= 8 or not tc_ok):
+            name, per = "decode_ffn_split_gemv", 16
+        else:
+            name, per = "decode_ffn_tcgen05", 32
+        n = min(rem, per)
+        u = int(case.mask[t0:t0 + n].any(axis=0).sum())
+        out[name] = out.get(name, 0) + 3 * u * gs * H * 2
+        t0 += n
+    # activations: on the kernel of the first launch
+    first = next(iter(out))
+    out[first] += io
+    out["total"] = sum(out.values())
+    out["union_groups"] = U
+    return out
 
 
 def _ffn_oracle_step(samples):
@@ -368,6 +403,11 @@ class LayerDevice:
         self.lc = lc
         self.x, self.wts, self.kc, self.vc, self.hm, self.fm, cap = layer_to_dev(lc, device=dev)
         a, f = lc.attn, lc.ffn
+        if a.seq_len == 1:
+            # decode: the FFN weights' packed copy, made once (outside timing)
+            self.wts = dict(self.wts)
+            self.wts["ffn_packed"] = w.wide_ffn_pack(self.wts["w_gate"], self.wts["w_up"],
+                                                     self.wts["w_down"])
         self.d = w.wide_layer_dims(a.n_seq, a.seq_len, a.cache_len, cap, a.H, f.I, f.gs, a.n_q,
                                    a.n_kv, a.hd, a.theta, a.eps)
         self.out = torch.empty_like(self.x)
@@ -439,7 +479,8 @@ class DecodeLayer8B:
     desc = ("decode_layer_8b: Llama-3.1-8B-shaped masked decode layer (RMSNorm, QKV with 32 "
             "query / 8 KV heads of 128, RoPE theta 5e5, GQA attention over a 2048-entry KV "
             "cache, o_proj, RMSNorm, SwiGLU FFN 14336 = 112 groups x 128), batch 16, head "
-            "groups Bernoulli(0.34), FFN groups Bernoulli(0.72); one step = one call")
+            "groups Bernoulli(0.34), FFN groups Bernoulli(0.72); one step = one call; FFN "
+            "weights also packed once (wide_ffn_pack, outside timing) for the decode FFN")
     bound = "hbm"
     dominant = None          # the kernel with the largest share of the step
     device = LayerDevice
@@ -464,15 +505,14 @@ class DecodeLayer8B:
         attn = kept_pairs * 2 * keys * hd * 2 + kept_pairs * rep * hd * 4 * 2
         oproj = H * Ua * rep * hd * 2 + kept_pairs * rep * hd * 4 + T * H * 2 * 2 + T * H * 4
         out = {"decode_qkv_rope_gemv": qkv, "decode_attention": attn}
-        if _split_decode_used(T, H, f.I, f.gs):
-            # FFN input norm (h1 fp32 in, bf16 out), then the FFN: bf16 x and
-            # h1 in (residual), ffn_out and out back
+        ffn = _ffn_decode_bytes(f, res_bytes=T * H * 4 + T * H * 2)
+        if "decode_down_gemv" not in ffn:
+            # FFN input norm (h1 fp32 in, bf16 out), then one persistent FFN
+            # kernel: bf16 x and h1 in (residual), ffn_out and out back
             out["rmsnorm"] = T * H * 4 + T * H * 2 + H * 2
-            ffn = _ffn_decode_bytes(f, res_bytes=T * H * 4 + T * H * 2)
             out["decode_down_gemv"] = oproj
         else:
             norm = T * H * 4 + T * H * 2 + H * 2
-            ffn = _ffn_decode_bytes(f, res_bytes=T * H * 4 + T * H * 2)
             out["rmsnorm"] = norm
             out["decode_down_gemv"] = oproj + ffn.pop("decode_down_gemv")
         for k, v in ffn.items():

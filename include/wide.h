@@ -220,8 +220,9 @@ int wide_ffn_masked(const void *d_x, const void *d_w_gate, const void *d_w_up,
 
 /* Kernels of the bf16 decode FFN (process-wide; the decode layer's FFN
  * follows it too).  All compute the same sums, in a different fp32 order:
- *   WIDE_DECODE_AUTO   the channel-split kernel for up to 8 tokens, the
- *                      tensor-core kernel above, each where its shape
+ *   WIDE_DECODE_AUTO   the channel-split kernel for up to 8 tokens per
+ *                      launch, the tensor-core kernel above (on a packed
+ *                      copy where the call has one), each where its shape
  *                      limits allow, else the GEMVs (default)
  *   WIDE_DECODE_TC     the tensor-core kernel: one persistent kernel per launch of
  *                      up to 32 tokens (hidden % 128 == 0, group size a
@@ -277,14 +278,20 @@ size_t wide_ffn_packed_bytes(int64_t hidden, int64_t inter);
 int wide_ffn_pack(const void *d_w_gate, const void *d_w_up, const void *d_w_down, int64_t hidden,
                   int64_t inter, void *d_packed, size_t packed_bytes, void *stream);
 
-/* The masked FFN of wide_ffn_masked, decode path, reading the packed copy:
- * the tensor-core kernel in launches of up to 32 tokens (any token count).
- * bf16 only; d->path WIDE_PATH_AUTO or WIDE_PATH_DECODE (PREFILL:
+/* The masked FFN of wide_ffn_masked, decode path, reading the packed copy
+ * in the tensor-core kernel (launches of up to 32 tokens, any token count).
+ * d_w_gate, d_w_up, d_w_down: the nn.Linear weights as well (all three) or
+ * NULL (all three).  With them the call picks the kernel per launch as the
+ * wide_set_decode_ffn_path mode says (AUTO: the channel-split kernel for up
+ * to 8 tokens, where it is faster, the tensor-core kernel on the packed copy
+ * above); without them the tensor-core kernel runs every launch.  bf16
+ * only; d->path WIDE_PATH_AUTO or WIDE_PATH_DECODE (PREFILL:
  * WIDE_EUNSUPPORTED); group size a multiple of 16 up to 256; the same
  * workspace as wide_ffn_masked's decode path (wide_ffn_workspace_bytes with
  * path WIDE_PATH_DECODE).  Atomics order the fp32 sums differently from
  * call to call (see WIDE_DECODE_TC). */
-int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const uint32_t *d_group_mask,
+int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const void *d_w_gate,
+                           const void *d_w_up, const void *d_w_down, const uint32_t *d_group_mask,
                            void *d_out, const wide_ffn_dims *d, void *d_workspace,
                            size_t workspace_bytes, void *stream);
 

@@ -156,15 +156,19 @@ def test_packed_weight_entry_points_check_on_the_host(native):
                            None) == native.WIDE_EUNSUPPORTED       # packed not 256-aligned
     D = native.WideFFNDims
     d = D(8, 256, 512, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)
-    assert L.wide_ffn_masked_packed(None, p, p, p, ctypes.byref(d), p, 1 << 30,
+    assert L.wide_ffn_masked_packed(None, p, None, None, None, p, p, ctypes.byref(d), p, 1 << 30,
+                                    None) == native.WIDE_EINVAL
+    # the nn.Linear weights come all three or none
+    assert L.wide_ffn_masked_packed(p, p, p, None, p, p, p, ctypes.byref(d), p, 1 << 30,
                                     None) == native.WIDE_EINVAL
     for bad in (D(8, 256, 512, 128, native.WIDE_BF16, native.WIDE_PATH_PREFILL),
                 D(8, 256, 512, 128, native.WIDE_F32, native.WIDE_PATH_DECODE),
                 D(8, 256 + 64, 512, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)):
-        assert L.wide_ffn_masked_packed(p, p, p, p, ctypes.byref(bad), p, 1 << 30,
-                                        None) == native.WIDE_EUNSUPPORTED
+        assert L.wide_ffn_masked_packed(p, p, None, None, None, p, p, ctypes.byref(bad), p,
+                                        1 << 30, None) == native.WIDE_EUNSUPPORTED
     z = D(0, 256, 512, 128, native.WIDE_BF16, native.WIDE_PATH_DECODE)
-    assert L.wide_ffn_masked_packed(p, p, p, p, ctypes.byref(z), p, 0, None) == native.WIDE_OK
+    assert L.wide_ffn_masked_packed(p, p, None, None, None, p, p, ctypes.byref(z), p, 0,
+                                    None) == native.WIDE_OK
 
 
 def test_binding_refuses_operands_on_two_devices():

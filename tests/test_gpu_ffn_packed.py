@@ -158,3 +158,30 @@ def test_decode_layer_reads_the_packed_copy():
     ref, p = layer_masked(lc, ret_parts=True)
     assert rel_l2(from_dev(ffn), p["ffn_out"]) <= TOL
     assert rel_l2(from_dev(out), ref) <= TOL
+
+
+@pytest.mark.parametrize("T,kernel", [(1, "decode_ffn_split_gemv"), (8, "decode_ffn_split_gemv"),
+                                      (16, "decode_ffn_tcgen05"), (32, "decode_ffn_tcgen05"),
+                                      (40, None)])
+def test_packed_with_linear_weights_picks_per_launch(T, kernel):
+    """Given the nn.Linear weights too, the call runs the channel-split
+    kernel for up to 8 tokens per launch and the tensor-core kernel on the
+    packed copy above (40 tokens: one launch of each); the result is the
+    oracle's either way."""
+    import torch
+    import token_level_dynamic_b200 as w
+    c = synth.ffn_case(T, 3072, 8192, 128, seed=70 + T, keep=0.5)
+    x, wg, wu, wd, m = ffn_to_dev(c)
+    pk = w.wide_ffn_pack(wg, wu, wd)
+    w.wide_clear_device_status()
+    w.wide_profile_start(64)
+    out = w.wide_ffn_masked_packed(x, pk, m, c.gs, c.I, weights=(wg, wu, wd))
+    w.wide_profile_stop()
+    names = [n for n, _ in w.wide_profile_read()]
+    torch.cuda.synchronize()
+    assert w.wide_get_device_status() == 0
+    if kernel is None:
+        assert names.count("decode_ffn_tcgen05") == 1 and names.count("decode_ffn_split_gemv") == 1
+    else:
+        assert names == [kernel], names
+    assert rel_l2(from_dev(out), _ref(c)) <= TOL

@@ -323,8 +323,11 @@ def wide_ffn_pack(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor
 
 def wide_ffn_masked_packed(x: torch.Tensor, packed: torch.Tensor, mask_words: torch.Tensor,
                            group_size: int, inter: int, out: torch.Tensor = None,
-                           workspace: torch.Tensor = None, stream=None) -> torch.Tensor:
-    """The decode-path masked FFN on a wide_ffn_pack copy of the weights."""
+                           workspace: torch.Tensor = None, stream=None,
+                           weights: tuple = None) -> torch.Tensor:
+    """The decode-path masked FFN on a wide_ffn_pack copy of the weights.
+    ``weights``: optionally the nn.Linear (w_gate, w_up, w_down) as well, so
+    the library can pick the faster kernel per launch (small batches)."""
     T, H = x.shape
     if x.dtype != torch.bfloat16:
         raise TypeError(f"x is {x.dtype}; the packed decode FFN is bf16")
@@ -335,8 +338,12 @@ def wide_ffn_masked_packed(x: torch.Tensor, packed: torch.Tensor, mask_words: to
         if mask_words.dtype != torch.int32 or tuple(mask_words.shape) != (T, W):
             raise ValueError(f"mask_words must be int32 [{T}][{W}], got {mask_words.dtype} "
                              f"{tuple(mask_words.shape)}")
+    wg = wu = wd = None
+    if weights is not None:
+        wg, wu, wd = weights
+        _check_ffn(x, wg, wu, wd, mask_words, group_size, out)
     dev = _one_device("wide_ffn_masked_packed", x=x, packed=packed, mask_words=mask_words, out=out,
-                      workspace=workspace)
+                      workspace=workspace, w_gate=wg, w_up=wu, w_down=wd)
     d = WideFFNDims(T, H, inter, group_size, WIDE_BF16, WIDE_PATH_DECODE)
     if out is None:
         out = torch.empty_like(x)
@@ -344,8 +351,10 @@ def wide_ffn_masked_packed(x: torch.Tensor, packed: torch.Tensor, mask_words: to
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     with torch.cuda.device(dev):
+        lin = [None, None, None] if weights is None else \
+            [_dev_ptr(wg, "w_gate"), _dev_ptr(wu, "w_up"), _dev_ptr(wd, "w_down")]
         _check("wide_ffn_masked_packed", _L.wide_ffn_masked_packed(
-            _dev_ptr(x, "x"), _dev_ptr(packed, "packed"), _dev_ptr(mask_words, "mask_words"),
+            _dev_ptr(x, "x"), _dev_ptr(packed, "packed"), *lin, _dev_ptr(mask_words, "mask_words"),
             _dev_ptr(out, "out"), ctypes.byref(d), workspace.data_ptr(), workspace.numel(),
             _stream(stream, dev)))
     return out

@@ -89,8 +89,9 @@ SIGNATURES = {
     "wide_ffn_packed_bytes": (c_size_t, [c_int64, c_int64]),
     "wide_ffn_pack": (c_int, [c_void_p, c_void_p, c_void_p, c_int64, c_int64, c_void_p, c_size_t,
                               c_void_p]),
-    "wide_ffn_masked_packed": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p,
-                                       ctypes.POINTER(WideFFNDims), c_void_p, c_size_t, c_void_p]),
+    "wide_ffn_masked_packed": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, ctypes.POINTER(WideFFNDims), c_void_p, c_size_t,
+                                       c_void_p]),
     "wide_ffn_masked_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                         c_void_p, ctypes.POINTER(WideFFNDims), c_void_p]),
     "wide_layer_workspace_bytes": (c_size_t, [ctypes.POINTER(WideLayerDims)]),

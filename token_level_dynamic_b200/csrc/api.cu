@@ -524,7 +524,8 @@ int wide_ffn_pack(const void *d_w_gate, const void *d_w_up, const void *d_w_down
                            static_cast<cudaStream_t>(stream));
 }
 
-int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const uint32_t *d_group_mask,
+int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const void *d_w_gate,
+                           const void *d_w_up, const void *d_w_down, const uint32_t *d_group_mask,
                            void *d_out, const wide_ffn_dims *d, void *d_workspace,
                            size_t workspace_bytes, void *stream)
 {
@@ -533,6 +534,9 @@ int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const uint32_t
     if (d->tokens == 0)
         return WIDE_OK;
     if (!d_x || !d_packed || !d_group_mask || !d_out || !d_workspace)
+        return WIDE_EINVAL;
+    const bool linear = d_w_gate || d_w_up || d_w_down;
+    if (linear && (!d_w_gate || !d_w_up || !d_w_down))
         return WIDE_EINVAL;
     if (d->dtype != WIDE_BF16 || d->path == WIDE_PATH_PREFILL ||
         ffn_packed_bytes(d->hidden, d->inter) == 0 || d->hidden > (1 << 20) ||
@@ -543,18 +547,22 @@ int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const uint32_t
     if (!decode_ffn_tc_packed_supported(T1, H, I, gs))
         return WIDE_EUNSUPPORTED;
     if (!aligned16(d_x) || !aligned16(d_out) || (reinterpret_cast<uintptr_t>(d_packed) & 255u) ||
-        (reinterpret_cast<uintptr_t>(d_workspace) & 255u) != 0)
+        (reinterpret_cast<uintptr_t>(d_workspace) & 255u) != 0 ||
+        (linear && (!aligned16(d_w_gate) || !aligned16(d_w_up) || !aligned16(d_w_down))))
         return WIDE_EUNSUPPORTED;
     wide_ffn_dims dd = *d;
     dd.path = WIDE_PATH_DECODE;
     const size_t need = wide_ffn_workspace_bytes(&dd);
     if (workspace_bytes < need)
         return WIDE_EWORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (linear)   // every decode kernel is open: the dispatcher picks per launch
+        return ffn_decode_launch(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, &dd,
+                                 d_workspace, s, d_packed);
     DownOutputs o = {};
     o.out_sum = d_out;
     return decode_ffn_persistent(d_x, nullptr, nullptr, nullptr, d_group_mask, o, d->tokens, H, I,
-                                 gs, d_workspace, need, static_cast<cudaStream_t>(stream),
-                                 d_packed);
+                                 gs, d_workspace, need, s, d_packed);
 }
 
 static bool layer_dims_ok(const wide_layer_dims *d, bool ffn)

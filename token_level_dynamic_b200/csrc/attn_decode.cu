@@ -773,12 +773,8 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
     fo.res_f32 = w.h1;
     fo.out_total = p.out;
     const size_t hcap = align_up((size_t)(T + 1) / 2 * 2 * I * 4, 256);
-    // the packed copy where the tensor-core kernel takes this shape, else
-    // the nn.Linear weights
-    const void *pk = p.ffn_packed && decode_ffn_persistent_available(T, H, I, gsf, hcap,
-                                                                     p.ffn_packed)
-                         ? p.ffn_packed
-                         : nullptr;
+    // the dispatcher reads the packed copy where the tensor-core kernel runs
+    const void *pk = p.ffn_packed;
     if (decode_ffn_persistent_available(T, H, I, gsf, hcap, pk)) {
         if ((rc = rmsnorm_f32_launch(w.h1, p.gamma2, w.xn2, T, H, d->eps, s)))
             return rc;

@@ -671,7 +671,7 @@ size_t ffn_decode_workspace(const wide_ffn_dims *d) { return ffn_decode_h_bytes(
 
 int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
                    const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
-                   size_t h_cap, uint32_t *bar, cudaStream_t s)
+                   size_t h_cap, uint32_t *bar, cudaStream_t s, const void *packed)
 {
     if (d->tokens == 0)
         return WIDE_OK;
@@ -679,10 +679,11 @@ int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd
     if (d->dtype == WIDE_BF16) {
         const int H = (int)d->hidden, I = (int)d->inter;
         const int64_t T = d->tokens;
-        if (decode_ffn_persistent_available(T, H, I, (int)gs, h_cap)) {
+        if (decode_ffn_persistent_available(T, H, I, (int)gs, h_cap, packed)) {
             DownOutputs o = {};
             o.out_sum = out;
-            return decode_ffn_persistent(x, wg, wu, wd, mask, o, T, H, I, (int)gs, h, h_cap, s);
+            return decode_ffn_persistent(x, wg, wu, wd, mask, o, T, H, I, (int)gs, h, h_cap, s,
+                                         packed);
         }
         if (gs == 128)
             return decode_all<__nv_bfloat16, 128>(x, wg, wu, wd, mask, out, d, h, s);
@@ -701,14 +702,14 @@ int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd
 
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
-                      cudaStream_t s)
+                      cudaStream_t s, const void *packed)
 {
     // h, then the 256 bytes of the barrier words: ffn_decode_h_bytes + 256
     // contiguous bytes
     char *base = static_cast<char *>(ws);
     return ffn_decode_run(x, wg, wu, wd, mask, out, d, reinterpret_cast<float *>(base),
                           ffn_decode_h_bytes(d) + 256,
-                          reinterpret_cast<uint32_t *>(base + ffn_decode_h_bytes(d)), s);
+                          reinterpret_cast<uint32_t *>(base + ffn_decode_h_bytes(d)), s, packed);
 }
 
 }  // namespace wide

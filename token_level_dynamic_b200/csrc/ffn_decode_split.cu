@@ -1033,59 +1033,61 @@ std::atomic<int> g_decode_mode{WIDE_DECODE_AUTO};
 
 // Which persistent kernel runs a bf16 decode FFN of T tokens (launches of
 // at most kTcMaxTok or kSplitMaxTok tokens) with `cap` bytes of scratch:
-// 2 the tensor-core kernel, 1 the channel-split kernel, 0 neither (the
-// GEMV kernels run).  AUTO and TC take the tensor-core kernel wherever it
-// applies (on B200 it is the fastest at every token count), FUSED the
-// channel-split kernel, GEMV neither except for group size 32, which has no
-// GEMV kernel.
-int persistent_choice(int64_t T, int H, int I, int gs, size_t cap, const void *packed)
+// 3 the tensor-core kernel on the packed copy, 2 the tensor-core kernel on
+// the nn.Linear weights, 1 the channel-split kernel, 0 none (the GEMV
+// kernels run).  `linear`: the nn.Linear weights are at hand (the split and
+// GEMV kernels need them).  AUTO: the channel-split kernel for up to 8
+// tokens (there it is the fastest on B200), the tensor-core kernel above,
+// on the packed copy when there is one.  TC and FUSED force the tensor-core
+// and the channel-split kernel where they apply; GEMV forces the GEMVs
+// (group size 32 has none: AUTO's choice).
+int persistent_choice(int64_t T, int H, int I, int gs, size_t cap, const void *packed, bool linear)
 {
     const int mode = g_decode_mode.load(std::memory_order_relaxed);
     const int Ttc = (int)(T < kTcMaxTok ? T : kTcMaxTok);
     const int Tsp = (int)(T < kSplitMaxTok ? T : kSplitMaxTok);
-    if (packed)
-        return Ttc >= 1 && decode_ffn_tc_packed_supported(Ttc, H, I, gs) &&
-                       decode_ffn_tc_scratch(Ttc, H) <= cap
-                   ? 2
-                   : 0;
-    const bool tc = Ttc >= 1 && decode_ffn_tc_supported(Ttc, H, I, gs) &&
-                    decode_ffn_tc_scratch(Ttc, H) <= cap;
-    const bool sp = Tsp >= 1 && decode_ffn_split_supported(Tsp, H, I, gs) &&
+    const bool tc_fits = Ttc >= 1 && decode_ffn_tc_scratch(Ttc, H) <= cap;
+    const bool tcp = packed && tc_fits && decode_ffn_tc_packed_supported(Ttc, H, I, gs);
+    const bool tcl = linear && tc_fits && decode_ffn_tc_supported(Ttc, H, I, gs);
+    const bool sp = linear && Tsp >= 1 && decode_ffn_split_supported(Tsp, H, I, gs) &&
                     decode_ffn_split_scratch(Tsp, H) <= cap;
+    const int tc = tcp ? 3 : tcl ? 2 : 0;
     if (mode == WIDE_DECODE_FUSED)
-        return sp ? 1 : tc && gs == 32 ? 2 : 0;
-    if (mode == WIDE_DECODE_GEMV && gs != 32)
-        return 0;
+        return sp ? 1 : tc;
     if (mode == WIDE_DECODE_TC)
-        return tc ? 2 : sp ? 1 : 0;
-    // AUTO on nn.Linear weights: the channel-split kernel up to 8 tokens per
-    // launch (there it streams the row-strided tiles faster), the tensor-core
-    // kernel above
+        return tc ? tc : sp ? 1 : 0;
+    if (mode == WIDE_DECODE_GEMV && gs != 32 && linear)
+        return 0;
     if (sp && T <= 8)
         return 1;
-    return tc ? 2 : sp ? 1 : 0;
+    return tc ? tc : sp ? 1 : 0;
 }
 }  // namespace
 
 bool decode_ffn_persistent_available(int64_t T, int H, int I, int gs, size_t cap,
-                                     const void *packed)
+                                     const void *packed, bool linear)
 {
-    return persistent_choice(T, H, I, gs, cap, packed) != 0;
+    return persistent_choice(T, H, I, gs, cap, packed, linear) != 0;
 }
 
 int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const void *wd,
                           const uint32_t *mask, const DownOutputs &o, int64_t T, int H, int I,
                           int gs, void *scratch, size_t cap, cudaStream_t s, const void *packed)
 {
-    const int which = persistent_choice(T, H, I, gs, cap, packed);
-    if (which == 0)
+    const bool linear = wg && wu && wd;
+    if (persistent_choice(T, H, I, gs, cap, packed, linear) == 0)
         return WIDE_EUNSUPPORTED;
-    const int per = which == 2 ? kTcMaxTok : kSplitMaxTok;
     const int W = (I / gs + 31) / 32;
     auto at = [](const void *p, int64_t off, size_t elem) -> const char * {
         return p ? static_cast<const char *>(p) + off * (int64_t)elem : nullptr;
     };
-    for (int64_t t0 = 0; t0 < T; t0 += per) {
+    // the kernel is chosen per launch from the tokens left (AUTO: a tail of
+    // up to 8 tokens goes to the channel-split kernel)
+    for (int64_t t0 = 0; t0 < T;) {
+        const int which = persistent_choice(T - t0, H, I, gs, cap, packed, linear);
+        if (which == 0)
+            return WIDE_EUNSUPPORTED;
+        const int per = which >= 2 ? kTcMaxTok : kSplitMaxTok;
         const int Tc = (int)(T - t0 < per ? T - t0 : per);
         const int64_t e = t0 * H;
         DownOutputs c = {};
@@ -1095,13 +1097,14 @@ int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const v
         c.out_total = const_cast<char *>(at(o.out_total, e, 2));
         c.out_total_f32 = reinterpret_cast<float *>(const_cast<char *>(at(o.out_total_f32, e, 4)));
         const void *xc = at(x, e, 2);
-        const int rc = which == 2
-                           ? decode_ffn_tc(xc, wg, wu, wd, packed, mask + t0 * W, c, Tc, H, I, gs,
-                                           scratch, s)
+        const int rc = which >= 2
+                           ? decode_ffn_tc(xc, wg, wu, wd, which == 3 ? packed : nullptr,
+                                           mask + t0 * W, c, Tc, H, I, gs, scratch, s)
                            : decode_ffn_split(xc, wg, wu, wd, mask + t0 * W, c, Tc, H, I, gs,
                                              scratch, s);
         if (rc)
             return rc;
+        t0 += Tc;
     }
     return WIDE_OK;
 }

@@ -288,9 +288,10 @@ int ffn_pack_launch(const void *wg, const void *wu, const void *wd, int64_t H, i
 // (tensor-core kernel) or 16 (channel-split kernel) tokens, with `cap` bytes
 // of scratch.  WIDE_EUNSUPPORTED, with nothing enqueued, when neither
 // applies: the caller then runs the GEMV kernels.
-// With `packed` non-NULL only the tensor-core kernel applies (any mode).
+// `packed`: the wide_ffn_pack copy or NULL; wg / wu / wd may be NULL when
+// only the packed copy is at hand (then only the tensor-core kernel applies).
 bool decode_ffn_persistent_available(int64_t T, int H, int I, int gs, size_t cap,
-                                     const void *packed = nullptr);
+                                     const void *packed = nullptr, bool linear = true);
 int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const void *wd,
                           const uint32_t *mask, const DownOutputs &o, int64_t T, int H, int I,
                           int gs, void *scratch, size_t cap, cudaStream_t s,
@@ -299,11 +300,13 @@ int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const v
 size_t ffn_decode_h_bytes(const wide_ffn_dims *d);
 // Runs the decode path with h scratch (h_cap contiguous bytes at h, at
 // least ffn_decode_h_bytes(d)) and grid-barrier words given apart.
+// packed: an optional wide_ffn_pack copy of the weights, which the
+// tensor-core kernel then reads.
 int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
                    const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
-                   size_t h_cap, uint32_t *bar, cudaStream_t s);
+                   size_t h_cap, uint32_t *bar, cudaStream_t s, const void *packed = nullptr);
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
-                      cudaStream_t s);
+                      cudaStream_t s, const void *packed = nullptr);
 
 }  // namespace wide
