@@ -136,3 +136,17 @@ def test_decode_layer_8b_full_config():
     groups Bernoulli(0.34), FFN groups Bernoulli(0.72)."""
     lc = synth.decode_layer()
     _check(lc, _run(lc))
+
+
+@pytest.mark.parametrize("mode", ["gemv", "fused"])
+def test_decode_layer_on_cuda_core_kernels(mode):
+    """The 8B decode layer with the decode mode forcing CUDA-core kernels
+    (o_proj on the GEMV, the FFN on the GEMVs or the channel-split kernel):
+    the same oracle outputs as the default tensor-core path."""
+    import token_level_dynamic_b200 as w
+    prev = w.wide_set_decode_ffn_path(w.WIDE_DECODE_GEMV if mode == "gemv" else w.WIDE_DECODE_FUSED)
+    try:
+        lc = synth.decode_layer()
+        _check(lc, _run(lc))
+    finally:
+        w.wide_set_decode_ffn_path(prev)

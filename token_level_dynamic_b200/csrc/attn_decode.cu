@@ -616,6 +616,7 @@ int launch_cluster(int32_t kid, void (*kernel)(KArgs...), dim3 grid, dim3 block,
 
 struct DecodeWs {
     float *q, *o, *h1, *hffn, *part_o;
+    size_t hffn_bytes;
     float2 *part_ml;
     __nv_bfloat16 *xn2;
     uint32_t *bar, *arrived;
@@ -639,7 +640,11 @@ DecodeWs decode_ws(const wide_layer_dims *d, void *base)
     w.q = reinterpret_cast<float *>(take(T * qd * 4));
     w.o = reinterpret_cast<float *>(take(Tp * qd * 4));
     w.h1 = reinterpret_cast<float *>(take(T * (size_t)d->hidden * 4));
-    w.hffn = reinterpret_cast<float *>(take(Tp * (size_t)d->inter * 4));
+    // FFN h, or a persistent kernel's accumulator (the o_proj's too)
+    const size_t hffn_bytes = Tp * (size_t)d->inter * 4;
+    const size_t acc_bytes = decode_ffn_tc_scratch((int)T, (int)d->hidden);
+    w.hffn_bytes = hffn_bytes > acc_bytes ? hffn_bytes : acc_bytes;
+    w.hffn = reinterpret_cast<float *>(take(w.hffn_bytes));
     w.xn2 = reinterpret_cast<__nv_bfloat16 *>(take(T * (size_t)d->hidden * 2));
     w.bar = reinterpret_cast<uint32_t *>(take(256));
     const int64_t nkeys = d->cache_len + 1;
@@ -772,7 +777,7 @@ int layer_decode_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws, 
     fo.out_sum = p.ffn_out;
     fo.res_f32 = w.h1;
     fo.out_total = p.out;
-    const size_t hcap = align_up((size_t)(T + 1) / 2 * 2 * I * 4, 256);
+    const size_t hcap = w.hffn_bytes;
     // the dispatcher reads the packed copy where the tensor-core kernel runs
     const void *pk = p.ffn_packed;
     if (decode_ffn_persistent_available(T, H, I, gsf, hcap, pk)) {

@@ -277,6 +277,7 @@ int decode_ffn_tc(const void *x, const void *wg, const void *wu, const void *wd,
                   const void *packed, const uint32_t *mask, const DownOutputs &o, int T, int H,
                   int I, int gs, void *scratch, cudaStream_t s);
 bool decode_ffn_tc_packed_supported(int T, int H, int I, int gs);
+
 // Packed decode weights (ffn_pack.cu): W_gate and W_up in 64-row panels,
 // each panel K-step-major ([I/64][H/64][64][64]), then W_down in 16-channel
 // column panels ([I/16][H][16]); 3 * I * H bf16 in all.
