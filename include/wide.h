@@ -179,8 +179,9 @@ int wide_reorder(const uint32_t *d_mask, int64_t T, int64_t G, int32_t tile_m,
  *
  * Supported: hidden % 128 == 0; group_size in {32, 64, 128} dividing inter;
  * G <= 1024; 16-byte aligned pointers.  The bf16 decode path with
- * group_size 32 needs hidden % 256 == 0 (it runs on the channel-split
- * kernel only).  WIDE_PATH_PREFILL needs bf16, group_size 64 or 128 and
+ * group_size 32 runs on the persistent kernels only (the GEMVs take 64 and
+ * 128).  WIDE_PATH_PREFILL needs bf16, group_size 64 or 128 (or 32 with
+ * inter % 64 == 0: the down projection takes the groups in pairs) and
  * hidden % 256 == 0.  The fp32 type runs the CUDA-core path at any T.
  */
 typedef struct wide_ffn_dims {
@@ -321,6 +322,7 @@ int wide_ffn_masked_packed(const void *d_x, const void *d_packed, const void *d_
  *           cache_len < 131072, cache_cap >= cache_len + 1;
  *   prefill (seq_len >= 1 with cache_len == 0, i.e. no earlier context):
  *           n_kv_heads even, 2..1024, n_q_heads / n_kv_heads in {2, 4},
+ *           ffn_group_size 32 also (with inter % 64 == 0),
  *           hidden % 256 == 0, inter / ffn_group_size <= 1024,
  *           cache_cap >= seq_len, n_seq * seq_len <= 2^24 and
  *           n_kv_heads * n_seq * seq_len <= 2^22.

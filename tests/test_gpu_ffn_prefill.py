@@ -117,6 +117,43 @@ def test_prefill_group_size_64_all_zero_and_dense():
     assert rel_l2(_run(c), ffn_dense(c.x, c.w_gate, c.w_up, c.w_down)) <= TOL
 
 
+@pytest.mark.parametrize("T,H,I,kind,keep", [
+    (300, 256, 512, "bernoulli", 0.5),        # 16 groups of 32, ragged tails
+    (1000, 512, 2048, "prototype", 0.5),      # 64 groups of 32: two mask words
+    (513, 1024, 4352, "prototype", 0.25),     # 136 groups of 32 over five mask words
+    (1024, 2048, 8192, "bernoulli", 0.5),     # 256 groups of 32, wider hidden
+])
+def test_prefill_group_size_32(T, H, I, kind, keep):
+    """32-channel groups: gate/up tiles are N = 64, and the down projection
+    takes the groups in pairs (one 64-column stage per pair that some token
+    of the tile keeps), zeroing each 32-channel half for the tokens that
+    skip that half's group."""
+    c = synth.ffn_case(T, H, I, 32, seed=T + 11, keep=keep, mask_kind=kind)
+    assert rel_l2(_run(c), _ref(c)) <= TOL
+
+
+def test_prefill_group_size_32_halves_of_a_pair():
+    """Tokens keep only odd groups, or only even ones, or one half of a
+    pair each: every pair's stage is loaded and the half a token skips is
+    zeroed for it (an all-zero or a both-halves mistake shows here)."""
+    c = synth.ffn_case(384, 512, 1024, 32, seed=21)         # 32 groups
+    G = c.I // c.gs
+    c.mask[:] = False
+    c.mask[:128, 1::2] = True                  # odd groups only
+    c.mask[128:256, 0::2] = True               # even groups only
+    c.mask[256:, 5] = True                     # one half of pair 2
+    c.mask[300:, 10] = True                    # the other tokens: pair 5's first half
+    assert rel_l2(_run(c), _ref(c)) <= TOL
+    assert G == 32
+
+
+def test_prefill_group_size_32_all_zero_and_dense():
+    c = synth.ffn_case(200, 256, 512, 32, seed=15, mask_kind="zeros")
+    assert not np.any(_run(c))
+    c = synth.ffn_case(260, 512, 1024, 32, seed=16, mask_kind="ones")
+    assert rel_l2(_run(c), ffn_dense(c.x, c.w_gate, c.w_up, c.w_down)) <= TOL
+
+
 @pytest.mark.parametrize("path", ["decode", "prefill"])
 def test_empty_batch_is_a_no_op(path):
     """Zero tokens: the call succeeds, launches nothing that fails, and

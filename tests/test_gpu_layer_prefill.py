@@ -82,6 +82,14 @@ def test_prefill_all_groups_kept():
     _check_full(lc, _run(lc))
 
 
+def test_prefill_layer_ffn_group_size_32():
+    """The prefill layer with 32-channel FFN groups (the down projection
+    takes them in pairs)."""
+    lc = synth.small_layer("prefill", seed=41, n_seq=2, seq_len=200, H=512, n_q=8, n_kv=2,
+                           hd=128, I=1024, gs=32, keep_a=0.5, keep_f=0.5)
+    _check_full(lc, _run(lc))
+
+
 @pytest.mark.parametrize("keep", [0.25, 0.5, 0.75, 1.0])
 def test_prefill_layer_8b_full_size_sampled(keep):
     """The Llama-3.1-8B-shaped prefill layer (4 sequences x 2048 tokens,

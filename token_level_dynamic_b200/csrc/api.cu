@@ -358,9 +358,10 @@ bool ffn_shape_supported(const wide_ffn_dims *d, int path)
                (gs == 32 && (decode_ffn_split_supported(T1, H, I, 32) ||
                              decode_ffn_tc_supported(T1, H, I, 32)));
     }
-    // prefill: tcgen05 kernels with 128-channel groups and 256-column output blocks
-    return d->dtype == WIDE_BF16 && (gs == 64 || gs == 128) && d->hidden % 256 == 0 &&
-           d->tokens <= (1 << 24);
+    // prefill: tcgen05 kernels, 256-column output blocks; 32-channel groups
+    // go through the down projection in pairs (64-column stages)
+    return d->dtype == WIDE_BF16 && (gs == 64 || gs == 128 || (gs == 32 && d->inter % 64 == 0)) &&
+           d->hidden % 256 == 0 && d->tokens <= (1 << 24);
 }
 
 }  // namespace wide

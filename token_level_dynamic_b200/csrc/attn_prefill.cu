@@ -463,7 +463,8 @@ bool layer_prefill_supported(const wide_layer_dims *d)
     return d->cache_len == 0 && d->seq_len >= 1 && T >= 1 && T <= (1 << 24) &&
            d->head_dim == kHD && d->n_kv_heads >= 2 && d->n_kv_heads % 2 == 0 &&
            d->n_kv_heads <= 1024 && (rep == 2 || rep == 4) && d->hidden % 256 == 0 &&
-           (d->ffn_group_size == 64 || d->ffn_group_size == 128) &&
+           (d->ffn_group_size == 64 || d->ffn_group_size == 128 ||
+            (d->ffn_group_size == 32 && d->inter % 64 == 0)) &&
            d->inter % d->ffn_group_size == 0 && d->inter / d->ffn_group_size <= 1024 &&
            d->cache_cap >= d->seq_len && (int64_t)d->n_kv_heads * T <= (1ll << 31) / 512;
 }

@@ -612,7 +612,14 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_sig = (a.T + kBM - 1) / kBM;
     const int n_tiles = n_sig * (a.N / kBN);
-    const int spg = a.gs / kBK;            // K stages per group
+    // K stages per group; 32-channel groups go in pairs (2p, 2p + 1), one
+    // 64-column stage per pair that holds either group (the pair's word bits
+    // folded onto the even bit)
+    const bool pairs = a.gs == 32;
+    const int spg = pairs ? 1 : a.gs / kBK;
+    auto stage_bits = [&](uint32_t bits) {
+        return pairs ? (bits | (bits >> 1)) & 0x55555555u : bits;
+    };
 
     if (threadIdx.x == 0) {
         // full: the producer's arrive with the A and B bytes; fixed: one
@@ -649,7 +656,7 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
             int s, nb;
             coords(tile, s, nb);
             for (int w = 0; w < a.W && ok; ++w) {
-                uint32_t bits = uword(s, w);
+                uint32_t bits = stage_bits(uword(s, w));
                 while (bits && ok) {
                     const int g = w * 32 + __ffs(bits) - 1;
                     bits &= bits - 1u;
@@ -703,7 +710,7 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
                 tok[i] = sr < a.T ? a.sig_perm[sr] : -1;
             }
             for (int w = 0; w < a.W && ok; ++w) {
-                uint32_t bits = uword(s, w);
+                uint32_t bits = stage_bits(uword(s, w));
                 if (!bits)
                     continue;
                 uint32_t mw[kBM / 8];
@@ -720,9 +727,13 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
                             break;
                         }
                         uint8_t *sa = smem + stage * kStageBytes;
+                        // chunk cc holds channels 8 cc .. 8 cc + 7 of the
+                        // stage: of group gb, or with 32-channel pairs of
+                        // group gb + cc / 4
+                        const int gbit = pairs ? gb + (cc >> 2) : gb;
 #pragma unroll
                         for (int i = 0; i < kBM / 8; ++i)
-                            if (!((mw[i] >> gb) & 1u))
+                            if (!((mw[i] >> gbit) & 1u))
                                 *reinterpret_cast<uint4 *>(sa + swz128(lr + 8 * i, cc)) =
                                     make_uint4(0u, 0u, 0u, 0u);
                         // the zeros are written by the generic proxy and read
@@ -751,7 +762,7 @@ __global__ void __launch_bounds__(kThreadsDown, 1)
                 const uint32_t d = tmem + acc * (uint32_t)kBN;
                 int kstep = 0;
                 for (int w = 0; w < a.W && ok; ++w) {
-                    const int nsteps = __popc(uword(s, w)) * spg;
+                    const int nsteps = __popc(stage_bits(uword(s, w))) * spg;
                     for (int n = 0; n < nsteps && ok; ++n) {
                         // fixed completes once the zero-filling warps (which
                         // waited for full) are done with the stage
