@@ -107,3 +107,29 @@ def test_clock_sampler_without_nvml(monkeypatch):
     with bench.ClockSampler(0) as c:
         pass
     assert c.summary()["source"] == "unavailable"
+
+
+def test_decode_bytes_follow_the_per_launch_kernel_choice():
+    """The decode FFN's algorithmic bytes are booked on the kernel each
+    launch runs: the channel-split kernel up to 8 tokens, the tensor-core
+    kernel for 32-token launches, and a 40-token batch as one 32-token
+    tensor-core launch plus an 8-token split launch, each streaming the
+    union of its own tokens' groups."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    H, I, gs = 3072, 8192, 128
+    for T, names in ((1, {"decode_ffn_split_gemv"}), (8, {"decode_ffn_split_gemv"}),
+                     (32, {"decode_ffn_tcgen05"}),
+                     (40, {"decode_ffn_tcgen05", "decode_ffn_split_gemv"})):
+        c = synth.ffn_case(T, H, I, gs, seed=T, keep=0.5)
+        b = bench._ffn_decode_bytes(c)
+        kern = set(b) - {"total", "union_groups"}
+        assert kern == names, (T, kern)
+        assert b["total"] == sum(b[k] for k in kern)
+        io = T * H * 2 + c.mask_words.nbytes + T * H * 2
+        w = 0
+        for t0, n in ((0, 32), (32, 8)) if T == 40 else ((0, T),):
+            u = int(c.mask[t0:t0 + n].any(axis=0).sum())
+            w += 3 * u * gs * H * 2
+        assert b["total"] == w + io

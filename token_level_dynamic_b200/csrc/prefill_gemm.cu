@@ -478,14 +478,20 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
         // -------------------------------------------- MMA issuer
         // SwiGLU: N = gate rows + up rows of one group (2 gs); router: the
         // bottleneck width; else 256
-        const uint32_t idesc = umma::idesc_bf16_f32(
-            kBM, MODE == GEMM_SWIGLU   ? 2u * (uint32_t)a.gs
-                 : MODE == GEMM_ROUTER ? (uint32_t)a.rn
-                                       : (uint32_t)kBN);
+        const uint32_t nd = MODE == GEMM_SWIGLU   ? 2u * (uint32_t)a.gs
+                            : MODE == GEMM_ROUTER ? (uint32_t)a.rn
+                                                  : (uint32_t)kBN;
+        const uint32_t idesc = umma::idesc_bf16_f32(kBM, nd);
+        // MMA-stage skip: a group's tile with at most 64 active tokens (its
+        // rows are the tile's first rows) runs M = 64 MMAs
+        const uint32_t idesc64 = umma::idesc_bf16_f32(64, nd);
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < nw && ok; it += gridDim.x) {
             if (lane == 0) {
+                const bool m64 = (MODE == GEMM_SWIGLU || MODE == GEMM_ROPE_Q) &&
+                                 decode_work<MODE>(a, it).nrows <= 64;
+                const uint32_t id = m64 ? idesc64 : idesc;
                 if (!wait_or_abort(&ctl->tempty[acc], acc_phase ^ 1u, ctl, a.status))
                     ok = false;
                 umma::fence_after_sync();
@@ -504,7 +510,7 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
                         umma::mma_bf16(d, umma::desc_kmajor_sw128(sa + 32u * k),
-                                       umma::desc_kmajor_sw128(sb + 32u * k), idesc,
+                                       umma::desc_kmajor_sw128(sb + 32u * k), id,
                                        (kt | k) != 0);
                     umma::commit(&ctl->empty[stage]);
                     if (++stage == nst) {
@@ -529,10 +535,14 @@ __global__ void __launch_bounds__(kThreadsGather, 1)
     } else {
         // -------------------------------------------- epilogue (warps 2-5)
         const int q = warp & 3;
-        const int r = q * 32 + lane;          // tile row = TMEM lane
         uint32_t acc = 0, acc_phase = 0;
         for (int it = blockIdx.x; it < nw; it += gridDim.x) {
             const Work w = decode_work<MODE>(a, it);
+            // tile row of this thread: the TMEM lane at M = 128; at M = 64
+            // (tiles of at most 64 rows) row m sits in lane (m % 16) + 32 (m /
+            // 16), so lanes 0..15 of warp q hold rows 16 q .. 16 q + 15
+            const bool m64 = (MODE == GEMM_SWIGLU || MODE == GEMM_ROPE_Q) && w.nrows <= 64;
+            const int r = m64 ? (lane < 16 ? q * 16 + lane : kBM) : q * 32 + lane;
             const bool live = r < w.nrows;
             const int t = live ? row_token<MODE>(a, w, r) : 0;
             if (!wait_or_abort(&ctl->tfull[acc], acc_phase, ctl, a.status))
