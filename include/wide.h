@@ -381,15 +381,18 @@ int wide_attn_masked(const void *d_x, const wide_layer_weights *w, void *d_k_cac
  * synchronise the device).
  *
  * Same operation, arguments and layouts as wide_ffn_masked on its decode
- * path (CUDA-core GEMV over the batch's union of groups), minus the
- * workspace: the kernels' scratch (fp32 h for up to 32 tokens x inter
- * channels) lives in a fixed device array inside the library of
- * WIDE_NOALLOC_SCRATCH_BYTES bytes, and the decode kernel's grid-barrier
- * words in a second one of 256 bytes, which every GPU that loads the library
- * holds until the process exits.  Limit: min(tokens, 32), rounded up to
- * an even count, * inter * 4 bytes must not exceed it (inter <= 16384 at
- * 32 tokens); larger problems return
- * WIDE_ETOOLARGE before anything is enqueued.  The call allocates nothing.
+ * path (the kernels the wide_set_decode_ffn_path mode picks, over the
+ * batch's union of groups), minus the workspace: the kernels' scratch (fp32
+ * h for up to 32 tokens x inter channels, or a persistent kernel's fp32
+ * accumulator and arrival counter) lives in a fixed device array inside the
+ * library of WIDE_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads
+ * the library holds until the process exits.  Limit: min(tokens, 32),
+ * rounded up to an even count, * inter * 4 bytes, and min(tokens, 32)
+ * rounded up to a multiple of 4, * hidden * 4 bytes, must not exceed it
+ * (inter <= 16384 at 32 tokens); larger problems return WIDE_ETOOLARGE
+ * before anything is enqueued.  A persistent kernel runs only where its
+ * accumulator and counter fit in the array (else the GEMV kernels).  The
+ * call allocates nothing.
  * Its first call on a device looks up the array's device address (once per
  * device and CUDA context, with that device current: after a
  * cudaDeviceReset the next call looks it up again); make that first call

@@ -102,7 +102,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     for I, expect_ok in ((16384, True), (16384 + 128, False)):
         d = _native.WideFFNDims(T, H, I, gs, _native.WIDE_BF16, _native.WIDE_PATH_DECODE)
         if expect_ok:
-            # the fixed array holds h; the grid-barrier words live apart
+            # the fixed array holds h (or a persistent kernel's accumulator)
             assert T * I * 4 <= w.WIDE_NOALLOC_SCRATCH_BYTES
             assert w.wide_ffn_workspace_bytes(T, H, I, gs) == T * I * 4 + 256
         else:

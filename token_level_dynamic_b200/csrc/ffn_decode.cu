@@ -666,12 +666,13 @@ size_t ffn_decode_h_bytes(const wide_ffn_dims *d)
     return align_up((h > acc ? h : acc) * sizeof(float), 256);
 }
 
-// h scratch, then 256 bytes holding the fused kernel's grid-barrier words.
+// h scratch, then 256 bytes: a persistent kernel's accumulator may take all
+// of h_bytes, its arrival counter sits after it
 size_t ffn_decode_workspace(const wide_ffn_dims *d) { return ffn_decode_h_bytes(d) + 256; }
 
 int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
                    const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
-                   size_t h_cap, uint32_t *bar, cudaStream_t s, const void *packed)
+                   size_t h_cap, cudaStream_t s, const void *packed)
 {
     if (d->tokens == 0)
         return WIDE_OK;
@@ -704,12 +705,9 @@ int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void 
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s, const void *packed)
 {
-    // h, then the 256 bytes of the barrier words: ffn_decode_h_bytes + 256
-    // contiguous bytes
-    char *base = static_cast<char *>(ws);
-    return ffn_decode_run(x, wg, wu, wd, mask, out, d, reinterpret_cast<float *>(base),
-                          ffn_decode_h_bytes(d) + 256,
-                          reinterpret_cast<uint32_t *>(base + ffn_decode_h_bytes(d)), s, packed);
+    // h and the 256 bytes after it: ffn_decode_h_bytes + 256 contiguous bytes
+    return ffn_decode_run(x, wg, wu, wd, mask, out, d, static_cast<float *>(ws),
+                          ffn_decode_h_bytes(d) + 256, s, packed);
 }
 
 }  // namespace wide

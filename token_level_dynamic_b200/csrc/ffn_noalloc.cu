@@ -6,26 +6,25 @@
 // latency-critical loop where cudaMalloc/cudaFree would synchronise the
 // device.  This entry point runs the same decode kernels as
 // wide_ffn_masked's decode path, but keeps their scratch in the file-scope
-// device arrays below instead of a caller workspace: for the channel-split
-// kernel (bf16, the usual case) its fp32 [T][hidden] accumulator and arrival
-// counter, for the GEMV kernels (fp32, and bf16 shapes outside the split
-// kernel's limits) the fp32 intermediate h = silu(gate) * up of up to 32
-// tokens.  The second array holds the barrier words the decode path's
-// interface carries (unused by the current kernels).
+// device array below instead of a caller workspace: for the persistent
+// kernels (bf16, the usual case) their fp32 accumulator and arrival counter,
+// for the GEMV kernels (fp32, and bf16 shapes outside the persistent
+// kernels' limits) the fp32 intermediate h = silu(gate) * up of up to 32
+// tokens.
 //
-// The arrays are module globals: every GPU that loads the library holds
-// WIDE_NOALLOC_SCRATCH_BYTES (+ 256) bytes of device memory for them until
-// the process exits.  All calls on a device share them and they keep the
-// last call's contents.  No call depends on those contents: the split
+// The array is a module global: every GPU that loads the library holds
+// WIDE_NOALLOC_SCRATCH_BYTES bytes of device memory for it until the
+// process exits.  All calls on a device share it and it keeps the last
+// call's contents.  No call depends on those contents: a persistent
 // kernel's launch zeroes, on the stream, the accumulator and counter it is
 // about to use, and the GEMV kernels read h only at the (token, group) pairs
 // the same call wrote.  Two calls whose work overlaps on the GPU (different
-// streams without ordering) race on the arrays.
+// streams without ordering) race on the array.
 //
-// In host code the arrays' names are host-side stand-ins, not device
-// addresses: the addresses are looked up with cudaGetSymbolAddress, with the
+// In host code the array's name is a host-side stand-in, not a device
+// address: the address is looked up with cudaGetSymbolAddress, with the
 // device current, once per device and CUDA context (device_symbol_address),
-// so after a cudaDeviceReset the next call looks them up again.  The first
+// so after a cudaDeviceReset the next call looks it up again.  The first
 // call on a device (or in a new context) does that lookup; make it before
 // any stream capture.
 #include <cuda_runtime.h>
@@ -35,19 +34,16 @@
 #include "wide.h"
 
 static __device__ __align__(256) float g_noalloc_scratch[WIDE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
-static __device__ __align__(256) uint32_t g_noalloc_bar[64];
 
 namespace wide {
 namespace {
 
-// Device addresses of this device's copies of g_noalloc_scratch and
-// g_noalloc_bar (see device_symbol_address).
-bool noalloc_arrays(float **scratch, uint32_t **bar)
+// Device address of this device's copy of g_noalloc_scratch (see
+// device_symbol_address).
+float *noalloc_scratch()
 {
-    static DeviceSymbolCache cs, cb;
-    *scratch = static_cast<float *>(device_symbol_address(cs, &g_noalloc_scratch));
-    *bar = static_cast<uint32_t *>(device_symbol_address(cb, &g_noalloc_bar));
-    return *scratch && *bar;
+    static DeviceSymbolCache cs;
+    return static_cast<float *>(device_symbol_address(cs, &g_noalloc_scratch));
 }
 
 }  // namespace
@@ -74,10 +70,9 @@ extern "C" int wide_ffn_masked_noalloc(const void *d_x, const void *d_w_gate, co
         return WIDE_EUNSUPPORTED;
     if (ffn_decode_h_bytes(d) > (size_t)WIDE_NOALLOC_SCRATCH_BYTES)
         return WIDE_ETOOLARGE;
-    float *scratch = nullptr;
-    uint32_t *bar = nullptr;
-    if (!noalloc_arrays(&scratch, &bar))
+    float *scratch = noalloc_scratch();
+    if (!scratch)
         return WIDE_CUDA_FAIL();
     return ffn_decode_run(d_x, d_w_gate, d_w_up, d_w_down, d_group_mask, d_out, d, scratch,
-                          WIDE_NOALLOC_SCRATCH_BYTES, bar, static_cast<cudaStream_t>(stream));
+                          WIDE_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
 }

@@ -299,13 +299,14 @@ int decode_ffn_persistent(const void *x, const void *wg, const void *wu, const v
                           const void *packed = nullptr);
 // Bytes of the fp32 h scratch of the decode path (tokens capped at 32).
 size_t ffn_decode_h_bytes(const wide_ffn_dims *d);
-// Runs the decode path with h scratch (h_cap contiguous bytes at h, at
-// least ffn_decode_h_bytes(d)) and grid-barrier words given apart.
+// Runs the decode path with h scratch of h_cap contiguous bytes at h (at
+// least ffn_decode_h_bytes(d); the persistent kernels run only where their
+// accumulator and counter fit in h_cap).
 // packed: an optional wide_ffn_pack copy of the weights, which the
 // tensor-core kernel then reads.
 int ffn_decode_run(const void *x, const void *wg, const void *wu, const void *wd,
                    const uint32_t *mask, void *out, const wide_ffn_dims *d, float *h,
-                   size_t h_cap, uint32_t *bar, cudaStream_t s, const void *packed = nullptr);
+                   size_t h_cap, cudaStream_t s, const void *packed = nullptr);
 int ffn_decode_launch(const void *x, const void *wg, const void *wu, const void *wd,
                       const uint32_t *mask, void *out, const wide_ffn_dims *d, void *ws,
                       cudaStream_t s, const void *packed = nullptr);
