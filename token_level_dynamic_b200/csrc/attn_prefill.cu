@@ -11,11 +11,14 @@
 //
 // prefill_attn: one CTA per (query tile, query head of the group, sequence x
 // KV head); warps 0-3 run the softmax (thread r = query row r = TMEM lane r),
-// warp 4 issues every TMA copy and tensor-core MMA; two CTAs per SM (112 KB
-// of shared memory and 256 TMEM columns each).  The warps hand work over
-// through mbarriers only (no block-wide barrier inside the loop), so the
-// softmax never waits for the issuer except for data.  Per 64-key tile up to
-// the tile's last query position:
+// one thread of warp 4 issues the tensor-core MMAs, one thread of warp 5 the
+// Q and K copies and one of warp 6 the V copies; two CTAs per SM (112 KB of
+// shared memory and 256 TMEM columns each).  The roles hand work over through
+// mbarriers only (no block-wide barrier inside the loop), and each role
+// blocks only on the barrier of its own next step, so no MMA waits for the
+// completion of an earlier one: the issuer queues S(t) as soon as K(t) has
+// landed and the softmax has read S(t-2), then P(t-1) V(t-1) as soon as P(t-1)
+// is written.  Per 64-key tile up to the tile's last query position:
 //   S  = Q K^T           tcgen05, M=128 N=64 K=128, fp32 in one of two
 //                        64-column TMEM buffers; S of the next tile is issued
 //                        before this tile's softmax runs
@@ -29,7 +32,8 @@
 //        P <= 256; when it grows further the row's O and sum are rescaled
 //        (TMEM load, multiply, store) and m_ref moves up.  Rescales are rare
 //        after the first tiles, so O never passes through registers per tile.
-// K and V tiles are double-buffered and prefetched by TMA two tiles ahead.
+// K and V tiles are double-buffered: K(t) is copied once S(t-2) has
+// completed, V(t) once P(t-2) V(t-2) has.
 // Then O / l is written (bf16) at the token's signature-order row of the
 // o_proj input.  Tiles with no query (ragged counts) exit at once.
 #include "common.cuh"
@@ -49,6 +53,15 @@ constexpr uint32_t kKTile = 2 * kKHalf;
 constexpr uint32_t kPTile = 128 * 128;  // P: 128 rows x 64 keys (16 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 
+// 2^x by the SFU's approximate base-2 exponential (PTX ex2.approx; results
+// below the normal range flush to 0, which a probability in bf16 loses anyway)
+__device__ __forceinline__ float exp2_sfu(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 struct AttnPArgs {
     const int32_t *count, *perm, *sig_pos;   // head-group work list
     int T, seq_len, n_kv, rep, qcols, ocols;
@@ -58,16 +71,22 @@ struct AttnPArgs {
     int32_t *status;
 };
 
+// Barrier phases: every barrier of a pair alternates by tile (tile t uses
+// [t & 1], phase t >> 1), so a waiter for tile t's phase can never see the
+// barrier two phases further on: that phase belongs to tile t + 2, whose
+// copy or MMA needs a step the waiter itself takes after this wait.
 struct __align__(8) ACtl {
-    uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_pv;
+    uint64_t bar_q, bar_k[2], bar_v[2], bar_s[2], bar_pv[2];
     uint64_t s_free[2];   // softmax warps have read S buffer b (4 warp arrivals)
     uint64_t p_full;      // softmax warps wrote P and rescaled O (4 warp arrivals)
+    uint64_t bar_end;     // error path: every MMA of the issuer has completed
     uint32_t tmem_base;
-    int lo, nq, pmax;
+    int bound[2], pmax;
     int abort;
 };
 constexpr int kSoftWarps = 4;
-constexpr int kAttnThreads = 32 * (kSoftWarps + 1);
+constexpr int kMmaWarp = kSoftWarps, kKWarp = kSoftWarps + 1, kVWarp = kSoftWarps + 2;
+constexpr int kAttnThreads = 32 * (kSoftWarps + 3);
 
 // Q | K[2] | V[2] | P | control.  No alignment slack: the kernel checks that
 // the dynamic shared memory starts 1024-byte aligned (it does when nothing
@@ -77,16 +96,22 @@ constexpr uint32_t kOffK = kQTile, kOffV = kOffK + 2 * kKTile, kOffP = kOffV + 2
 constexpr uint32_t kOffCtl = kOffP + kPTile;
 constexpr size_t kAttnSmem = kOffCtl + sizeof(ACtl);
 
-// first index i in [0, n) with v[i] >= key (v ascending)
-__device__ __forceinline__ int lower_bound(const int32_t *v, int n, int key)
+// First index i in [0, n) with v[i] >= key (v ascending; n if none), by one
+// warp: each round the 32 lanes test 32 evenly spaced entries of the current
+// range [lo, hi], which shrinks it about 32-fold (a 4096-entry list takes 3
+// rounds of loads instead of the 12 dependent loads of a one-thread search).
+// Invariant: v[lo - 1] < key (or lo = 0) and v[hi] >= key (or hi = n).
+__device__ __forceinline__ int warp_lower_bound(const int32_t *v, int n, int key, int lane)
 {
     int lo = 0, hi = n;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (v[mid] < key)
-            lo = mid + 1;
-        else
-            hi = mid;
+    while (hi > lo) {
+        const int step = (hi - lo + 32) / 32;         // 32 probes reach hi
+        const int p = lo + (lane + 1) * step - 1;
+        const bool ge = p >= hi || v[p] >= key;
+        const int f = __ffs(__ballot_sync(0xffffffffu, ge)) - 1;   // lane 31 always tests true
+        const int pf = lo + (f + 1) * step - 1;
+        hi = min(pf, hi);
+        lo += f * step;                                // just past the last probe below key
     }
     return lo;
 }
@@ -129,67 +154,57 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int s = blockIdx.z / a.n_kv, j = blockIdx.z % a.n_kv;
     const int32_t *pj = a.perm + (size_t)j * a.T;
 
+    // this sequence's queries of group j: [lo, hi) of the group's token list
+    // (warp 0 finds lo, warp 1 hi, at the same time)
+    if (warp < 2) {
+        const int r = warp_lower_bound(pj, a.count[j], (s + warp) * a.seq_len, lane);
+        if (lane == 0)
+            ctl->bound[warp] = r;
+    }
     if (tid == 0) {
-        const int cnt = a.count[j];
-        const int lo = lower_bound(pj, cnt, s * a.seq_len);
-        const int hi = lower_bound(pj, cnt, (s + 1) * a.seq_len);
-        ctl->lo = lo;
-        ctl->nq = hi - lo;
-        const int last = min(hi - 1, lo + (qt + 1) * kBQ - 1);
-        ctl->pmax = last >= lo ? pj[last] - s * a.seq_len : -1;
         ctl->abort = 0;
         mbar_init(&ctl->bar_q, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&ctl->bar_k[b], 1);
             mbar_init(&ctl->bar_v[b], 1);
             mbar_init(&ctl->bar_s[b], 1);
+            mbar_init(&ctl->bar_pv[b], 1);
             mbar_init(&ctl->s_free[b], kSoftWarps);
         }
-        mbar_init(&ctl->bar_pv, 1);
         mbar_init(&ctl->p_full, kSoftWarps);
+        mbar_init(&ctl->bar_end, 1);
         fence_mbar_init();
     }
     __syncthreads();
-    const int lo = ctl->lo, nq = ctl->nq, pmax = ctl->pmax;
+    const int lo = ctl->bound[0], nq = ctl->bound[1] - lo;
     if (qt * kBQ >= nq)
         return;  // no query of this group in this tile: nothing to compute
     if (warp == 0) {
         umma::tmem_alloc(&ctl->tmem_base, 256);
         umma::tmem_relinquish();
+    } else if (tid == 32) {
+        // position of the tile's last query: how far its keys reach
+        ctl->pmax = pj[min(lo + nq - 1, lo + (qt + 1) * kBQ - 1)] - s * a.seq_len;
     }
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
+    const int pmax = ctl->pmax;
     const uint32_t t_pv = tmem + 128;             // S buffers at columns 0 and 64
     const int64_t kvrow0 = ((int64_t)s * a.n_kv + j) * a.cache_cap;
     const int nkt = pmax / kBKV + 1;
 
-    if (warp == kSoftWarps) {
-        // ---------------------------------------- TMA + MMA issuer (one lane)
+    if (warp == kMmaWarp) {
+        // ---------------------------------------- MMA issuer (one lane)
+        // Program order S(0), then per t: S(t+1), P(t) V(t).  Each MMA group
+        // completes on its own barrier; the issuer never waits for one.
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma::idesc_bf16_f32(kBQ, kBKV);
             constexpr uint32_t idesc_pv = umma::idesc_bf16_f32_bmn(kBQ, kHD);
-            int nk[2] = {0, 0}, nv[2] = {0, 0}, npv = 0, ns[2] = {0, 0};
-            auto load_k = [&](int t) {
-                ++nk[t & 1];
-                uint8_t *dst = smem + kOffK + (t & 1) * kKTile;
-                const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
-                mbar_arrive_expect_tx(&ctl->bar_k[t & 1], kKTile);
-                tma_load_2d(dst, &tm_k, 0, krow, &ctl->bar_k[t & 1]);
-                tma_load_2d(dst + kKHalf, &tm_k, 64, krow, &ctl->bar_k[t & 1]);
-            };
-            auto load_v = [&](int t) {
-                ++nv[t & 1];
-                uint8_t *dst = smem + kOffV + (t & 1) * kKTile;
-                const int krow = (int)(kvrow0 + (int64_t)t * kBKV);
-                mbar_arrive_expect_tx(&ctl->bar_v[t & 1], kKTile);
-                tma_load_2d(dst, &tm_v, 0, krow, &ctl->bar_v[t & 1]);
-                tma_load_2d(dst + kKHalf, &tm_v, 64, krow, &ctl->bar_v[t & 1]);
-            };
+            const uint32_t q0 = smem_u32(sq), p0 = smem_u32(sp);
             auto issue_s = [&](int t) {
-                ++ns[t & 1];
-                const uint32_t q0 = smem_u32(sq), k0 = smem_u32(smem + kOffK + (t & 1) * kKTile);
+                const uint32_t k0 = smem_u32(smem + kOffK + (t & 1) * kKTile);
 #pragma unroll
                 for (int k = 0; k < kHD / 16; ++k) {
                     const uint32_t qo = (uint32_t)(k >> 2) * kQHalf + (uint32_t)(k & 3) * 32u;
@@ -200,51 +215,36 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                 }
                 umma::commit(&ctl->bar_s[t & 1]);
             };
-            bool ok = true;
-            mbar_arrive_expect_tx(&ctl->bar_q, kQTile);
-            const int qrow = j * a.T + lo + qt * kBQ;
-            tma_load_2d(sq, &tm_q, hh * kHD, qrow, &ctl->bar_q);
-            tma_load_2d(sq + kQHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
-            for (int t = 0; t < 2 && t < nkt; ++t) {
-                load_k(t);
-                load_v(t);
-            }
-            ok = attn_wait(&ctl->bar_q, 0, ctl, a.status) &&
-                 attn_wait(&ctl->bar_k[0], 0, ctl, a.status);
+            // S(t): K(t) landed and the softmax has read S(t-2) (same buffer)
+            auto ready_s = [&](int t) {
+                return attn_wait(&ctl->bar_k[t & 1], (uint32_t)(t >> 1) & 1u, ctl, a.status) &&
+                       (t < 2 || attn_wait(&ctl->s_free[t & 1], (uint32_t)((t - 2) >> 1) & 1u, ctl,
+                                           a.status));
+            };
+            bool ok = attn_wait(&ctl->bar_q, 0, ctl, a.status) && ready_s(0);
             if (ok) {
                 umma::fence_after_sync();
                 issue_s(0);
             }
-            for (int kt = 0; kt < nkt && ok; ++kt) {
-                const int b = kt & 1;
-                // S(kt+1): K(kt+1) landed and the softmax is done with S(kt-1)
-                if (kt + 1 < nkt) {
-                    ok = (kt == 0 || attn_wait(&ctl->s_free[b ^ 1], (uint32_t)((kt - 1) >> 1) & 1u,
-                                               ctl, a.status)) &&
-                         attn_wait(&ctl->bar_k[b ^ 1], (uint32_t)((kt + 1) >> 1) & 1u, ctl,
-                                   a.status);
-                    if (!ok)
+            for (int t = 0; t < nkt && ok; ++t) {
+                if (t + 1 < nkt) {
+                    if (!(ok = ready_s(t + 1)))
                         break;
                     umma::fence_after_sync();
-                    issue_s(kt + 1);
+                    issue_s(t + 1);
                 }
-                // K(b) is free once S(kt) has completed: prefetch K(kt+2)
-                if (kt + 2 < nkt) {
-                    if (!(ok = attn_wait(&ctl->bar_s[b], (uint32_t)(kt >> 1) & 1u, ctl, a.status)))
-                        break;
-                    load_k(kt + 2);
-                }
-                // O += P(kt) V(kt) once P is written and V(kt) landed
-                ok = attn_wait(&ctl->p_full, (uint32_t)kt & 1u, ctl, a.status) &&
-                     attn_wait(&ctl->bar_v[b], (uint32_t)(kt >> 1) & 1u, ctl, a.status);
+                // O += P(t) V(t): P(t) written (which the softmax does only
+                // after P(t-1) V(t-1) completed) and V(t) landed
+                ok = attn_wait(&ctl->p_full, (uint32_t)t & 1u, ctl, a.status) &&
+                     attn_wait(&ctl->bar_v[t & 1], (uint32_t)(t >> 1) & 1u, ctl, a.status);
                 if (!ok)
                     break;
-                const int kmax = a.seq_len - 1 - kt * kBKV;   // last valid key row in tile
+                const int kmax = a.seq_len - 1 - t * kBKV;   // last valid key row in tile
+                uint8_t *sv = smem + kOffV + (t & 1) * kKTile;
                 if (kmax < kBKV - 1) {
                     // keys past the sequence's end may be uninitialised cache
                     // memory: clear those V rows so that 0 * garbage cannot
                     // reach P V
-                    uint8_t *sv = smem + kOffV + b * kKTile;
                     for (int rr = max(kmax + 1, 0); rr < kBKV; ++rr)
                         for (int c = 0; c < 16; ++c)
                             *reinterpret_cast<uint4 *>(sv + (c >> 3) * kKHalf + rr * 128 +
@@ -252,36 +252,56 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                     fence_proxy_async_smem();
                 }
                 umma::fence_after_sync();
-                const uint32_t p0 = smem_u32(sp), v0 = smem_u32(smem + kOffV + b * kKTile);
+                const uint32_t v0 = smem_u32(sv);
 #pragma unroll
                 for (int k = 0; k < kBKV / 16; ++k) {
                     const uint32_t aoff = (uint32_t)k * 32u;          // 16 keys of the P row
                     const uint32_t boff = (uint32_t)k * 16u * 128u;   // 16 key rows of V
                     umma::mma_bf16(t_pv, umma::desc_kmajor_sw128(p0 + aoff),
                                    umma::desc_mnmajor_sw128(v0 + boff, kKHalf), idesc_pv,
-                                   (kt | k) != 0);
+                                   (t | k) != 0);
                 }
-                umma::commit(&ctl->bar_pv);
-                ++npv;
-                // V(b) is free once PV(kt) has completed: prefetch V(kt+2)
-                if (kt + 2 < nkt) {
-                    if (!(ok = attn_wait(&ctl->bar_pv, (uint32_t)kt & 1u, ctl, a.status)))
-                        break;
-                    load_v(kt + 2);
-                }
+                umma::commit(&ctl->bar_pv[t & 1]);
             }
             if (!ok) {
-                // let this CTA's copies and MMAs in flight land
-                for (int b = 0; b < 2; ++b) {
-                    if (nk[b] > 0)
-                        mbar_wait(&ctl->bar_k[b], (uint32_t)(nk[b] - 1) & 1u);
-                    if (nv[b] > 0)
-                        mbar_wait(&ctl->bar_v[b], (uint32_t)(nv[b] - 1) & 1u);
-                }
-                umma::commit(&ctl->bar_pv);
-                mbar_wait(&ctl->bar_pv, (uint32_t)npv & 1u);
+                // let every MMA issued so far complete before TMEM is freed
+                umma::commit(&ctl->bar_end);
+                mbar_wait(&ctl->bar_end, 0);
             }
-            (void)ns;
+        }
+    } else if (warp == kKWarp || warp == kVWarp) {
+        // ---------------------------------------- TMA copies (one lane each)
+        // K(t) [V(t)] overwrites the buffer of K(t-2) [V(t-2)] once S(t-2)
+        // [P(t-2) V(t-2)] has completed.
+        if (lane == 0) {
+            const bool is_k = warp == kKWarp;
+            const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+            uint8_t *buf0 = smem + (is_k ? kOffK : kOffV);
+            uint64_t *full = is_k ? ctl->bar_k : ctl->bar_v;
+            uint64_t *done = is_k ? ctl->bar_s : ctl->bar_pv;
+            if (is_k) {
+                mbar_arrive_expect_tx(&ctl->bar_q, kQTile);
+                const int qrow = j * a.T + lo + qt * kBQ;
+                tma_load_2d(sq, &tm_q, hh * kHD, qrow, &ctl->bar_q);
+                tma_load_2d(sq + kQHalf, &tm_q, hh * kHD + 64, qrow, &ctl->bar_q);
+            }
+            int n = 0;                   // copies issued
+            for (; n < nkt; ++n) {
+                if (n >= 2 && !attn_wait(&done[n & 1], (uint32_t)((n - 2) >> 1) & 1u, ctl, a.status))
+                    break;
+                uint8_t *dst = buf0 + (n & 1) * kKTile;
+                const int krow = (int)(kvrow0 + (int64_t)n * kBKV);
+                mbar_arrive_expect_tx(&full[n & 1], kKTile);
+                tma_load_2d(dst, tm, 0, krow, &full[n & 1]);
+                tma_load_2d(dst + kKHalf, tm, 64, krow, &full[n & 1]);
+            }
+            if (n < nkt) {
+                // error path: the last copy into each buffer must land before exit
+                for (int t = n - 1; t >= 0 && t >= n - 2; --t)
+                    mbar_wait(&full[t & 1], (uint32_t)(t >> 1) & 1u);
+                if (is_k)
+                    mbar_wait(&ctl->bar_q, 0);
+            }
         }
     } else {
         // ---------------------------------------- softmax warps (rows 0..127)
@@ -320,10 +340,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                     if (!(live && k0 + e <= pos))
                         v[e] = -INFINITY;
             }
-            float vmax = v[0];
+            // row max over 8 independent chains
+            float vm[8];
 #pragma unroll
-            for (int e = 1; e < kBKV; ++e)
-                vmax = fmaxf(vmax, v[e]);
+            for (int e = 0; e < 8; ++e)
+                vm[e] = v[e];
+#pragma unroll
+            for (int e = 8; e < kBKV; ++e)
+                vm[e & 7] = fmaxf(vm[e & 7], v[e]);
+            const float vmax = fmaxf(fmaxf(fmaxf(vm[0], vm[1]), fmaxf(vm[2], vm[3])),
+                                     fmaxf(fmaxf(vm[4], vm[5]), fmaxf(vm[6], vm[7])));
             const float mt = vmax * sc;                       // -inf if no key is visible
             // move the reference max when the running max passes it by > 8
             float alpha = 1.f;
@@ -334,18 +360,20 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             // probabilities (bf16 pairs) while the previous tile's P V may
             // still run: only storing P and rescaling O wait for it
             const float mb = m_ref > -INFINITY ? m_ref : 0.f;
-            float lsum = 0.f;
+            float ls[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pw[kBKV / 2];
 #pragma unroll
             for (int e = 0; e < kBKV; e += 2) {
-                const float p0 = exp2f(fmaf(v[e], sc, -mb)), p1 = exp2f(fmaf(v[e + 1], sc, -mb));
-                lsum += p0 + p1;
+                const float p0 = exp2_sfu(fmaf(v[e], sc, -mb)),
+                            p1 = exp2_sfu(fmaf(v[e + 1], sc, -mb));
+                ls[(e >> 1) & 3] += p0 + p1;
                 const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
                 pw[e / 2] = *reinterpret_cast<const uint32_t *>(&b2);
             }
             // the previous tile's P V is done: P is free, O is stable
             if (kt > 0) {
-                w = attn_wait(&ctl->bar_pv, (uint32_t)(kt - 1) & 1u, ctl, a.status);
+                w = attn_wait(&ctl->bar_pv[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, ctl,
+                              a.status);
                 if (!__all_sync(0xffffffffu, w)) {
                     ok = false;
                     break;
@@ -370,7 +398,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
             for (int g8 = 0; g8 < kBKV / 8; ++g8)
                 *reinterpret_cast<uint4 *>(sp + swz128(tid, g8)) =
                     make_uint4(pw[4 * g8], pw[4 * g8 + 1], pw[4 * g8 + 2], pw[4 * g8 + 3]);
-            l = l * alpha + lsum;
+            l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
             fence_proxy_async_smem();       // P written by threads, read by the tensor core
             umma::fence_before_sync();
             __syncwarp();
@@ -378,7 +406,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                 mbar_arrive(&ctl->p_full);
         }
         if (ok) {
-            const bool w = attn_wait(&ctl->bar_pv, (uint32_t)(nkt - 1) & 1u, ctl, a.status);
+            const bool w = attn_wait(&ctl->bar_pv[(nkt - 1) & 1], (uint32_t)((nkt - 1) >> 1) & 1u,
+                                     ctl, a.status);
             ok = __all_sync(0xffffffffu, w);
         }
         if (ok) {
