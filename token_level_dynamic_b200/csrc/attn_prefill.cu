@@ -65,6 +65,7 @@ __device__ __forceinline__ float exp2_sfu(float x)
 struct AttnPArgs {
     const int32_t *count, *perm, *sig_pos;   // head-group work list
     int T, seq_len, n_kv, rep, qcols, ocols;
+    int n_seq, q_tiles;                      // grid: q_tiles x rep x n_seq x n_kv CTAs
     int64_t cache_cap;
     float scale_log2;                        // log2(e) / sqrt(hd)
     __nv_bfloat16 *o_sig;                    // [T][n_q * hd]
@@ -150,8 +151,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     uint8_t *sq = smem, *sp = smem + kOffP;
     ACtl *ctl = reinterpret_cast<ACtl *>(smem + kOffCtl);
-    const int qt = blockIdx.x, hh = blockIdx.y;
-    const int s = blockIdx.z / a.n_kv, j = blockIdx.z % a.n_kv;
+    // one-dimensional grid, query tile slowest and in descending order: the
+    // tiles with the most key steps start first and the short ones fill in
+    // at the end (empty tiles, the highest, come first and exit at once)
+    const int nsk = a.n_seq * a.n_kv, per_qt = nsk * a.rep;
+    const int qt = a.q_tiles - 1 - (int)(blockIdx.x / (unsigned)per_qt);
+    const int rem = (int)(blockIdx.x % (unsigned)per_qt);
+    const int hh = rem / nsk, s = (rem % nsk) / a.n_kv, j = rem % a.n_kv;
     const int32_t *pj = a.perm + (size_t)j * a.T;
 
     // this sequence's queries of group j: [lo, hi) of the group's token list
@@ -572,6 +578,8 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
     aa.seq_len = (int)d->seq_len;
     aa.n_kv = n_kv;
     aa.rep = rep;
+    aa.n_seq = (int)d->n_seq;
+    aa.q_tiles = (int)((d->seq_len + kBQ - 1) / kBQ);
     aa.qcols = qcols;
     aa.ocols = qd;
     aa.cache_cap = d->cache_cap;
@@ -582,8 +590,7 @@ int layer_prefill_launch(const LayerPtrs &p, const wide_layer_dims *d, void *ws,
         return WIDE_CUDA_FAIL();
     {
         LaunchScope scope(KID_PREFILL_ATTN, s);
-        const dim3 grid((unsigned)((d->seq_len + kBQ - 1) / kBQ), (unsigned)rep,
-                        (unsigned)(d->n_seq * n_kv));
+        const unsigned grid = (unsigned)aa.q_tiles * (unsigned)rep * (unsigned)(d->n_seq * n_kv);
         prefill_attn<<<grid, kAttnThreads, kAttnSmem, s>>>(tqc, tkc, tvc, aa);
     }
     if ((rc = launch_status()))
