@@ -1,5 +1,6 @@
-"""bench.py's host side on CPU: the reference arm's JSON line, and the
-algorithmic units the router workload divides by (no GPU needed)."""
+"""bench.py's host side on CPU: the reference arm's JSON line, the CPU
+leg, the clock record, and the algorithmic units (bytes or kept FLOPs) that
+the workloads divide by, against independent counts (no GPU needed)."""
 import json
 import os
 import subprocess
@@ -133,3 +134,67 @@ def test_decode_bytes_follow_the_per_launch_kernel_choice():
             u = int(c.mask[t0:t0 + n].any(axis=0).sum())
             w += 3 * u * gs * H * 2
         assert b["total"] == w + io
+
+
+def _prefill_flops_by_loops(lc, all_kept=False):
+    """Multiply-adds of the masked prefill layer counted one (token, group,
+    head) at a time, 2 FLOPs each: Q and o_proj per kept (token, head
+    group) pair and query head, attention over the query's causal keys
+    (QK^T and PV), K and V for every token, gate/up and down per kept
+    (token, channel group) pair."""
+    a, f = lc.attn, lc.ffn
+    rep = a.n_q // a.n_kv
+    n = {"q": 0, "kv": 0, "att": 0, "oproj": 0, "gateup": 0, "down": 0}
+    for t in range(a.T):
+        pos = t % a.seq_len + a.cache_len
+        n["kv"] += 2 * (2 * a.n_kv * a.hd) * a.H
+        for g in range(a.n_kv):
+            if all_kept or a.mask[t, g]:
+                for _ in range(rep):
+                    n["q"] += 2 * a.hd * a.H
+                    n["att"] += 2 * a.hd * (pos + 1) + 2 * (pos + 1) * a.hd
+                    n["oproj"] += 2 * a.hd * a.H
+        for g in range(f.I // f.gs):
+            if all_kept or f.mask[t, g]:
+                n["gateup"] += 2 * (2 * f.gs) * a.H
+                n["down"] += 2 * a.H * f.gs
+    return n
+
+
+def test_prefill_layer_kept_flops():
+    """The kept FLOPs that the prefill-layer line divides by, against a
+    per-pair count on a small layer; the dense figure is the same count
+    with every group kept."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    lc = synth.small_layer("prefill", seed=3, n_seq=2, seq_len=37, H=256, n_q=8, n_kv=2, hd=128,
+                           I=512, gs=64, keep_a=0.5, keep_f=0.5)
+    u = bench.WORKLOADS["prefill_layer_8b"].units(lc)
+    n = _prefill_flops_by_loops(lc)
+    assert (u["prefill_q_rope_tcgen05"], u["prefill_kv_rope_tcgen05"],
+            u["prefill_attention_tcgen05"], u["prefill_oproj_tcgen05"],
+            u["prefill_gateup_tcgen05"], u["prefill_down_tcgen05"]) == \
+        (n["q"], n["kv"], n["att"], n["oproj"], n["gateup"], n["down"])
+    assert u["total"] == sum(n.values())
+    assert u["dense_flops"] == sum(_prefill_flops_by_loops(lc, all_kept=True).values())
+    assert 0 < u["total"] < u["dense_flops"]
+
+
+def test_prefill_ffn_kept_flops():
+    """The prefill FFN line's kept FLOPs equal the per-pair count of the
+    layer test above (its FFN part) on a small masked FFN."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    c = synth.ffn_case(T=29, H=256, I=512, gs=64, seed=5, keep=0.5)
+    u = bench.WORKLOADS["prefill_ffn_8b"].units(c)
+    gateup = down = 0
+    for t in range(c.T):
+        for g in range(c.I // c.gs):
+            if c.mask[t, g]:
+                gateup += 2 * (2 * c.gs) * c.H
+                down += 2 * c.H * c.gs
+    assert (u["prefill_gateup_tcgen05"], u["prefill_down_tcgen05"]) == (gateup, down)
+    assert u["total"] == gateup + down and u["pairs"] == int(c.mask.sum())
+    assert u["dense_flops"] == 3 * 2 * c.T * c.H * c.I
